@@ -1,0 +1,543 @@
+#!/usr/bin/env python
+"""Benchmark of rank-major MoE EP dispatch + combine on B200 (virtual EP ranks).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: the routing plan and
+EPLB gather, the dispatch row copy, and the BF16 combine, on the prefill
+workload (ep 8, 256 experts, top_k 8, 4096 tokens per rank, hidden 7168 BF16,
+64 extra bytes per token, EPLB statistics).  Inputs are resident in HBM when
+the timed region starts; they are larger than L2, so no flush is needed.
+Rank 0 prints one JSON line.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own independent
+replica of the workload (the path has no exchange between GPUs: all EP ranks
+are virtual ranks of one GPU); the timed region is bracketed by barriers and
+the max over ranks is reported (weak scaling).
+
+`--impl reference` times the plain CPU oracle on the host cores instead (rank 0
+only), on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "c4_ep8_prefill"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------------------- #
+# Process group helpers (also exercised on CPU with gloo by the tests)
+# --------------------------------------------------------------------------- #
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_group(backend: str, timeout_s: float = 120.0):
+    import torch.distributed as dist
+    ws, rank, _ = dist_env()
+    if ws > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return dist if ws > 1 else None
+
+
+def reduce_max(value: float, dist, device=None) -> float:
+    """Max over ranks (identity on one rank)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device=None):
+    if dist is None:
+        return
+    if device is not None and device.type == "cuda":
+        dist.barrier(device_ids=[device.index])
+    else:
+        dist.barrier()
+
+
+class CudaTimer:
+    """Device time between two events on the launching stream."""
+
+    def __init__(self, stream):
+        import torch
+        self.torch = torch
+        self.stream = stream
+        self.a = torch.cuda.Event(enable_timing=True)
+        self.b = torch.cuda.Event(enable_timing=True)
+
+    def start(self):
+        self.torch.cuda.synchronize()
+        self.a.record(self.stream)
+
+    def stop(self) -> float:
+        self.b.record(self.stream)
+        self.torch.cuda.synchronize()
+        return float(self.a.elapsed_time(self.b))
+
+
+class WallTimer:
+    """Host clock; used only by the CPU tests of the harness and the oracle arm."""
+
+    def start(self):
+        self.t = time.perf_counter()
+
+    def stop(self) -> float:
+        return (time.perf_counter() - self.t) * 1e3
+
+
+def run_timed(step, steps: int, warmup: int, timer, dist, device=None,
+              during=None, on_start=None) -> float:
+    """W untimed steps, then exactly K timed steps bracketed by barriers and
+    synchronisation; returns the max over ranks of the elapsed milliseconds.
+    `on_start` runs after the warm-up, before the timed region opens."""
+    for _ in range(warmup):
+        step()
+    if on_start is not None:
+        on_start()
+    barrier(dist, device)
+    timer.start()
+    if during is not None:
+        during.start()
+    for _ in range(steps):
+        step()
+    ms = timer.stop()
+    if during is not None:
+        during.stop()
+    barrier(dist, device)
+    return reduce_max(ms, dist, device)
+
+
+# --------------------------------------------------------------------------- #
+# Clocks during the timed region (NVML reads only; nothing is changed)
+# --------------------------------------------------------------------------- #
+
+_REASONS = [(0x1, "gpu_idle"), (0x2, "applications_clocks_setting"), (0x4, "sw_power_cap"),
+            (0x8, "hw_slowdown"), (0x10, "sync_boost"), (0x20, "sw_thermal_slowdown"),
+            (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"),
+            (0x100, "display_clock_setting")]
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.error = None
+        self.handle = None
+        try:
+            import pynvml
+            self.nvml = pynvml
+            pynvml.nvmlInit()
+            try:
+                import torch
+                p = torch.cuda.get_device_properties(device_index)
+                bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+                self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self.reason_fn = fn
+        except Exception as e:  # no NVML: report it, do not fail the bench
+            self.error = f"{type(e).__name__}: {e}"
+
+    def _loop(self):
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.handle,
+                                                                     self.nvml.NVML_CLOCK_SM))
+                self.reasons |= int(self.reason_fn(self.handle))
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                return
+            time.sleep(self.period)
+
+    def start(self):
+        self.stop_flag = threading.Event()
+        if self.handle is None:
+            return
+        self.thread = threading.Thread(target=self._loop, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        self.stop_flag.set()
+        if self.handle is not None:
+            self.thread.join()
+
+    def record(self):
+        r = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+             "sm_max_mhz": self.max_mhz,
+             "reasons": [n for bit, n in _REASONS if self.reasons & bit],
+             "samples": len(self.samples)}
+        if self.error:
+            r["error"] = self.error
+        return r
+
+
+# --------------------------------------------------------------------------- #
+# Algorithmic bytes (what the method must move; invalid rows and the dense
+# ep x tpr capacity excluded)
+# --------------------------------------------------------------------------- #
+
+@dataclasses.dataclass
+class Bytes:
+    copy: int          # dispatch row copy: rows read once + written once per destination
+    combine: int       # combine: valid rows read + output written
+    route: int         # ids read, per-destination ids / valid rows, plan, counts, EPLB
+    step: int
+
+
+def algorithmic_bytes(w, n_tok: int, sum_d: int, live: int, fp8: bool) -> Bytes:
+    rb = sum(w.payload_row_bytes())
+    k, ep, tpr, E, H = w.top_k, w.ep_size, w.tokens_per_rank, w.num_experts, w.hidden
+    copy = n_tok * rb + sum_d * rb
+    combine = sum_d * H * (1 if fp8 else 2) + n_tok * H * 2
+    route = n_tok * k * 4 * (1 + 0) + sum_d * k * 4 + live * ep * tpr + ep * ep * 4
+    if w.eplb:
+        route += ep * E * 4 + live * ep * E * 4
+    return Bytes(copy, combine, route, copy + combine + route)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sources_hash() -> str:
+    """Hash of the CUDA sources, to tell whether committed ncu counters still
+    describe the kernels that run."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "combine_route_plan_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel: str, workload: str):
+    """dram bytes per launch from profiles/dram_traffic.json, if it was taken on
+    these exact kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        if d.get("sources_hash") != kernel_sources_hash():
+            return None
+        e = d["kernels"][kernel]
+        if e.get("workload") != workload:
+            return None
+        return int(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------------------- #
+# Our arm
+# --------------------------------------------------------------------------- #
+
+def run_ours(args):
+    import torch
+    from combine_route_plan_b200 import ep_a2a
+    from combine_route_plan_b200 import workloads as W
+
+    ws, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_group("nccl")
+    w = W.BY_NAME[args.workload]
+    x = W.make_inputs(w)
+    stream = torch.cuda.current_stream()
+
+    ids = x.token_selected_experts.to(device)
+    payloads = [p.to(device) for p in x.payloads]
+    stats = x.eplb_local_stats.to(device) if x.eplb_local_stats is not None else None
+    xo = x.expert_output.to(device)
+    xo8 = ep_a2a.quantize_e4m3(xo)
+    n = x.local_num_tokens
+    mask = x.active_rank_mask
+    comm = ep_a2a.EpA2A(w.ep_size, w.num_experts, w.top_k, w.tokens_per_rank, w.hidden,
+                        w.payload_row_bytes(), eplb_stats_num_experts=w.num_experts if w.eplb else 0,
+                        enable_rank_mask=mask is not None)
+    out = torch.empty((w.ep_size, w.tokens_per_rank, w.hidden), dtype=torch.bfloat16, device=device)
+    tpr = w.tokens_per_rank
+    fp8 = args.combine == "fp8"
+    comb_in = xo8 if fp8 else xo
+
+    def step():
+        comm.dispatch(ids, n, payloads, tpr, stats, mask, views=False)
+        comm.combine(comb_in, out)
+
+    step()
+    torch.cuda.synchronize()
+    d = comm.dispatch(ids, n, payloads, tpr, stats, mask)
+    torch.cuda.synchronize()
+    assert comm.get_status() == ep_a2a.OK
+    sum_d = int(d.send_counts.sum().item())
+    live = w.ep_size - len(w.masked_ranks)
+    n_tok = int(sum(int(n[r]) for r in range(w.ep_size) if r not in w.masked_ranks))
+    by = algorithmic_bytes(w, n_tok, sum_d, live, fp8)
+
+    clocks = ClockSampler(local)
+    ms = run_timed(step, args.steps, args.warmup, CudaTimer(stream), dist, device, during=clocks,
+                   on_start=lambda: ep_a2a.ep_a2a_profile_start(comm.handle, 4 * args.steps + 8))
+    kt = ep_a2a.ep_a2a_profile_stop(comm.handle)
+    assert comm.get_status() == ep_a2a.OK
+    ms_per_step = ms / args.steps
+    tokens_total = ws * n_tok * args.steps
+    value = tokens_total / (ms / 1e3)
+    peak, peak_kind = load_peaks()
+
+    per_kernel = {}
+    for name, (cnt, tot) in kt.items():
+        if cnt:
+            per_kernel[name] = {"launches": cnt, "avg_ms": tot / cnt}
+    kbytes = {"route_plan": by.route, "copy_bulk": by.copy, "copy_vec": by.copy,
+              "combine": by.combine}
+    for name, e in per_kernel.items():
+        e["algorithmic_bytes"] = kbytes[name]
+        e["achieved_gbs"] = kbytes[name] / (e["avg_ms"] / 1e3) / 1e9
+        e["frac_of_peak"] = e["achieved_gbs"] / peak
+    dominant = max(per_kernel, key=lambda k: per_kernel[k]["avg_ms"] * per_kernel[k]["launches"])
+    dk = per_kernel[dominant]
+    step_gbs = by.step / (ms_per_step / 1e3) / 1e9
+
+    # FP8 combine, timed alone on the same plan (context, not the headline)
+    fp8_ctx = None
+    if not fp8 and args.fp8_steps > 0:
+        comm.dispatch(ids, n, payloads, tpr, stats, mask)
+        t8 = run_timed(lambda: comm.combine(xo8, out), args.fp8_steps, 3, CudaTimer(stream),
+                       dist, device, on_start=lambda: ep_a2a.ep_a2a_profile_start(
+                           comm.handle, args.fp8_steps + 4))
+        k8 = ep_a2a.ep_a2a_profile_stop(comm.handle)["combine"]
+        b8 = algorithmic_bytes(w, n_tok, sum_d, live, True).combine
+        avg8 = k8[1] / k8[0]
+        fp8_ctx = {"avg_ms": avg8, "algorithmic_bytes": b8,
+                   "achieved_gbs": b8 / (avg8 / 1e3) / 1e9, "frac_of_peak": b8 / (avg8 / 1e3) / 1e9 / peak,
+                   "loop_ms_per_launch": t8 / args.fp8_steps}
+
+    e2e = None
+    if args.e2e_steps > 0:
+        e2e = run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws)
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_seconds)
+
+    if rank == 0:
+        rec = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": f"{w.name}: ep_size {w.ep_size}, num_experts {w.num_experts}, "
+                            f"top_k {w.top_k}, {tpr} tokens/rank, hidden {w.hidden} BF16, "
+                            f"extra {w.extra_bytes} B/token, EPLB stats, "
+                            f"{'FP8 E4M3' if fp8 else 'BF16'} combine (fp32 accumulate)",
+                "tokens_per_step_per_gpu": n_tok, "mean_distinct_ranks": sum_d / n_tok,
+                "l2": "inputs larger than L2 (no flush)",
+                "parallelism": f"{ws} independent replicas" if ws > 1 else "1 GPU, virtual ranks",
+            },
+            "hbm": {"step_algorithmic_bytes": by.step, "achieved_gbs": step_gbs,
+                    "peak_gbs": peak, "peak_kind": peak_kind, "frac": step_gbs / peak},
+            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": dk["achieved_gbs"],
+                         "peak": peak, "unit": "GB/s", "frac": dk["frac_of_peak"],
+                         "peak_kind": peak_kind,
+                         "traffic": committed_traffic(dominant, w.name)},
+            "kernels": per_kernel,
+            "gpu_launches": sum(e["launches"] for e in per_kernel.values()),
+            "clocks": clocks.record(),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "kernel_sources": kernel_sources_hash(),
+        }
+        if fp8_ctx:
+            rec["fp8_combine"] = fp8_ctx
+        print(json.dumps(rec), flush=True)
+    comm.destroy()
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws):
+    """Same step through the public API with the inputs in pinned host memory:
+    every step copies the inputs host->device and the result device->host."""
+    import torch
+    h_ids = x.token_selected_experts.pin_memory()
+    h_pay = [p.pin_memory() for p in x.payloads]
+    h_stats = x.eplb_local_stats.pin_memory() if x.eplb_local_stats is not None else None
+    h_xo = x.expert_output.pin_memory()
+    h_out = torch.empty((w.ep_size, w.tokens_per_rank, w.hidden), dtype=torch.bfloat16).pin_memory()
+    d_ids = torch.empty_like(h_ids, device=device)
+    d_pay = [torch.empty_like(p, device=device) for p in h_pay]
+    d_stats = torch.empty_like(h_stats, device=device) if h_stats is not None else None
+    d_xo = torch.empty_like(h_xo, device=device)
+    d_out = torch.empty_like(h_out, device=device)
+    h2d = h_ids.nbytes + sum(p.nbytes for p in h_pay) + h_xo.nbytes + \
+        (h_stats.nbytes if h_stats is not None else 0)
+    d2h = h_out.nbytes
+
+    def step():
+        d_ids.copy_(h_ids, non_blocking=True)
+        for d, h in zip(d_pay, h_pay):
+            d.copy_(h, non_blocking=True)
+        if d_stats is not None:
+            d_stats.copy_(h_stats, non_blocking=True)
+        d_xo.copy_(h_xo, non_blocking=True)
+        comm.dispatch(d_ids, x.local_num_tokens, d_pay, w.tokens_per_rank, d_stats,
+                      x.active_rank_mask, views=False)
+        comm.combine(d_xo, d_out)
+        h_out.copy_(d_out, non_blocking=True)
+
+    ms = run_timed(step, args.e2e_steps, 2, CudaTimer(stream), dist, device)
+    return {"value": ws * n_tok * args.e2e_steps / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": args.e2e_steps, "ms_per_step": ms / args.e2e_steps}
+
+
+# --------------------------------------------------------------------------- #
+# The oracle on the host cores
+# --------------------------------------------------------------------------- #
+
+def oracle_step(w, x):
+    """One pass of the whole path in the CPU oracle."""
+    import oracle
+    plan = oracle.route(w.ep_size, w.num_experts, w.top_k, w.tokens_per_rank,
+                        x.token_selected_experts.numpy(), x.local_num_tokens, x.active_rank_mask)
+    for p in x.payloads:
+        oracle.dispatch_payload(plan, p.numpy())
+    if x.eplb_local_stats is not None:
+        oracle.eplb_gather(w.ep_size, x.eplb_local_stats.numpy(), x.active_rank_mask)
+    xo = x.expert_output.view(__import__("torch").int16).numpy().view(np.uint16)
+    oracle.combine(plan, xo, w.hidden)
+    return int(sum(int(x.local_num_tokens[r]) for r in range(w.ep_size)
+                   if r not in w.masked_ranks))
+
+
+def cpu_baseline(w, seconds: float, tokens_per_rank: int = 1024):
+    """The oracle as it stands, single-threaded, on a bounded sample of the
+    workload: the same shapes with fewer tokens per rank, repeated for at
+    least `seconds`."""
+    from combine_route_plan_b200 import workloads as W
+    import oracle
+    oracle.build()
+    ws = W.scaled(w, min(tokens_per_rank, w.tokens_per_rank))
+    xs = W.make_inputs(ws)
+    oracle_step(ws, xs)            # untimed: page in buffers
+    t0 = time.perf_counter()
+    toks = reps = 0
+    while True:
+        toks += oracle_step(ws, xs)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": toks / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{ws.name}: {ws.tokens_per_rank} tokens/rank "
+                      f"({toks // reps} tokens) x {reps} steps, route + dispatch + EPLB + "
+                      f"BF16 combine, {dt:.1f} s, single thread",
+            "host_cpus": os.cpu_count()}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return                      # rank 0 alone runs the CPU oracle
+    from combine_route_plan_b200 import workloads as W
+    import oracle
+    oracle.build()
+    w = W.BY_NAME[args.workload]
+    # size each step's sample so that warm-up + K steps take about args.ref_budget_s
+    probe = W.scaled(w, 64)
+    xp = W.make_inputs(probe)
+    oracle_step(probe, xp)
+    t0 = time.perf_counter()
+    tok = oracle_step(probe, xp)
+    per_tok = (time.perf_counter() - t0) / max(tok, 1)
+    per_step_s = args.ref_budget_s / max(1, args.steps + args.warmup)
+    tpr = int(min(w.tokens_per_rank, max(8, per_step_s / per_tok / w.ep_size)))
+    ws_ = W.scaled(w, tpr)
+    xs = W.make_inputs(ws_)
+    n_tok = [0]
+
+    def step():
+        n_tok[0] = oracle_step(ws_, xs)
+
+    ms = run_timed(step, args.steps, args.warmup, WallTimer(), None)
+    value = n_tok[0] * args.steps / (ms / 1e3)
+    sample = (f"{ws_.name}: {tpr} tokens/rank ({n_tok[0]} tokens) per step, route + dispatch + "
+              f"EPLB + BF16 combine, single thread")
+    rec = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name} (bounded samples of {tpr} tokens/rank per step)",
+                   "l2": "host run"},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample, "host_cpus": os.cpu_count()},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(rec), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--combine", choices=["bf16", "fp8"], default="bf16")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--fp8-steps", type=int, default=100)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget-s", type=float, default=120.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

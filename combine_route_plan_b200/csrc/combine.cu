@@ -1,0 +1,221 @@
+// Combine of rank-major MoE dispatch (flashinfer.moe_ep.NVLinkTwoSidedAlltoAll,
+// combine()): each existing token (src, t) gets the sum of the rows its
+// destination ranks return, already weighted and reduced over each rank's local
+// experts.  The sum is an fp32 accumulator that starts at +0.0f and adds the
+// rows in ascending destination-rank order with round-to-nearest adds, then is
+// rounded once to bf16 (nearest-even).  With the low-precision combine
+// (flashinfer.moe_ep.NVLinkOneSidedConfig, use_low_precision_combine) the rows
+// are E4M3, widened exactly to fp32 before the same sum.
+//
+// Memory plan: one CTA per token (grid-stride); each thread owns 16-byte column
+// vectors of the row and issues the loads of all (up to 8 at a time)
+// destination rows before the adds, so one thread keeps up to 128 bytes in
+// flight.  Loads bypass L1 (each row is read exactly once).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include "ep_a2a_internal.cuh"
+
+namespace ep_a2a {
+namespace {
+
+__device__ __forceinline__ int dst_rank(uint64_t w0, uint64_t w1, uint64_t w2, uint64_t w3,
+                                        int i) {
+  const uint64_t w = i < 8 ? w0 : (i < 16 ? w1 : (i < 24 ? w2 : w3));
+  return (int)((w >> ((i & 7) * 8)) & 0xFFu);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) {
+  return __uint_as_float(bits16 << 16);
+}
+
+__device__ __forceinline__ uint32_t f32_to_bf16_bits(float f) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+// Add the 8 bf16 of a 16-byte vector into acc[0..8).
+__device__ __forceinline__ void add_bf16x8(float* acc, const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] = __fadd_rn(acc[2 * i], bf16_bits_to_f32(w[i] & 0xFFFFu));
+    acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], bf16_bits_to_f32(w[i] >> 16));
+  }
+}
+
+// Add the 16 E4M3 of a 16-byte vector into acc[0..16) (exact widening).
+__device__ __forceinline__ void add_e4m3x16(float* acc, const uint4& v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * h)) & 0xFFFFu);
+      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+      __half_raw lo, hi;
+      lo.x = hr.x;
+      hi.x = hr.y;
+      acc[4 * i + 2 * h] = __fadd_rn(acc[4 * i + 2 * h], __half2float(__half(lo)));
+      acc[4 * i + 2 * h + 1] = __fadd_rn(acc[4 * i + 2 * h + 1], __half2float(__half(hi)));
+    }
+  }
+}
+
+template <bool kFp8>
+__global__ void combine_vec_kernel(const CombineArgs a) {
+  constexpr int kElems = kFp8 ? 16 : 8;       // elements per 16-byte input vector
+  constexpr int kElemBytes = kFp8 ? 1 : 2;
+  const int nvec = a.H / kElems;
+  const int words = a.plan_stride / 8;
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    const int nd = a.plan_nd[tok];
+    if (nd == kNoToken) continue;
+    const uint64_t* row = reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    const uint64_t w0 = row[0];
+    const uint64_t w1 = words > 1 ? row[1] : 0;
+    const uint64_t w2 = words > 2 ? row[2] : 0;
+    const uint64_t w3 = words > 3 ? row[3] : 0;
+    const uint8_t* xt = a.x + tok * (int64_t)a.H * kElemBytes;           // rank 0's row
+    const int64_t rank_stride = a.ntok * (int64_t)a.H * kElemBytes;      // bytes per rank
+    uint16_t* out = a.out + tok * (int64_t)a.H;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      float acc[kElems];
+#pragma unroll
+      for (int e = 0; e < kElems; ++e) acc[e] = 0.0f;
+      for (int c0 = 0; c0 < nd; c0 += 8) {
+        uint4 raw[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (c0 + i < nd)
+            raw[i] = ld_stream_v4(xt + (int64_t)dst_rank(w0, w1, w2, w3, c0 + i) * rank_stride +
+                                  (int64_t)v * 16);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (c0 + i < nd) {
+            if (kFp8)
+              add_e4m3x16(acc, raw[i]);
+            else
+              add_bf16x8(acc, raw[i]);
+          }
+        }
+      }
+      uint4* o = reinterpret_cast<uint4*>(out + (int64_t)v * kElems);
+#pragma unroll
+      for (int q = 0; q < kElems / 8; ++q) {
+        uint4 pk;
+        pk.x = f32_to_bf16_bits(acc[8 * q + 0]) | (f32_to_bf16_bits(acc[8 * q + 1]) << 16);
+        pk.y = f32_to_bf16_bits(acc[8 * q + 2]) | (f32_to_bf16_bits(acc[8 * q + 3]) << 16);
+        pk.z = f32_to_bf16_bits(acc[8 * q + 4]) | (f32_to_bf16_bits(acc[8 * q + 5]) << 16);
+        pk.w = f32_to_bf16_bits(acc[8 * q + 6]) | (f32_to_bf16_bits(acc[8 * q + 7]) << 16);
+        o[q] = pk;
+      }
+    }
+  }
+}
+
+// Any hidden size and alignment: one element per thread step.
+template <bool kFp8>
+__global__ void combine_scalar_kernel(const CombineArgs a) {
+  const int words = a.plan_stride / 8;
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    const int nd = a.plan_nd[tok];
+    if (nd == kNoToken) continue;
+    const uint64_t* row = reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    const uint64_t w0 = row[0];
+    const uint64_t w1 = words > 1 ? row[1] : 0;
+    const uint64_t w2 = words > 2 ? row[2] : 0;
+    const uint64_t w3 = words > 3 ? row[3] : 0;
+    for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
+      float acc = 0.0f;
+      for (int i = 0; i < nd; ++i) {
+        const int64_t idx = ((int64_t)dst_rank(w0, w1, w2, w3, i) * a.ntok + tok) * a.H + h;
+        float x;
+        if (kFp8) {
+          const __half_raw hr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)a.x[idx], __NV_E4M3);
+          x = __half2float(__half(hr));
+        } else {
+          x = bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(a.x)[idx]);
+        }
+        acc = __fadd_rn(acc, x);
+      }
+      a.out[tok * (int64_t)a.H + h] = (uint16_t)f32_to_bf16_bits(acc);
+    }
+  }
+}
+
+// bf16 -> E4M3, round to nearest even, saturating (satfinite).
+__global__ void quantize_e4m3_kernel(const uint16_t* __restrict__ in, uint8_t* __restrict__ out,
+                                     int64_t n, bool vec) {
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  int64_t n_vec = 0;
+  if (vec) {
+    n_vec = n / 8;
+    for (int64_t i = tid; i < n_vec; i += stride) {
+      const uint4 v = reinterpret_cast<const uint4*>(in)[i];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o[2] = {0u, 0u};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = make_float2(bf16_bits_to_f32(w[q] & 0xFFFFu), bf16_bits_to_f32(w[q] >> 16));
+        const uint32_t pair = (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+        o[q >> 1] |= pair << (16 * (q & 1));
+      }
+      reinterpret_cast<uint2*>(out)[i] = make_uint2(o[0], o[1]);
+    }
+    n_vec *= 8;
+  }
+  for (int64_t i = n_vec + tid; i < n; i += stride)
+    out[i] = (uint8_t)__nv_cvt_float_to_fp8(bf16_bits_to_f32(in[i]), __NV_SATFINITE, __NV_E4M3);
+}
+
+// Failure-detection probe: waits on a barrier whose byte count never arrives,
+// with a bounded wait; on expiry it sets the error word and returns.
+__global__ void wait_timeout_probe_kernel(uint32_t* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_addr(&bar);
+  mbar_init(b, 1);
+  mbar_init_fence();
+  mbar_arrive_expect_tx(b, 16);   // no copy will ever complete these 16 bytes
+  if (!mbar_wait_bounded(b, 0, limit_ns)) atomicOr(err, kErrWaitTimeout);
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, int threads, int grid,
+                           cudaStream_t stream) {
+  if (vec) {
+    if (fp8)
+      combine_vec_kernel<true><<<grid, threads, 0, stream>>>(a);
+    else
+      combine_vec_kernel<false><<<grid, threads, 0, stream>>>(a);
+  } else {
+    if (fp8)
+      combine_scalar_kernel<true><<<grid, threads, 0, stream>>>(a);
+    else
+      combine_scalar_kernel<false><<<grid, threads, 0, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n,
+                                 cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const bool vec = (reinterpret_cast<uintptr_t>(in) % 16 == 0) &&
+                   (reinterpret_cast<uintptr_t>(out) % 8 == 0);
+  const int threads = 256;
+  const int64_t work = vec ? (n / 8 + 1) : n;
+  const int grid = (int)std::min<int64_t>((work + threads - 1) / threads, 148 * 16);
+  quantize_e4m3_kernel<<<grid, threads, 0, stream>>>(in, out, n, vec);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_timeout_probe(uint32_t* err, unsigned long long limit_ns,
+                                      cudaStream_t stream) {
+  wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace ep_a2a

@@ -1,0 +1,577 @@
+// Host side of the C ABI declared in include/ep_a2a.h: argument validation,
+// workspace layout, and kernel launches.  No device memory is allocated here;
+// the caller owns the workspace and every input / output buffer.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "ep_a2a_internal.cuh"
+
+#define EP_API extern "C" __attribute__((visibility("default")))
+
+namespace ep_a2a {
+namespace {
+
+constexpr uint32_t kMagic = 0x45504132u;   // "EPA2"
+constexpr int64_t kAlign = 256;
+
+thread_local std::string g_last_error;
+
+ep_a2a_status fail(ep_a2a_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+ep_a2a_status fail(ep_a2a_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+ep_a2a_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(EP_A2A_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Byte offsets of everything in the workspace.
+struct Layout {
+  int64_t off_err, off_count_acc, off_ticket, off_counts, off_plan_nd, off_plan_dst;
+  int64_t ctrl_bytes;        // [0, ctrl_bytes) is cleared at init
+  int64_t rank_base;         // rank 0's region
+  int64_t rank_stride;       // bytes per rank region
+  int64_t off_payload[kMaxPayloads];
+  int64_t off_ids, off_valid, off_eplb;   // inside a rank region
+  int64_t total;
+  int plan_stride;
+};
+
+ep_a2a_status check_params(const ep_a2a_params* p) {
+  if (!p) return fail(EP_A2A_ERR_INVALID_ARG, "params is NULL");
+  if (p->ep_size < 1 || p->ep_size > kMaxRanks)
+    return fail(EP_A2A_ERR_UNSUPPORTED, "ep_size %d outside 1..%d", p->ep_size, kMaxRanks);
+  if (p->num_experts <= 0 || p->num_experts % 4 != 0)
+    return fail(EP_A2A_ERR_INVALID_ARG, "num_experts %d must be a positive multiple of 4",
+                p->num_experts);
+  if (p->num_experts % p->ep_size != 0)
+    return fail(EP_A2A_ERR_INVALID_ARG, "num_experts %d must be divisible by ep_size %d",
+                p->num_experts, p->ep_size);
+  if (p->top_k < 1 || p->top_k > kMaxTopK)
+    return fail(EP_A2A_ERR_UNSUPPORTED, "top_k %d outside 1..%d", p->top_k, kMaxTopK);
+  if (p->max_tokens_per_rank < 1)
+    return fail(EP_A2A_ERR_INVALID_ARG, "max_tokens_per_rank %d must be >= 1",
+                p->max_tokens_per_rank);
+  if ((int64_t)p->ep_size * p->max_tokens_per_rank > (int64_t)1 << 30)
+    return fail(EP_A2A_ERR_UNSUPPORTED, "ep_size * max_tokens_per_rank too large");
+  if (p->hidden_size < 1)
+    return fail(EP_A2A_ERR_INVALID_ARG, "hidden_size %d must be >= 1", p->hidden_size);
+  if (p->num_payloads < 0 || p->num_payloads > kMaxPayloads)
+    return fail(EP_A2A_ERR_UNSUPPORTED, "num_payloads %d outside 0..%d", p->num_payloads,
+                kMaxPayloads);
+  for (int i = 0; i < p->num_payloads; ++i)
+    if (p->payload_row_bytes[i] < 1 || p->payload_row_bytes[i] > ((int64_t)1 << 24))
+      return fail(EP_A2A_ERR_INVALID_ARG, "payload_row_bytes[%d] = %lld outside 1..2^24", i,
+                  (long long)p->payload_row_bytes[i]);
+  if (p->eplb_stats_num_experts != 0 && p->eplb_stats_num_experts != p->num_experts)
+    return fail(EP_A2A_ERR_INVALID_ARG,
+                "eplb_stats_num_experts %d must be 0 or num_experts %d (statistics must cover "
+                "all experts)",
+                p->eplb_stats_num_experts, p->num_experts);
+  if (p->enable_rank_mask != 0 && p->enable_rank_mask != 1)
+    return fail(EP_A2A_ERR_INVALID_ARG, "enable_rank_mask must be 0 or 1");
+  if (p->reserved != 0) return fail(EP_A2A_ERR_INVALID_ARG, "reserved must be 0");
+  return EP_A2A_OK;
+}
+
+Layout make_layout(const ep_a2a_params& p) {
+  Layout L{};
+  const int64_t ep = p.ep_size, cap = p.max_tokens_per_rank, slots = ep * cap;
+  L.plan_stride = (int)align_up(p.top_k, 8);
+  int64_t c = 0;
+  L.off_err = c;        c = align_up(c + 16, kAlign);
+  L.off_count_acc = c;  c = align_up(c + ep * ep * 4, kAlign);
+  L.off_ticket = c;     c = align_up(c + ep * 4, kAlign);
+  L.off_counts = c;     c = align_up(c + ep * ep * 4, kAlign);
+  L.off_plan_nd = c;    c = align_up(c + slots, kAlign);
+  L.off_plan_dst = c;   c = align_up(c + slots * L.plan_stride, kAlign);
+  L.ctrl_bytes = c;
+  L.rank_base = c;
+  int64_t r = 0;
+  for (int i = 0; i < kMaxPayloads; ++i) {
+    L.off_payload[i] = r;
+    if (i < p.num_payloads) r = align_up(r + slots * p.payload_row_bytes[i], kAlign);
+  }
+  L.off_ids = r;    r = align_up(r + slots * p.top_k * 4, kAlign);
+  L.off_valid = r;  r = align_up(r + slots, kAlign);
+  L.off_eplb = r;   r = align_up(r + ep * p.eplb_stats_num_experts * 4, kAlign);
+  L.rank_stride = r;
+  L.total = L.rank_base + ep * L.rank_stride;
+  return L;
+}
+
+}  // namespace
+}  // namespace ep_a2a
+
+using namespace ep_a2a;
+
+struct ep_a2a_handle_s {
+  uint32_t magic;
+  ep_a2a_params p;
+  Layout L;
+  uint8_t* ws;
+  size_t ws_bytes;
+  int device;
+  int num_sms;
+  int max_smem_optin;
+  bool have_plan;
+  int last_tpr;
+  // tuning
+  int copy_path;          // 0 bulk where possible, 1 vector only
+  int copy_ctas_per_sm;
+  int copy_stages;        // 0 = choose from the row size
+  int combine_threads;
+  // profiling (ep_a2a_profile_start / _stop)
+  bool profiling;
+  int prof_max;
+  std::vector<cudaEvent_t> prof_events;   // 2 per timed launch
+  std::vector<int> prof_kernel;           // kernel id per timed launch
+};
+
+namespace {
+
+ep_a2a_status check_handle(ep_a2a_handle h) {
+  if (!h || h->magic != kMagic)
+    return fail(EP_A2A_ERR_NOT_INITIALIZED, "handle is NULL or destroyed");
+  return EP_A2A_OK;
+}
+
+// Record the start event of a timed launch; returns the slot or -1.
+int prof_begin(ep_a2a_handle h, int kernel, cudaStream_t stream) {
+  if (!h->profiling || (int)h->prof_kernel.size() >= h->prof_max) return -1;
+  const int slot = (int)h->prof_kernel.size();
+  if (cudaEventRecord(h->prof_events[2 * slot], stream) != cudaSuccess) return -1;
+  h->prof_kernel.push_back(kernel);
+  return slot;
+}
+
+void prof_end(ep_a2a_handle h, int slot, cudaStream_t stream) {
+  if (slot >= 0) cudaEventRecord(h->prof_events[2 * slot + 1], stream);
+}
+
+void prof_free(ep_a2a_handle h) {
+  for (cudaEvent_t e : h->prof_events) cudaEventDestroy(e);
+  h->prof_events.clear();
+  h->prof_kernel.clear();
+  h->profiling = false;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+uint32_t vec_bytes(const void* src, const void* dst_base, int64_t rank_stride, int64_t rb) {
+  for (uint32_t v : {16u, 8u, 4u, 2u}) {
+    if (rb % v == 0 && aligned(src, v) && aligned(dst_base, v) && rank_stride % v == 0) return v;
+  }
+  return 1u;
+}
+
+}  // namespace
+
+EP_API const char* ep_a2a_status_string(ep_a2a_status s) {
+  switch (s) {
+    case EP_A2A_OK: return "ok";
+    case EP_A2A_ERR_INVALID_ARG: return "invalid argument";
+    case EP_A2A_ERR_CAPACITY: return "step exceeds the capacity given at init";
+    case EP_A2A_ERR_UNSUPPORTED: return "unsupported size";
+    case EP_A2A_ERR_CUDA: return "CUDA runtime error";
+    case EP_A2A_ERR_NOT_INITIALIZED: return "handle not initialised";
+    case EP_A2A_ERR_NO_PLAN: return "combine called before any dispatch";
+    case EP_A2A_ERR_DEVICE_TIMEOUT: return "a bounded device wait ran out";
+  }
+  return "unknown status";
+}
+
+EP_API const char* ep_a2a_last_error(void) { return g_last_error.c_str(); }
+
+EP_API ep_a2a_status ep_a2a_workspace_size(const ep_a2a_params* params, size_t* bytes) {
+  ep_a2a_status st = check_params(params);
+  if (st != EP_A2A_OK) return st;
+  if (!bytes) return fail(EP_A2A_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = (size_t)make_layout(*params).total;
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
+                                 size_t workspace_bytes, void* stream,
+                                 ep_a2a_handle* out_handle) {
+  ep_a2a_status st = check_params(params);
+  if (st != EP_A2A_OK) return st;
+  if (!out_handle) return fail(EP_A2A_ERR_INVALID_ARG, "out_handle is NULL");
+  *out_handle = nullptr;
+  if (!workspace) return fail(EP_A2A_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned(workspace, kAlign))
+    return fail(EP_A2A_ERR_INVALID_ARG, "workspace must be %lld-byte aligned", (long long)kAlign);
+  const Layout L = make_layout(*params);
+  if ((int64_t)workspace_bytes < L.total)
+    return fail(EP_A2A_ERR_INVALID_ARG, "workspace has %zu bytes, needs %lld", workspace_bytes,
+                (long long)L.total);
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, workspace);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaPointerGetAttributes(workspace)");
+  if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+    return fail(EP_A2A_ERR_INVALID_ARG, "workspace is not device memory");
+  int dev = 0, sms = 0, smem = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (attr.device != dev)
+    return fail(EP_A2A_ERR_INVALID_ARG, "workspace is on device %d, current device is %d",
+                attr.device, dev);
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+  if ((e = cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) !=
+      cudaSuccess)
+    return cuda_fail(e, "cudaDeviceGetAttribute(shared memory)");
+  e = cudaMemsetAsync(workspace, 0, (size_t)L.ctrl_bytes, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(control region)");
+
+  ep_a2a_handle h = new (std::nothrow) ep_a2a_handle_s();
+  if (!h) return fail(EP_A2A_ERR_INVALID_ARG, "out of host memory");
+  h->magic = kMagic;
+  h->p = *params;
+  if (h->p.invalid_expert_id < 0) h->p.invalid_expert_id = h->p.num_experts;
+  h->L = L;
+  h->ws = static_cast<uint8_t*>(workspace);
+  h->ws_bytes = workspace_bytes;
+  h->device = dev;
+  h->num_sms = sms;
+  h->max_smem_optin = smem;
+  h->have_plan = false;
+  h->last_tpr = 0;
+  h->copy_path = 0;
+  h->copy_ctas_per_sm = 1;
+  h->copy_stages = 0;
+  h->combine_threads = 128;
+  h->profiling = false;
+  h->prof_max = 0;
+  *out_handle = h;
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, int64_t value) {
+  ep_a2a_status st = check_handle(h);
+  if (st != EP_A2A_OK) return st;
+  switch (option) {
+    case EP_A2A_OPT_COPY_PATH:
+      if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "copy path must be 0 or 1");
+      h->copy_path = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_COPY_CTAS_PER_SM:
+      if (value < 1 || value > 8) return fail(EP_A2A_ERR_INVALID_ARG, "CTAs per SM must be 1..8");
+      h->copy_ctas_per_sm = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_COPY_STAGES:
+      if (value != 0 && (value < 2 || value > kMaxStages))
+        return fail(EP_A2A_ERR_INVALID_ARG, "stages must be 0 (automatic) or 2..%d", kMaxStages);
+      h->copy_stages = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_COMBINE_THREADS:
+      if (value < 64 || value > 1024 || value % 32 != 0)
+        return fail(EP_A2A_ERR_INVALID_ARG, "combine threads must be a multiple of 32 in 64..1024");
+      h->combine_threads = (int)value;
+      return EP_A2A_OK;
+  }
+  return fail(EP_A2A_ERR_INVALID_ARG, "unknown option %d", (int)option);
+}
+
+EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selected_experts,
+                                     const int32_t* local_num_tokens,
+                                     int32_t runtime_max_tokens_per_rank,
+                                     const void* const* payloads,
+                                     const int64_t* payload_row_bytes, int32_t num_payloads,
+                                     const int32_t* eplb_local_stats,
+                                     const uint64_t* active_rank_mask, void* stream_v,
+                                     ep_a2a_dispatch_result* result) {
+  ep_a2a_status st = check_handle(h);
+  if (st != EP_A2A_OK) return st;
+  const ep_a2a_params& p = h->p;
+  const Layout& L = h->L;
+  cudaStream_t stream = (cudaStream_t)stream_v;
+  const int ep = p.ep_size;
+  if (!token_selected_experts) return fail(EP_A2A_ERR_INVALID_ARG, "token_selected_experts is NULL");
+  if (!local_num_tokens) return fail(EP_A2A_ERR_INVALID_ARG, "local_num_tokens is NULL");
+  if (!result) return fail(EP_A2A_ERR_INVALID_ARG, "result is NULL");
+  const int tpr = runtime_max_tokens_per_rank <= 0 ? p.max_tokens_per_rank
+                                                   : runtime_max_tokens_per_rank;
+  if (tpr > p.max_tokens_per_rank)
+    return fail(EP_A2A_ERR_CAPACITY, "runtime_max_tokens_per_rank %d exceeds capacity %d", tpr,
+                p.max_tokens_per_rank);
+  if (num_payloads < 0 || num_payloads > p.num_payloads)
+    return fail(EP_A2A_ERR_INVALID_ARG, "num_payloads %d outside 0..%d", num_payloads,
+                p.num_payloads);
+  if (num_payloads > 0 && !payloads) return fail(EP_A2A_ERR_INVALID_ARG, "payloads is NULL");
+  int64_t rb[kMaxPayloads] = {0};
+  for (int i = 0; i < num_payloads; ++i) {
+    rb[i] = payload_row_bytes ? payload_row_bytes[i] : p.payload_row_bytes[i];
+    if (rb[i] < 1 || rb[i] > p.payload_row_bytes[i])
+      return fail(EP_A2A_ERR_CAPACITY, "payload %d row bytes %lld outside 1..%lld", i,
+                  (long long)rb[i], (long long)p.payload_row_bytes[i]);
+    if (!payloads[i]) return fail(EP_A2A_ERR_INVALID_ARG, "payload %d is NULL", i);
+  }
+  if (eplb_local_stats && p.eplb_stats_num_experts == 0)
+    return fail(EP_A2A_ERR_INVALID_ARG,
+                "eplb_local_stats given but the handle was created with eplb_stats_num_experts=0");
+  if (eplb_local_stats && !aligned(eplb_local_stats, 16))
+    return fail(EP_A2A_ERR_INVALID_ARG, "eplb_local_stats must be 16-byte aligned");
+  if (active_rank_mask && !p.enable_rank_mask)
+    return fail(EP_A2A_ERR_INVALID_ARG, "active_rank_mask needs enable_rank_mask");
+
+  RouteArgs ra;
+  std::memset(&ra, 0, sizeof(ra));
+  for (int w = 0; w < kMaskWords; ++w) ra.live[w] = ~0ull;
+  if (active_rank_mask) {
+    bool any = false;
+    for (int w = 0; w < kMaskWords; ++w) ra.live[w] = active_rank_mask[w];
+    for (int r = 0; r < ep; ++r) any |= ((ra.live[r >> 6] >> (r & 63)) & 1ull) != 0;
+    if (!any) return fail(EP_A2A_ERR_INVALID_ARG, "active_rank_mask has no active rank");
+  }
+  for (int r = 0; r < ep; ++r) {
+    const int n = local_num_tokens[r];
+    if (n < 0 || n > tpr)
+      return fail(EP_A2A_ERR_INVALID_ARG, "local_num_tokens[%d] = %d outside 0..%d", r, n, tpr);
+    const bool live = ((ra.live[r >> 6] >> (r & 63)) & 1ull) != 0;
+    ra.n[r] = live ? n : 0;
+  }
+
+  uint8_t* ws = h->ws;
+  uint8_t* rank0 = ws + L.rank_base;
+  const int64_t ntok = (int64_t)ep * tpr;
+  ra.ids = token_selected_experts;
+  ra.eplb_stats = eplb_local_stats;
+  ra.plan_nd = ws + L.off_plan_nd;
+  ra.plan_dst = ws + L.off_plan_dst;
+  ra.count_acc = reinterpret_cast<int32_t*>(ws + L.off_count_acc);
+  ra.count_ticket = reinterpret_cast<uint32_t*>(ws + L.off_ticket);
+  ra.send_counts = reinterpret_cast<int32_t*>(ws + L.off_counts);
+  ra.rank0 = rank0;
+  ra.rank_stride = L.rank_stride;
+  ra.off_ids = L.off_ids;
+  ra.off_valid = L.off_valid;
+  ra.off_eplb = L.off_eplb;
+  ra.ep = ep;
+  ra.E = p.num_experts;
+  ra.k = p.top_k;
+  ra.tpr = tpr;
+  ra.epr = p.num_experts / ep;
+  ra.plan_stride = L.plan_stride;
+  ra.eplb_n = p.eplb_stats_num_experts;
+  ra.invalid_id = p.invalid_expert_id;
+  int slot = prof_begin(h, EP_A2A_KERNEL_ROUTE_PLAN, stream);
+  cudaError_t e = launch_route_plan(ra, active_rank_mask != nullptr, stream);
+  prof_end(h, slot, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "routing-plan kernel launch");
+
+  // split payloads between the bulk-async copy and the vector copy
+  CopyArgs bulk, vec;
+  std::memset(&bulk, 0, sizeof(bulk));
+  bulk.plan_nd = ra.plan_nd;
+  bulk.plan_dst = ra.plan_dst;
+  bulk.rank0 = rank0;
+  bulk.rank_stride = L.rank_stride;
+  bulk.ntok = ntok;
+  bulk.plan_stride = L.plan_stride;
+  bulk.err = reinterpret_cast<uint32_t*>(ws + L.off_err);
+  vec = bulk;
+  uint32_t stage = 0;
+  for (int i = 0; i < num_payloads; ++i) {
+    const uint8_t* src = static_cast<const uint8_t*>(payloads[i]);
+    const bool bulk_ok = h->copy_path == 0 && rb[i] % 16 == 0 && aligned(src, 16);
+    CopyArgs& c = bulk_ok ? bulk : vec;
+    const int j = c.np++;
+    c.src[j] = src;
+    c.rb[j] = rb[i];
+    c.dst_off[j] = L.off_payload[i];
+    if (bulk_ok) {
+      c.smem_off[j] = stage;
+      stage += (uint32_t)rb[i];
+    } else {
+      c.vec[j] = vec_bytes(src, rank0 + L.off_payload[i], L.rank_stride, rb[i]);
+    }
+  }
+  if (bulk.np > 0) {
+    bulk.tx_bytes = stage;
+    bulk.stage_bytes = (uint32_t)align_up(stage, 128);
+    // shared memory per CTA when `ctas` CTAs share an SM (1 KB per block is
+    // reserved by the hardware; 2 KB covers the kernel's static arrays)
+    const int ctas = h->copy_ctas_per_sm;
+    const int64_t per_cta =
+        std::min<int64_t>(h->max_smem_optin, (int64_t)228 * 1024 / ctas - 1024) - 2048;
+    int64_t stages = h->copy_stages > 0 ? h->copy_stages : 16;
+    stages = std::min<int64_t>(stages, per_cta / bulk.stage_bytes);
+    if (stages < 2) {
+      // rows too large to stage: move them with the vector copy instead
+      for (int j = 0; j < bulk.np; ++j) {
+        const int k = vec.np++;
+        vec.src[k] = bulk.src[j];
+        vec.rb[k] = bulk.rb[j];
+        vec.dst_off[k] = bulk.dst_off[j];
+        vec.vec[k] = vec_bytes(bulk.src[j], rank0 + bulk.dst_off[j], L.rank_stride, bulk.rb[j]);
+      }
+      bulk.np = 0;
+    } else {
+      bulk.stages = (int)stages;
+      const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)h->num_sms * ctas, ntok));
+      slot = prof_begin(h, EP_A2A_KERNEL_COPY_BULK, stream);
+      e = launch_dispatch_bulk(bulk, grid, stream);
+      prof_end(h, slot, stream);
+      if (e != cudaSuccess) return cuda_fail(e, "bulk copy kernel launch");
+    }
+  }
+  if (vec.np > 0) {
+    const int64_t warps_needed = ntok;
+    const int grid = (int)std::max<int64_t>(
+        1, std::min<int64_t>((warps_needed + 7) / 8, (int64_t)h->num_sms * 8));
+    slot = prof_begin(h, EP_A2A_KERNEL_COPY_VEC, stream);
+    e = launch_dispatch_vec(vec, grid, stream);
+    prof_end(h, slot, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "vector copy kernel launch");
+  }
+
+  std::memset(result, 0, sizeof(*result));
+  result->tokens_per_rank = tpr;
+  result->num_payloads = num_payloads;
+  result->rank_stride_bytes = L.rank_stride;
+  for (int i = 0; i < num_payloads; ++i) result->recv_payloads[i] = rank0 + L.off_payload[i];
+  result->recv_topk_ids = reinterpret_cast<int32_t*>(rank0 + L.off_ids);
+  result->recv_valid = rank0 + L.off_valid;
+  result->eplb_gathered_stats =
+      eplb_local_stats ? reinterpret_cast<int32_t*>(rank0 + L.off_eplb) : nullptr;
+  result->send_counts = ra.send_counts;
+  result->plan_num_dst = ra.plan_nd;
+  result->plan_dst_ranks = ra.plan_dst;
+  result->plan_stride = L.plan_stride;
+  h->have_plan = true;
+  h->last_tpr = tpr;
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
+                                    ep_a2a_combine_dtype dtype, void* output, void* stream_v) {
+  ep_a2a_status st = check_handle(h);
+  if (st != EP_A2A_OK) return st;
+  if (!h->have_plan) return fail(EP_A2A_ERR_NO_PLAN, "combine needs a preceding dispatch");
+  if (!expert_output || !output)
+    return fail(EP_A2A_ERR_INVALID_ARG, "expert_output / output is NULL");
+  if (dtype != EP_A2A_COMBINE_BF16 && dtype != EP_A2A_COMBINE_FP8_E4M3)
+    return fail(EP_A2A_ERR_INVALID_ARG, "unknown combine dtype %d", (int)dtype);
+  const bool fp8 = dtype == EP_A2A_COMBINE_FP8_E4M3;
+  CombineArgs a;
+  a.plan_nd = h->ws + h->L.off_plan_nd;
+  a.plan_dst = h->ws + h->L.off_plan_dst;
+  a.x = static_cast<const uint8_t*>(expert_output);
+  a.out = static_cast<uint16_t*>(output);
+  a.ntok = (int64_t)h->p.ep_size * h->last_tpr;
+  a.H = h->p.hidden_size;
+  a.plan_stride = h->L.plan_stride;
+  const int elems = fp8 ? 16 : 8;
+  const bool vec = a.H % elems == 0 && aligned(expert_output, 16) && aligned(output, 16);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(a.ntok, (int64_t)h->num_sms * 16));
+  const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);
+  cudaError_t e = launch_combine(a, fp8, vec, h->combine_threads, grid, (cudaStream_t)stream_v);
+  prof_end(h, slot, (cudaStream_t)stream_v);
+  if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_quantize_e4m3(const void* bf16_in, void* e4m3_out, int64_t n,
+                                          void* stream) {
+  if (n < 0) return fail(EP_A2A_ERR_INVALID_ARG, "n < 0");
+  if (n > 0 && (!bf16_in || !e4m3_out)) return fail(EP_A2A_ERR_INVALID_ARG, "NULL buffer");
+  cudaError_t e = launch_quantize_e4m3(static_cast<const uint16_t*>(bf16_in),
+                                       static_cast<uint8_t*>(e4m3_out), n, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize kernel launch");
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_get_status(ep_a2a_handle h, void* stream) {
+  ep_a2a_status st = check_handle(h);
+  if (st != EP_A2A_OK) return st;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  uint32_t word = 0;
+  uint32_t* dev_word = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
+  e = cudaMemcpy(&word, dev_word, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (word != 0) {
+    e = cudaMemset(dev_word, 0, sizeof(word));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    if (word & kErrWaitTimeout)
+      return fail(EP_A2A_ERR_DEVICE_TIMEOUT, "a bounded wait in a kernel ran out (word 0x%x)",
+                  word);
+  }
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_debug_wait_probe(ep_a2a_handle h, int64_t limit_ns, void* stream) {
+  ep_a2a_status st = check_handle(h);
+  if (st != EP_A2A_OK) return st;
+  if (limit_ns < 1 || limit_ns > 10000000000ll)
+    return fail(EP_A2A_ERR_INVALID_ARG, "limit_ns must be in 1..1e10");
+  cudaError_t e = launch_wait_timeout_probe(reinterpret_cast<uint32_t*>(h->ws + h->L.off_err),
+                                            (unsigned long long)limit_ns, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "probe kernel launch");
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_profile_start(ep_a2a_handle h, int32_t max_launches) {
+  ep_a2a_status st = check_handle(h);
+  if (st != EP_A2A_OK) return st;
+  if (max_launches < 1 || max_launches > (1 << 20))
+    return fail(EP_A2A_ERR_INVALID_ARG, "max_launches must be in 1..2^20");
+  prof_free(h);
+  h->prof_events.resize(2 * (size_t)max_launches);
+  for (size_t i = 0; i < h->prof_events.size(); ++i) {
+    cudaError_t e = cudaEventCreate(&h->prof_events[i]);
+    if (e != cudaSuccess) {
+      h->prof_events.resize(i);
+      prof_free(h);
+      return cuda_fail(e, "cudaEventCreate");
+    }
+  }
+  h->prof_kernel.reserve(max_launches);
+  h->prof_max = max_launches;
+  h->profiling = true;
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_profile_stop(ep_a2a_handle h, ep_a2a_kernel_times* times) {
+  ep_a2a_status st = check_handle(h);
+  if (st != EP_A2A_OK) return st;
+  if (!h->profiling) return fail(EP_A2A_ERR_INVALID_ARG, "profiling was not started");
+  ep_a2a_kernel_times t;
+  std::memset(&t, 0, sizeof(t));
+  for (size_t i = 0; i < h->prof_kernel.size(); ++i) {
+    cudaError_t e = cudaEventSynchronize(h->prof_events[2 * i + 1]);
+    float ms = 0.f;
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, h->prof_events[2 * i], h->prof_events[2 * i + 1]);
+    if (e != cudaSuccess) {
+      prof_free(h);
+      return cuda_fail(e, "reading profiling events");
+    }
+    t.launches[h->prof_kernel[i]] += 1;
+    t.total_ms[h->prof_kernel[i]] += ms;
+  }
+  prof_free(h);
+  if (times) *times = t;
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_destroy(ep_a2a_handle* hp) {
+  if (!hp || !*hp) return EP_A2A_OK;
+  ep_a2a_handle h = *hp;
+  if (h->magic != kMagic) return fail(EP_A2A_ERR_NOT_INITIALIZED, "handle is not valid");
+  prof_free(h);
+  h->magic = 0;
+  delete h;
+  *hp = nullptr;
+  return EP_A2A_OK;
+}

@@ -1,0 +1,193 @@
+// Internal declarations of libep_a2a: kernel argument blocks, launchers and
+// small PTX wrappers (mbarrier, bulk-async copies).  Not part of the C ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "ep_a2a.h"
+
+namespace ep_a2a {
+
+constexpr int kMaxRanks = EP_A2A_MAX_RANKS;
+constexpr int kMaskWords = EP_A2A_RANK_MASK_WORDS;
+constexpr int kMaxPayloads = EP_A2A_MAX_PAYLOADS;
+constexpr int kMaxTopK = EP_A2A_MAX_TOP_K;
+constexpr uint8_t kNoToken = 0xFF;       // plan_num_dst of a token that does not exist
+constexpr uint8_t kPad = 0xFF;           // plan_dst_ranks entries past the count
+constexpr int kMaxStages = 32;           // shared-memory row stages per bulk-copy CTA
+
+// Bits of the device error word.
+enum : uint32_t { kErrWaitTimeout = 1u };
+
+// Bounded waits give up after this many nanoseconds of %globaltimer.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+__host__ __device__ inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------
+// Routing plan (+ EPLB gather)
+// ---------------------------------------------------------------------------
+struct RouteArgs {
+  const int32_t* ids;          // [ep, tpr, k]
+  const int32_t* eplb_stats;   // [ep, eplb_n] or nullptr
+  uint8_t* plan_nd;            // [ep*tpr]
+  uint8_t* plan_dst;           // [ep*tpr, plan_stride]
+  int32_t* count_acc;          // [ep*ep] scratch; zero between calls
+  uint32_t* count_ticket;      // [ep] scratch; zero between calls
+  int32_t* send_counts;        // [ep*ep]
+  uint8_t* rank0;              // rank 0's region of the workspace
+  int64_t rank_stride;         // bytes between rank regions
+  int64_t off_ids, off_valid, off_eplb;  // offsets inside a rank region
+  int ep, E, k, tpr, epr, plan_stride, eplb_n;
+  int32_t invalid_id;
+  int32_t n[kMaxRanks];        // local_num_tokens, 0 for masked-off ranks
+  uint64_t live[kMaskWords];   // bit r = rank r active
+};
+
+cudaError_t launch_route_plan(const RouteArgs& a, bool use_mask, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
+// Dispatch row copy
+// ---------------------------------------------------------------------------
+struct CopyArgs {
+  const uint8_t* plan_nd;
+  const uint8_t* plan_dst;
+  uint8_t* rank0;
+  int64_t rank_stride;
+  int64_t ntok;                          // ep * tpr token slots
+  int plan_stride;
+  int np;                                // payloads handled by this launch
+  const uint8_t* src[kMaxPayloads];      // [ep*tpr, rb] each
+  int64_t rb[kMaxPayloads];              // row bytes
+  int64_t dst_off[kMaxPayloads];         // receive array offset inside a rank region
+  uint32_t smem_off[kMaxPayloads];       // bulk path: offset of the row in a stage
+  uint32_t vec[kMaxPayloads];            // vector path: bytes per access (16/8/4/2/1)
+  uint32_t stage_bytes;                  // bulk path: bytes of one stage
+  uint32_t tx_bytes;                     // bulk path: bytes one token brings in
+  int stages;                            // bulk path
+  uint32_t* err;
+};
+
+cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t stream);
+cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, cudaStream_t stream);
+int bulk_queue_depth(int stages);        // groups allowed in flight for `stages`
+
+// ---------------------------------------------------------------------------
+// Combine and the E4M3 helper
+// ---------------------------------------------------------------------------
+struct CombineArgs {
+  const uint8_t* plan_nd;
+  const uint8_t* plan_dst;
+  const uint8_t* x;            // [ep, ep*tpr, H] bf16 or E4M3
+  uint16_t* out;               // [ep, tpr, H] bf16
+  int64_t ntok;                // ep * tpr
+  int H;
+  int plan_stride;
+};
+
+cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, int threads, int grid,
+                           cudaStream_t stream);
+cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n, cudaStream_t stream);
+cudaError_t launch_wait_timeout_probe(uint32_t* err, unsigned long long limit_ns,
+                                      cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
+// PTX wrappers (sm_90+; built for sm_100a).  All forms are CTA-local.
+// ---------------------------------------------------------------------------
+#if defined(__CUDACC__)
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// Make barrier initialisation visible to the async proxy (the bulk-copy unit).
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long global_timer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `parity` of the barrier, for at most limit_ns.  Returns false
+// if the limit ran out (the caller records an error and stops).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0u && global_timer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// Global -> this CTA's shared memory, completion counted on `bar` in bytes.
+__device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_smem),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// This CTA's shared memory -> global, tracked by bulk groups.
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(src_smem), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// At most N committed groups may still be reading shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// All committed groups complete (writes performed).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+#endif  // __CUDACC__
+
+}  // namespace ep_a2a

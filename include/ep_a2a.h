@@ -1,0 +1,264 @@
+/*
+ * ep_a2a.h — C ABI of libep_a2a.so: rank-major MoE expert-parallel token
+ * dispatch and combine for one NVIDIA B200 (sm_100a), all EP ranks virtual.
+ *
+ * Every EP rank is a virtual rank whose receive arrays live in one GPU's HBM,
+ * inside one caller-owned workspace.  A "send" from rank src to rank d is a
+ * copy into rank d's slice of that workspace.  All entry points take plain
+ * pointers and sizes; device pointers are CUDA device addresses on the current
+ * device, host pointers are ordinary process memory.  No entry point allocates
+ * device memory, and none throws: each returns an ep_a2a_status, and on failure
+ * ep_a2a_last_error() gives a one-line message (per calling thread).
+ *
+ * GPU work is enqueued asynchronously on the caller's stream (a cudaStream_t
+ * passed as void*; NULL = the legacy default stream).  Arguments are validated
+ * synchronously on the host before anything is enqueued; a call that returns an
+ * error has enqueued nothing.
+ *
+ * Sources (page title, then section):
+ *   flashinfer.moe_ep.NVLinkOneSidedConfig — options paragraph
+ *     (extra_payload_bytes_per_token, eplb_stats_num_experts, enable_rank_mask,
+ *     use_low_precision_combine) and the `lamport` paragraph (slot
+ *     src * tokens_per_rank + t; tokens_per_rank = runtime_max_tokens_per_rank).
+ *   flashinfer.moe_ep.NVLinkTwoSidedAlltoAll — class constraints (num_experts
+ *     divisible by 4; EPLB statistics cover all experts), dispatch(), combine(),
+ *     destroy().
+ *   flashinfer.comm.moe_a2a_dispatch — Parameters (token_selected_experts,
+ *     input_payloads, workspace, runtime_max_tokens_per_rank, eplb_local_stats,
+ *     enable_rank_mask, active_rank_mask) and Returns.
+ *   vllm.distributed.device_communicators.all2all —
+ *     FlashInferNVLinkTwoSidedManager.get_communication (invalid_expert_id =
+ *     num_experts for received rows past a source's token count).
+ */
+#ifndef EP_A2A_H
+#define EP_A2A_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Limits of this implementation. */
+#define EP_A2A_MAX_RANKS 256          /* ep_size */
+#define EP_A2A_RANK_MASK_WORDS 4      /* uint64 words of active_rank_mask */
+#define EP_A2A_MAX_PAYLOADS 8         /* entries of the payload list */
+#define EP_A2A_MAX_TOP_K 32
+
+typedef struct ep_a2a_handle_s* ep_a2a_handle;   /* opaque, library-owned host object */
+
+typedef enum {
+  EP_A2A_OK = 0,
+  EP_A2A_ERR_INVALID_ARG = 1,     /* a size, pointer or flag breaks a rule below */
+  EP_A2A_ERR_CAPACITY = 2,        /* step larger than the capacity given at init */
+  EP_A2A_ERR_UNSUPPORTED = 3,     /* beyond this implementation's limits */
+  EP_A2A_ERR_CUDA = 4,            /* a CUDA runtime call failed (launch, device query) */
+  EP_A2A_ERR_NOT_INITIALIZED = 5, /* NULL or destroyed handle */
+  EP_A2A_ERR_NO_PLAN = 6,         /* combine without a preceding dispatch */
+  EP_A2A_ERR_DEVICE_TIMEOUT = 7   /* a bounded wait inside a kernel ran out */
+} ep_a2a_status;
+
+typedef enum {
+  EP_A2A_COMBINE_BF16 = 0,        /* expert_output is bf16 */
+  EP_A2A_COMBINE_FP8_E4M3 = 1     /* expert_output is E4M3 (fn), unscaled */
+} ep_a2a_combine_dtype;
+
+/*
+ * Sizes fixed at init (the pages' MoEEpCommParams plus the one-sided config
+ * options).  Capacity values bound every later step.
+ */
+typedef struct {
+  int32_t ep_size;                /* 1..EP_A2A_MAX_RANKS */
+  int32_t num_experts;            /* E: divisible by 4 (NVLinkTwoSidedAlltoAll) and by
+                                     ep_size; expert e is owned by rank e / (E / ep_size) */
+  int32_t top_k;                  /* 1..EP_A2A_MAX_TOP_K */
+  int32_t max_tokens_per_rank;    /* capacity: largest runtime_max_tokens_per_rank */
+  int32_t hidden_size;            /* elements per combine row (bf16 or E4M3) */
+  int32_t num_payloads;           /* 0..EP_A2A_MAX_PAYLOADS dispatch payloads */
+  int64_t payload_row_bytes[EP_A2A_MAX_PAYLOADS];  /* capacity of each payload's row,
+                                     bytes (> 0): token rows, block scales, topk_weights,
+                                     extra_payload_bytes_per_token, ... */
+  int32_t eplb_stats_num_experts; /* 0 = no EPLB gather; else must equal num_experts */
+  int32_t enable_rank_mask;       /* 0: every rank always active and no mask may be
+                                     passed; 1: dispatch accepts active_rank_mask */
+  int32_t invalid_expert_id;      /* id written into invalid received rows; < 0 means
+                                     num_experts (no rank owns it) */
+  int32_t reserved;               /* must be 0 */
+} ep_a2a_params;
+
+/*
+ * Everything dispatch produced, as device pointers into the workspace (the
+ * pages' "workspace-backed views").  They stay valid, and keep their contents,
+ * until the next dispatch on the same handle or its destruction.  Every
+ * per-rank array of rank d sits at (rank-0 pointer + d * rank_stride_bytes).
+ * Let tpr = tokens_per_rank and slot s = src * tpr + t.
+ */
+typedef struct {
+  int32_t tokens_per_rank;        /* this step's runtime_max_tokens_per_rank */
+  int32_t num_payloads;
+  int64_t rank_stride_bytes;      /* bytes between consecutive ranks' arrays */
+  void* recv_payloads[EP_A2A_MAX_PAYLOADS]; /* [ep*tpr, row_bytes_i]: row s = payload i of
+                                     token t of rank src, for valid s; invalid rows are
+                                     not written */
+  int32_t* recv_topk_ids;         /* [ep*tpr, top_k]: the token's global ids for valid s,
+                                     else invalid_expert_id in all top_k entries */
+  uint8_t* recv_valid;            /* [ep*tpr]: 1 if row s was received, else 0 */
+  int32_t* eplb_gathered_stats;   /* [ep, E] per rank: row r = rank r's eplb_local_stats
+                                     (zeros for a masked-off r); NULL if not gathered */
+  int32_t* send_counts;           /* [ep(src), ep(dst)]: tokens src sent to dst (one
+                                     array, not per rank) */
+  uint8_t* plan_num_dst;          /* [ep(src), tpr]: distinct destination ranks of token
+                                     (src, t); 0xFF if the token does not exist */
+  uint8_t* plan_dst_ranks;        /* [ep(src), tpr, plan_stride]: those ranks ascending;
+                                     entries past plan_num_dst are 0xFF */
+  int32_t plan_stride;            /* bytes per plan_dst_ranks row: top_k rounded up to 8 */
+  int32_t reserved;
+} ep_a2a_dispatch_result;
+
+/*
+ * Bytes of device workspace needed for `params`.  Host only; no CUDA call.
+ * INVALID_ARG / UNSUPPORTED when params break the rules of ep_a2a_params.
+ */
+ep_a2a_status ep_a2a_workspace_size(const ep_a2a_params* params, size_t* bytes);
+
+/*
+ * Bind a caller-owned device workspace (>= ep_a2a_workspace_size bytes, 256-byte
+ * aligned) and create a handle.  The pages' moe_a2a_initialize / create_communication,
+ * for all virtual ranks at once.  Clears the workspace's small control region on
+ * `stream` (the caller keeps the workspace alive until ep_a2a_destroy).
+ * The library owns the returned handle; free it with ep_a2a_destroy.
+ */
+ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
+                          size_t workspace_bytes, void* stream, ep_a2a_handle* out_handle);
+
+/*
+ * Dispatch (flashinfer.comm.moe_a2a_dispatch; NVLinkTwoSidedAlltoAll.dispatch()):
+ * send each token of every live source rank, with all its payload rows, once to
+ * every live rank owning any of its top_k experts, landing at slot
+ * src * tokens_per_rank + t of that rank's receive arrays.
+ *
+ *   token_selected_experts  device int32 [ep, tpr, top_k]: global expert ids; an id
+ *                           outside [0, E) is owned by no rank and not routed.
+ *   local_num_tokens        host int32 [ep]: tokens of each rank, <= tpr.  Rows
+ *                           t >= local_num_tokens[r] of the inputs are ignored.
+ *   runtime_max_tokens_per_rank  tpr of this step, <= max_tokens_per_rank; <= 0
+ *                           means max_tokens_per_rank.
+ *   payloads                host array of num_payloads device pointers; payload i is
+ *                           [ep, tpr, payload_row_bytes[i]] bytes, rank-major.  The
+ *                           bytes are copied verbatim (no sentinel rewriting: NaN,
+ *                           -0 and any other pattern arrive unchanged).
+ *   payload_row_bytes       host int64 [num_payloads]: this step's row bytes
+ *                           (<= the init capacity); NULL = the init values.
+ *   num_payloads            <= the init num_payloads.
+ *   eplb_local_stats        device int32 [ep, eplb_stats_num_experts], or NULL.
+ *                           Must be NULL when init had eplb_stats_num_experts = 0.
+ *   active_rank_mask        host uint64 [EP_A2A_RANK_MASK_WORDS] (bit r = rank r
+ *                           alive), or NULL = all alive.  Needs enable_rank_mask and
+ *                           at least one live rank below ep_size; bits >= ep_size are
+ *                           ignored.  A masked-off rank neither sends nor receives:
+ *                           tokens routed to it are dropped, its receive arrays are
+ *                           not written, its tokens are not sent.
+ *   result                  filled on success (pointers into the workspace).
+ *
+ * The routing plan is kept in the workspace for the next ep_a2a_combine.
+ * Input buffers must stay untouched until the enqueued work has run.
+ */
+ep_a2a_status ep_a2a_dispatch(ep_a2a_handle handle, const int32_t* token_selected_experts,
+                              const int32_t* local_num_tokens,
+                              int32_t runtime_max_tokens_per_rank,
+                              const void* const* payloads, const int64_t* payload_row_bytes,
+                              int32_t num_payloads, const int32_t* eplb_local_stats,
+                              const uint64_t* active_rank_mask, void* stream,
+                              ep_a2a_dispatch_result* result);
+
+/*
+ * Combine (NVLinkTwoSidedAlltoAll.combine()): for each existing token (src, t) of
+ * the last dispatch, out[src][t][:] = bf16 of the fp32 sum, in ascending
+ * destination-rank order starting from +0.0f, of expert_output[d][src*tpr + t][:]
+ * over the token's destination ranks d; one round-to-nearest-even at the end.
+ * A token whose destinations were all masked off gets +0.0.
+ *
+ *   expert_output   device [ep, ep*tpr, hidden_size] of `dtype` (bf16 or E4M3),
+ *                   each rank's rows already weighted and reduced over its local
+ *                   experts.  Only rows of valid slots are read.
+ *   output          device bf16 [ep, tpr, hidden_size].  Rows of tokens that do
+ *                   not exist (t >= local_num_tokens[src], masked-off src) are not
+ *                   written.
+ * NO_PLAN if no dispatch has run on this handle.
+ */
+ep_a2a_status ep_a2a_combine(ep_a2a_handle handle, const void* expert_output,
+                             ep_a2a_combine_dtype dtype, void* output, void* stream);
+
+/*
+ * FP8 helper (flashinfer.moe_ep.NVLinkOneSidedConfig, use_low_precision_combine):
+ * e4m3_out[i] = E4M3(bf16_in[i]), round to nearest even, saturating to +-448.
+ * Device pointers; n elements.  Not part of a dispatch / combine step.
+ */
+ep_a2a_status ep_a2a_quantize_e4m3(const void* bf16_in, void* e4m3_out, int64_t n,
+                                   void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the handle's device error word.
+ * DEVICE_TIMEOUT if a kernel's bounded wait ran out since the last check.
+ */
+ep_a2a_status ep_a2a_get_status(ep_a2a_handle handle, void* stream);
+
+/*
+ * Failure-detection check (the pages' timeout_sec bounds waits on peers,
+ * flashinfer.moe_ep.NVLinkOneSidedConfig, `timeout_sec`; here a wait that runs
+ * out returns an error status instead of trapping): enqueues one kernel whose
+ * bounded wait on a shared-memory barrier can never complete; after limit_ns
+ * (1..1e10) of GPU time it sets the handle's error word and returns, leaving the
+ * context usable.  ep_a2a_get_status then reports EP_A2A_ERR_DEVICE_TIMEOUT.
+ */
+ep_a2a_status ep_a2a_debug_wait_probe(ep_a2a_handle handle, int64_t limit_ns, void* stream);
+
+/* Tuning knobs of the kernels (performance only; results never change). */
+typedef enum {
+  EP_A2A_OPT_COPY_PATH = 0,       /* 0 = bulk-async (TMA) copy where rows allow it,
+                                     1 = vector load/store copy for every payload */
+  EP_A2A_OPT_COPY_CTAS_PER_SM = 1,/* CTAs per SM of the bulk copy kernel (1..8) */
+  EP_A2A_OPT_COPY_STAGES = 2,     /* shared-memory row stages per copy CTA (2..32) */
+  EP_A2A_OPT_COMBINE_THREADS = 3  /* threads per CTA of the combine kernel (64..1024) */
+} ep_a2a_option;
+ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
+
+/*
+ * Per-kernel device timing.  Between ep_a2a_profile_start and ep_a2a_profile_stop
+ * every kernel this handle launches is bracketed by two CUDA events recorded on
+ * the launch stream; stop waits for them and returns, per kernel, the launch count
+ * and the summed event-to-event milliseconds.  Meant for benchmarks: recording
+ * adds two event records per launch.  At most max_launches launches are timed
+ * (later ones run untimed); start allocates the events (host-side CUDA objects,
+ * no device memory), stop frees them.
+ */
+typedef enum {
+  EP_A2A_KERNEL_ROUTE_PLAN = 0,   /* routing plan + EPLB gather */
+  EP_A2A_KERNEL_COPY_BULK = 1,    /* dispatch rows, bulk-async path */
+  EP_A2A_KERNEL_COPY_VEC = 2,     /* dispatch rows, vector path */
+  EP_A2A_KERNEL_COMBINE = 3,
+  EP_A2A_KERNEL_COUNT = 4
+} ep_a2a_kernel;
+typedef struct {
+  int64_t launches[EP_A2A_KERNEL_COUNT];
+  double total_ms[EP_A2A_KERNEL_COUNT];
+} ep_a2a_kernel_times;
+ep_a2a_status ep_a2a_profile_start(ep_a2a_handle handle, int32_t max_launches);
+ep_a2a_status ep_a2a_profile_stop(ep_a2a_handle handle, ep_a2a_kernel_times* times);
+
+/*
+ * Release the handle (NVLinkTwoSidedAlltoAll.destroy(): idempotent).  Sets
+ * *handle to NULL; NULL or *handle == NULL is a no-op returning OK.  Does not
+ * free the workspace, which the caller owns.
+ */
+ep_a2a_status ep_a2a_destroy(ep_a2a_handle* handle);
+
+const char* ep_a2a_status_string(ep_a2a_status status);
+const char* ep_a2a_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_A2A_H */

@@ -1,0 +1,347 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle,
+element by element, on the five synthetic workloads at full size and on edge
+cases.  Dispatch, the plan, EPLB gather and the BF16 combine are bit-exact;
+the FP8 combine is checked against the 2^-3 relative bar and, since both sides
+take the same E4M3 decisions, also for bit-exactness."""
+import functools
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+from combine_route_plan_b200 import workloads as W
+import parity_util as U
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from combine_route_plan_b200 import build
+    build.build()
+    yield
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+@functools.lru_cache(maxsize=1)
+def _inputs(name):
+    return W.make_inputs(W.BY_NAME[name])
+
+
+def _full_check(w, copy_path=0, options=None):
+    x = _inputs(w.name)
+    run = U.Run(w, x, copy_path=copy_path, options=options)
+    plan = U.oracle_plan(w, x)
+    U.check_plan(run, plan, w)
+    U.check_payloads(run, plan, w, x)
+    U.check_eplb(run, w, x)
+    U.check_combine(run, plan, w, x)
+    del run
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", [w.name for w in W.ALL])
+def test_workload_bit_exact(name):
+    _full_check(W.BY_NAME[name])
+
+
+@pytest.mark.parametrize("name", ["c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked"])
+def test_vector_copy_path_bit_exact(name):
+    from combine_route_plan_b200 import ep_a2a
+    _full_check(W.BY_NAME[name], copy_path=1)
+
+
+@pytest.mark.parametrize("stages,ctas", [(2, 1), (3, 2), (4, 4), (8, 1), (16, 1), (32, 1), (5, 3)])
+def test_copy_tuning_does_not_change_results(stages, ctas):
+    from combine_route_plan_b200 import ep_a2a
+    w = W.scaled(W.C2, 96)
+    x = W.make_inputs(w, with_expert_output=False)
+    run = U.Run(w, x, options={ep_a2a.OPT_COPY_STAGES: stages, ep_a2a.OPT_COPY_CTAS_PER_SM: ctas})
+    plan = U.oracle_plan(w, x)
+    U.check_plan(run, plan, w)
+    U.check_payloads(run, plan, w, x)
+
+
+@pytest.mark.parametrize("threads", [64, 96, 256, 1024])
+def test_combine_threads_do_not_change_results(threads):
+    from combine_route_plan_b200 import ep_a2a
+    w = W.C2
+    x = _inputs(w.name)
+    run = U.Run(w, x, options={ep_a2a.OPT_COMBINE_THREADS: threads})
+    U.check_combine(run, U.oracle_plan(w, x), w, x)
+
+
+def test_fp8_quantize_all_bf16_patterns():
+    from combine_route_plan_b200 import ep_a2a
+    table = U.oracle_e4m3_table()
+    allbits = torch.arange(65536, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    for lead in (0, 1, 3, 8):        # misaligned starts and odd lengths take the scalar path
+        src = torch.cat([torch.zeros(lead, dtype=torch.bfloat16), allbits]).cuda()[lead:]
+        n = src.numel() - (lead % 3)
+        out = torch.empty(n + 1, dtype=torch.uint8, device="cuda")[1:] if lead else \
+            torch.empty(n, dtype=torch.uint8, device="cuda")
+        ep_a2a.ep_a2a_quantize_e4m3(src.data_ptr(), out.data_ptr(), n)
+        torch.cuda.synchronize()
+        got = out.cpu().numpy()
+        f = (np.arange(n, dtype=np.uint32) << 16).view(np.float32)
+        nan = np.isnan(f)
+        assert np.array_equal(got[~nan], table[:n][~nan]), f"quantize lead={lead}"
+        assert np.all((got[nan] & 0x7F) == 0x7F)      # NaN stays NaN (its sign is not fixed)
+
+
+@pytest.mark.parametrize("name", ["c4_ep8_prefill", "c2_ep8_decode"])
+def test_fp8_combine(name):
+    w = W.BY_NAME[name]
+    x = _inputs(w.name)
+    run = U.Run(w, x, fp8=True)
+    plan = U.oracle_plan(w, x)
+    xq = U.oracle_quantize_big(U.to_np(x.expert_output), U.oracle_e4m3_table())
+    U.assert_equal(run.xq, xq, "quantized expert_output")
+    want = U.oracle.combine(plan, xq, w.hidden, input_is_e4m3=True, out_init=U.oracle_out_init(w))
+    got = U.to_np(run.out)
+    exists = plan.num_dst >= 0
+    gf = (got[exists].astype(np.uint32) << 16).view(np.float32)
+    wf = (want[exists].astype(np.uint32) << 16).view(np.float32)
+    rel = np.abs(gf.astype(np.float64) - wf) / np.maximum(np.abs(wf.astype(np.float64)), 1e-30)
+    rel[(gf == wf)] = 0.0
+    assert rel.max() <= 2.0 ** -3, rel.max()          # the stated bar
+    U.assert_equal(run.out, want, "fp8 combine (bit-exact)")
+    assert np.all(got[~exists] == 0xEEEE)
+
+
+# --------------------------------------------------------------------------- #
+# Edge cases
+# --------------------------------------------------------------------------- #
+
+def _custom(ep, E, k, tpr, H, rows, n=None, mask=None, seed=0, ids=None):
+    """A workload-like object with arbitrary payload rows of random bytes."""
+    g = torch.Generator().manual_seed(seed)
+    if ids is None:
+        ids = torch.stack([torch.randperm(E, generator=g)[:k] for _ in range(ep * tpr)]) \
+            .to(torch.int32).view(ep, tpr, k)
+    n = np.full(ep, tpr, np.int32) if n is None else np.asarray(n, np.int32)
+    payloads = [W.random_bytes_payload(ep, tpr, rb, seed + 17 * i) for i, rb in enumerate(rows)]
+    xo = torch.randn((ep, ep * tpr, H), generator=g).to(torch.bfloat16)
+
+    class Cfg:
+        pass
+    w = Cfg()
+    w.ep_size, w.num_experts, w.top_k, w.tokens_per_rank, w.hidden = ep, E, k, tpr, H
+    w.eplb = False
+    w.masked_ranks = () if mask is None else tuple(r for r in range(ep)
+                                                   if not (int(mask[r // 64]) >> (r % 64)) & 1)
+    w.payload_row_bytes = lambda: list(rows)
+    x = W.Inputs(w, ids.contiguous(), n, payloads, None,
+                 None if mask is None else np.asarray(mask, np.uint64), xo)
+    return w, x
+
+
+@pytest.mark.parametrize("ep,E,k,tpr,H,rows", [
+    (3, 12, 3, 37, 100, [1, 3, 13, 100]),          # odd rows: vector path, 1-byte vectors
+    (5, 20, 5, 33, 24, [16, 48, 8, 4]),            # k not a power of two
+    (16, 64, 16, 20, 64, [4096 + 16, 32]),         # 16 lanes per token
+    (16, 64, 32, 9, 32, [64, 2]),                  # top_k 32: a whole warp per token
+    (1, 8, 4, 50, 40, [272, 12]),                  # ep_size 1: identity
+    (2, 4, 1, 64, 8, [16]),                        # top_k 1
+    (4, 8, 2, 300, 128, [256, 8, 8]),              # several route blocks per rank, ragged tail
+])
+def test_edge_shapes(ep, E, k, tpr, H, rows):
+    w, x = _custom(ep, E, k, tpr, H, rows, seed=ep * 100 + k)
+    run = U.Run(w, x)
+    plan = U.oracle_plan(w, x)
+    U.check_plan(run, plan, w)
+    U.check_payloads(run, plan, w, x)
+    U.check_combine(run, plan, w, x)
+
+
+def test_misaligned_payload_pointers():
+    ep, E, k, tpr, H = 4, 16, 4, 25, 64
+    w, x = _custom(ep, E, k, tpr, H, [64, 32], seed=5)
+    from combine_route_plan_b200 import ep_a2a
+    comm = ep_a2a.EpA2A(ep, E, k, tpr, H, [64, 32], workspace_fill=U.CANARY)
+    ids = x.token_selected_experts.cuda()
+    shifted = []
+    for i, p in enumerate(x.payloads):
+        buf = torch.empty(p.numel() + 8, dtype=torch.uint8, device="cuda")
+        v = buf[1 + 2 * i: 1 + 2 * i + p.numel()].view(p.shape)
+        v.copy_(p.cuda())
+        shifted.append(v)
+    d = comm.dispatch(ids, x.local_num_tokens, shifted, tpr)
+    torch.cuda.synchronize()
+    plan = U.oracle_plan(w, x)
+    for i, p in enumerate(x.payloads):
+        for dst in range(ep):
+            want = U.oracle.dispatch_payload(plan, p.numpy(), only_dst=dst, recv_init=np.full(
+                (1, ep * tpr, p.shape[2]), U.CANARY, np.uint8))
+            U.assert_equal(d.recv_payloads[i][dst], want, f"payload {i} rank {dst}")
+
+
+def test_out_of_range_ids_and_duplicates():
+    ep, E, k, tpr, H = 4, 16, 4, 8, 32
+    ids = torch.tensor([[[-1, 16, 100, 3], [0, 1, 2, 3], [15, 15, 15, 15], [4, 8, 12, 0],
+                         [-5, -5, 7, 7], [16, 17, 18, 19], [3, 2, 1, 0], [12, 9, 6, 3]]] * ep,
+                       dtype=torch.int32)
+    w, x = _custom(ep, E, k, tpr, H, [32], ids=ids, seed=9)
+    run = U.Run(w, x)
+    plan = U.oracle_plan(w, x)
+    assert plan.num_dst[0].tolist() == [1, 1, 1, 4, 2, 0, 1, 4]
+    U.check_plan(run, plan, w)
+    U.check_payloads(run, plan, w, x)
+    U.check_combine(run, plan, w, x)
+
+
+@pytest.mark.parametrize("live", [[0], [3], [0, 5], list(range(1, 8))])
+def test_rank_masks(live):
+    ep, E, k, tpr, H = 8, 64, 6, 40, 64
+    mask = [0, 0, 0, 0]
+    for r in live:
+        mask[0] |= 1 << r
+    w, x = _custom(ep, E, k, tpr, H, [128, 24], n=[40, 1, 0, 39, 17, 40, 2, 33], mask=mask, seed=3)
+    run = U.Run(w, x)
+    plan = U.oracle_plan(w, x)
+    U.check_plan(run, plan, w)
+    U.check_payloads(run, plan, w, x)
+    U.check_combine(run, plan, w, x)
+
+
+def test_runtime_max_below_capacity_and_redispatch():
+    """tokens_per_rank follows runtime_max_tokens_per_rank (slots src*tpr+t);
+    a second dispatch on the same handle with another tpr fully replaces the plan."""
+    from combine_route_plan_b200 import ep_a2a
+    ep, E, k, H, cap = 8, 64, 4, 64, 96
+    comm = ep_a2a.EpA2A(ep, E, k, cap, H, [64, 16], workspace_fill=U.CANARY)
+    for tpr, seed in ((96, 1), (40, 2), (7, 3), (96, 4)):
+        w, x = _custom(ep, E, k, tpr, H, [64, 16], n=[min(tpr, v) for v in
+                                                         (tpr, 3, tpr, 0, 5, tpr - 1, 1, tpr)],
+                       seed=seed)
+        d = comm.dispatch(x.token_selected_experts.cuda(), x.local_num_tokens,
+                          [p.cuda() for p in x.payloads], tpr if seed != 4 else 0)
+        assert d.tokens_per_rank == tpr
+        out = comm.combine(x.expert_output.cuda(), tokens_per_rank=tpr)
+        torch.cuda.synchronize()
+        plan = U.oracle_plan(w, x)
+        nd = plan.num_dst.copy()
+        nd[nd < 0] = 0xFF
+        U.assert_equal(d.plan_num_dst, nd.astype(np.uint8), "plan_num_dst")
+        U.assert_equal(d.recv_valid, plan.recv_valid, "recv_valid")
+        U.assert_equal(d.recv_topk_ids, plan.recv_topk_ids, "recv_topk_ids")
+        U.assert_equal(d.send_counts, plan.send_counts, "send_counts")
+        want = U.oracle.combine(plan, U.to_np(x.expert_output), H,
+                                out_init=U.to_np(out))  # absent rows: whatever out held
+        exists = plan.num_dst >= 0
+        got = U.to_np(out)
+        assert np.array_equal(got[exists], want[exists])
+        for i, p in enumerate(x.payloads):
+            for dst in range(ep):
+                g = d.recv_payloads[i][dst]
+                pw = U.oracle.dispatch_payload(plan, p.numpy(), only_dst=dst)[0]
+                valid = plan.recv_valid[dst] == 1
+                U.assert_equal(g[torch.from_numpy(valid).cuda()], pw[valid], f"p{i} d{dst}")
+
+
+def test_counts_scratch_resets_between_calls():
+    w = W.scaled(W.C2, 64)
+    x = W.make_inputs(w, with_expert_output=False)
+    run = U.Run(w, x)
+    plan = U.oracle_plan(w, x)
+    for _ in range(4):
+        run.comm.dispatch(run.ids, x.local_num_tokens, run.payloads, w.tokens_per_rank)
+        torch.cuda.synchronize()
+        U.assert_equal(run.d.send_counts, plan.send_counts, "send_counts after repeat")
+
+
+def test_nan_in_invalid_rows_never_reaches_output():
+    w = W.C1
+    x = W.make_inputs(w)
+    plan = U.oracle_plan(w, x)
+    xo = x.expert_output.clone()
+    flat = xo.view(w.ep_size, -1, w.hidden)
+    for d in range(w.ep_size):
+        invalid = torch.from_numpy(plan.recv_valid[d] != 1)
+        flat[d][invalid] = float("nan")
+    x2 = W.Inputs(w, x.token_selected_experts, x.local_num_tokens, x.payloads, None, None, xo)
+    run = U.Run(w, x2)
+    assert not torch.isnan(run.out.float()).any()
+    U.check_combine(run, plan, w, x2)
+
+
+def test_ones_combine_counts_destinations():
+    w = W.C5
+    x = _inputs(w.name)
+    ones = torch.ones_like(x.expert_output)
+    x2 = W.Inputs(w, x.token_selected_experts, x.local_num_tokens, x.payloads[:0], None,
+                  x.active_rank_mask, ones)
+    run = U.Run(w, x2)
+    plan = U.oracle_plan(w, x)
+    got = run.out.float().cpu().numpy()
+    for r in range(w.ep_size):
+        for t in range(w.tokens_per_rank):
+            if plan.num_dst[r, t] >= 0:
+                assert np.all(got[r, t] == plan.num_dst[r, t])
+
+
+# --------------------------------------------------------------------------- #
+# Host validation that needs a live handle, and the bounded-wait status path
+# --------------------------------------------------------------------------- #
+
+def test_dispatch_and_combine_validation():
+    from combine_route_plan_b200 import ep_a2a
+    ep, E, k, tpr, H = 4, 16, 2, 8, 32
+    comm = ep_a2a.EpA2A(ep, E, k, tpr, H, [32], eplb_stats_num_experts=0)
+    ids = torch.zeros((ep, tpr, k), dtype=torch.int32, device="cuda")
+    pay = torch.zeros((ep, tpr, 32), dtype=torch.uint8, device="cuda")
+    stats = torch.zeros((ep, E), dtype=torch.int32, device="cuda")
+    xo = torch.zeros((ep, ep * tpr, H), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ep_a2a.EpA2AError) as e:
+        comm.combine(xo)
+    assert e.value.status == ep_a2a.ERR_NO_PLAN
+
+    def raw(handle=None, n=None, runtime=tpr, rb=(32,), stats_ptr=0, mask=None):
+        return ep_a2a.ep_a2a_dispatch(handle or comm.handle, ids.data_ptr(),
+                                      n if n is not None else [tpr] * ep, runtime,
+                                      [pay.data_ptr()], list(rb), stats_ptr, mask)
+
+    cases = [
+        (dict(runtime=tpr + 1), ep_a2a.ERR_CAPACITY),
+        (dict(n=[tpr + 1, 0, 0, 0]), ep_a2a.ERR_INVALID_ARG),
+        (dict(n=[-1, 0, 0, 0]), ep_a2a.ERR_INVALID_ARG),
+        (dict(mask=[0b1111]), ep_a2a.ERR_INVALID_ARG),          # mask without enable_rank_mask
+        (dict(stats_ptr=stats.data_ptr()), ep_a2a.ERR_INVALID_ARG),  # EPLB not enabled
+        (dict(rb=(48,)), ep_a2a.ERR_CAPACITY),                  # row above capacity
+        (dict(rb=(0,)), ep_a2a.ERR_CAPACITY),
+    ]
+    for kw, status in cases:
+        with pytest.raises(ep_a2a.EpA2AError) as e:
+            raw(**kw)
+        assert e.value.status == status, kw
+    masked = ep_a2a.EpA2A(ep, E, k, tpr, H, [32], enable_rank_mask=True)
+    with pytest.raises(ep_a2a.EpA2AError) as e:       # no live rank below ep_size
+        raw(handle=masked.handle, mask=[0b10000])
+    assert e.value.status == ep_a2a.ERR_INVALID_ARG
+    comm.dispatch(ids, [1] * ep, [pay])
+    comm.combine(xo)
+    torch.cuda.synchronize()
+    comm.destroy()
+    comm.destroy()                                    # idempotent
+    with pytest.raises(ep_a2a.EpA2AError) as e:
+        comm.combine(xo)
+    assert e.value.status == ep_a2a.ERR_NOT_INITIALIZED
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    from combine_route_plan_b200 import ep_a2a
+    w = W.C1
+    x = W.make_inputs(w)
+    run = U.Run(w, x)
+    ep_a2a.ep_a2a_debug_wait_probe(run.comm.handle, 20_000_000)     # 20 ms
+    assert run.comm.get_status() == ep_a2a.ERR_DEVICE_TIMEOUT
+    assert run.comm.get_status() == ep_a2a.OK                       # the word was cleared
+    run2 = U.Run(w, x)                                               # context still usable
+    plan = U.oracle_plan(w, x)
+    U.check_plan(run2, plan, w)
+    U.check_combine(run2, plan, w, x)
