@@ -15,6 +15,8 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include <algorithm>
+
 #include "ep_a2a_internal.cuh"
 
 namespace ep_a2a {
@@ -63,7 +65,7 @@ __device__ __forceinline__ void add_e4m3x16(float* acc, const uint4& v) {
 }
 
 template <bool kFp8>
-__global__ void combine_vec_kernel(const CombineArgs a) {
+__global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
   constexpr int kElems = kFp8 ? 16 : 8;       // elements per 16-byte input vector
   constexpr int kElemBytes = kFp8 ? 1 : 2;
   const int nvec = a.H / kElems;
@@ -116,7 +118,7 @@ __global__ void combine_vec_kernel(const CombineArgs a) {
 
 // Any hidden size and alignment: one element per thread step.
 template <bool kFp8>
-__global__ void combine_scalar_kernel(const CombineArgs a) {
+__global__ void __launch_bounds__(512) combine_scalar_kernel(const CombineArgs a) {
   const int words = a.plan_stride / 8;
   for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
     const int nd = a.plan_nd[tok];

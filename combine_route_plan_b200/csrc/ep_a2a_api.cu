@@ -275,8 +275,8 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       h->copy_stages = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_COMBINE_THREADS:
-      if (value < 64 || value > 1024 || value % 32 != 0)
-        return fail(EP_A2A_ERR_INVALID_ARG, "combine threads must be a multiple of 32 in 64..1024");
+      if (value < 64 || value > 512 || value % 32 != 0)
+        return fail(EP_A2A_ERR_INVALID_ARG, "combine threads must be a multiple of 32 in 64..512");
       h->combine_threads = (int)value;
       return EP_A2A_OK;
   }

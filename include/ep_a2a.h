@@ -220,7 +220,7 @@ typedef enum {
                                      1 = vector load/store copy for every payload */
   EP_A2A_OPT_COPY_CTAS_PER_SM = 1,/* CTAs per SM of the bulk copy kernel (1..8) */
   EP_A2A_OPT_COPY_STAGES = 2,     /* shared-memory row stages per copy CTA (2..32) */
-  EP_A2A_OPT_COMBINE_THREADS = 3  /* threads per CTA of the combine kernel (64..1024) */
+  EP_A2A_OPT_COMBINE_THREADS = 3  /* threads per CTA of the combine kernel (64..512) */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

@@ -67,7 +67,7 @@ def test_copy_tuning_does_not_change_results(stages, ctas):
     U.check_payloads(run, plan, w, x)
 
 
-@pytest.mark.parametrize("threads", [64, 96, 256, 1024])
+@pytest.mark.parametrize("threads", [64, 96, 256, 512])
 def test_combine_threads_do_not_change_results(threads):
     from combine_route_plan_b200 import ep_a2a
     w = W.C2
@@ -189,7 +189,7 @@ def test_out_of_range_ids_and_duplicates():
     w, x = _custom(ep, E, k, tpr, H, [32], ids=ids, seed=9)
     run = U.Run(w, x)
     plan = U.oracle_plan(w, x)
-    assert plan.num_dst[0].tolist() == [1, 1, 1, 4, 2, 0, 1, 4]
+    assert plan.num_dst[0].tolist() == [1, 1, 1, 4, 1, 0, 1, 4]
     U.check_plan(run, plan, w)
     U.check_payloads(run, plan, w, x)
     U.check_combine(run, plan, w, x)
