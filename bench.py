@@ -282,6 +282,8 @@ def run_ours(args):
     device = torch.device("cuda", local)
     dist = init_group("nccl")
     w = W.BY_NAME[args.workload]
+    if args.tokens_per_rank:
+        w = W.scaled(w, args.tokens_per_rank)
     x = W.make_inputs(w)
     stream = torch.cuda.current_stream()
 
@@ -524,6 +526,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--tokens-per-rank", type=int, default=0,
+                    help="run the workload with this many tokens per rank (small profiling cases)")
     ap.add_argument("--combine", choices=["bf16", "fp8"], default="bf16")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--fp8-steps", type=int, default=100)
