@@ -112,6 +112,9 @@ Layout make_layout(const ep_a2a_params& p) {
 }
 
 }  // namespace
+
+void record_last_error(const char* msg) { g_last_error = msg; }
+
 }  // namespace ep_a2a
 
 using namespace ep_a2a;

@@ -92,6 +92,9 @@ cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n, cu
 cudaError_t launch_wait_timeout_probe(uint32_t* err, unsigned long long limit_ns,
                                       cudaStream_t stream);
 
+// Message returned by ep_a2a_last_error() on the calling thread.
+void record_last_error(const char* msg);
+
 // ---------------------------------------------------------------------------
 // PTX wrappers (sm_90+; built for sm_100a).  All forms are CTA-local.
 // ---------------------------------------------------------------------------

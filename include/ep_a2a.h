@@ -257,6 +257,49 @@ ep_a2a_status ep_a2a_destroy(ep_a2a_handle* handle);
 const char* ep_a2a_status_string(ep_a2a_status status);
 const char* ep_a2a_last_error(void);
 
+/*
+ * Routing plan without a workspace, for callers that cannot allocate device
+ * memory.  The pages have no counterpart: it exists for callers whose device
+ * memory belongs to an outer allocator (for example a serving engine that
+ * reserves nearly all of HBM for its own pools at start-up, or a host
+ * application that does not let plug-in libraries call cudaMalloc) and who
+ * therefore cannot give ep_a2a_init a workspace that includes the routing
+ * kernel's scratch.  This call runs the same routing-plan kernel as
+ * ep_a2a_dispatch with that scratch (send-count accumulators and tickets) in a
+ * fixed array inside the library, and allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.  The caller passes every input and
+ * output.  It writes what ep_a2a_dispatch writes into plan_num_dst,
+ * plan_dst_ranks, send_counts, recv_topk_ids and recv_valid (no EPLB gather,
+ * no payload copy), with the same meaning and layout:
+ *
+ *   token_selected_experts  device int32 [ep, tpr, top_k]
+ *   local_num_tokens        host int32 [ep], each 0..tpr
+ *   active_rank_mask        host uint64 [EP_A2A_RANK_MASK_WORDS] or NULL (all active)
+ *   invalid_expert_id       < 0 means num_experts
+ *   plan_num_dst            device [ep, tpr]
+ *   plan_dst_ranks          device [ep, tpr, round_up(top_k, 8)]
+ *   send_counts             device int32 [ep, ep]
+ *   recv_topk_ids           device, rank 0's int32 [ep*tpr, top_k]; 4-byte aligned
+ *   recv_valid              device, rank 0's uint8 [ep*tpr]
+ *   recv_rank_stride_bytes  bytes from rank d's recv_topk_ids / recv_valid to rank
+ *                           d+1's (the same for both arrays; a multiple of 4)
+ *
+ * Limit: ep_size <= EP_A2A_NOALLOC_MAX_RANKS (64); larger sizes return
+ * EP_A2A_ERR_UNSUPPORTED.  The array takes 16,640 bytes on every GPU that loads
+ * the library, until the process exits.  The first call on each device looks up
+ * the array's device address with that device current (cudaGetSymbolAddress);
+ * make that first call before any stream capture.  Every call shares the array
+ * and clears the part it uses on `stream` before its kernel, so calls in stream
+ * order are independent; calls whose work overlaps on the GPU race on the array.
+ */
+#define EP_A2A_NOALLOC_MAX_RANKS 64
+ep_a2a_status ep_a2a_route_plan_noalloc(
+    int32_t ep_size, int32_t num_experts, int32_t top_k, int32_t tokens_per_rank,
+    int32_t invalid_expert_id, const int32_t* token_selected_experts,
+    const int32_t* local_num_tokens, const uint64_t* active_rank_mask, uint8_t* plan_num_dst,
+    uint8_t* plan_dst_ranks, int32_t* send_counts, int32_t* recv_topk_ids, uint8_t* recv_valid,
+    int64_t recv_rank_stride_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
