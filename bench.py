@@ -331,7 +331,7 @@ def run_ours(args):
         if cnt:
             per_kernel[name] = {"launches": cnt, "avg_ms": tot / cnt}
     kbytes = {"route_plan": by.route, "copy_bulk": by.copy, "copy_vec": by.copy,
-              "combine": by.combine}
+              "copy_staged": by.copy, "combine": by.combine}
     for name, e in per_kernel.items():
         e["algorithmic_bytes"] = kbytes[name]
         e["achieved_gbs"] = kbytes[name] / (e["avg_ms"] / 1e3) / 1e9

@@ -10,7 +10,9 @@
 // Memory plan: one CTA per token (grid-stride); each thread owns 16-byte column
 // vectors of the row and issues the loads of all (up to 8 at a time)
 // destination rows before the adds, so one thread keeps up to 128 bytes in
-// flight.  Loads bypass L1 (each row is read exactly once).
+// flight.  Loads bypass L1 (each row is read exactly once).  The widening and
+// the add are one sm_100 mixed-precision instruction per element
+// (add.rn.f32.bf16 / add.rn.f32.f16).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -36,17 +38,37 @@ __device__ __forceinline__ uint32_t f32_to_bf16_bits(float f) {
   return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
-// Add the 8 bf16 of a 16-byte vector into acc[0..8).
-__device__ __forceinline__ void add_bf16x8(float* acc, const uint4& v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    acc[2 * i] = __fadd_rn(acc[2 * i], bf16_bits_to_f32(w[i] & 0xFFFFu));
-    acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], bf16_bits_to_f32(w[i] >> 16));
-  }
+// acc0 += widen(lo half of w), acc1 += widen(hi half of w), BF16 halves.  The
+// mixed-precision add widens exactly and rounds once to nearest, so it equals
+// __fadd_rn(acc, (float)bf16) with one instruction per element.
+__device__ __forceinline__ void add_bf16x2(float& acc0, float& acc1, uint32_t w) {
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\t"
+      "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(acc0), "+f"(acc1)
+      : "r"(w));
 }
 
-// Add the 16 E4M3 of a 16-byte vector into acc[0..16) (exact widening).
+// The same for two FP16 values held as raw halves.
+__device__ __forceinline__ void add_f16x2(float& acc0, float& acc1, uint16_t lo, uint16_t hi) {
+  asm("add.rn.f32.f16 %0, %2, %0;\n\t"
+      "add.rn.f32.f16 %1, %3, %1;"
+      : "+f"(acc0), "+f"(acc1)
+      : "h"(lo), "h"(hi));
+}
+
+// Add the 8 bf16 of a 16-byte vector into acc[0..8).
+__device__ __forceinline__ void add_bf16x8(float* acc, const uint4& v) {
+  add_bf16x2(acc[0], acc[1], v.x);
+  add_bf16x2(acc[2], acc[3], v.y);
+  add_bf16x2(acc[4], acc[5], v.z);
+  add_bf16x2(acc[6], acc[7], v.w);
+}
+
+// Add the 16 E4M3 of a 16-byte vector into acc[0..16): each pair is widened
+// exactly to FP16 (every E4M3 value is an FP16 normal or zero), then added in
+// fp32 by the mixed-precision add.
 __device__ __forceinline__ void add_e4m3x16(float* acc, const uint4& v) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -55,13 +77,15 @@ __device__ __forceinline__ void add_e4m3x16(float* acc, const uint4& v) {
     for (int h = 0; h < 2; ++h) {
       const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * h)) & 0xFFFFu);
       const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-      __half_raw lo, hi;
-      lo.x = hr.x;
-      hi.x = hr.y;
-      acc[4 * i + 2 * h] = __fadd_rn(acc[4 * i + 2 * h], __half2float(__half(lo)));
-      acc[4 * i + 2 * h + 1] = __fadd_rn(acc[4 * i + 2 * h + 1], __half2float(__half(hi)));
+      add_f16x2(acc[4 * i + 2 * h], acc[4 * i + 2 * h + 1], hr.x, hr.y);
     }
   }
+}
+
+// Two fp32 -> packed bf16x2 (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&p);
 }
 
 template <bool kFp8>
@@ -106,10 +130,10 @@ __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
 #pragma unroll
       for (int q = 0; q < kElems / 8; ++q) {
         uint4 pk;
-        pk.x = f32_to_bf16_bits(acc[8 * q + 0]) | (f32_to_bf16_bits(acc[8 * q + 1]) << 16);
-        pk.y = f32_to_bf16_bits(acc[8 * q + 2]) | (f32_to_bf16_bits(acc[8 * q + 3]) << 16);
-        pk.z = f32_to_bf16_bits(acc[8 * q + 4]) | (f32_to_bf16_bits(acc[8 * q + 5]) << 16);
-        pk.w = f32_to_bf16_bits(acc[8 * q + 6]) | (f32_to_bf16_bits(acc[8 * q + 7]) << 16);
+        pk.x = pack_bf16x2(acc[8 * q + 0], acc[8 * q + 1]);
+        pk.y = pack_bf16x2(acc[8 * q + 2], acc[8 * q + 3]);
+        pk.z = pack_bf16x2(acc[8 * q + 4], acc[8 * q + 5]);
+        pk.w = pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]);
         o[q] = pk;
       }
     }

@@ -4,8 +4,19 @@
 // flashinfer.moe_ep.NVLinkOneSidedConfig, `lamport` paragraph, for the slot).
 // Bytes are moved verbatim, so every bit pattern arrives unchanged.
 //
-// Two kernels:
-//   * dispatch_bulk_kernel — for payloads whose rows are 16-byte multiples at
+// Three kernels:
+//   * dispatch_staged_kernel (default) — for payloads whose rows are 16-byte
+//     multiples at 16-byte-aligned addresses.  A producer warp streams each
+//     token's rows from HBM into a ring of shared-memory stages with bulk-async
+//     loads (completion counted on a "full" mbarrier per stage); consumer warps
+//     copy the token from shared memory into registers, release the stage
+//     ("empty" mbarrier), and write the rows to every destination with 16-byte
+//     vector stores, all threads of the CTA sharing each token.  Loads run as
+//     far ahead as the ring allows and cost no registers; the SM's threads only
+//     issue stores.
+//   * dispatch_bulk_kernel — the same staging, but the copy engine also does
+//     the stores (one bulk-async store per destination and payload).  For rows
+//     that are 16-byte multiples at
 //     16-byte-aligned addresses.  One warp per CTA; lane 0 drives a ring of
 //     shared-memory stages: a bulk-async load (cp.async.bulk, completion on an
 //     mbarrier) brings one token's rows of all such payloads into a stage, then
@@ -24,25 +35,27 @@ namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
-// Warp-collective iterator over the tokens of [begin, end) that exist and have
-// at least one destination.  All 32 lanes call next() together; the result is
-// the same in every lane.
+// Warp-collective iterator over the tokens begin, begin + stride, ... (< end)
+// that exist and have at least one destination.  All 32 lanes call next()
+// together; the result is the same in every lane.
 struct TokenStream {
   const uint8_t* plan_nd;
   const uint8_t* plan_dst;
   int plan_words;      // plan_stride / 8
   int64_t base, end;   // next batch starts at base
+  int64_t stride;      // distance between consecutive tokens of this stream
   int64_t batch;       // first token of the current batch
   unsigned pending;    // lanes of the current batch still to hand out
   int my_nd;
   uint64_t my_dst[kMaxTopK / 8];
 
-  __device__ void init(const CopyArgs& a, int64_t b, int64_t e) {
+  __device__ void init(const CopyArgs& a, int64_t b, int64_t e, int64_t st) {
     plan_nd = a.plan_nd;
     plan_dst = a.plan_dst;
     plan_words = a.plan_stride / 8;
     base = b;
     end = e;
+    stride = st;
     batch = b;
     pending = 0u;
   }
@@ -51,7 +64,7 @@ struct TokenStream {
   __device__ int64_t next(int lane, int& nd, uint64_t (&dst)[kMaxTopK / 8]) {
     while (pending == 0u) {
       if (base >= end) return -1;
-      const int64_t tok = base + lane;
+      const int64_t tok = base + lane * stride;
       int v = kNoToken;
       if (tok < end) {
         v = plan_nd[tok];
@@ -65,7 +78,7 @@ struct TokenStream {
       my_nd = v;
       pending = __ballot_sync(kFull, v != kNoToken && v > 0);
       batch = base;
-      base += 32;
+      base += 32 * stride;
     }
     const int src_lane = __ffs(pending) - 1;
     pending &= pending - 1u;
@@ -73,9 +86,25 @@ struct TokenStream {
 #pragma unroll
     for (int w = 0; w < kMaxTopK / 8; ++w)
       if (w < plan_words) dst[w] = __shfl_sync(kFull, my_dst[w], src_lane);
-    return batch + src_lane;
+    return batch + src_lane * stride;
   }
 };
+
+// This CTA's token stream: a contiguous chunk, or every gridDim.x-th token
+// (interleaved, so that the CTAs of the grid work on neighbouring slots).
+__device__ __forceinline__ void cta_tokens(const CopyArgs& a, int64_t& begin, int64_t& end,
+                                           int64_t& stride) {
+  if (a.interleave) {
+    begin = blockIdx.x;
+    end = a.ntok;
+    stride = gridDim.x;
+  } else {
+    const int64_t chunk = (a.ntok + gridDim.x - 1) / gridDim.x;
+    begin = min(a.ntok, (int64_t)blockIdx.x * chunk);
+    end = min(a.ntok, begin + chunk);
+    stride = 1;
+  }
+}
 
 // i-th destination rank of a packed plan row (byte i of words w0..w3); the
 // words are chosen with selects so they stay in registers.
@@ -96,9 +125,8 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(const CopyArgs a) {
   const int lane = threadIdx.x;
   const int S = a.stages;
   const int L = S - Q;                      // loads issued ahead of stores
-  const int64_t chunk = (a.ntok + gridDim.x - 1) / gridDim.x;
-  const int64_t begin = min(a.ntok, (int64_t)blockIdx.x * chunk);
-  const int64_t end = min(a.ntok, begin + chunk);
+  int64_t begin, end, stride;
+  cta_tokens(a, begin, end, stride);
   const uint32_t smem0 = smem_addr(stage_mem);
   const uint32_t bar0 = smem_addr(bars);
 
@@ -109,7 +137,7 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(const CopyArgs a) {
   __syncwarp();
 
   TokenStream ts;
-  ts.init(a, begin, end);
+  ts.init(a, begin, end, stride);
   int nd;
   uint64_t dst[kMaxTopK / 8];
   const int words = a.plan_stride / 8;
@@ -189,11 +217,35 @@ __global__ void __launch_bounds__(32) dispatch_bulk_kernel(const CopyArgs a) {
   }
 }
 
+template <typename T>
+__device__ __forceinline__ T load_src(const T* p) {
+  return *p;
+}
+template <typename T>
+__device__ __forceinline__ void store_dst(T* p, const T& v, bool) {
+  *p = v;
+}
+// 16-byte accesses: the source is read once (no L1 allocation); with
+// `streaming` the stores carry the evict-first (.cs) hint.
+template <>
+__device__ __forceinline__ uint4 load_src<uint4>(const uint4* p) {
+  return ld_stream_v4(p);
+}
+template <>
+__device__ __forceinline__ void store_dst<uint4>(uint4* p, const uint4& v, bool streaming) {
+  if (streaming)
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+  else
+    *p = v;
+}
+
 template <typename T, int U>
 __device__ __forceinline__ void copy_row(const uint8_t* __restrict__ src, int64_t rb,
                                          uint8_t* rank0, int64_t rank_stride, int64_t off,
                                          uint64_t w0, uint64_t w1, uint64_t w2, uint64_t w3,
-                                         int nd, int lane) {
+                                         int nd, int lane, bool streaming) {
   const int64_t n = rb / (int64_t)sizeof(T);
   const T* s = reinterpret_cast<const T*>(src);
   for (int64_t i0 = lane; i0 < n; i0 += 32 * U) {
@@ -201,7 +253,7 @@ __device__ __forceinline__ void copy_row(const uint8_t* __restrict__ src, int64_
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int64_t i = i0 + (int64_t)u * 32;
-      if (i < n) v[u] = s[i];
+      if (i < n) v[u] = load_src<T>(s + i);
     }
     for (int q = 0; q < nd; ++q) {
       T* d = reinterpret_cast<T*>(rank0 + (int64_t)dst_rank(w0, w1, w2, w3, q) * rank_stride +
@@ -209,7 +261,7 @@ __device__ __forceinline__ void copy_row(const uint8_t* __restrict__ src, int64_
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t i = i0 + (int64_t)u * 32;
-        if (i < n) d[i] = v[u];
+        if (i < n) store_dst<T>(d + i, v[u], streaming);
       }
     }
   }
@@ -217,6 +269,9 @@ __device__ __forceinline__ void copy_row(const uint8_t* __restrict__ src, int64_
 
 constexpr int kVecThreads = 256;
 
+// kAll16: every payload of the launch moves in 16-byte vectors (one code path,
+// fewer registers); otherwise each payload picks its own vector width.
+template <int U, bool kAll16, bool kStreaming>
 __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArgs a) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -233,31 +288,191 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
     for (int p = 0; p < a.np; ++p) {
       const uint8_t* src = a.src[p] + tok * a.rb[p];
       const int64_t off = a.dst_off[p] + tok * a.rb[p];
+      if (kAll16) {
+        copy_row<uint4, U>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd, lane,
+                           kStreaming);
+        continue;
+      }
       switch (a.vec[p]) {
         case 16:
-          copy_row<uint4, 4>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd, lane);
+          copy_row<uint4, U>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd, lane,
+                             kStreaming);
           break;
         case 8:
-          copy_row<uint2, 4>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd, lane);
+          copy_row<uint2, U>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd, lane,
+                             false);
           break;
         case 4:
-          copy_row<uint32_t, 4>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
-                                lane);
+          copy_row<uint32_t, U>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
+                                lane, false);
           break;
         case 2:
-          copy_row<uint16_t, 4>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
-                                lane);
+          copy_row<uint16_t, U>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
+                                lane, false);
           break;
         default:
-          copy_row<uint8_t, 4>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
-                               lane);
+          copy_row<uint8_t, U>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
+                               lane, false);
           break;
       }
     }
   }
 }
 
+template <int NCW, int MAXV>
+__global__ void __launch_bounds__(32 * (NCW + 1)) dispatch_staged_kernel(const CopyArgs a) {
+  extern __shared__ __align__(128) uint8_t stage_mem[];
+  __shared__ __align__(8) uint64_t full_bar[kMaxStages];
+  __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
+  __shared__ int64_t st_tok[kMaxStages];
+  __shared__ int st_nd[kMaxStages];
+  __shared__ uint64_t st_dst[kMaxStages][kMaxTopK / 8];
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int S = a.stages;
+  int64_t begin, end, stride;
+  cta_tokens(a, begin, end, stride);
+  const uint32_t smem0 = smem_addr(stage_mem);
+  const uint32_t full0 = smem_addr(full_bar);
+  const uint32_t empty0 = smem_addr(empty_bar);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, NCW);
+    }
+    mbar_init_fence();
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // producer: one token per stage, in order; the token after the last one is
+    // a sentinel (index -1) that tells the consumers to stop
+    TokenStream ts;
+    ts.init(a, begin, end, stride);
+    const int words = a.plan_stride / 8;
+    for (int64_t i = 0;; ++i) {
+      int nd = 0;
+      uint64_t dst[kMaxTopK / 8];
+      const int64_t tok = ts.next(lane, nd, dst);
+      const int s = (int)(i % S);
+      const uint32_t use = (uint32_t)(i / S);
+      bool ok = true;
+      if (lane == 0) {
+        if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1u, kWaitLimitNs)) {
+          atomicOr(a.err, kErrWaitTimeout);
+          ok = false;
+        } else {
+          st_tok[s] = tok;
+          st_nd[s] = nd;
+#pragma unroll
+          for (int w = 0; w < kMaxTopK / 8; ++w)
+            if (w < words) st_dst[s][w] = dst[w];
+          if (tok < 0) {
+            mbar_arrive(full0 + 8 * s);
+          } else {
+            mbar_arrive_expect_tx(full0 + 8 * s, a.tx_bytes);
+            const uint32_t stage = smem0 + (uint32_t)s * a.stage_bytes;
+            for (int p = 0; p < a.np; ++p)
+              bulk_load(stage + a.smem_off[p], a.src[p] + tok * a.rb[p], (uint32_t)a.rb[p],
+                        full0 + 8 * s);
+          }
+        }
+      }
+      ok = __shfl_sync(kFull, ok, 0);
+      if (tok < 0 || !ok) break;
+    }
+    return;
+  }
+
+  // consumers: thread c owns the stage's 16-byte vectors c, c + 32*NCW, ...
+  // (at most MAXV of them); for each, the receive-array offset of its bytes
+  // and the row length of its payload
+  constexpr int kCons = 32 * NCW;
+  const int c = threadIdx.x - 32;
+  const int nvec_total = (int)(a.tx_bytes / 16);
+  int64_t dbase[MAXV];
+  uint32_t drow[MAXV];
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j) {
+    const int f = c + j * kCons;
+    dbase[j] = 0;
+    drow[j] = 0;
+    if (f < nvec_total) {
+      const uint32_t byte = (uint32_t)f * 16u;
+      int p = 0;
+      while (p + 1 < a.np && byte >= a.smem_off[p + 1]) ++p;
+      dbase[j] = a.dst_off[p] + (int64_t)(byte - a.smem_off[p]);
+      drow[j] = (uint32_t)a.rb[p];
+    }
+  }
+  const int words = a.plan_stride / 8;
+  for (int64_t i = 0;; ++i) {
+    const int s = (int)(i % S);
+    const uint32_t use = (uint32_t)(i / S);
+    if (!mbar_wait_bounded(full0 + 8 * s, use & 1u, kWaitLimitNs)) {
+      atomicOr(a.err, kErrWaitTimeout);
+      break;
+    }
+    const int64_t tok = st_tok[s];
+    if (tok < 0) break;
+    const int nd = st_nd[s];
+    const uint64_t w0 = st_dst[s][0];
+    const uint64_t w1 = words > 1 ? st_dst[s][1] : 0;
+    const uint64_t w2 = words > 2 ? st_dst[s][2] : 0;
+    const uint64_t w3 = words > 3 ? st_dst[s][3] : 0;
+    const uint8_t* stage = stage_mem + (size_t)s * a.stage_bytes;
+    uint4 v[MAXV];
+#pragma unroll
+    for (int j = 0; j < MAXV; ++j)
+      if (c + j * kCons < nvec_total)
+        v[j] = *reinterpret_cast<const uint4*>(stage + (uint32_t)(c + j * kCons) * 16u);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * s);      // this warp is done with the stage
+    int64_t off[MAXV];
+#pragma unroll
+    for (int j = 0; j < MAXV; ++j) off[j] = dbase[j] + tok * (int64_t)drow[j];
+    for (int q = 0; q < nd; ++q) {
+      uint8_t* rank = a.rank0 + (int64_t)dst_rank(w0, w1, w2, w3, q) * a.rank_stride;
+#pragma unroll
+      for (int j = 0; j < MAXV; ++j)
+        if (c + j * kCons < nvec_total) *reinterpret_cast<uint4*>(rank + off[j]) = v[j];
+    }
+  }
+}
+
+template <int NCW, int MAXV>
+cudaError_t launch_staged(const CopyArgs& a, int grid, size_t smem, cudaStream_t stream) {
+  cudaError_t err = cudaFuncSetAttribute(dispatch_staged_kernel<NCW, MAXV>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  dispatch_staged_kernel<NCW, MAXV><<<grid, 32 * (NCW + 1), smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int NCW>
+cudaError_t launch_staged_v(const CopyArgs& a, int grid, size_t smem, cudaStream_t stream) {
+  const int per_thread = (int)((a.tx_bytes / 16 + 32 * NCW - 1) / (32 * NCW));
+  if (per_thread <= 1) return launch_staged<NCW, 1>(a, grid, smem, stream);
+  if (per_thread <= 2) return launch_staged<NCW, 2>(a, grid, smem, stream);
+  if (per_thread <= 4) return launch_staged<NCW, 4>(a, grid, smem, stream);
+  if (per_thread <= 8) return launch_staged<NCW, 8>(a, grid, smem, stream);
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
+
+cudaError_t launch_dispatch_staged(const CopyArgs& a, int consumer_warps, int grid,
+                                   cudaStream_t stream) {
+  const size_t smem = (size_t)a.stage_bytes * a.stages;
+  switch (consumer_warps) {
+    case 4: return launch_staged_v<4>(a, grid, smem, stream);
+    case 8: return launch_staged_v<8>(a, grid, smem, stream);
+    case 16: return launch_staged_v<16>(a, grid, smem, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 int bulk_queue_depth(int stages) {
   // store groups allowed to be reading shared memory when a stage is refilled
@@ -297,9 +512,32 @@ cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t strea
   return cudaGetLastError();
 }
 
-cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, cudaStream_t stream) {
-  dispatch_vec_kernel<<<grid, kVecThreads, 0, stream>>>(a);
+template <int U>
+cudaError_t launch_vec_u(const CopyArgs& a, int grid, bool streaming, cudaStream_t stream) {
+  bool all16 = true;
+  for (int p = 0; p < a.np; ++p) all16 &= a.vec[p] == 16;
+  if (all16) {
+    if (streaming)
+      dispatch_vec_kernel<U, true, true><<<grid, kVecThreads, 0, stream>>>(a);
+    else
+      dispatch_vec_kernel<U, true, false><<<grid, kVecThreads, 0, stream>>>(a);
+  } else {
+    if (streaming)
+      dispatch_vec_kernel<U, false, true><<<grid, kVecThreads, 0, stream>>>(a);
+    else
+      dispatch_vec_kernel<U, false, false><<<grid, kVecThreads, 0, stream>>>(a);
+  }
   return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, int unroll, bool streaming,
+                                cudaStream_t stream) {
+  switch (unroll) {
+    case 2: return launch_vec_u<2>(a, grid, streaming, stream);
+    case 4: return launch_vec_u<4>(a, grid, streaming, stream);
+    case 8: return launch_vec_u<8>(a, grid, streaming, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace ep_a2a

@@ -66,11 +66,16 @@ struct CopyArgs {
   uint32_t stage_bytes;                  // bulk path: bytes of one stage
   uint32_t tx_bytes;                     // bulk path: bytes one token brings in
   int stages;                            // bulk path
+  int interleave;                        // bulk paths: 1 = CTA b takes tokens b, b+grid, ...
   uint32_t* err;
 };
 
 cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t stream);
-cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, cudaStream_t stream);
+cudaError_t launch_dispatch_staged(const CopyArgs& a, int consumer_warps, int grid,
+                                   cudaStream_t stream);
+constexpr int kStagedMaxVec = 8;         // 16-byte vectors per consumer thread per token
+cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, int unroll, bool streaming,
+                                cudaStream_t stream);
 int bulk_queue_depth(int stages);        // groups allowed in flight for `stages`
 
 // ---------------------------------------------------------------------------
@@ -111,6 +116,10 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 __device__ __forceinline__ void mbar_init_fence() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {

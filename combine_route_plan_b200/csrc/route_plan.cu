@@ -36,7 +36,7 @@ namespace {
 
 constexpr int kRouteThreads = 256;
 constexpr int kRouteWarps = kRouteThreads / 32;
-constexpr int kTokPerBlock = 128;
+constexpr int kTokPerBlock = 32;
 
 template <bool kMask>
 __device__ __forceinline__ bool rank_live(const uint64_t* live, int r) {

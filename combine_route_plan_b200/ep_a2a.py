@@ -30,7 +30,9 @@ MAX_TOP_K = 32
 OK, ERR_INVALID_ARG, ERR_CAPACITY, ERR_UNSUPPORTED, ERR_CUDA, ERR_NOT_INITIALIZED, \
     ERR_NO_PLAN, ERR_DEVICE_TIMEOUT = range(8)
 COMBINE_BF16, COMBINE_FP8_E4M3 = 0, 1
-OPT_COPY_PATH, OPT_COPY_CTAS_PER_SM, OPT_COPY_STAGES, OPT_COMBINE_THREADS = range(4)
+OPT_COPY_PATH, OPT_COPY_CTAS_PER_SM, OPT_COPY_STAGES, OPT_COMBINE_THREADS, \
+    OPT_BULK_MIN_ROW_BYTES, OPT_COMBINE_CTAS_PER_SM, OPT_COPY_CONSUMER_WARPS, \
+    OPT_COPY_INTERLEAVE, OPT_VEC_UNROLL, OPT_VEC_CTAS_PER_SM, OPT_STORE_STREAMING = range(11)
 
 
 class EpA2AError(RuntimeError):
@@ -72,11 +74,11 @@ class DispatchResult(ctypes.Structure):
     ]
 
 
-KERNEL_NAMES = ["route_plan", "copy_bulk", "copy_vec", "combine"]
+KERNEL_NAMES = ["route_plan", "copy_bulk", "copy_vec", "combine", "copy_staged"]
 
 
 class KernelTimes(ctypes.Structure):
-    _fields_ = [("launches", ctypes.c_int64 * 4), ("total_ms", ctypes.c_double * 4)]
+    _fields_ = [("launches", ctypes.c_int64 * 5), ("total_ms", ctypes.c_double * 5)]
 
 
 def _load():

@@ -216,11 +216,27 @@ ep_a2a_status ep_a2a_debug_wait_probe(ep_a2a_handle handle, int64_t limit_ns, vo
 
 /* Tuning knobs of the kernels (performance only; results never change). */
 typedef enum {
-  EP_A2A_OPT_COPY_PATH = 0,       /* 0 = bulk-async (TMA) copy where rows allow it,
-                                     1 = vector load/store copy for every payload */
+  EP_A2A_OPT_COPY_PATH = 0,       /* 1 = vector load/store copy for every payload
+                                     (default); for rows that are 16-byte multiples at
+                                     16-byte-aligned addresses: 0 = bulk-async loads into
+                                     shared memory + vector stores, 2 = bulk-async loads
+                                     and bulk-async stores (other rows take the vector
+                                     copy) */
   EP_A2A_OPT_COPY_CTAS_PER_SM = 1,/* CTAs per SM of the bulk copy kernel (1..8) */
-  EP_A2A_OPT_COPY_STAGES = 2,     /* shared-memory row stages per copy CTA (2..32) */
-  EP_A2A_OPT_COMBINE_THREADS = 3  /* threads per CTA of the combine kernel (64..512) */
+  EP_A2A_OPT_COPY_STAGES = 2,     /* shared-memory row stages per copy CTA (2..32; 0 = as
+                                     many as fit, up to 8 / 16) */
+  EP_A2A_OPT_COMBINE_THREADS = 3, /* threads per CTA of the combine kernel (64..512;
+                                     default 64) */
+  EP_A2A_OPT_BULK_MIN_ROW_BYTES = 4, /* rows shorter than this take the vector copy (0..2^24) */
+  EP_A2A_OPT_COMBINE_CTAS_PER_SM = 5, /* combine grid = min(tokens, SMs x this) (1..1024);
+                                       0 = 128 */
+  EP_A2A_OPT_COPY_CONSUMER_WARPS = 6, /* store warps per CTA of copy path 0 (4, 8 or 16) */
+  EP_A2A_OPT_COPY_INTERLEAVE = 7, /* paths 0 and 2: 1 = CTA b copies tokens b, b + grid, ...
+                                     (default); 0 = each CTA copies a contiguous chunk */
+  EP_A2A_OPT_VEC_UNROLL = 8,      /* vector copy: vectors per lane in flight (2, 4 = default, 8) */
+  EP_A2A_OPT_VEC_CTAS_PER_SM = 9, /* vector copy grid = SMs x this (1..64; default 32) */
+  EP_A2A_OPT_STORE_STREAMING = 10 /* vector copy: 1 = evict-first (.cs) 16-byte stores
+                                     (default), 0 = plain stores */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 
@@ -235,10 +251,11 @@ ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int6
  */
 typedef enum {
   EP_A2A_KERNEL_ROUTE_PLAN = 0,   /* routing plan + EPLB gather */
-  EP_A2A_KERNEL_COPY_BULK = 1,    /* dispatch rows, bulk-async path */
+  EP_A2A_KERNEL_COPY_BULK = 1,    /* dispatch rows, bulk-async loads and stores */
   EP_A2A_KERNEL_COPY_VEC = 2,     /* dispatch rows, vector path */
   EP_A2A_KERNEL_COMBINE = 3,
-  EP_A2A_KERNEL_COUNT = 4
+  EP_A2A_KERNEL_COPY_STAGED = 4,  /* dispatch rows, bulk-async loads + vector stores */
+  EP_A2A_KERNEL_COUNT = 5
 } ep_a2a_kernel;
 typedef struct {
   int64_t launches[EP_A2A_KERNEL_COUNT];

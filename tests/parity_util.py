@@ -42,13 +42,14 @@ def assert_equal(gpu: torch.Tensor, want: np.ndarray, what: str):
 class Run:
     """One dispatch + combine through the C ABI."""
 
-    def __init__(self, w, x, copy_path=0, options=None, capacity=None, fp8=False):
+    def __init__(self, w, x, copy_path=None, options=None, capacity=None, fp8=False):
         from combine_route_plan_b200 import ep_a2a
         ep, tpr, k, E, H = w.ep_size, w.tokens_per_rank, w.top_k, w.num_experts, w.hidden
         self.comm = ep_a2a.EpA2A(ep, E, k, capacity or tpr, H, w.payload_row_bytes(),
                                  eplb_stats_num_experts=E if w.eplb else 0,
                                  enable_rank_mask=bool(w.masked_ranks), workspace_fill=CANARY)
-        self.comm.set_option(ep_a2a.OPT_COPY_PATH, copy_path)
+        if copy_path is not None:               # None: the library's default path
+            self.comm.set_option(ep_a2a.OPT_COPY_PATH, copy_path)
         for opt, val in (options or {}).items():
             self.comm.set_option(opt, val)
         self.ids = x.token_selected_experts.cuda()

@@ -32,7 +32,7 @@ def _inputs(name):
     return W.make_inputs(W.BY_NAME[name])
 
 
-def _full_check(w, copy_path=0, options=None):
+def _full_check(w, copy_path=None, options=None):
     x = _inputs(w.name)
     run = U.Run(w, x, copy_path=copy_path, options=options)
     plan = U.oracle_plan(w, x)
@@ -50,29 +50,64 @@ def test_workload_bit_exact(name):
     _full_check(W.BY_NAME[name])
 
 
-@pytest.mark.parametrize("name", ["c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked"])
-def test_vector_copy_path_bit_exact(name):
-    from combine_route_plan_b200 import ep_a2a
-    _full_check(W.BY_NAME[name], copy_path=1)
+@pytest.mark.parametrize("name,path", [
+    (n, p) for n in ("c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked", "c3_ep16_zipf_nvfp4")
+    for p in (0, 2)])
+def test_bulk_copy_paths_bit_exact(name, path):
+    """The two bulk-async copy paths (loads into shared memory + vector stores;
+    bulk loads + bulk stores) on the workloads, next to the default vector path."""
+    _full_check(W.BY_NAME[name], copy_path=path)
 
 
-@pytest.mark.parametrize("stages,ctas", [(2, 1), (3, 2), (4, 4), (8, 1), (16, 1), (32, 1), (5, 3)])
-def test_copy_tuning_does_not_change_results(stages, ctas):
+@pytest.mark.parametrize("path,stages,ctas,cw,inter", [
+    (0, 0, 1, 8, 0), (0, 2, 1, 4, 1), (0, 3, 2, 16, 0), (0, 5, 3, 8, 1), (0, 32, 1, 8, 0),
+    (0, 4, 4, 4, 1), (2, 2, 1, 8, 0), (2, 3, 2, 8, 1), (2, 4, 4, 8, 0), (2, 8, 1, 8, 1),
+    (2, 16, 1, 8, 0), (2, 32, 1, 8, 1), (2, 5, 3, 8, 0),
+])
+def test_copy_tuning_does_not_change_results(path, stages, ctas, cw, inter):
+    """Every copy path and staging configuration writes the same bytes."""
     from combine_route_plan_b200 import ep_a2a
     w = W.scaled(W.C2, 96)
     x = W.make_inputs(w, with_expert_output=False)
-    run = U.Run(w, x, options={ep_a2a.OPT_COPY_STAGES: stages, ep_a2a.OPT_COPY_CTAS_PER_SM: ctas})
+    run = U.Run(w, x, copy_path=path,
+                options={ep_a2a.OPT_COPY_STAGES: stages, ep_a2a.OPT_COPY_CTAS_PER_SM: ctas,
+                         ep_a2a.OPT_COPY_CONSUMER_WARPS: cw, ep_a2a.OPT_COPY_INTERLEAVE: inter})
     plan = U.oracle_plan(w, x)
     U.check_plan(run, plan, w)
     U.check_payloads(run, plan, w, x)
 
 
-@pytest.mark.parametrize("threads", [64, 96, 256, 512])
-def test_combine_threads_do_not_change_results(threads):
+@pytest.mark.parametrize("unroll,ctas,streaming,rows", [
+    (2, 1, 0, [14336, 32]), (4, 8, 1, [14336, 64, 32]), (8, 64, 0, [14336, 32]),
+    (8, 3, 1, [100, 13, 16]), (2, 16, 1, [7, 4096 + 8]),
+])
+def test_vector_copy_variants(unroll, ctas, streaming, rows):
+    from combine_route_plan_b200 import ep_a2a
+    w, x = _custom(8, 64, 8, 50, 32, rows, seed=unroll * 31 + ctas)
+    run = U.Run(w, x, copy_path=1, options={ep_a2a.OPT_VEC_UNROLL: unroll,
+                                            ep_a2a.OPT_VEC_CTAS_PER_SM: ctas,
+                                            ep_a2a.OPT_STORE_STREAMING: streaming})
+    plan = U.oracle_plan(w, x)
+    U.check_payloads(run, plan, w, x)
+
+
+@pytest.mark.parametrize("rows", [[16], [4096 + 16, 32], [65536 + 16, 48]])
+def test_staged_copy_row_sizes(rows):
+    """Rows from one vector per token up to more than the staged kernel holds in
+    registers (which then falls back to the vector copy)."""
+    w, x = _custom(4, 16, 4, 40, 32, rows, seed=len(rows) * 7 + rows[0] % 97)
+    run = U.Run(w, x)
+    plan = U.oracle_plan(w, x)
+    U.check_payloads(run, plan, w, x)
+
+
+@pytest.mark.parametrize("threads,ctas", [(64, 0), (96, 3), (256, 64), (512, 1), (128, 1024)])
+def test_combine_launch_shape_does_not_change_results(threads, ctas):
     from combine_route_plan_b200 import ep_a2a
     w = W.C2
     x = _inputs(w.name)
-    run = U.Run(w, x, options={ep_a2a.OPT_COMBINE_THREADS: threads})
+    run = U.Run(w, x, options={ep_a2a.OPT_COMBINE_THREADS: threads,
+                               ep_a2a.OPT_COMBINE_CTAS_PER_SM: ctas})
     U.check_combine(run, U.oracle_plan(w, x), w, x)
 
 
