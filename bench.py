@@ -101,6 +101,34 @@ class CudaTimer:
         return float(self.a.elapsed_time(self.b))
 
 
+def run_timed_flushed(step, flush, steps: int, warmup: int, stream, dist, device=None,
+                      during=None) -> float:
+    """Like run_timed, but L2 is flushed before every step and only the steps
+    are timed (one event pair around each); returns the summed milliseconds,
+    max over ranks."""
+    import torch
+    for _ in range(warmup):
+        flush()
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    if during is not None:
+        during.start()
+    for a, b in ev:
+        flush()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    if during is not None:
+        during.stop()
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    barrier(dist, device)
+    return reduce_max(ms, dist, device)
+
+
 class WallTimer:
     """Host clock; used only by the CPU tests of the harness and the oracle arm."""
 
@@ -297,6 +325,8 @@ def run_ours(args):
     comm = ep_a2a.EpA2A(w.ep_size, w.num_experts, w.top_k, w.tokens_per_rank, w.hidden,
                         w.payload_row_bytes(), eplb_stats_num_experts=w.num_experts if w.eplb else 0,
                         enable_rank_mask=mask is not None)
+    if args.no_pdl:
+        comm.set_option(ep_a2a.OPT_PDL, 0)
     out = torch.empty((w.ep_size, w.tokens_per_rank, w.hidden), dtype=torch.bfloat16, device=device)
     tpr = w.tokens_per_rank
     fp8 = args.combine == "fp8"
@@ -317,9 +347,44 @@ def run_ours(args):
     by = algorithmic_bytes(w, n_tok, sum_d, live, fp8)
 
     clocks = ClockSampler(local)
-    ms = run_timed(step, args.steps, args.warmup, CudaTimer(stream), dist, device, during=clocks,
-                   on_start=lambda: ep_a2a.ep_a2a_profile_start(comm.handle, 4 * args.steps + 8))
-    kt = ep_a2a.ep_a2a_profile_stop(comm.handle)
+    flush_buf = None
+    if args.l2_flush:
+        flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    if args.graph or flush_buf is not None:
+        # per-kernel times from an eager profiled pass (flushing L2 before each
+        # step when the timed loop does), then the timed loop without events
+        # between the kernels
+        def flushed_step():
+            if flush_buf is not None:
+                flush_buf.zero_()
+            step()
+        run_timed(flushed_step, args.steps, args.warmup, CudaTimer(stream), dist, device,
+                  on_start=lambda: ep_a2a.ep_a2a_profile_start(comm.handle, 4 * args.steps + 8))
+        kt = ep_a2a.ep_a2a_profile_stop(comm.handle)
+        timed_step = step
+        if args.graph:
+            graph = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                step()
+            torch.cuda.current_stream().wait_stream(side)
+            with torch.cuda.graph(graph):
+                step()
+            timed_step = graph.replay
+        if flush_buf is not None:
+            ms = run_timed_flushed(timed_step, lambda: flush_buf.zero_(), args.steps, args.warmup,
+                                   stream, dist, device, during=clocks)
+        else:
+            ms = run_timed(timed_step, args.steps, args.warmup, CudaTimer(stream), dist, device,
+                           during=clocks)
+    else:
+        ms = run_timed(step, args.steps, args.warmup, CudaTimer(stream), dist, device,
+                       during=clocks,
+                       on_start=lambda: ep_a2a.ep_a2a_profile_start(comm.handle,
+                                                                    4 * args.steps + 8))
+        kt = ep_a2a.ep_a2a_profile_stop(comm.handle)
+    torch.cuda.synchronize()
     assert comm.get_status() == ep_a2a.OK
     ms_per_step = ms / args.steps
     tokens_total = ws * n_tok * args.steps
@@ -373,7 +438,10 @@ def run_ours(args):
                             f"extra {w.extra_bytes} B/token, EPLB stats, "
                             f"{'FP8 E4M3' if fp8 else 'BF16'} combine (fp32 accumulate)",
                 "tokens_per_step_per_gpu": n_tok, "mean_distinct_ranks": sum_d / n_tok,
-                "l2": "inputs larger than L2 (no flush)",
+                "l2": ("512 MB L2 flush before every step, each step timed alone"
+                       if args.l2_flush else "inputs larger than L2 (no flush)"),
+                "launch": ("CUDA graph replay" if args.graph else "eager") +
+                          (", programmatic dependent launch" if not args.no_pdl else ""),
                 "parallelism": f"{ws} independent replicas" if ws > 1 else "1 GPU, virtual ranks",
             },
             "hbm": {"step_algorithmic_bytes": by.step, "achieved_gbs": step_gbs,
@@ -534,6 +602,12 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget-s", type=float, default=120.0)
+    ap.add_argument("--graph", action="store_true",
+                    help="time CUDA-graph replays of the step (small workloads)")
+    ap.add_argument("--l2-flush", action="store_true",
+                    help="flush L2 before every step and time steps alone (small workloads)")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch without programmatic dependent launch")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")

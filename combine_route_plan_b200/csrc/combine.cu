@@ -90,6 +90,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 template <bool kFp8>
 __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
+  pdl_wait();
   constexpr int kElems = kFp8 ? 16 : 8;       // elements per 16-byte input vector
   constexpr int kElemBytes = kFp8 ? 1 : 2;
   const int nvec = a.H / kElems;
@@ -143,6 +144,7 @@ __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
 // Any hidden size and alignment: one element per thread step.
 template <bool kFp8>
 __global__ void __launch_bounds__(512) combine_scalar_kernel(const CombineArgs a) {
+  pdl_wait();
   const int words = a.plan_stride / 8;
   for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
     const int nd = a.plan_nd[tok];
@@ -211,19 +213,14 @@ __global__ void wait_timeout_probe_kernel(uint32_t* err, unsigned long long limi
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, int threads, int grid,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, bool pdl) {
+  const dim3 g(grid), b(threads);
   if (vec) {
-    if (fp8)
-      combine_vec_kernel<true><<<grid, threads, 0, stream>>>(a);
-    else
-      combine_vec_kernel<false><<<grid, threads, 0, stream>>>(a);
-  } else {
-    if (fp8)
-      combine_scalar_kernel<true><<<grid, threads, 0, stream>>>(a);
-    else
-      combine_scalar_kernel<false><<<grid, threads, 0, stream>>>(a);
+    if (fp8) return launch_kernel(combine_vec_kernel<true>, g, b, 0, stream, pdl, a);
+    return launch_kernel(combine_vec_kernel<false>, g, b, 0, stream, pdl, a);
   }
-  return cudaGetLastError();
+  if (fp8) return launch_kernel(combine_scalar_kernel<true>, g, b, 0, stream, pdl, a);
+  return launch_kernel(combine_scalar_kernel<false>, g, b, 0, stream, pdl, a);
 }
 
 cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n,

@@ -116,6 +116,7 @@ __device__ __forceinline__ int dst_rank(uint64_t w0, uint64_t w1, uint64_t w2, u
 
 template <int Q>
 __global__ void __launch_bounds__(32) dispatch_bulk_kernel(const CopyArgs a) {
+  pdl_wait();
   extern __shared__ __align__(128) uint8_t stage_mem[];
   __shared__ __align__(8) uint64_t bars[kMaxStages];
   __shared__ int64_t st_tok[kMaxStages];
@@ -273,6 +274,7 @@ constexpr int kVecThreads = 256;
 // fewer registers); otherwise each payload picks its own vector width.
 template <int U, bool kAll16, bool kStreaming>
 __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArgs a) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int words = a.plan_stride / 8;
@@ -321,6 +323,7 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
 
 template <int NCW, int MAXV>
 __global__ void __launch_bounds__(32 * (NCW + 1)) dispatch_staged_kernel(const CopyArgs a) {
+  pdl_wait();
   extern __shared__ __align__(128) uint8_t stage_mem[];
   __shared__ __align__(8) uint64_t full_bar[kMaxStages];
   __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
@@ -443,33 +446,35 @@ __global__ void __launch_bounds__(32 * (NCW + 1)) dispatch_staged_kernel(const C
 }
 
 template <int NCW, int MAXV>
-cudaError_t launch_staged(const CopyArgs& a, int grid, size_t smem, cudaStream_t stream) {
+cudaError_t launch_staged(const CopyArgs& a, int grid, size_t smem, cudaStream_t stream,
+                          bool pdl) {
   cudaError_t err = cudaFuncSetAttribute(dispatch_staged_kernel<NCW, MAXV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  dispatch_staged_kernel<NCW, MAXV><<<grid, 32 * (NCW + 1), smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_kernel(dispatch_staged_kernel<NCW, MAXV>, dim3(grid), dim3(32 * (NCW + 1)), smem,
+                       stream, pdl, a);
 }
 
 template <int NCW>
-cudaError_t launch_staged_v(const CopyArgs& a, int grid, size_t smem, cudaStream_t stream) {
+cudaError_t launch_staged_v(const CopyArgs& a, int grid, size_t smem, cudaStream_t stream,
+                            bool pdl) {
   const int per_thread = (int)((a.tx_bytes / 16 + 32 * NCW - 1) / (32 * NCW));
-  if (per_thread <= 1) return launch_staged<NCW, 1>(a, grid, smem, stream);
-  if (per_thread <= 2) return launch_staged<NCW, 2>(a, grid, smem, stream);
-  if (per_thread <= 4) return launch_staged<NCW, 4>(a, grid, smem, stream);
-  if (per_thread <= 8) return launch_staged<NCW, 8>(a, grid, smem, stream);
+  if (per_thread <= 1) return launch_staged<NCW, 1>(a, grid, smem, stream, pdl);
+  if (per_thread <= 2) return launch_staged<NCW, 2>(a, grid, smem, stream, pdl);
+  if (per_thread <= 4) return launch_staged<NCW, 4>(a, grid, smem, stream, pdl);
+  if (per_thread <= 8) return launch_staged<NCW, 8>(a, grid, smem, stream, pdl);
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
 cudaError_t launch_dispatch_staged(const CopyArgs& a, int consumer_warps, int grid,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, bool pdl) {
   const size_t smem = (size_t)a.stage_bytes * a.stages;
   switch (consumer_warps) {
-    case 4: return launch_staged_v<4>(a, grid, smem, stream);
-    case 8: return launch_staged_v<8>(a, grid, smem, stream);
-    case 16: return launch_staged_v<16>(a, grid, smem, stream);
+    case 4: return launch_staged_v<4>(a, grid, smem, stream, pdl);
+    case 8: return launch_staged_v<8>(a, grid, smem, stream, pdl);
+    case 16: return launch_staged_v<16>(a, grid, smem, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -482,60 +487,44 @@ int bulk_queue_depth(int stages) {
   return 1;
 }
 
-cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t stream) {
-  const size_t smem = (size_t)a.stage_bytes * a.stages;
-  const int q = bulk_queue_depth(a.stages);
-  cudaError_t err = cudaSuccess;
-  switch (q) {
-    case 8:
-      err = cudaFuncSetAttribute(dispatch_bulk_kernel<8>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (err == cudaSuccess) dispatch_bulk_kernel<8><<<grid, 32, smem, stream>>>(a);
-      break;
-    case 4:
-      err = cudaFuncSetAttribute(dispatch_bulk_kernel<4>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (err == cudaSuccess) dispatch_bulk_kernel<4><<<grid, 32, smem, stream>>>(a);
-      break;
-    case 2:
-      err = cudaFuncSetAttribute(dispatch_bulk_kernel<2>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (err == cudaSuccess) dispatch_bulk_kernel<2><<<grid, 32, smem, stream>>>(a);
-      break;
-    default:
-      err = cudaFuncSetAttribute(dispatch_bulk_kernel<1>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (err == cudaSuccess) dispatch_bulk_kernel<1><<<grid, 32, smem, stream>>>(a);
-      break;
-  }
+template <int Q>
+cudaError_t launch_bulk_q(const CopyArgs& a, int grid, size_t smem, cudaStream_t stream, bool pdl) {
+  cudaError_t err = cudaFuncSetAttribute(dispatch_bulk_kernel<Q>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  return cudaGetLastError();
+  return launch_kernel(dispatch_bulk_kernel<Q>, dim3(grid), dim3(32), smem, stream, pdl, a);
+}
+
+cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t stream, bool pdl) {
+  const size_t smem = (size_t)a.stage_bytes * a.stages;
+  switch (bulk_queue_depth(a.stages)) {
+    case 8: return launch_bulk_q<8>(a, grid, smem, stream, pdl);
+    case 4: return launch_bulk_q<4>(a, grid, smem, stream, pdl);
+    case 2: return launch_bulk_q<2>(a, grid, smem, stream, pdl);
+    default: return launch_bulk_q<1>(a, grid, smem, stream, pdl);
+  }
 }
 
 template <int U>
-cudaError_t launch_vec_u(const CopyArgs& a, int grid, bool streaming, cudaStream_t stream) {
+cudaError_t launch_vec_u(const CopyArgs& a, int grid, bool streaming, cudaStream_t stream,
+                         bool pdl) {
   bool all16 = true;
   for (int p = 0; p < a.np; ++p) all16 &= a.vec[p] == 16;
+  const dim3 g(grid), b(kVecThreads);
   if (all16) {
-    if (streaming)
-      dispatch_vec_kernel<U, true, true><<<grid, kVecThreads, 0, stream>>>(a);
-    else
-      dispatch_vec_kernel<U, true, false><<<grid, kVecThreads, 0, stream>>>(a);
-  } else {
-    if (streaming)
-      dispatch_vec_kernel<U, false, true><<<grid, kVecThreads, 0, stream>>>(a);
-    else
-      dispatch_vec_kernel<U, false, false><<<grid, kVecThreads, 0, stream>>>(a);
+    if (streaming) return launch_kernel(dispatch_vec_kernel<U, true, true>, g, b, 0, stream, pdl, a);
+    return launch_kernel(dispatch_vec_kernel<U, true, false>, g, b, 0, stream, pdl, a);
   }
-  return cudaGetLastError();
+  if (streaming) return launch_kernel(dispatch_vec_kernel<U, false, true>, g, b, 0, stream, pdl, a);
+  return launch_kernel(dispatch_vec_kernel<U, false, false>, g, b, 0, stream, pdl, a);
 }
 
 cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, int unroll, bool streaming,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, bool pdl) {
   switch (unroll) {
-    case 2: return launch_vec_u<2>(a, grid, streaming, stream);
-    case 4: return launch_vec_u<4>(a, grid, streaming, stream);
-    case 8: return launch_vec_u<8>(a, grid, streaming, stream);
+    case 2: return launch_vec_u<2>(a, grid, streaming, stream, pdl);
+    case 4: return launch_vec_u<4>(a, grid, streaming, stream, pdl);
+    case 8: return launch_vec_u<8>(a, grid, streaming, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -137,6 +137,7 @@ struct ep_a2a_handle_s {
   int vec_unroll;
   int vec_ctas_per_sm;
   int store_streaming;
+  int pdl;                // programmatic dependent launch for the path's kernels
   int copy_ctas_per_sm;
   int copy_stages;        // 0 = choose from the row size
   int combine_threads;
@@ -267,6 +268,7 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   h->vec_unroll = 4;
   h->vec_ctas_per_sm = 32;
   h->store_streaming = 1;
+  h->pdl = 1;
   h->copy_ctas_per_sm = 1;
   h->copy_stages = 4;
   h->combine_threads = 64;
@@ -322,6 +324,10 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
     case EP_A2A_OPT_STORE_STREAMING:
       if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "streaming must be 0 or 1");
       h->store_streaming = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_PDL:
+      if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "pdl must be 0 or 1");
+      h->pdl = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_BULK_MIN_ROW_BYTES:
       if (value < 0 || value > (1 << 24))
@@ -420,7 +426,8 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
   ra.eplb_n = p.eplb_stats_num_experts;
   ra.invalid_id = p.invalid_expert_id;
   int slot = prof_begin(h, EP_A2A_KERNEL_ROUTE_PLAN, stream);
-  cudaError_t e = launch_route_plan(ra, active_rank_mask != nullptr, stream);
+  const bool pdl = h->pdl != 0;
+  cudaError_t e = launch_route_plan(ra, active_rank_mask != nullptr, stream, pdl);
   prof_end(h, slot, stream);
   if (e != cudaSuccess) return cuda_fail(e, "routing-plan kernel launch");
 
@@ -483,10 +490,10 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
           (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)h->num_sms * ctas, ntok));
       if (staged) {
         slot = prof_begin(h, EP_A2A_KERNEL_COPY_STAGED, stream);
-        e = launch_dispatch_staged(bulk, h->copy_consumer_warps, grid, stream);
+        e = launch_dispatch_staged(bulk, h->copy_consumer_warps, grid, stream, pdl);
       } else {
         slot = prof_begin(h, EP_A2A_KERNEL_COPY_BULK, stream);
-        e = launch_dispatch_bulk(bulk, grid, stream);
+        e = launch_dispatch_bulk(bulk, grid, stream, pdl);
       }
       prof_end(h, slot, stream);
       if (e != cudaSuccess) return cuda_fail(e, "bulk copy kernel launch");
@@ -497,7 +504,7 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
     const int grid = (int)std::max<int64_t>(
         1, std::min<int64_t>((warps_needed + 7) / 8, (int64_t)h->num_sms * h->vec_ctas_per_sm));
     slot = prof_begin(h, EP_A2A_KERNEL_COPY_VEC, stream);
-    e = launch_dispatch_vec(vec, grid, h->vec_unroll, h->store_streaming != 0, stream);
+    e = launch_dispatch_vec(vec, grid, h->vec_unroll, h->store_streaming != 0, stream, pdl);
     prof_end(h, slot, stream);
     if (e != cudaSuccess) return cuda_fail(e, "vector copy kernel launch");
   }
@@ -543,7 +550,8 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   const int grid = (int)std::max<int64_t>(
       1, std::min<int64_t>(a.ntok, (int64_t)h->num_sms * h->combine_ctas_per_sm));
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);
-  cudaError_t e = launch_combine(a, fp8, vec, h->combine_threads, grid, (cudaStream_t)stream_v);
+  cudaError_t e = launch_combine(a, fp8, vec, h->combine_threads, grid, (cudaStream_t)stream_v,
+                                 h->pdl != 0);
   prof_end(h, slot, (cudaStream_t)stream_v);
   if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
   return EP_A2A_OK;

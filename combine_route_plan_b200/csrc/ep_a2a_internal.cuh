@@ -4,6 +4,7 @@
 
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <utility>
 
 #include "ep_a2a.h"
 
@@ -45,7 +46,8 @@ struct RouteArgs {
   uint64_t live[kMaskWords];   // bit r = rank r active
 };
 
-cudaError_t launch_route_plan(const RouteArgs& a, bool use_mask, cudaStream_t stream);
+cudaError_t launch_route_plan(const RouteArgs& a, bool use_mask, cudaStream_t stream,
+                              bool pdl = false);
 
 // ---------------------------------------------------------------------------
 // Dispatch row copy
@@ -70,12 +72,12 @@ struct CopyArgs {
   uint32_t* err;
 };
 
-cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t stream);
+cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t stream, bool pdl);
 cudaError_t launch_dispatch_staged(const CopyArgs& a, int consumer_warps, int grid,
-                                   cudaStream_t stream);
+                                   cudaStream_t stream, bool pdl);
 constexpr int kStagedMaxVec = 8;         // 16-byte vectors per consumer thread per token
 cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, int unroll, bool streaming,
-                                cudaStream_t stream);
+                                cudaStream_t stream, bool pdl);
 int bulk_queue_depth(int stages);        // groups allowed in flight for `stages`
 
 // ---------------------------------------------------------------------------
@@ -92,7 +94,7 @@ struct CombineArgs {
 };
 
 cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, int threads, int grid,
-                           cudaStream_t stream);
+                           cudaStream_t stream, bool pdl);
 cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n, cudaStream_t stream);
 cudaError_t launch_wait_timeout_probe(uint32_t* err, unsigned long long limit_ns,
                                       cudaStream_t stream);
@@ -100,10 +102,34 @@ cudaError_t launch_wait_timeout_probe(uint32_t* err, unsigned long long limit_ns
 // Message returned by ep_a2a_last_error() on the calling thread.
 void record_last_error(const char* msg);
 
+// Launch `kernel` on `stream`; with `pdl` the launch may begin while the
+// previous kernel of the stream finishes (programmatic dependent launch), and
+// the kernel itself waits for that kernel (pdl_wait) before touching memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------------------
 // PTX wrappers (sm_90+; built for sm_100a).  All forms are CTA-local.
 // ---------------------------------------------------------------------------
 #if defined(__CUDACC__)
+// Wait until the grid this one depends on (programmatic dependent launch) has
+// completed and its writes are visible; returns at once otherwise.  Every
+// kernel of the path calls it before its first global memory access.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -67,6 +67,7 @@ __device__ void eplb_gather(const RouteArgs& a) {
 
 template <int G, bool kMask>
 __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteArgs a) {
+  pdl_wait();
   const int r = blockIdx.y;
   if (r == a.ep) {  // the extra row of blocks gathers EPLB statistics
     eplb_gather<kMask>(a);
@@ -158,17 +159,15 @@ __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteAr
 }
 
 template <int G>
-cudaError_t launch_g(const RouteArgs& a, bool use_mask, dim3 grid, cudaStream_t stream) {
+cudaError_t launch_g(const RouteArgs& a, bool use_mask, dim3 grid, cudaStream_t stream, bool pdl) {
   if (use_mask)
-    route_plan_kernel<G, true><<<grid, kRouteThreads, 0, stream>>>(a);
-  else
-    route_plan_kernel<G, false><<<grid, kRouteThreads, 0, stream>>>(a);
-  return cudaGetLastError();
+    return launch_kernel(route_plan_kernel<G, true>, grid, dim3(kRouteThreads), 0, stream, pdl, a);
+  return launch_kernel(route_plan_kernel<G, false>, grid, dim3(kRouteThreads), 0, stream, pdl, a);
 }
 
 }  // namespace
 
-cudaError_t launch_route_plan(const RouteArgs& a, bool use_mask, cudaStream_t stream) {
+cudaError_t launch_route_plan(const RouteArgs& a, bool use_mask, cudaStream_t stream, bool pdl) {
   const int tok_blocks = (a.tpr + kTokPerBlock - 1) / kTokPerBlock;
   int gx = tok_blocks > 0 ? tok_blocks : 1;
   int gy = a.ep;
@@ -182,12 +181,12 @@ cudaError_t launch_route_plan(const RouteArgs& a, bool use_mask, cudaStream_t st
   int G = 1;
   while (G < a.k) G <<= 1;
   switch (G) {
-    case 1: return launch_g<1>(a, use_mask, grid, stream);
-    case 2: return launch_g<2>(a, use_mask, grid, stream);
-    case 4: return launch_g<4>(a, use_mask, grid, stream);
-    case 8: return launch_g<8>(a, use_mask, grid, stream);
-    case 16: return launch_g<16>(a, use_mask, grid, stream);
-    case 32: return launch_g<32>(a, use_mask, grid, stream);
+    case 1: return launch_g<1>(a, use_mask, grid, stream, pdl);
+    case 2: return launch_g<2>(a, use_mask, grid, stream, pdl);
+    case 4: return launch_g<4>(a, use_mask, grid, stream, pdl);
+    case 8: return launch_g<8>(a, use_mask, grid, stream, pdl);
+    case 16: return launch_g<16>(a, use_mask, grid, stream, pdl);
+    case 32: return launch_g<32>(a, use_mask, grid, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -235,8 +235,13 @@ typedef enum {
                                      (default); 0 = each CTA copies a contiguous chunk */
   EP_A2A_OPT_VEC_UNROLL = 8,      /* vector copy: vectors per lane in flight (2, 4 = default, 8) */
   EP_A2A_OPT_VEC_CTAS_PER_SM = 9, /* vector copy grid = SMs x this (1..64; default 32) */
-  EP_A2A_OPT_STORE_STREAMING = 10 /* vector copy: 1 = evict-first (.cs) 16-byte stores
+  EP_A2A_OPT_STORE_STREAMING = 10,/* vector copy: 1 = evict-first (.cs) 16-byte stores
                                      (default), 0 = plain stores */
+  EP_A2A_OPT_PDL = 11             /* 1 (default): launch the routing, copy and combine
+                                     kernels with programmatic dependent launch
+                                     (flashinfer.moe_ep.NVLinkOneSidedConfig, enable_pdl);
+                                     each kernel waits for the previous one before it
+                                     touches memory, so results do not change */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

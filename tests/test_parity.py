@@ -101,6 +101,53 @@ def test_staged_copy_row_sizes(rows):
     U.check_payloads(run, plan, w, x)
 
 
+@pytest.mark.parametrize("name", ["c2_ep8_decode", "c5_ep64_wide_masked"])
+def test_without_programmatic_dependent_launch(name):
+    from combine_route_plan_b200 import ep_a2a
+    _full_check(W.BY_NAME[name], options={ep_a2a.OPT_PDL: 0})
+
+
+def test_cuda_graph_capture_and_replay():
+    """Dispatch + combine captured into a CUDA graph give the oracle's result on
+    every replay (new inputs are copied into the captured buffers between replays)."""
+    from combine_route_plan_b200 import ep_a2a
+    w = W.C2
+    x = _inputs(w.name)
+    comm = ep_a2a.EpA2A(w.ep_size, w.num_experts, w.top_k, w.tokens_per_rank, w.hidden,
+                        w.payload_row_bytes(), workspace_fill=U.CANARY)
+    ids = x.token_selected_experts.cuda()
+    pays = [p.cuda() for p in x.payloads]
+    xo = x.expert_output.cuda()
+    out = torch.empty((w.ep_size, w.tokens_per_rank, w.hidden), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        comm.dispatch(ids, x.local_num_tokens, pays, w.tokens_per_rank, views=False)
+        comm.combine(xo, out)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    plan = U.oracle_plan(w, x)
+    for _ in range(2):
+        out.fill_(0)
+        g.replay()
+        torch.cuda.synchronize()
+        U.check_combine(type("R", (), {"out": out})(), plan, w, x)
+    # new routing and rows through the same captured pointers
+    ids.copy_(torch.roll(x.token_selected_experts, 1, dims=1).cuda())
+    x3 = W.Inputs(w, torch.roll(x.token_selected_experts, 1, dims=1), x.local_num_tokens,
+                  x.payloads, None, None, x.expert_output)
+    g.replay()
+    torch.cuda.synchronize()
+    U.check_combine(type("R", (), {"out": out})(), U.oracle_plan(w, x3), w, x3)
+    assert comm.get_status() == ep_a2a.OK
+
+
 @pytest.mark.parametrize("threads,ctas", [(64, 0), (96, 3), (256, 64), (512, 1), (128, 1024)])
 def test_combine_launch_shape_does_not_change_results(threads, ctas):
     from combine_route_plan_b200 import ep_a2a
