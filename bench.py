@@ -379,10 +379,14 @@ def run_ours(args):
             ms = run_timed(timed_step, args.steps, args.warmup, CudaTimer(stream), dist, device,
                            during=clocks)
     else:
+        # the headline: K steps with nothing recorded between the kernels (an
+        # event between two kernels would stop them from overlapping)
         ms = run_timed(step, args.steps, args.warmup, CudaTimer(stream), dist, device,
-                       during=clocks,
-                       on_start=lambda: ep_a2a.ep_a2a_profile_start(comm.handle,
-                                                                    4 * args.steps + 8))
+                       during=clocks)
+        # per-kernel durations: a second timed region of K steps, each kernel
+        # bracketed by CUDA events on its launch stream
+        run_timed(step, args.steps, 0, CudaTimer(stream), dist, device,
+                  on_start=lambda: ep_a2a.ep_a2a_profile_start(comm.handle, 4 * args.steps + 8))
         kt = ep_a2a.ep_a2a_profile_stop(comm.handle)
     torch.cuda.synchronize()
     assert comm.get_status() == ep_a2a.OK
@@ -442,6 +446,8 @@ def run_ours(args):
                        if args.l2_flush else "inputs larger than L2 (no flush)"),
                 "launch": ("CUDA graph replay" if args.graph else "eager") +
                           (", programmatic dependent launch" if not args.no_pdl else ""),
+                "kernel_times": "CUDA events around each launch, in a second timed region of "
+                                "the same K steps (events between kernels stop them overlapping)",
                 "parallelism": f"{ws} independent replicas" if ws > 1 else "1 GPU, virtual ranks",
             },
             "hbm": {"step_algorithmic_bytes": by.step, "achieved_gbs": step_gbs,

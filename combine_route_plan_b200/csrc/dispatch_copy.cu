@@ -24,9 +24,9 @@
 //     Loads run `L = stages - Q` tokens ahead of the stores, and at most Q
 //     tokens' store groups are still reading shared memory when a stage is
 //     refilled.  The copy engine generates the addresses; the SM only issues.
-//   * dispatch_vec_kernel — any row size and alignment.  One warp per token:
-//     lanes load the row in the widest aligned vectors into registers once and
-//     store them to each destination.
+//   * dispatch_vec_kernel (default) — any row size and alignment.  A group of
+//     32..256 threads per token loads the row in the widest aligned vectors
+//     into registers once and stores them to each destination.
 // Both read the plan (plan_nd / plan_dst) the routing kernel wrote just before.
 #include "ep_a2a_internal.cuh"
 
@@ -242,18 +242,20 @@ __device__ __forceinline__ void store_dst<uint4>(uint4* p, const uint4& v, bool 
     *p = v;
 }
 
-template <typename T, int U>
+// Copy one payload row of a token to its nd destinations: the TPT threads of a
+// token group each take vectors gl, gl + TPT, ... (U of them in flight).
+template <typename T, int U, int TPT>
 __device__ __forceinline__ void copy_row(const uint8_t* __restrict__ src, int64_t rb,
                                          uint8_t* rank0, int64_t rank_stride, int64_t off,
                                          uint64_t w0, uint64_t w1, uint64_t w2, uint64_t w3,
-                                         int nd, int lane, bool streaming) {
+                                         int nd, int gl, bool streaming) {
   const int64_t n = rb / (int64_t)sizeof(T);
   const T* s = reinterpret_cast<const T*>(src);
-  for (int64_t i0 = lane; i0 < n; i0 += 32 * U) {
+  for (int64_t i0 = gl; i0 < n; i0 += TPT * U) {
     T v[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int64_t i = i0 + (int64_t)u * 32;
+      const int64_t i = i0 + (int64_t)u * TPT;
       if (i < n) v[u] = load_src<T>(s + i);
     }
     for (int q = 0; q < nd; ++q) {
@@ -261,7 +263,7 @@ __device__ __forceinline__ void copy_row(const uint8_t* __restrict__ src, int64_
                                   off);
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const int64_t i = i0 + (int64_t)u * 32;
+        const int64_t i = i0 + (int64_t)u * TPT;
         if (i < n) store_dst<T>(d + i, v[u], streaming);
       }
     }
@@ -270,55 +272,96 @@ __device__ __forceinline__ void copy_row(const uint8_t* __restrict__ src, int64_
 
 constexpr int kVecThreads = 256;
 
-// kAll16: every payload of the launch moves in 16-byte vectors (one code path,
-// fewer registers); otherwise each payload picks its own vector width.
-template <int U, bool kAll16, bool kStreaming>
+// Destinations of token `tok` (all lanes of the warp call it together): lanes
+// j < k look at expert slot j, the owners are de-duplicated with a warp match,
+// and the distinct live owners are packed as bytes into w0..w3.  The same rule
+// as the routing kernel (owner = e / epr for e in [0, E), live ranks only);
+// returns the number of destinations, or 0 for a token that does not exist.
+__device__ __forceinline__ int token_destinations(const CopyArgs& a, int64_t tok, int lane,
+                                                  uint64_t& w0, uint64_t& w1, uint64_t& w2,
+                                                  uint64_t& w3) {
+  const int r = (int)(tok / a.tpr);
+  const int t = (int)(tok - (int64_t)r * a.tpr);
+  w0 = w1 = w2 = w3 = 0;
+  if (t >= a.n[r]) return 0;              // n[r] is 0 for masked-off ranks
+  int d = -1;
+  if (lane < a.k) {
+    const int32_t e = a.ids[tok * a.k + lane];
+    if (e >= 0 && e < a.E) {
+      const int owner = e / a.epr;
+      if (!a.use_mask || ((a.live[owner >> 6] >> (owner & 63)) & 1ull)) d = owner;
+    }
+  }
+  const unsigned peers = __match_any_sync(kFull, d);
+  const bool leader = d >= 0 && (__ffs(peers) - 1) == lane;
+  unsigned leaders = __ballot_sync(kFull, leader);
+  int nd = 0;
+  while (leaders) {
+    const int l = __ffs(leaders) - 1;
+    leaders &= leaders - 1u;
+    const uint64_t dd = (uint64_t)(__shfl_sync(kFull, d, l) & 0xFF);
+    const int sh = (nd & 7) * 8;
+    if (nd < 8) w0 |= dd << sh;
+    else if (nd < 16) w1 |= dd << sh;
+    else if (nd < 24) w2 |= dd << sh;
+    else w3 |= dd << sh;
+    ++nd;
+  }
+  return nd;
+}
+
+// TPT threads per token (a warp for many tokens, up to the whole CTA for few,
+// so that short steps still fill the GPU).  Each warp finds its token's
+// destinations from the routing ids itself, so the kernel does not depend on
+// the routing kernel's plan and may run alongside it (programmatic dependent
+// launch); it waits for the preceding grid only before it exits, so that work
+// after it sees the plan complete.  kAll16: every payload of the launch moves
+// in 16-byte vectors (one code path, fewer registers); otherwise each payload
+// picks its own vector width.
+template <int U, bool kAll16, bool kStreaming, int TPT>
 __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArgs a) {
-  pdl_wait();
+  constexpr int kGroups = kVecThreads / TPT;
+  const int gl = threadIdx.x % TPT;
+  const int group = threadIdx.x / TPT;
   const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int words = a.plan_stride / 8;
-  for (int64_t tok = (int64_t)blockIdx.x * (kVecThreads / 32) + warp; tok < a.ntok;
-       tok += (int64_t)gridDim.x * (kVecThreads / 32)) {
-    const int nd = a.plan_nd[tok];
-    if (nd == kNoToken || nd == 0) continue;
-    const uint64_t* row = reinterpret_cast<const uint64_t*>(a.plan_dst + tok * words * 8);
-    const uint64_t w0 = row[0];
-    const uint64_t w1 = words > 1 ? row[1] : 0;
-    const uint64_t w2 = words > 2 ? row[2] : 0;
-    const uint64_t w3 = words > 3 ? row[3] : 0;
+  for (int64_t tok = (int64_t)blockIdx.x * kGroups + group; tok < a.ntok;
+       tok += (int64_t)gridDim.x * kGroups) {
+    uint64_t w0, w1, w2, w3;
+    const int nd = token_destinations(a, tok, lane, w0, w1, w2, w3);
+    if (nd == 0) continue;
     for (int p = 0; p < a.np; ++p) {
       const uint8_t* src = a.src[p] + tok * a.rb[p];
       const int64_t off = a.dst_off[p] + tok * a.rb[p];
       if (kAll16) {
-        copy_row<uint4, U>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd, lane,
-                           kStreaming);
+        copy_row<uint4, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
+                                gl, kStreaming);
         continue;
       }
       switch (a.vec[p]) {
         case 16:
-          copy_row<uint4, U>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd, lane,
-                             kStreaming);
+          copy_row<uint4, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
+                                  gl, kStreaming);
           break;
         case 8:
-          copy_row<uint2, U>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd, lane,
-                             false);
+          copy_row<uint2, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
+                                  gl, false);
           break;
         case 4:
-          copy_row<uint32_t, U>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
-                                lane, false);
+          copy_row<uint32_t, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3,
+                                     nd, gl, false);
           break;
         case 2:
-          copy_row<uint16_t, U>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
-                                lane, false);
+          copy_row<uint16_t, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3,
+                                     nd, gl, false);
           break;
         default:
-          copy_row<uint8_t, U>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
-                               lane, false);
+          copy_row<uint8_t, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3,
+                                    nd, gl, false);
           break;
       }
     }
   }
+  pdl_wait();
 }
 
 template <int NCW, int MAXV>
@@ -505,26 +548,40 @@ cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t strea
   }
 }
 
-template <int U>
-cudaError_t launch_vec_u(const CopyArgs& a, int grid, bool streaming, cudaStream_t stream,
-                         bool pdl) {
+template <int U, int TPT>
+cudaError_t launch_vec_ut(const CopyArgs& a, int grid, bool streaming, cudaStream_t stream,
+                          bool pdl) {
   bool all16 = true;
   for (int p = 0; p < a.np; ++p) all16 &= a.vec[p] == 16;
   const dim3 g(grid), b(kVecThreads);
   if (all16) {
-    if (streaming) return launch_kernel(dispatch_vec_kernel<U, true, true>, g, b, 0, stream, pdl, a);
-    return launch_kernel(dispatch_vec_kernel<U, true, false>, g, b, 0, stream, pdl, a);
+    if (streaming)
+      return launch_kernel(dispatch_vec_kernel<U, true, true, TPT>, g, b, 0, stream, pdl, a);
+    return launch_kernel(dispatch_vec_kernel<U, true, false, TPT>, g, b, 0, stream, pdl, a);
   }
-  if (streaming) return launch_kernel(dispatch_vec_kernel<U, false, true>, g, b, 0, stream, pdl, a);
-  return launch_kernel(dispatch_vec_kernel<U, false, false>, g, b, 0, stream, pdl, a);
+  if (streaming)
+    return launch_kernel(dispatch_vec_kernel<U, false, true, TPT>, g, b, 0, stream, pdl, a);
+  return launch_kernel(dispatch_vec_kernel<U, false, false, TPT>, g, b, 0, stream, pdl, a);
 }
 
-cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, int unroll, bool streaming,
-                                cudaStream_t stream, bool pdl) {
+template <int U>
+cudaError_t launch_vec_u(const CopyArgs& a, int grid, int tpt, bool streaming,
+                         cudaStream_t stream, bool pdl) {
+  switch (tpt) {
+    case 32: return launch_vec_ut<U, 32>(a, grid, streaming, stream, pdl);
+    case 64: return launch_vec_ut<U, 64>(a, grid, streaming, stream, pdl);
+    case 128: return launch_vec_ut<U, 128>(a, grid, streaming, stream, pdl);
+    case 256: return launch_vec_ut<U, 256>(a, grid, streaming, stream, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, int unroll, int threads_per_token,
+                                bool streaming, cudaStream_t stream, bool pdl) {
   switch (unroll) {
-    case 2: return launch_vec_u<2>(a, grid, streaming, stream, pdl);
-    case 4: return launch_vec_u<4>(a, grid, streaming, stream, pdl);
-    case 8: return launch_vec_u<8>(a, grid, streaming, stream, pdl);
+    case 2: return launch_vec_u<2>(a, grid, threads_per_token, streaming, stream, pdl);
+    case 4: return launch_vec_u<4>(a, grid, threads_per_token, streaming, stream, pdl);
+    case 8: return launch_vec_u<8>(a, grid, threads_per_token, streaming, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

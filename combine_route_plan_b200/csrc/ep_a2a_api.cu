@@ -138,6 +138,7 @@ struct ep_a2a_handle_s {
   int vec_ctas_per_sm;
   int store_streaming;
   int pdl;                // programmatic dependent launch for the path's kernels
+  int vec_threads_per_token;  // 0 = from the token count
   int copy_ctas_per_sm;
   int copy_stages;        // 0 = choose from the row size
   int combine_threads;
@@ -177,6 +178,12 @@ void prof_free(ep_a2a_handle h) {
   h->prof_kernel.clear();
   h->profiling = false;
 }
+
+// Threads per token of the vector copy.  Measured on the workloads: with
+// 8192 or more token slots a warp per token is fastest (enough tokens to fill
+// the GPU; 32 beat 64-256 by 2-30 %), below that a whole 256-thread CTA per
+// token is (fewer tokens, each spread over more threads).
+int copy_threads_per_token(int64_t tokens) { return tokens >= 8192 ? 32 : 256; }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -269,9 +276,10 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   h->vec_ctas_per_sm = 32;
   h->store_streaming = 1;
   h->pdl = 1;
+  h->vec_threads_per_token = 0;
   h->copy_ctas_per_sm = 1;
   h->copy_stages = 4;
-  h->combine_threads = 64;
+  h->combine_threads = 0;
   h->bulk_min_row = 0;
   h->combine_ctas_per_sm = 128;
   h->profiling = false;
@@ -298,8 +306,9 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       h->copy_stages = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_COMBINE_THREADS:
-      if (value < 64 || value > 512 || value % 32 != 0)
-        return fail(EP_A2A_ERR_INVALID_ARG, "combine threads must be a multiple of 32 in 64..512");
+      if (value != 0 && (value < 64 || value > 512 || value % 32 != 0))
+        return fail(EP_A2A_ERR_INVALID_ARG,
+                    "combine threads must be 0 (automatic) or a multiple of 32 in 64..512");
       h->combine_threads = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_COPY_CONSUMER_WARPS:
@@ -324,6 +333,11 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
     case EP_A2A_OPT_STORE_STREAMING:
       if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "streaming must be 0 or 1");
       h->store_streaming = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_VEC_THREADS_PER_TOKEN:
+      if (value != 0 && value != 32 && value != 64 && value != 128 && value != 256)
+        return fail(EP_A2A_ERR_INVALID_ARG, "threads per token must be 0, 32, 64, 128 or 256");
+      h->vec_threads_per_token = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_PDL:
       if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "pdl must be 0 or 1");
@@ -442,6 +456,14 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
   bulk.plan_stride = L.plan_stride;
   bulk.err = reinterpret_cast<uint32_t*>(ws + L.off_err);
   bulk.interleave = h->copy_interleave;
+  bulk.ids = token_selected_experts;
+  bulk.E = p.num_experts;
+  bulk.k = p.top_k;
+  bulk.epr = p.num_experts / ep;
+  bulk.tpr = tpr;
+  bulk.use_mask = active_rank_mask != nullptr;
+  std::memcpy(bulk.n, ra.n, sizeof(bulk.n));
+  std::memcpy(bulk.live, ra.live, sizeof(bulk.live));
   vec = bulk;
   uint32_t stage = 0;
   for (int i = 0; i < num_payloads; ++i) {
@@ -500,11 +522,14 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
     }
   }
   if (vec.np > 0) {
-    const int64_t warps_needed = ntok;
+    const int tpt = h->vec_threads_per_token > 0 ? h->vec_threads_per_token
+                                                 : copy_threads_per_token(ntok);
+    const int64_t groups_per_cta = 256 / tpt;
     const int grid = (int)std::max<int64_t>(
-        1, std::min<int64_t>((warps_needed + 7) / 8, (int64_t)h->num_sms * h->vec_ctas_per_sm));
+        1, std::min<int64_t>((ntok + groups_per_cta - 1) / groups_per_cta,
+                             (int64_t)h->num_sms * h->vec_ctas_per_sm));
     slot = prof_begin(h, EP_A2A_KERNEL_COPY_VEC, stream);
-    e = launch_dispatch_vec(vec, grid, h->vec_unroll, h->store_streaming != 0, stream, pdl);
+    e = launch_dispatch_vec(vec, grid, h->vec_unroll, tpt, h->store_streaming != 0, stream, pdl);
     prof_end(h, slot, stream);
     if (e != cudaSuccess) return cuda_fail(e, "vector copy kernel launch");
   }
@@ -549,8 +574,11 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   const bool vec = a.H % elems == 0 && aligned(expert_output, 16) && aligned(output, 16);
   const int grid = (int)std::max<int64_t>(
       1, std::min<int64_t>(a.ntok, (int64_t)h->num_sms * h->combine_ctas_per_sm));
+  // 64-thread CTAs measured best for every token count (16-1024 CTAs per SM,
+  // 64-512 threads swept on the decode, wide-EP and prefill workloads)
+  const int threads = h->combine_threads > 0 ? h->combine_threads : 64;
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);
-  cudaError_t e = launch_combine(a, fp8, vec, h->combine_threads, grid, (cudaStream_t)stream_v,
+  cudaError_t e = launch_combine(a, fp8, vec, threads, grid, (cudaStream_t)stream_v,
                                  h->pdl != 0);
   prof_end(h, slot, (cudaStream_t)stream_v);
   if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");

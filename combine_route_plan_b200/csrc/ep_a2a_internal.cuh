@@ -70,14 +70,20 @@ struct CopyArgs {
   int stages;                            // bulk path
   int interleave;                        // bulk paths: 1 = CTA b takes tokens b, b+grid, ...
   uint32_t* err;
+  // vector path: the routing inputs, so that it finds each token's
+  // destinations itself instead of reading the plan
+  const int32_t* ids;                    // [ep, tpr, k]
+  int E, k, epr, tpr, use_mask;
+  int32_t n[kMaxRanks];                  // local_num_tokens (0 for masked-off ranks)
+  uint64_t live[kMaskWords];
 };
 
 cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t stream, bool pdl);
 cudaError_t launch_dispatch_staged(const CopyArgs& a, int consumer_warps, int grid,
                                    cudaStream_t stream, bool pdl);
 constexpr int kStagedMaxVec = 8;         // 16-byte vectors per consumer thread per token
-cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, int unroll, bool streaming,
-                                cudaStream_t stream, bool pdl);
+cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, int unroll, int threads_per_token,
+                                bool streaming, cudaStream_t stream, bool pdl);
 int bulk_queue_depth(int stages);        // groups allowed in flight for `stages`
 
 // ---------------------------------------------------------------------------
@@ -129,6 +135,13 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
 // completed and its writes are visible; returns at once otherwise.  Every
 // kernel of the path calls it before its first global memory access.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next kernel of the stream (if launched with programmatic
+// dependent launch) to start; it still waits for this grid with pdl_wait
+// before it reads anything this grid writes.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -68,6 +68,10 @@ __device__ void eplb_gather(const RouteArgs& a) {
 template <int G, bool kMask>
 __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteArgs a) {
   pdl_wait();
+  // The vector copy that follows routes its tokens itself and does not read
+  // what this kernel writes, so it may run alongside; the combine after it
+  // still waits for this grid (through the copy's final wait).
+  pdl_launch_dependents();
   const int r = blockIdx.y;
   if (r == a.ep) {  // the extra row of blocks gathers EPLB statistics
     eplb_gather<kMask>(a);
@@ -90,20 +94,29 @@ __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteAr
   const int t_begin = blockIdx.x * kTokPerBlock;
   const int t_end = min(a.tpr, t_begin + kTokPerBlock);
 
-  for (int t0 = t_begin; t0 < t_end; t0 += kRouteWarps * kTokPerWarp) {
-    const int t = t0 + warp * kTokPerWarp + g;
-    const bool in_range = t < t_end;
-    const bool exists = in_range && t < n_r;
-    const int64_t s = (int64_t)r * a.tpr + t;
-    int32_t e = 0;
-    int d = -1;
+  // Expert slot j of token t: its global id e and owning live rank d (-1 if none).
+  auto owner_of = [&](int t, int32_t& e, int& d, bool& in_range, bool& exists) {
+    in_range = t < t_end;
+    exists = in_range && t < n_r;
+    e = 0;
+    d = -1;
     if (exists && j < a.k) {
-      e = a.ids[s * a.k + j];
+      e = a.ids[((int64_t)r * a.tpr + t) * a.k + j];
       if (e >= 0 && e < a.E) {
         const int owner = e / a.epr;
         if (rank_live<kMask>(a.live, owner)) d = owner;
       }
     }
+  };
+
+  // Pass 1: the plan (this rank's tokens) and the per-block send counts.
+  for (int t0 = t_begin; t0 < t_end; t0 += kRouteWarps * kTokPerWarp) {
+    const int t = t0 + warp * kTokPerWarp + g;
+    int32_t e;
+    int d;
+    bool in_range, exists;
+    owner_of(t, e, d, in_range, exists);
+    const int64_t s = (int64_t)r * a.tpr + t;
     // de-duplicate owners within the token
     const unsigned key = ((unsigned)g << 9) | ((unsigned)d & 0x1FFu);
     const unsigned peers = __match_any_sync(kFull, key);
@@ -126,26 +139,20 @@ __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteAr
       for (int c = j; c < a.plan_stride; c += G)
         if (c >= nd) row[c] = kPad;
     }
-    // receive-side rows of slot s in every live destination
-    for (int dd = 0; dd < a.ep; ++dd) {
-      const bool got = (__ballot_sync(kFull, d == dd) & gmask) != 0u;
-      if (!in_range || !rank_live<kMask>(a.live, dd)) continue;
-      uint8_t* base = a.rank0 + dd * a.rank_stride;
-      if (j < a.k)
-        reinterpret_cast<int32_t*>(base + a.off_ids)[s * a.k + j] = got ? e : a.invalid_id;
-      if (j == 0) base[a.off_valid + s] = got ? 1 : 0;
-    }
   }
 
-  // send_counts[r][:] = sum over this rank's blocks
+  // send_counts[r][:] = sum over this rank's blocks.  The block's totals go to
+  // the accumulators; the last block to take a ticket writes the row and
+  // resets the scratch.  Only plan writes precede the fence, so the ticket
+  // chain stays short; the receive rows are written afterwards.
   __syncthreads();
   for (int i = threadIdx.x; i < a.ep; i += kRouteThreads) {
     const int v = s_cnt[i];
     if (v) atomicAdd(&a.count_acc[r * a.ep + i], v);
   }
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
+    __threadfence();
     const unsigned prev = atomicAdd(&a.count_ticket[r], 1u);
     s_last = (prev == gridDim.x - 1);
   }
@@ -155,6 +162,24 @@ __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteAr
     for (int i = threadIdx.x; i < a.ep; i += kRouteThreads)
       a.send_counts[r * a.ep + i] = atomicExch(&a.count_acc[r * a.ep + i], 0);
     if (threadIdx.x == 0) atomicExch(&a.count_ticket[r], 0u);
+  }
+
+  // Pass 2: receive-side rows of every slot in every live destination.
+  for (int t0 = t_begin; t0 < t_end; t0 += kRouteWarps * kTokPerWarp) {
+    const int t = t0 + warp * kTokPerWarp + g;
+    int32_t e;
+    int d;
+    bool in_range, exists;
+    owner_of(t, e, d, in_range, exists);
+    const int64_t s = (int64_t)r * a.tpr + t;
+    for (int dd = 0; dd < a.ep; ++dd) {
+      const bool got = (__ballot_sync(kFull, d == dd) & gmask) != 0u;
+      if (!in_range || !rank_live<kMask>(a.live, dd)) continue;
+      uint8_t* base = a.rank0 + dd * a.rank_stride;
+      if (j < a.k)
+        reinterpret_cast<int32_t*>(base + a.off_ids)[s * a.k + j] = got ? e : a.invalid_id;
+      if (j == 0) base[a.off_valid + s] = got ? 1 : 0;
+    }
   }
 }
 

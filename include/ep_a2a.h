@@ -225,8 +225,8 @@ typedef enum {
   EP_A2A_OPT_COPY_CTAS_PER_SM = 1,/* CTAs per SM of the bulk copy kernel (1..8) */
   EP_A2A_OPT_COPY_STAGES = 2,     /* shared-memory row stages per copy CTA (2..32; 0 = as
                                      many as fit, up to 8 / 16) */
-  EP_A2A_OPT_COMBINE_THREADS = 3, /* threads per CTA of the combine kernel (64..512;
-                                     default 64) */
+  EP_A2A_OPT_COMBINE_THREADS = 3, /* threads per CTA of the combine kernel (64..512);
+                                     0 (default) = 64 */
   EP_A2A_OPT_BULK_MIN_ROW_BYTES = 4, /* rows shorter than this take the vector copy (0..2^24) */
   EP_A2A_OPT_COMBINE_CTAS_PER_SM = 5, /* combine grid = min(tokens, SMs x this) (1..1024);
                                        0 = 128 */
@@ -237,11 +237,13 @@ typedef enum {
   EP_A2A_OPT_VEC_CTAS_PER_SM = 9, /* vector copy grid = SMs x this (1..64; default 32) */
   EP_A2A_OPT_STORE_STREAMING = 10,/* vector copy: 1 = evict-first (.cs) 16-byte stores
                                      (default), 0 = plain stores */
-  EP_A2A_OPT_PDL = 11             /* 1 (default): launch the routing, copy and combine
+  EP_A2A_OPT_PDL = 11,            /* 1 (default): launch the routing, copy and combine
                                      kernels with programmatic dependent launch
                                      (flashinfer.moe_ep.NVLinkOneSidedConfig, enable_pdl);
                                      each kernel waits for the previous one before it
                                      touches memory, so results do not change */
+  EP_A2A_OPT_VEC_THREADS_PER_TOKEN = 12 /* vector copy: threads per token (32, 64, 128,
+                                     256); 0 (default) = from the token count */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

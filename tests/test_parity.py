@@ -77,16 +77,18 @@ def test_copy_tuning_does_not_change_results(path, stages, ctas, cw, inter):
     U.check_payloads(run, plan, w, x)
 
 
-@pytest.mark.parametrize("unroll,ctas,streaming,rows", [
-    (2, 1, 0, [14336, 32]), (4, 8, 1, [14336, 64, 32]), (8, 64, 0, [14336, 32]),
-    (8, 3, 1, [100, 13, 16]), (2, 16, 1, [7, 4096 + 8]),
+@pytest.mark.parametrize("unroll,ctas,streaming,tpt,rows", [
+    (2, 1, 0, 32, [14336, 32]), (4, 8, 1, 64, [14336, 64, 32]), (8, 64, 0, 128, [14336, 32]),
+    (8, 3, 1, 256, [100, 13, 16]), (2, 16, 1, 0, [7, 4096 + 8]), (4, 32, 1, 256, [14336, 32]),
+    (4, 2, 0, 128, [1, 2, 4, 8, 16]),
 ])
-def test_vector_copy_variants(unroll, ctas, streaming, rows):
+def test_vector_copy_variants(unroll, ctas, streaming, tpt, rows):
     from combine_route_plan_b200 import ep_a2a
     w, x = _custom(8, 64, 8, 50, 32, rows, seed=unroll * 31 + ctas)
     run = U.Run(w, x, copy_path=1, options={ep_a2a.OPT_VEC_UNROLL: unroll,
                                             ep_a2a.OPT_VEC_CTAS_PER_SM: ctas,
-                                            ep_a2a.OPT_STORE_STREAMING: streaming})
+                                            ep_a2a.OPT_STORE_STREAMING: streaming,
+                                            ep_a2a.OPT_VEC_THREADS_PER_TOKEN: tpt})
     plan = U.oracle_plan(w, x)
     U.check_payloads(run, plan, w, x)
 
@@ -148,7 +150,8 @@ def test_cuda_graph_capture_and_replay():
     assert comm.get_status() == ep_a2a.OK
 
 
-@pytest.mark.parametrize("threads,ctas", [(64, 0), (96, 3), (256, 64), (512, 1), (128, 1024)])
+@pytest.mark.parametrize("threads,ctas", [(64, 0), (96, 3), (256, 64), (512, 1), (128, 1024),
+                                          (0, 0)])
 def test_combine_launch_shape_does_not_change_results(threads, ctas):
     from combine_route_plan_b200 import ep_a2a
     w = W.C2
