@@ -33,6 +33,9 @@
  *          past a source's token count keep expert id num_experts.
  *   [OSCu] flashinfer.moe_ep.NVLinkOneSidedConfig, `use_low_precision_combine`:
  *          combine payloads travel as FP8.
+ *   [TSCi] flashinfer.moe_ep.NVLinkTwoSidedAlltoAll, combine(): its input rows
+ *          are "already weighted and reduced over this rank's local experts";
+ *          oracle_expert_reduce states that step.
  *
  * Readings where the pages are silent (each is one deliberate choice):
  *   - expert e is owned by rank e / (E / ep_size) (contiguous blocks);
@@ -43,7 +46,12 @@
  *     clear neither sends nor receives; its receive arrays are left untouched;
  *   - the combine sum is an fp32 accumulator starting at +0.0f, adding the rows
  *     in ascending destination-rank order, rounded once to bf16 (nearest-even);
- *   - the FP8 combine format is E4M3 ("fn": no infinities, max 448), unscaled.
+ *   - the FP8 combine format is E4M3 ("fn": no infinities, max 448), unscaled;
+ *   - expert outputs before that reduction are one BF16 row per (source token,
+ *     top_k slot), [ep, tpr, k, hidden]; rank d's combine row for the token is
+ *     bf16(sum over the slots j whose expert d owns, ascending j, of
+ *     w_j * y_j), each term added with one fused multiply-add (fmaf) to an fp32
+ *     accumulator that starts at +0.0f.
  */
 #include <math.h>
 #include <stdint.h>
@@ -316,6 +324,51 @@ void oracle_combine(int ep_size, int top_k, int tokens_per_rank, int hidden,
                 acc = acc + x;
             }
             out[s * hidden + h] = oracle_bf16_from_f32(acc);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Weighted reduction over each rank's local experts (the combine's input).  */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * For a token (r, t) that exists and every rank d in its destination set,
+ * rank d's combine row [TSCi] is
+ *   z[d][r*tpr + t][h] = bf16( sum over j ascending with owner(ids[j]) == d of
+ *                              w[r][t][j] * y[r][t][j][h] )
+ * where the sum is an fp32 accumulator starting at +0.0f and each term is one
+ * fmaf (product and add rounded once).  Slots whose expert is owned by no rank
+ * or by a masked-off rank are not in any destination's sum.  Rows of z that no
+ * token fills are left as they were.  Feeding z to oracle_combine gives the
+ * combine of the per-expert outputs.
+ */
+void oracle_expert_reduce(int ep_size, int num_experts, int top_k, int tokens_per_rank,
+                          int hidden, const int32_t* num_dst, const int32_t* dst_ranks,
+                          const int32_t* token_selected_experts, /* [ep, tpr, k] */
+                          const float* topk_weights,             /* [ep, tpr, k] */
+                          const uint16_t* expert_out,            /* [ep, tpr, k, hidden] */
+                          uint16_t* z)                           /* [ep, ep*tpr, hidden] */
+{
+    const int ep = ep_size, k = top_k, tpr = tokens_per_rank;
+    const int experts_per_rank = num_experts / ep;
+    const int64_t slots = (int64_t)ep * tpr;
+    for (int64_t s = 0; s < slots; ++s) {
+        const int nd = num_dst[s];
+        const int32_t* ids = token_selected_experts + s * k;
+        const float* w = topk_weights + s * k;
+        for (int i = 0; i < nd; ++i) {
+            const int d = dst_ranks[s * k + i];
+            for (int h = 0; h < hidden; ++h) {
+                float acc = 0.0f;
+                for (int j = 0; j < k; ++j) {
+                    const int32_t e = ids[j];
+                    if (e < 0 || e >= num_experts || e / experts_per_rank != d) continue;
+                    const float y = oracle_bf16_to_f32(expert_out[(s * k + j) * hidden + h]);
+                    acc = fmaf(w[j], y, acc);
+                }
+                z[((int64_t)d * slots + s) * hidden + h] = oracle_bf16_from_f32(acc);
+            }
         }
     }
 }

@@ -57,6 +57,8 @@ def _load():
         lib.oracle_eplb_gather.restype = None
         lib.oracle_combine.argtypes = [I, I, I, I, P, P, P, I, P, P, I64]
         lib.oracle_combine.restype = None
+        lib.oracle_expert_reduce.argtypes = [I, I, I, I, I, P, P, P, P, P, P]
+        lib.oracle_expert_reduce.restype = None
         lib.oracle_quantize_e4m3.argtypes = [P, P, I64]
         lib.oracle_quantize_e4m3.restype = None
         lib.oracle_bf16_from_f32.argtypes = [ctypes.c_float]
@@ -194,6 +196,35 @@ def combine(plan: RoutePlan, expert_output, hidden, input_is_e4m3=False,
     return out
 
 
+def expert_reduce(plan: RoutePlan, num_experts, token_selected_experts, topk_weights,
+                  expert_out, hidden, z_init=None):
+    """Each destination's combine row from per-(token, slot) expert outputs
+    (see ``oracle_expert_reduce``): uint16 bf16 bits ``[ep, ep*tpr, hidden]``.
+
+    ``expert_out`` holds bf16 bits shaped ``[ep, tpr, k, hidden]``; rows of z no
+    token fills keep ``z_init`` (default 0xEEEE)."""
+    lib = _load()
+    ep, tpr, k = plan.ep_size, plan.tokens_per_rank, plan.top_k
+    ids = np.ascontiguousarray(token_selected_experts, dtype=np.int32).reshape(ep, tpr, k)
+    w = np.ascontiguousarray(topk_weights, dtype=np.float32).reshape(ep, tpr, k)
+    y = np.ascontiguousarray(expert_out).view(np.uint16).reshape(ep, tpr, k, hidden)
+    if z_init is None:
+        z = np.full((ep, ep * tpr, hidden), 0xEEEE, np.uint16)
+    else:
+        z = np.array(z_init, dtype=np.uint16, copy=True).reshape(ep, ep * tpr, hidden)
+    lib.oracle_expert_reduce(ep, num_experts, k, tpr, hidden, _ptr(plan.num_dst),
+                             _ptr(plan.dst_ranks), _ptr(ids), _ptr(w), _ptr(y), _ptr(z))
+    return z
+
+
+def combine_experts(plan: RoutePlan, num_experts, token_selected_experts, topk_weights,
+                    expert_out, hidden, out_init=None):
+    """The combine of per-expert outputs: the expert reduction, then combine."""
+    z = expert_reduce(plan, num_experts, token_selected_experts, topk_weights, expert_out,
+                      hidden)
+    return combine(plan, z, hidden, out_init=out_init)
+
+
 def quantize_e4m3(bf16_bits):
     """E4M3 bytes of bf16 values (round to nearest even, saturate to +-448)."""
     lib = _load()
@@ -219,6 +250,7 @@ def e4m3_to_f32(b: int) -> float:
     return float(_load().oracle_e4m3_to_f32(int(b)))
 
 
-__all__ = ["build", "route", "dispatch_payload", "eplb_gather", "combine",
+__all__ = ["build", "route", "dispatch_payload", "eplb_gather", "combine", "expert_reduce",
+           "combine_experts",
            "quantize_e4m3", "bf16_from_f32", "bf16_to_f32", "e4m3_from_f32",
            "e4m3_to_f32", "RoutePlan"]

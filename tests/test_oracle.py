@@ -436,3 +436,84 @@ def test_mean_distinct_ranks_closed_form(oracle_mod, w):
     assert abs(nd.mean() - mean) < 4 * math.sqrt(var / nd.size), (nd.mean(), mean)
     if w is W.C2:
         assert abs(mean - 5.295) < 1e-3          # the 5.295 quoted for EP 8, E 256, k 8
+
+
+# --------------------------------------------------------------------------- #
+# Weighted reduction over local experts (the combine's input) and its combine
+# --------------------------------------------------------------------------- #
+
+def test_expert_reduce_uses_one_rounding_per_term(oracle_mod):
+    """Two slots owned by the same rank, worked by hand: with w0 = -(1 + 2^-7 +
+    2^-20), y0 = 1, w1 = 1 + 2^-20, y1 = 1 + 2^-7 the exact sum is 2^-27.
+    fmaf keeps it (the product w1*y1 = 1 + 2^-7 + 2^-20 + 2^-27 is never
+    rounded on its own); a rounded product followed by an add would give 0."""
+    ids = np.array([[[0, 1]], [[2, 3]]], np.int32)          # ep 2, E 4: experts 0, 1 -> rank 0
+    plan = oracle_mod.route(2, 4, 2, 1, ids, np.array([1, 0], np.int32))
+    w = np.zeros((2, 1, 2), np.float32)
+    w[0, 0] = [-(1 + 2.0 ** -7 + 2.0 ** -20), 1 + 2.0 ** -20]
+    y = np.zeros((2, 1, 2, 1), np.uint16)
+    y[0, 0, :, 0] = bf16_bits([1.0, 1 + 2.0 ** -7])
+    z = oracle_mod.expert_reduce(plan, 4, ids, w, y, 1)
+    assert bits_to_f32(z[0, 0])[0] == 2.0 ** -27
+    out = oracle_mod.combine_experts(plan, 4, ids, w, y, 1)
+    assert bits_to_f32(out[0, 0])[0] == 2.0 ** -27
+
+
+@pytest.mark.parametrize("w", [W.C1, W.C2, W.C5], ids=lambda w: w.name)
+def test_combine_experts_matches_vectorised_restatement(oracle_mod, w):
+    """Power-of-two weights make every product exact, so fmaf equals a plain
+    multiply and add; the reduction and the combine are then restated with
+    numpy fp32 arrays, looping over destination rank and slot and vectorising
+    over tokens and columns."""
+    H = 64
+    x = W.make_inputs(w, with_expert_output=False)
+    ep, tpr, k, E = w.ep_size, w.tokens_per_rank, w.top_k, w.num_experts
+    rng = np.random.default_rng(11)
+    ids = x.token_selected_experts.numpy()
+    wts = (2.0 ** rng.integers(-3, 4, (ep, tpr, k))).astype(np.float32)
+    wts *= np.where(rng.random((ep, tpr, k)) < 0.3, -1, 1).astype(np.float32)
+    y = bf16_bits(rng.standard_normal(ep * tpr * k * H).astype(np.float32)).reshape(ep, tpr, k, H)
+    plan = oracle_mod.route(ep, E, k, tpr, ids, x.local_num_tokens, x.active_rank_mask)
+    got = oracle_mod.combine_experts(plan, E, ids, wts, y, H).reshape(ep * tpr, H)
+
+    live = np.ones(ep, bool)
+    for r in w.masked_ranks:
+        live[r] = False
+    owner = np.where((ids >= 0) & (ids < E), ids // (E // ep), -1).reshape(ep * tpr, k)
+    exists = ((np.arange(tpr)[None, :] < x.local_num_tokens[:, None]) & live[:, None]).reshape(-1)
+    yf = bits_to_f32(y.reshape(ep * tpr, k, H))
+    wf = wts.reshape(ep * tpr, k)
+    acc = np.zeros((ep * tpr, H), np.float32)
+    for d in range(ep):
+        if not live[d]:
+            continue
+        z = np.zeros((ep * tpr, H), np.float32)
+        for j in range(k):
+            sel = (owner[:, j] == d)[:, None]
+            z = np.where(sel, (z + wf[:, j:j + 1] * yf[:, j, :]).astype(np.float32), z)
+        zb = torch.from_numpy(z).to(torch.bfloat16).float().numpy()
+        has = (owner == d).any(axis=1)[:, None]
+        acc = np.where(has, (acc + zb).astype(np.float32), acc)
+    want = torch.from_numpy(acc).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got[exists], want[exists])
+    assert np.all(got[~exists] == 0xEEEE)
+
+
+def test_expert_reduce_single_slot_is_the_weighted_row(oracle_mod):
+    """top_k 1: every token's only destination gets bf16(w * y)."""
+    ep, E, tpr, H = 4, 8, 20, 16
+    rng = np.random.default_rng(2)
+    ids = rng.integers(0, E, (ep, tpr, 1)).astype(np.int32)
+    wts = rng.standard_normal((ep, tpr, 1)).astype(np.float32)
+    y = bf16_bits(rng.standard_normal(ep * tpr * H).astype(np.float32)).reshape(ep, tpr, 1, H)
+    plan = oracle_mod.route(ep, E, 1, tpr, ids, np.full(ep, tpr, np.int32))
+    z = oracle_mod.expert_reduce(plan, E, ids, wts, y, H)
+    for r in range(ep):
+        for t in range(tpr):
+            d = ids[r, t, 0] // 2
+            # the fp64 product is exact; one fmaf onto +0 rounds it once to fp32,
+            # then the row is rounded to bf16
+            prod = wts[r, t, 0].astype(np.float64) * bits_to_f32(y[r, t, 0]).astype(np.float64)
+            want = torch.from_numpy(prod.astype(np.float32)).to(torch.bfloat16) \
+                .view(torch.int16).numpy().view(np.uint16)
+            assert np.array_equal(z[d, r * tpr + t], want)
