@@ -243,11 +243,17 @@ class Bytes:
     step: int
 
 
-def algorithmic_bytes(w, n_tok: int, sum_d: int, live: int, fp8: bool) -> Bytes:
+def algorithmic_bytes(w, n_tok: int, sum_d: int, live: int, fp8: bool,
+                      live_slots: int = 0) -> Bytes:
+    """live_slots > 0: the combine of per-expert outputs, which reads one bf16
+    row per (token, slot) whose expert a live rank owns, plus ids and weights."""
     rb = sum(w.payload_row_bytes())
     k, ep, tpr, E, H = w.top_k, w.ep_size, w.tokens_per_rank, w.num_experts, w.hidden
     copy = n_tok * rb + sum_d * rb
-    combine = sum_d * H * (1 if fp8 else 2) + n_tok * H * 2
+    if live_slots:
+        combine = live_slots * H * 2 + n_tok * k * 8 + n_tok * H * 2
+    else:
+        combine = sum_d * H * (1 if fp8 else 2) + n_tok * H * 2
     route = n_tok * k * 4 * (1 + 0) + sum_d * k * 4 + live * ep * tpr + ep * ep * 4
     if w.eplb:
         route += ep * E * 4 + live * ep * E * 4
@@ -320,6 +326,13 @@ def run_ours(args):
     stats = x.eplb_local_stats.to(device) if x.eplb_local_stats is not None else None
     xo = x.expert_output.to(device)
     xo8 = ep_a2a.quantize_e4m3(xo)
+    experts = args.combine == "experts"
+    if experts:
+        # one bf16 row per (token, slot), drawn on the device (seeded)
+        gen = torch.Generator(device=device).manual_seed(w.seed + 77)
+        y = torch.randn((w.ep_size, w.tokens_per_rank, w.top_k, w.hidden), generator=gen,
+                        device=device).to(torch.bfloat16)
+        wts = payloads[-1].view(torch.float32).view(w.ep_size, w.tokens_per_rank, w.top_k)
     n = x.local_num_tokens
     mask = x.active_rank_mask
     comm = ep_a2a.EpA2A(w.ep_size, w.num_experts, w.top_k, w.tokens_per_rank, w.hidden,
@@ -334,7 +347,10 @@ def run_ours(args):
 
     def step():
         comm.dispatch(ids, n, payloads, tpr, stats, mask, views=False)
-        comm.combine(comb_in, out)
+        if experts:
+            comm.combine_experts(wts, y, out)
+        else:
+            comm.combine(comb_in, out)
 
     step()
     torch.cuda.synchronize()
@@ -344,7 +360,14 @@ def run_ours(args):
     sum_d = int(d.send_counts.sum().item())
     live = w.ep_size - len(w.masked_ranks)
     n_tok = int(sum(int(n[r]) for r in range(w.ep_size) if r not in w.masked_ranks))
-    by = algorithmic_bytes(w, n_tok, sum_d, live, fp8)
+    live_slots = 0
+    if experts:
+        idn = x.token_selected_experts.numpy()
+        owner = np.where((idn >= 0) & (idn < w.num_experts), idn // w.experts_per_rank, -1)
+        alive = np.array([r not in w.masked_ranks for r in range(w.ep_size)] + [False])
+        exists = (np.arange(tpr)[None, :] < n[:, None]) & alive[:w.ep_size, None]
+        live_slots = int((alive[owner] & exists[:, :, None]).sum())
+    by = algorithmic_bytes(w, n_tok, sum_d, live, fp8, live_slots)
 
     clocks = ClockSampler(local)
     flush_buf = None
@@ -400,7 +423,7 @@ def run_ours(args):
         if cnt:
             per_kernel[name] = {"launches": cnt, "avg_ms": tot / cnt}
     kbytes = {"route_plan": by.route, "copy_bulk": by.copy, "copy_vec": by.copy,
-              "copy_staged": by.copy, "combine": by.combine}
+              "copy_staged": by.copy, "combine": by.combine, "combine_experts": by.combine}
     for name, e in per_kernel.items():
         e["algorithmic_bytes"] = kbytes[name]
         e["achieved_gbs"] = kbytes[name] / (e["avg_ms"] / 1e3) / 1e9
@@ -411,7 +434,7 @@ def run_ours(args):
 
     # FP8 combine, timed alone on the same plan (context, not the headline)
     fp8_ctx = None
-    if not fp8 and args.fp8_steps > 0:
+    if not fp8 and not experts and args.fp8_steps > 0:
         comm.dispatch(ids, n, payloads, tpr, stats, mask)
         t8 = run_timed(lambda: comm.combine(xo8, out), args.fp8_steps, 3, CudaTimer(stream),
                        dist, device, on_start=lambda: ep_a2a.ep_a2a_profile_start(
@@ -425,7 +448,8 @@ def run_ours(args):
 
     e2e = None
     if args.e2e_steps > 0:
-        e2e = run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws)
+        e2e = run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws,
+                      y_dev=y if experts else None)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -440,7 +464,9 @@ def run_ours(args):
                 "workload": f"{w.name}: ep_size {w.ep_size}, num_experts {w.num_experts}, "
                             f"top_k {w.top_k}, {tpr} tokens/rank, hidden {w.hidden} BF16, "
                             f"extra {w.extra_bytes} B/token, EPLB stats, "
-                            f"{'FP8 E4M3' if fp8 else 'BF16'} combine (fp32 accumulate)",
+                            + ("combine of per-expert outputs (weighted local reduction "
+                               "fused, fp32 accumulate)" if experts else
+                               f"{'FP8 E4M3' if fp8 else 'BF16'} combine (fp32 accumulate)"),
                 "tokens_per_step_per_gpu": n_tok, "mean_distinct_ranks": sum_d / n_tok,
                 "l2": ("512 MB L2 flush before every step, each step timed alone"
                        if args.l2_flush else "inputs larger than L2 (no flush)"),
@@ -471,14 +497,16 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws):
+def run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws, y_dev=None):
     """Same step through the public API with the inputs in pinned host memory:
-    every step copies the inputs host->device and the result device->host."""
+    every step copies the inputs host->device and the result device->host.
+    With y_dev (the combine of per-expert outputs) the combine input is the
+    per-(token, slot) expert outputs instead of per-rank rows."""
     import torch
     h_ids = x.token_selected_experts.pin_memory()
     h_pay = [p.pin_memory() for p in x.payloads]
     h_stats = x.eplb_local_stats.pin_memory() if x.eplb_local_stats is not None else None
-    h_xo = x.expert_output.pin_memory()
+    h_xo = (y_dev.cpu() if y_dev is not None else x.expert_output).pin_memory()
     h_out = torch.empty((w.ep_size, w.tokens_per_rank, w.hidden), dtype=torch.bfloat16).pin_memory()
     d_ids = torch.empty_like(h_ids, device=device)
     d_pay = [torch.empty_like(p, device=device) for p in h_pay]
@@ -498,7 +526,11 @@ def run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws):
         d_xo.copy_(h_xo, non_blocking=True)
         comm.dispatch(d_ids, x.local_num_tokens, d_pay, w.tokens_per_rank, d_stats,
                       x.active_rank_mask, views=False)
-        comm.combine(d_xo, d_out)
+        if y_dev is not None:
+            wts = d_pay[-1].view(torch.float32).view(w.ep_size, w.tokens_per_rank, w.top_k)
+            comm.combine_experts(wts, d_xo, d_out)
+        else:
+            comm.combine(d_xo, d_out)
         h_out.copy_(d_out, non_blocking=True)
 
     ms = run_timed(step, args.e2e_steps, 2, CudaTimer(stream), dist, device)
@@ -602,7 +634,9 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--tokens-per-rank", type=int, default=0,
                     help="run the workload with this many tokens per rank (small profiling cases)")
-    ap.add_argument("--combine", choices=["bf16", "fp8"], default="bf16")
+    ap.add_argument("--combine", choices=["bf16", "fp8", "experts"], default="bf16",
+                    help="combine input: bf16 or fp8 rows per rank, or bf16 outputs per "
+                         "(token, slot) reduced with topk_weights inside the combine")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--fp8-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -172,6 +172,129 @@ __global__ void __launch_bounds__(512) combine_scalar_kernel(const CombineArgs a
   }
 }
 
+// Round to bf16 (nearest even) and widen back: the value a bf16 combine row holds.
+__device__ __forceinline__ float bf16_round(float z) {
+  return __bfloat162float(__float2bfloat16_rn(z));
+}
+
+// Per-token routing seen by the expert combine: for each slot j, the owner rank
+// of its expert if that rank is one of the token's destinations, else -1
+// (ids outside [0, E) and masked-off owners are in no destination's sum).
+template <int KMAX>
+__device__ __forceinline__ void slot_owners(const CombineExpertsArgs& a, int64_t tok, int nd,
+                                            uint64_t w0, uint64_t w1, uint64_t w2, uint64_t w3,
+                                            int (&own)[KMAX], float (&wt)[KMAX]) {
+  const int first = dst_rank(w0, w1, w2, w3, 0);
+  const int32_t* ids =
+      reinterpret_cast<const int32_t*>(a.recv_ids0 + (int64_t)first * a.rank_stride) + tok * a.k;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    own[j] = -1;
+    wt[j] = 0.0f;
+    if (j < a.k) {
+      const int32_t e = ids[j];
+      int o = (e >= 0 && e < a.E) ? e / a.epr : -1;
+      bool in_set = false;
+      for (int q = 0; q < nd; ++q) in_set |= dst_rank(w0, w1, w2, w3, q) == o;
+      own[j] = in_set ? o : -1;
+      wt[j] = a.w[tok * a.k + j];
+    }
+  }
+}
+
+// top_k <= 8, hidden a multiple of 8, 16-byte aligned rows: each thread owns
+// 16-byte column vectors; the loads of all needed slots are issued first.
+__global__ void __launch_bounds__(512) combine_experts_vec_kernel(const CombineExpertsArgs a) {
+  pdl_wait();
+  constexpr int KMAX = 8;
+  const int nvec = a.H / 8;
+  const int words = a.plan_stride / 8;
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    const int nd = a.plan_nd[tok];
+    if (nd == kNoToken) continue;
+    uint16_t* out = a.out + tok * (int64_t)a.H;
+    if (nd == 0) {           // every owner masked off: the sum is empty
+      for (int v = threadIdx.x; v < nvec; v += blockDim.x)
+        reinterpret_cast<uint4*>(out)[v] = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const uint64_t* row = reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    const uint64_t w0 = row[0];
+    const uint64_t w1 = words > 1 ? row[1] : 0;
+    const uint64_t w2 = words > 2 ? row[2] : 0;
+    const uint64_t w3 = words > 3 ? row[3] : 0;
+    int own[KMAX];
+    float wt[KMAX];
+    slot_owners<KMAX>(a, tok, nd, w0, w1, w2, w3, own, wt);
+    const uint16_t* yt = a.y + tok * (int64_t)a.k * a.H;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      uint4 raw[KMAX];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (own[j] >= 0) raw[j] = ld_stream_v4(yt + (int64_t)j * a.H + (int64_t)v * 8);
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+      for (int q = 0; q < nd; ++q) {
+        const int d = dst_rank(w0, w1, w2, w3, q);
+        float z[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) z[e] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          if (own[j] != d) continue;
+          const uint32_t wv[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            z[2 * i] = __fmaf_rn(wt[j], bf16_bits_to_f32(wv[i] & 0xFFFFu), z[2 * i]);
+            z[2 * i + 1] = __fmaf_rn(wt[j], bf16_bits_to_f32(wv[i] >> 16), z[2 * i + 1]);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], bf16_round(z[e]));
+      }
+      uint4 pk;
+      pk.x = pack_bf16x2(acc[0], acc[1]);
+      pk.y = pack_bf16x2(acc[2], acc[3]);
+      pk.z = pack_bf16x2(acc[4], acc[5]);
+      pk.w = pack_bf16x2(acc[6], acc[7]);
+      reinterpret_cast<uint4*>(out)[v] = pk;
+    }
+  }
+}
+
+// Any top_k (<= 32) and hidden size: one element per thread step.
+__global__ void __launch_bounds__(512) combine_experts_any_kernel(const CombineExpertsArgs a) {
+  pdl_wait();
+  constexpr int KMAX = kMaxTopK;
+  const int words = a.plan_stride / 8;
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    const int nd = a.plan_nd[tok];
+    if (nd == kNoToken) continue;
+    uint16_t* out = a.out + tok * (int64_t)a.H;
+    const uint64_t* row = reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    const uint64_t w0 = row[0];
+    const uint64_t w1 = words > 1 ? row[1] : 0;
+    const uint64_t w2 = words > 2 ? row[2] : 0;
+    const uint64_t w3 = words > 3 ? row[3] : 0;
+    int own[KMAX];
+    float wt[KMAX];
+    if (nd > 0) slot_owners<KMAX>(a, tok, nd, w0, w1, w2, w3, own, wt);
+    const uint16_t* yt = a.y + tok * (int64_t)a.k * a.H;
+    for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
+      float acc = 0.0f;
+      for (int q = 0; q < nd; ++q) {
+        const int d = dst_rank(w0, w1, w2, w3, q);
+        float z = 0.0f;
+        for (int j = 0; j < a.k; ++j)
+          if (own[j] == d) z = __fmaf_rn(wt[j], bf16_bits_to_f32(yt[(int64_t)j * a.H + h]), z);
+        acc = __fadd_rn(acc, bf16_round(z));
+      }
+      out[h] = (uint16_t)f32_to_bf16_bits(acc);
+    }
+  }
+}
+
 // bf16 -> E4M3, round to nearest even, saturating (satfinite).
 __global__ void quantize_e4m3_kernel(const uint16_t* __restrict__ in, uint8_t* __restrict__ out,
                                      int64_t n, bool vec) {
@@ -221,6 +344,13 @@ cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, int threads
   }
   if (fp8) return launch_kernel(combine_scalar_kernel<true>, g, b, 0, stream, pdl, a);
   return launch_kernel(combine_scalar_kernel<false>, g, b, 0, stream, pdl, a);
+}
+
+cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, int threads, int grid,
+                                   cudaStream_t stream, bool pdl) {
+  const dim3 g(grid), b(threads);
+  if (vec) return launch_kernel(combine_experts_vec_kernel, g, b, 0, stream, pdl, a);
+  return launch_kernel(combine_experts_any_kernel, g, b, 0, stream, pdl, a);
 }
 
 cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n,

@@ -585,6 +585,41 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   return EP_A2A_OK;
 }
 
+EP_API ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle h, const float* topk_weights,
+                                            const void* expert_output_per_slot, void* output,
+                                            void* stream_v) {
+  ep_a2a_status st = check_handle(h);
+  if (st != EP_A2A_OK) return st;
+  if (!h->have_plan) return fail(EP_A2A_ERR_NO_PLAN, "combine needs a preceding dispatch");
+  if (!topk_weights || !expert_output_per_slot || !output)
+    return fail(EP_A2A_ERR_INVALID_ARG, "topk_weights / expert output / output is NULL");
+  CombineExpertsArgs a;
+  a.plan_nd = h->ws + h->L.off_plan_nd;
+  a.plan_dst = h->ws + h->L.off_plan_dst;
+  a.recv_ids0 = h->ws + h->L.rank_base + h->L.off_ids;
+  a.rank_stride = h->L.rank_stride;
+  a.w = topk_weights;
+  a.y = static_cast<const uint16_t*>(expert_output_per_slot);
+  a.out = static_cast<uint16_t*>(output);
+  a.ntok = (int64_t)h->p.ep_size * h->last_tpr;
+  a.H = h->p.hidden_size;
+  a.k = h->p.top_k;
+  a.E = h->p.num_experts;
+  a.epr = h->p.num_experts / h->p.ep_size;
+  a.plan_stride = h->L.plan_stride;
+  const bool vec = a.k <= 8 && a.H % 8 == 0 && aligned(expert_output_per_slot, 16) &&
+                   aligned(output, 16);
+  const int grid = (int)std::max<int64_t>(
+      1, std::min<int64_t>(a.ntok, (int64_t)h->num_sms * h->combine_ctas_per_sm));
+  const int threads = h->combine_threads > 0 ? h->combine_threads : 64;
+  const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE_EXPERTS, (cudaStream_t)stream_v);
+  cudaError_t e = launch_combine_experts(a, vec, threads, grid, (cudaStream_t)stream_v,
+                                         h->pdl != 0);
+  prof_end(h, slot, (cudaStream_t)stream_v);
+  if (e != cudaSuccess) return cuda_fail(e, "expert combine kernel launch");
+  return EP_A2A_OK;
+}
+
 EP_API ep_a2a_status ep_a2a_quantize_e4m3(const void* bf16_in, void* e4m3_out, int64_t n,
                                           void* stream) {
   if (n < 0) return fail(EP_A2A_ERR_INVALID_ARG, "n < 0");

@@ -101,6 +101,23 @@ struct CombineArgs {
 
 cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, int threads, int grid,
                            cudaStream_t stream, bool pdl);
+
+// Combine of per-(token, slot) expert outputs: the weighted reduction over each
+// destination's local experts fused into the combine.
+struct CombineExpertsArgs {
+  const uint8_t* plan_nd;
+  const uint8_t* plan_dst;
+  const uint8_t* recv_ids0;    // rank 0's recv_topk_ids ([ep*tpr, k] int32 per rank)
+  int64_t rank_stride;         // bytes between ranks' recv_topk_ids
+  const float* w;              // topk_weights [ep*tpr, k]
+  const uint16_t* y;           // bf16 [ep*tpr, k, H]
+  uint16_t* out;               // bf16 [ep*tpr, H]
+  int64_t ntok;
+  int H, k, E, epr, plan_stride;
+};
+
+cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, int threads, int grid,
+                                   cudaStream_t stream, bool pdl);
 cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n, cudaStream_t stream);
 cudaError_t launch_wait_timeout_probe(uint32_t* err, unsigned long long limit_ns,
                                       cudaStream_t stream);

@@ -75,11 +75,12 @@ class DispatchResult(ctypes.Structure):
     ]
 
 
-KERNEL_NAMES = ["route_plan", "copy_bulk", "copy_vec", "combine", "copy_staged"]
+KERNEL_NAMES = ["route_plan", "copy_bulk", "copy_vec", "combine", "copy_staged",
+                "combine_experts"]
 
 
 class KernelTimes(ctypes.Structure):
-    _fields_ = [("launches", ctypes.c_int64 * 5), ("total_ms", ctypes.c_double * 5)]
+    _fields_ = [("launches", ctypes.c_int64 * 6), ("total_ms", ctypes.c_double * 6)]
 
 
 def _load():
@@ -95,6 +96,7 @@ def _load():
                                  P(DispatchResult)]),
         "ep_a2a_combine": (st, [VP, VP, ctypes.c_int, VP, VP]),
         "ep_a2a_quantize_e4m3": (st, [VP, VP, I64, VP]),
+        "ep_a2a_combine_experts": (st, [VP, VP, VP, VP, VP]),
         "ep_a2a_get_status": (st, [VP, VP]),
         "ep_a2a_debug_wait_probe": (st, [VP, I64, VP]),
         "ep_a2a_set_option": (st, [VP, ctypes.c_int, I64]),
@@ -170,6 +172,13 @@ def ep_a2a_combine(handle: int, expert_output_ptr: int, dtype: int, output_ptr: 
     _check(lib.ep_a2a_combine(ctypes.c_void_p(handle), ctypes.c_void_p(expert_output_ptr),
                               int(dtype), ctypes.c_void_p(output_ptr),
                               ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def ep_a2a_combine_experts(handle: int, topk_weights_ptr: int, expert_out_ptr: int,
+                           output_ptr: int, stream=None):
+    _check(lib.ep_a2a_combine_experts(ctypes.c_void_p(handle), ctypes.c_void_p(topk_weights_ptr),
+                                      ctypes.c_void_p(expert_out_ptr), ctypes.c_void_p(output_ptr),
+                                      ctypes.c_void_p(_stream_ptr(stream))))
 
 
 def ep_a2a_quantize_e4m3(bf16_ptr: int, e4m3_ptr: int, n: int, stream=None):
@@ -352,6 +361,25 @@ class EpA2A:
         if tpr is not None:
             assert output.numel() == self.ep_size * tpr * self.hidden_size, output.shape
         ep_a2a_combine(self.handle, x.data_ptr(), dt, output.data_ptr(), stream)
+        return output
+
+    def combine_experts(self, topk_weights: torch.Tensor, expert_output_per_slot: torch.Tensor,
+                        output: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """topk_weights fp32 [ep, tpr, k]; expert_output_per_slot bf16 [ep, tpr, k, hidden];
+        returns bf16 [ep, tpr, hidden] (see ep_a2a_combine_experts)."""
+        tpr = self.last_tokens_per_rank
+        assert tpr is not None, "combine needs a preceding dispatch"
+        w, y = topk_weights, expert_output_per_slot
+        assert w.is_cuda and w.dtype == torch.float32 and w.is_contiguous()
+        assert w.numel() == self.ep_size * tpr * self.top_k, w.shape
+        assert y.is_cuda and y.dtype == torch.bfloat16 and y.is_contiguous()
+        assert y.numel() == self.ep_size * tpr * self.top_k * self.hidden_size, y.shape
+        if output is None:
+            output = torch.empty((self.ep_size, tpr, self.hidden_size), dtype=torch.bfloat16,
+                                 device=y.device)
+        assert output.is_cuda and output.dtype == torch.bfloat16 and output.is_contiguous()
+        assert output.numel() == self.ep_size * tpr * self.hidden_size, output.shape
+        ep_a2a_combine_experts(self.handle, w.data_ptr(), y.data_ptr(), output.data_ptr(), stream)
         return output
 
     def get_status(self, stream=None) -> int:

@@ -191,6 +191,33 @@ ep_a2a_status ep_a2a_combine(ep_a2a_handle handle, const void* expert_output,
                              ep_a2a_combine_dtype dtype, void* output, void* stream);
 
 /*
+ * Combine of per-expert outputs: the step that makes the combine's input
+ * (NVLinkTwoSidedAlltoAll.combine(): rows "already weighted and reduced over
+ * this rank's local experts") fused into the combine, so the per-rank rows are
+ * never written to memory.  For each existing token (src, t) of the last
+ * dispatch:
+ *   z_d = bf16( fp32 sum over the token's slots j whose expert rank d owns,
+ *               ascending j, of topk_weights[j] * y[j] (one fused multiply-add
+ *               per term, accumulator starting at +0.0f) )
+ *   out[src][t] = bf16( fp32 sum of z_d over the token's destination ranks d in
+ *                       ascending order, starting at +0.0f )
+ * which equals ep_a2a_combine applied to the rows z.  Slots whose expert is
+ * owned by no rank or by a masked-off rank take no part.
+ *
+ *   topk_weights            device fp32 [ep, tpr, top_k] (source layout)
+ *   expert_output_per_slot  device bf16 [ep, tpr, top_k, hidden_size]: row
+ *                           (src, t, j) = output of expert j of token t of src;
+ *                           rows of slots that take no part are not read
+ *   output                  device bf16 [ep, tpr, hidden_size]; rows of tokens that
+ *                           do not exist are not written
+ * The routing ids are the ones the last dispatch received (read from the
+ * workspace).  NO_PLAN if no dispatch has run on this handle.
+ */
+ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle handle, const float* topk_weights,
+                                     const void* expert_output_per_slot, void* output,
+                                     void* stream);
+
+/*
  * FP8 helper (flashinfer.moe_ep.NVLinkOneSidedConfig, use_low_precision_combine):
  * e4m3_out[i] = E4M3(bf16_in[i]), round to nearest even, saturating to +-448.
  * Device pointers; n elements.  Not part of a dispatch / combine step.
@@ -262,7 +289,8 @@ typedef enum {
   EP_A2A_KERNEL_COPY_VEC = 2,     /* dispatch rows, vector path */
   EP_A2A_KERNEL_COMBINE = 3,
   EP_A2A_KERNEL_COPY_STAGED = 4,  /* dispatch rows, bulk-async loads + vector stores */
-  EP_A2A_KERNEL_COUNT = 5
+  EP_A2A_KERNEL_COMBINE_EXPERTS = 5, /* combine of per-expert outputs */
+  EP_A2A_KERNEL_COUNT = 6
 } ep_a2a_kernel;
 typedef struct {
   int64_t launches[EP_A2A_KERNEL_COUNT];

@@ -430,3 +430,73 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     plan = U.oracle_plan(w, x)
     U.check_plan(run2, plan, w)
     U.check_combine(run2, plan, w, x)
+
+
+# --------------------------------------------------------------------------- #
+# Combine of per-expert outputs (weighted local reduction fused into combine)
+# --------------------------------------------------------------------------- #
+
+def _expert_outputs(w, seed):
+    """bf16 [ep, tpr, k, H] N(0,1) expert outputs, one row per (token, slot)."""
+    g = torch.Generator().manual_seed(seed)
+    n = w.ep_size * w.tokens_per_rank * w.top_k * w.hidden
+    y = torch.empty(n, dtype=torch.bfloat16)
+    step = 1 << 26
+    for s in range(0, n, step):
+        e = min(n, s + step)
+        y[s:e] = torch.randn(e - s, generator=g).to(torch.bfloat16)
+    return y.view(w.ep_size, w.tokens_per_rank, w.top_k, w.hidden)
+
+
+def _check_combine_experts(w, x, y, wts, options=None):
+    from combine_route_plan_b200 import ep_a2a
+    run = U.Run(w, W.Inputs(w, x.token_selected_experts, x.local_num_tokens, x.payloads,
+                            x.eplb_local_stats, x.active_rank_mask, None), options=options)
+    out = torch.full((w.ep_size, w.tokens_per_rank, w.hidden), U.OUT_CANARY, dtype=torch.int16,
+                     device="cuda").view(torch.bfloat16)
+    run.comm.combine_experts(wts.cuda(), y.cuda(), out)
+    torch.cuda.synchronize()
+    assert run.comm.get_status() == ep_a2a.OK
+    plan = U.oracle_plan(w, x)
+    want = U.oracle.combine_experts(plan, w.num_experts, x.token_selected_experts.numpy(),
+                                    wts.numpy(), U.to_np(y), w.hidden,
+                                    out_init=U.oracle_out_init(w))
+    U.assert_equal(out, want, "combine of expert outputs")
+
+
+@pytest.mark.parametrize("name", ["c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked",
+                                  "c4_ep8_prefill"])
+def test_combine_experts_bit_exact(name):
+    w = W.BY_NAME[name]
+    x = _inputs(w.name)
+    wts = x.payloads[-1].view(torch.float32).view(w.ep_size, w.tokens_per_rank, w.top_k)
+    y = _expert_outputs(w, seed=w.seed + 77)
+    _check_combine_experts(w, x, y, wts)
+
+
+@pytest.mark.parametrize("ep,E,k,tpr,H", [
+    (3, 12, 3, 37, 100),     # hidden not a multiple of 8: element path
+    (16, 64, 16, 20, 64),    # top_k above 8: element path
+    (4, 16, 5, 33, 40),      # top_k 5, vector path
+    (8, 64, 8, 40, 64),
+])
+def test_combine_experts_edge_shapes(ep, E, k, tpr, H):
+    w, x = _custom(ep, E, k, tpr, H, [16], seed=ep * 13 + k)
+    g = torch.Generator().manual_seed(k)
+    wts = torch.randn((ep, tpr, k), generator=g)
+    y = torch.randn((ep, tpr, k, H), generator=g).to(torch.bfloat16)
+    _check_combine_experts(w, x, y, wts)
+
+
+def test_combine_experts_with_masks_and_invalid_ids():
+    ep, E, k, tpr, H = 8, 64, 6, 40, 64
+    mask = [0b10110111, 0, 0, 0]
+    w, x = _custom(ep, E, k, tpr, H, [32], n=[40, 1, 0, 39, 17, 40, 2, 33], mask=mask, seed=21)
+    ids = x.token_selected_experts.clone()
+    ids[0, :5, 0] = -3
+    ids[1, 0, 1] = 64
+    x = W.Inputs(w, ids, x.local_num_tokens, x.payloads, None, x.active_rank_mask, None)
+    g = torch.Generator().manual_seed(5)
+    wts = torch.randn((ep, tpr, k), generator=g)
+    y = torch.randn((ep, tpr, k, H), generator=g).to(torch.bfloat16)
+    _check_combine_experts(w, x, y, wts)
