@@ -88,6 +88,24 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&p);
 }
 
+// Thread 0 asks for the rows of token `tok` (if it exists) to be brought into
+// L2, so that this CTA's loads of it hit L2 when it gets there.
+template <int kElemBytes>
+__device__ __forceinline__ void prefetch_token_rows(const CombineArgs& a, int64_t tok) {
+  if (tok >= a.ntok) return;
+  const int nd = a.plan_nd[tok];
+  if (nd == kNoToken || nd == 0) return;
+  const uint64_t* row = reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+  const int words = a.plan_stride / 8;
+  const uint32_t bytes = (uint32_t)a.H * kElemBytes;
+  const int64_t rank_stride = a.ntok * (int64_t)a.H * kElemBytes;
+  for (int q = 0; q < nd; ++q) {
+    const uint64_t w = q < 8 ? row[0] : row[min(q >> 3, words - 1)];
+    const int d = (int)((w >> ((q & 7) * 8)) & 0xFFu);
+    prefetch_l2(a.x + (int64_t)d * rank_stride + tok * (int64_t)bytes, bytes);
+  }
+}
+
 template <bool kFp8>
 __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
   pdl_wait();
@@ -95,7 +113,9 @@ __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
   constexpr int kElemBytes = kFp8 ? 1 : 2;
   const int nvec = a.H / kElems;
   const int words = a.plan_stride / 8;
+  if (a.prefetch && threadIdx.x == 0) prefetch_token_rows<kElemBytes>(a, blockIdx.x);
   for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    if (a.prefetch && threadIdx.x == 0) prefetch_token_rows<kElemBytes>(a, tok + gridDim.x);
     const int nd = a.plan_nd[tok];
     if (nd == kNoToken) continue;
     const uint64_t* row = reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
@@ -209,7 +229,13 @@ __global__ void __launch_bounds__(512) combine_experts_vec_kernel(const CombineE
   constexpr int KMAX = 8;
   const int nvec = a.H / 8;
   const int words = a.plan_stride / 8;
+  // the k slot rows of a token are contiguous: one prefetch per token
+  const uint32_t tok_bytes = (uint32_t)a.k * a.H * 2;
+  if (a.prefetch && threadIdx.x == 0 && blockIdx.x < a.ntok)
+    prefetch_l2(a.y + (int64_t)blockIdx.x * a.k * a.H, tok_bytes);
   for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    if (a.prefetch && threadIdx.x == 0 && tok + gridDim.x < a.ntok)
+      prefetch_l2(a.y + (tok + gridDim.x) * a.k * a.H, tok_bytes);
     const int nd = a.plan_nd[tok];
     if (nd == kNoToken) continue;
     uint16_t* out = a.out + tok * (int64_t)a.H;

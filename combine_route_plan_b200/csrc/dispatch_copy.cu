@@ -324,8 +324,13 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
   const int gl = threadIdx.x % TPT;
   const int group = threadIdx.x / TPT;
   const int lane = threadIdx.x & 31;
-  for (int64_t tok = (int64_t)blockIdx.x * kGroups + group; tok < a.ntok;
-       tok += (int64_t)gridDim.x * kGroups) {
+  const int64_t tok_step = (int64_t)gridDim.x * kGroups;
+  for (int64_t tok = (int64_t)blockIdx.x * kGroups + group; tok < a.ntok; tok += tok_step) {
+    if (kAll16 && a.prefetch && gl == 0 && tok + tok_step < a.ntok) {
+      // the group's next token: its rows into L2 while this one is copied
+      for (int p = 0; p < a.np; ++p)
+        prefetch_l2(a.src[p] + (tok + tok_step) * a.rb[p], (uint32_t)a.rb[p]);
+    }
     uint64_t w0, w1, w2, w3;
     const int nd = token_destinations(a, tok, lane, w0, w1, w2, w3);
     if (nd == 0) continue;

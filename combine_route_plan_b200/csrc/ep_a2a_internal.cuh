@@ -74,6 +74,7 @@ struct CopyArgs {
   // destinations itself instead of reading the plan
   const int32_t* ids;                    // [ep, tpr, k]
   int E, k, epr, tpr, use_mask;
+  int prefetch;                          // vector path: prefetch the next token's rows into L2
   int32_t n[kMaxRanks];                  // local_num_tokens (0 for masked-off ranks)
   uint64_t live[kMaskWords];
 };
@@ -97,6 +98,7 @@ struct CombineArgs {
   int64_t ntok;                // ep * tpr
   int H;
   int plan_stride;
+  int prefetch;                // 1: prefetch the CTA's next token's rows into L2
 };
 
 cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, int threads, int grid,
@@ -114,6 +116,7 @@ struct CombineExpertsArgs {
   uint16_t* out;               // bf16 [ep*tpr, H]
   int64_t ntok;
   int H, k, E, epr, plan_stride;
+  int prefetch;                // 1: prefetch the CTA's next token's rows into L2
 };
 
 cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, int threads, int grid,
@@ -247,6 +250,12 @@ __device__ __forceinline__ void bulk_wait_all() {
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Ask the copy engine to bring `bytes` (a multiple of 16, 16-byte aligned)
+// into L2 ahead of use; no registers or shared memory are involved.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {

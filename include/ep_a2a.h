@@ -269,8 +269,13 @@ typedef enum {
                                      (flashinfer.moe_ep.NVLinkOneSidedConfig, enable_pdl);
                                      each kernel waits for the previous one before it
                                      touches memory, so results do not change */
-  EP_A2A_OPT_VEC_THREADS_PER_TOKEN = 12 /* vector copy: threads per token (32, 64, 128,
+  EP_A2A_OPT_VEC_THREADS_PER_TOKEN = 12,/* vector copy: threads per token (32, 64, 128,
                                      256); 0 (default) = from the token count */
+  EP_A2A_OPT_COMBINE_PREFETCH = 13,/* combines: 1 = each CTA asks for its next token's rows
+                                     to be brought into L2 (cp.async.bulk.prefetch.L2)
+                                     while it sums the current one; 0 = never; -1
+                                     (default) = for the FP8 combine only */
+  EP_A2A_OPT_COPY_PREFETCH = 14   /* vector copy: the same for the next token's rows */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

@@ -150,6 +150,22 @@ def test_cuda_graph_capture_and_replay():
     assert comm.get_status() == ep_a2a.OK
 
 
+@pytest.mark.parametrize("prefetch,ctas", [(1, 4), (1, 12), (1, 128), (0, 8)])
+def test_prefetch_options_do_not_change_results(prefetch, ctas):
+    from combine_route_plan_b200 import ep_a2a
+    for name in ("c2_ep8_decode", "c5_ep64_wide_masked"):
+        _full_check(W.BY_NAME[name], options={ep_a2a.OPT_COMBINE_PREFETCH: prefetch,
+                                              ep_a2a.OPT_COPY_PREFETCH: prefetch,
+                                              ep_a2a.OPT_COMBINE_CTAS_PER_SM: ctas,
+                                              ep_a2a.OPT_VEC_CTAS_PER_SM: min(ctas, 64)})
+    w = W.C2
+    x = _inputs(w.name)
+    wts = x.payloads[-1].view(torch.float32).view(w.ep_size, w.tokens_per_rank, w.top_k)
+    _check_combine_experts(w, x, _expert_outputs(w, seed=3), wts,
+                           options={ep_a2a.OPT_COMBINE_PREFETCH: prefetch,
+                                    ep_a2a.OPT_COMBINE_CTAS_PER_SM: ctas})
+
+
 @pytest.mark.parametrize("threads,ctas", [(64, 0), (96, 3), (256, 64), (512, 1), (128, 1024),
                                           (0, 0)])
 def test_combine_launch_shape_does_not_change_results(threads, ctas):
