@@ -46,7 +46,11 @@
  *     clear neither sends nor receives; its receive arrays are left untouched;
  *   - the combine sum is an fp32 accumulator starting at +0.0f, adding the rows
  *     in ascending destination-rank order, rounded once to bf16 (nearest-even);
- *   - the FP8 combine format is E4M3 ("fn": no infinities, max 448), unscaled;
+ *   - the FP8 combine format is E4M3 ("fn": no infinities, max 448), unscaled,
+ *     or, in the scaled variant, E4M3 with one fp32 scale per row: with
+ *     amax = max |x| over the row, scale = amax / 448 and the codes are
+ *     E4M3(x * (448 / amax)) (each fp32 operation rounded to nearest); a zero
+ *     row has scale 1; the combine adds fmaf(decode(q), scale, acc);
  *   - expert outputs before that reduction are one BF16 row per (source token,
  *     top_k slot), [ep, tpr, k, hidden]; rank d's combine row for the token is
  *     bf16(sum over the slots j whose expert d owns, ascending j, of
@@ -369,6 +373,66 @@ void oracle_expert_reduce(int ep_size, int num_experts, int top_k, int tokens_pe
                 }
                 z[((int64_t)d * slots + s) * hidden + h] = oracle_bf16_from_f32(acc);
             }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* FP8 combine with one scale per row.                                        */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Per row of `hidden` bf16 values: amax = max |x|; scale = amax / 448 and
+ * inv = 448 / amax, each an fp32 division rounded to nearest (1 and 1 for a
+ * zero row); code[h] = E4M3(x[h] * inv) with the product rounded to fp32 and
+ * the E4M3 rounding of oracle_e4m3_from_f32 (nearest even, saturating).
+ */
+void oracle_quantize_e4m3_rows(const uint16_t* bf16_in, int64_t rows, int hidden,
+                               uint8_t* e4m3_out, float* scales) {
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* x = bf16_in + r * hidden;
+        float amax = 0.0f;
+        for (int h = 0; h < hidden; ++h) {
+            const float a = fabsf(oracle_bf16_to_f32(x[h]));
+            if (a > amax) amax = a;
+        }
+        float scale = 1.0f, inv = 1.0f;
+        if (amax > 0.0f) {
+            scale = amax / 448.0f;
+            inv = 448.0f / amax;
+        }
+        scales[r] = scale;
+        for (int h = 0; h < hidden; ++h) {
+            const float v = oracle_bf16_to_f32(x[h]) * inv;
+            e4m3_out[r * hidden + h] = oracle_e4m3_from_f32(v);
+        }
+    }
+}
+
+/*
+ * As oracle_combine with E4M3 rows, each destination row carrying its scale
+ * (row_scales [ep(dst), ep*tpr]):  acc = fmaf(decode(q), scale, acc) for d in
+ * the token's destination set, ascending, from +0.0f; out = bf16(acc).
+ */
+void oracle_combine_scaled(int ep_size, int top_k, int tokens_per_rank, int hidden,
+                           const int32_t* num_dst, const int32_t* dst_ranks,
+                           const uint8_t* expert_output, const float* row_scales,
+                           uint16_t* out)
+{
+    const int ep = ep_size, k = top_k, tpr = tokens_per_rank;
+    const int64_t slots = (int64_t)ep * tpr;
+    for (int64_t s = 0; s < slots; ++s) {
+        const int nd = num_dst[s];
+        if (nd < 0) continue;
+        const int32_t* list = dst_ranks + s * k;
+        for (int h = 0; h < hidden; ++h) {
+            float acc = 0.0f;
+            for (int j = 0; j < nd; ++j) {
+                const int d = list[j];
+                const int64_t row = (int64_t)d * slots + s;
+                acc = fmaf(oracle_e4m3_to_f32(expert_output[row * hidden + h]), row_scales[row], acc);
+            }
+            out[s * hidden + h] = oracle_bf16_from_f32(acc);
         }
     }
 }

@@ -59,6 +59,10 @@ def _load():
         lib.oracle_combine.restype = None
         lib.oracle_expert_reduce.argtypes = [I, I, I, I, I, P, P, P, P, P, P]
         lib.oracle_expert_reduce.restype = None
+        lib.oracle_quantize_e4m3_rows.argtypes = [P, I64, I, P, P]
+        lib.oracle_quantize_e4m3_rows.restype = None
+        lib.oracle_combine_scaled.argtypes = [I, I, I, I, P, P, P, P, P]
+        lib.oracle_combine_scaled.restype = None
         lib.oracle_quantize_e4m3.argtypes = [P, P, I64]
         lib.oracle_quantize_e4m3.restype = None
         lib.oracle_bf16_from_f32.argtypes = [ctypes.c_float]
@@ -225,6 +229,32 @@ def combine_experts(plan: RoutePlan, num_experts, token_selected_experts, topk_w
     return combine(plan, z, hidden, out_init=out_init)
 
 
+def quantize_e4m3_rows(bf16_bits, hidden):
+    """(E4M3 codes uint8 [rows, hidden], fp32 scales [rows]) of bf16 rows, one
+    scale per row (see ``oracle_quantize_e4m3_rows``)."""
+    lib = _load()
+    x = np.ascontiguousarray(bf16_bits).view(np.uint16).reshape(-1, hidden)
+    codes = np.empty(x.shape, np.uint8)
+    scales = np.empty(x.shape[0], np.float32)
+    lib.oracle_quantize_e4m3_rows(_ptr(x), x.shape[0], hidden, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def combine_scaled(plan: RoutePlan, codes, row_scales, hidden, out_init=None):
+    """Combine of E4M3 rows with one fp32 scale per row: bf16 bits [ep, tpr, hidden]."""
+    lib = _load()
+    ep, tpr = plan.ep_size, plan.tokens_per_rank
+    x = np.ascontiguousarray(codes).view(np.uint8).reshape(ep, ep * tpr, hidden)
+    sc = np.ascontiguousarray(row_scales, dtype=np.float32).reshape(ep, ep * tpr)
+    if out_init is None:
+        out = np.full((ep, tpr, hidden), 0xEEEE, np.uint16)
+    else:
+        out = np.array(out_init, dtype=np.uint16, copy=True).reshape(ep, tpr, hidden)
+    lib.oracle_combine_scaled(ep, plan.top_k, tpr, hidden, _ptr(plan.num_dst),
+                              _ptr(plan.dst_ranks), _ptr(x), _ptr(sc), _ptr(out))
+    return out
+
+
 def quantize_e4m3(bf16_bits):
     """E4M3 bytes of bf16 values (round to nearest even, saturate to +-448)."""
     lib = _load()
@@ -251,6 +281,6 @@ def e4m3_to_f32(b: int) -> float:
 
 
 __all__ = ["build", "route", "dispatch_payload", "eplb_gather", "combine", "expert_reduce",
-           "combine_experts",
+           "combine_experts", "quantize_e4m3_rows", "combine_scaled",
            "quantize_e4m3", "bf16_from_f32", "bf16_to_f32", "e4m3_from_f32",
            "e4m3_to_f32", "RoutePlan"]

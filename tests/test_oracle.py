@@ -517,3 +517,83 @@ def test_expert_reduce_single_slot_is_the_weighted_row(oracle_mod):
             want = torch.from_numpy(prod.astype(np.float32)).to(torch.bfloat16) \
                 .view(torch.int16).numpy().view(np.uint16)
             assert np.array_equal(z[d, r * tpr + t], want)
+
+
+# --------------------------------------------------------------------------- #
+# FP8 combine with one scale per row
+# --------------------------------------------------------------------------- #
+
+def test_row_quantize_with_amax_448_is_plain_e4m3(oracle_mod):
+    """amax = 448 gives scale = inv = 1: the codes are plain E4M3 (torch's
+    float8_e4m3fn conversion in range)."""
+    rng = np.random.default_rng(4)
+    x = (rng.standard_normal((6, 64)) * 40).clip(-447, 447).astype(np.float32)
+    x[:, 3] = 448.0
+    xb = bf16_bits(x.ravel()).reshape(x.shape)
+    codes, scales = oracle_mod.quantize_e4m3_rows(xb, 64)
+    assert np.all(scales == 1.0)
+    ref = torch.from_numpy(bits_to_f32(xb)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, ref)
+
+
+def test_row_quantize_is_invariant_to_powers_of_two(oracle_mod):
+    rng = np.random.default_rng(6)
+    x = bf16_bits(rng.standard_normal(8 * 96).astype(np.float32)).reshape(8, 96)
+    c0, s0 = oracle_mod.quantize_e4m3_rows(x, 96)
+    for m in (-20, -3, 5, 30):
+        xm = bf16_bits((bits_to_f32(x) * np.float32(2.0 ** m)).ravel()).reshape(x.shape)
+        cm, sm = oracle_mod.quantize_e4m3_rows(xm, 96)
+        assert np.array_equal(cm, c0)
+        assert np.all(sm == s0 * np.float32(2.0 ** m))
+
+
+def test_row_quantize_error_bound_and_zero_rows(oracle_mod):
+    rng = np.random.default_rng(8)
+    x = (rng.standard_normal((20, 128)) * rng.lognormal(0, 3, (20, 1))).astype(np.float32)
+    x[5] = 0.0
+    xb = bf16_bits(x.ravel()).reshape(x.shape)
+    codes, scales = oracle_mod.quantize_e4m3_rows(xb, 128)
+    assert scales[5] == 1.0 and np.all(codes[5] == 0)
+    xf = bits_to_f32(xb).astype(np.float64)
+    dec = np.vectorize(oracle_mod.e4m3_to_f32)(codes).astype(np.float64) * scales[:, None]
+    # 3 mantissa bits: half an ulp is 2^-4 relative for normals; subnormal step 2^-9
+    bound = np.maximum(2.0 ** -4 * np.abs(xf), 2.0 ** -10 * scales[:, None]) * (1 + 2.0 ** -20)
+    assert np.all(np.abs(dec - xf) <= bound)
+
+
+def test_combine_scaled_unit_scales_equal_plain_fp8(oracle_mod):
+    w = W.C2
+    x = W.make_inputs(w)
+    plan = oracle_mod.route(w.ep_size, w.num_experts, w.top_k, w.tokens_per_rank,
+                            x.token_selected_experts.numpy(), x.local_num_tokens)
+    q = oracle_mod.quantize_e4m3(x.expert_output.view(torch.int16).numpy().view(np.uint16))
+    ones = np.ones((w.ep_size, w.ep_size * w.tokens_per_rank), np.float32)
+    a = oracle_mod.combine_scaled(plan, q, ones, w.hidden)
+    b = oracle_mod.combine(plan, q, w.hidden, input_is_e4m3=True)
+    assert np.array_equal(a, b)
+
+
+def test_combine_scaled_hand_example(oracle_mod):
+    # token (0, 0) -> ranks {0, 1}; codes 1.0 (0x38) with scales 0.5 and 2: 0.5 + 2 = 2.5
+    ids = np.array([[[0, 2]], [[0, 0]]], np.int32)
+    plan = oracle_mod.route(2, 4, 2, 1, ids, np.array([1, 0], np.int32))
+    codes = np.zeros((2, 2, 4), np.uint8)
+    codes[0, 0, :] = 0x38
+    codes[1, 0, :] = 0x38
+    sc = np.array([[0.5, 1.0], [2.0, 1.0]], np.float32)
+    out = oracle_mod.combine_scaled(plan, codes, sc, 4)
+    assert np.all(bits_to_f32(out[0, 0]) == 2.5)
+
+
+def test_combine_scaled_uses_fused_multiply_add(oracle_mod):
+    """Rank 0's row: code -1.875 (0xBF) with scale 1; rank 1's row: 1.875 (0x3F)
+    with scale 1 + 2^-23.  fmaf(1.875, 1 + 2^-23, -1.875) is exactly
+    1.875 * 2^-23; rounding the product first would give 2^-22."""
+    ids = np.array([[[0, 2]], [[0, 0]]], np.int32)
+    plan = oracle_mod.route(2, 4, 2, 1, ids, np.array([1, 0], np.int32))
+    codes = np.zeros((2, 2, 1), np.uint8)
+    codes[0, 0, 0] = 0xBF
+    codes[1, 0, 0] = 0x3F
+    sc = np.array([[1.0, 1.0], [1.0 + 2.0 ** -23, 1.0]], np.float32)
+    out = oracle_mod.combine_scaled(plan, codes, sc, 1)
+    assert bits_to_f32(out[0, 0])[0] == 1.875 * 2.0 ** -23
