@@ -33,6 +33,9 @@
  *          past a source's token count keep expert id num_experts.
  *   [OSCu] flashinfer.moe_ep.NVLinkOneSidedConfig, `use_low_precision_combine`:
  *          combine payloads travel as FP8.
+ *   [AGRS] vllm.distributed.device_communicators.all2all, AgRsAll2AllManager:
+ *          dispatch as an all-gather of every rank's rows, combine as a
+ *          reduce-scatter (each rank gets its own rows summed over all ranks).
  *   [TSCi] flashinfer.moe_ep.NVLinkTwoSidedAlltoAll, combine(): its input rows
  *          are "already weighted and reduced over this rank's local experts";
  *          oracle_expert_reduce states that step.
@@ -433,6 +436,61 @@ void oracle_combine_scaled(int ep_size, int top_k, int tokens_per_rank, int hidd
                 acc = fmaf(oracle_e4m3_to_f32(expert_output[row * hidden + h]), row_scales[row], acc);
             }
             out[s * hidden + h] = oracle_bf16_from_f32(acc);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Dense variant: all-gather dispatch and reduce-scatter combine [AGRS].      */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Every live rank receives every token of every live source rank:
+ * recv[d][r*tpr + t] = in[r][t] for live d, live r, t < n[r].  Other rows
+ * are left as they were.  (The rank-major slot layout is kept, so that the
+ * two variants read and write the same arrays.)
+ */
+void oracle_allgather(int ep_size, int tokens_per_rank, int64_t row_bytes,
+                      const int32_t* local_num_tokens, const uint64_t* active_rank_mask,
+                      const uint8_t* in, uint8_t* recv)
+{
+    const int ep = ep_size, tpr = tokens_per_rank;
+    const int64_t slots = (int64_t)ep * tpr;
+    for (int r = 0; r < ep; ++r) {
+        if (!rank_is_live(active_rank_mask, r)) continue;
+        for (int t = 0; t < local_num_tokens[r]; ++t) {
+            const int64_t s = (int64_t)r * tpr + t;
+            for (int d = 0; d < ep; ++d) {
+                if (!rank_is_live(active_rank_mask, d)) continue;
+                memcpy(recv + ((int64_t)d * slots + s) * row_bytes, in + s * row_bytes,
+                       (size_t)row_bytes);
+            }
+        }
+    }
+}
+
+/*
+ * out[r][t][h] = bf16( fp32 sum over live ranks d, ascending, from +0.0f, of
+ * x[d][r*tpr + t][h] ) for live r, t < n[r]; other rows are left as they were.
+ */
+void oracle_reduce_scatter(int ep_size, int tokens_per_rank, int hidden,
+                           const int32_t* local_num_tokens, const uint64_t* active_rank_mask,
+                           const uint16_t* x, uint16_t* out)
+{
+    const int ep = ep_size, tpr = tokens_per_rank;
+    const int64_t slots = (int64_t)ep * tpr;
+    for (int r = 0; r < ep; ++r) {
+        if (!rank_is_live(active_rank_mask, r)) continue;
+        for (int t = 0; t < local_num_tokens[r]; ++t) {
+            const int64_t s = (int64_t)r * tpr + t;
+            for (int h = 0; h < hidden; ++h) {
+                float acc = 0.0f;
+                for (int d = 0; d < ep; ++d) {
+                    if (!rank_is_live(active_rank_mask, d)) continue;
+                    acc = acc + oracle_bf16_to_f32(x[((int64_t)d * slots + s) * hidden + h]);
+                }
+                out[s * hidden + h] = oracle_bf16_from_f32(acc);
+            }
         }
     }
 }

@@ -63,6 +63,10 @@ def _load():
         lib.oracle_quantize_e4m3_rows.restype = None
         lib.oracle_combine_scaled.argtypes = [I, I, I, I, P, P, P, P, P]
         lib.oracle_combine_scaled.restype = None
+        lib.oracle_allgather.argtypes = [I, I, I64, P, P, P, P]
+        lib.oracle_allgather.restype = None
+        lib.oracle_reduce_scatter.argtypes = [I, I, I, P, P, P, P]
+        lib.oracle_reduce_scatter.restype = None
         lib.oracle_quantize_e4m3.argtypes = [P, P, I64]
         lib.oracle_quantize_e4m3.restype = None
         lib.oracle_bf16_from_f32.argtypes = [ctypes.c_float]
@@ -255,6 +259,39 @@ def combine_scaled(plan: RoutePlan, codes, row_scales, hidden, out_init=None):
     return out
 
 
+def allgather(ep_size, tokens_per_rank, local_num_tokens, payload, active_rank_mask=None,
+              recv_init=None):
+    """Dense dispatch: uint8 ``[ep, ep*tpr, row_bytes]`` (see ``oracle_allgather``)."""
+    lib = _load()
+    ep, tpr = ep_size, tokens_per_rank
+    src = np.ascontiguousarray(payload).view(np.uint8).reshape(ep, tpr, -1)
+    rb = src.shape[2]
+    n = np.ascontiguousarray(local_num_tokens, dtype=np.int32).reshape(ep)
+    if recv_init is None:
+        recv = np.full((ep, ep * tpr, rb), 0xCD, np.uint8)
+    else:
+        recv = np.array(recv_init, dtype=np.uint8, copy=True).reshape(ep, ep * tpr, rb)
+    lib.oracle_allgather(ep, tpr, rb, _ptr(n), _ptr(_mask_words(active_rank_mask, ep)),
+                         _ptr(src), _ptr(recv))
+    return recv
+
+
+def reduce_scatter(ep_size, tokens_per_rank, hidden, local_num_tokens, x, active_rank_mask=None,
+                   out_init=None):
+    """Dense combine: bf16 bits ``[ep, tpr, hidden]`` (see ``oracle_reduce_scatter``)."""
+    lib = _load()
+    ep, tpr = ep_size, tokens_per_rank
+    xx = np.ascontiguousarray(x).view(np.uint16).reshape(ep, ep * tpr, hidden)
+    n = np.ascontiguousarray(local_num_tokens, dtype=np.int32).reshape(ep)
+    if out_init is None:
+        out = np.full((ep, tpr, hidden), 0xEEEE, np.uint16)
+    else:
+        out = np.array(out_init, dtype=np.uint16, copy=True).reshape(ep, tpr, hidden)
+    lib.oracle_reduce_scatter(ep, tpr, hidden, _ptr(n), _ptr(_mask_words(active_rank_mask, ep)),
+                              _ptr(xx), _ptr(out))
+    return out
+
+
 def quantize_e4m3(bf16_bits):
     """E4M3 bytes of bf16 values (round to nearest even, saturate to +-448)."""
     lib = _load()
@@ -281,6 +318,7 @@ def e4m3_to_f32(b: int) -> float:
 
 
 __all__ = ["build", "route", "dispatch_payload", "eplb_gather", "combine", "expert_reduce",
-           "combine_experts", "quantize_e4m3_rows", "combine_scaled",
+           "combine_experts", "quantize_e4m3_rows", "combine_scaled", "allgather",
+           "reduce_scatter",
            "quantize_e4m3", "bf16_from_f32", "bf16_to_f32", "e4m3_from_f32",
            "e4m3_to_f32", "RoutePlan"]

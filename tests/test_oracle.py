@@ -597,3 +597,62 @@ def test_combine_scaled_uses_fused_multiply_add(oracle_mod):
     sc = np.array([[1.0, 1.0], [1.0 + 2.0 ** -23, 1.0]], np.float32)
     out = oracle_mod.combine_scaled(plan, codes, sc, 1)
     assert bits_to_f32(out[0, 0])[0] == 1.875 * 2.0 ** -23
+
+
+# --------------------------------------------------------------------------- #
+# Dense variant: all-gather dispatch, reduce-scatter combine
+# --------------------------------------------------------------------------- #
+
+def test_allgather_equals_dispatch_when_every_rank_is_an_owner(oracle_mod):
+    """With top_k = ep_size and one expert of every rank per token, the
+    rank-major dispatch sends each token to every rank: it must equal the
+    all-gather (two different definitions of the same movement)."""
+    ep, E, tpr, rb = 4, 16, 9, 24
+    rng = np.random.default_rng(12)
+    ids = np.zeros((ep, tpr, ep), np.int32)
+    for r in range(ep):
+        for t in range(tpr):
+            ids[r, t] = rng.permutation([d * 4 + rng.integers(0, 4) for d in range(ep)])
+    n = np.array([9, 3, 0, 7], np.int32)
+    data = rng.integers(0, 256, (ep, tpr, rb)).astype(np.uint8)
+    plan = oracle_mod.route(ep, E, ep, tpr, ids, n)
+    assert np.all(plan.num_dst[plan.num_dst >= 0] == ep)
+    assert np.array_equal(oracle_mod.dispatch_payload(plan, data),
+                          oracle_mod.allgather(ep, tpr, n, data))
+    mask = np.array([0b1011], np.uint64)
+    plan = oracle_mod.route(ep, E, ep, tpr, ids, n, mask)
+    assert np.array_equal(oracle_mod.dispatch_payload(plan, data),
+                          oracle_mod.allgather(ep, tpr, n, data, mask))
+
+
+@pytest.mark.parametrize("w", [W.C1, W.C5], ids=lambda w: w.name)
+def test_reduce_scatter_equals_combine_of_zero_padded_rows(oracle_mod, w):
+    """The reduce-scatter of rows that are +0.0 wherever the rank-major plan
+    sends nothing equals the combine (adding +0.0 to an fp32 sum that is never
+    -0.0 changes nothing)."""
+    x = W.make_inputs(w)
+    ep, tpr, H = w.ep_size, w.tokens_per_rank, w.hidden
+    plan = oracle_mod.route(ep, w.num_experts, w.top_k, tpr, x.token_selected_experts.numpy(),
+                            x.local_num_tokens, x.active_rank_mask)
+    xo = x.expert_output.view(torch.int16).numpy().view(np.uint16).copy()
+    for d in range(ep):
+        if d in w.masked_ranks:
+            continue
+        xo[d][plan.recv_valid[d] != 1] = 0
+    a = oracle_mod.reduce_scatter(ep, tpr, H, x.local_num_tokens, xo, x.active_rank_mask)
+    b = oracle_mod.combine(plan, xo, H)
+    assert np.array_equal(a, b)
+
+
+def test_reduce_scatter_hand_example(oracle_mod):
+    # 3 ranks, 1 token each, rank 1 masked off: out[r] = x[0][r] + x[2][r]
+    x = np.zeros((3, 3, 2), np.float32)
+    for d in range(3):
+        for s in range(3):
+            x[d, s] = [10.0 ** d, s + 0.5]
+    xb = bf16_bits(x.ravel()).reshape(x.shape)
+    out = oracle_mod.reduce_scatter(3, 1, 2, np.array([1, 1, 1], np.int32), xb,
+                                    np.array([0b101], np.uint64))
+    assert bits_to_f32(out[0, 0]).tolist() == [101.0, 1.0]
+    assert bits_to_f32(out[2, 0]).tolist() == [101.0, 5.0]
+    assert np.all(out[1, 0] == 0xEEEE)
