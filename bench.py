@@ -327,6 +327,9 @@ def run_ours(args):
     xo = x.expert_output.to(device)
     xo8 = ep_a2a.quantize_e4m3(xo)
     experts = args.combine == "experts"
+    scaled = args.combine == "fp8s"
+    if scaled:
+        codes, row_scales = ep_a2a.quantize_e4m3_rows(xo)
     if experts:
         # one bf16 row per (token, slot), drawn on the device (seeded)
         gen = torch.Generator(device=device).manual_seed(w.seed + 77)
@@ -345,10 +348,30 @@ def run_ours(args):
     fp8 = args.combine == "fp8"
     comb_in = xo8 if fp8 else xo
 
+    dense = args.variant == "agrs"
+    if dense:
+        # the all-gather writes into the same receive arrays the rank-major
+        # dispatch uses (taken from one dispatch result)
+        res0 = comm.dispatch(ids, n, payloads, tpr, stats, mask, views=False)
+        recv_ptrs = [res0.recv_payloads[i] for i in range(len(payloads))]
+        pay_ptrs = [p.data_ptr() for p in payloads]
+        rows = w.payload_row_bytes()
+        dense_calls = [
+            lambda: ep_a2a.ep_a2a_allgather(w.ep_size, tpr, n, pay_ptrs, rows, recv_ptrs,
+                                            res0.rank_stride_bytes, mask),
+            lambda: ep_a2a.ep_a2a_reduce_scatter(w.ep_size, tpr, w.hidden, n, xo.data_ptr(),
+                                                 out.data_ptr(), mask)]
+
     def step():
+        if dense:
+            for call in dense_calls:
+                call()
+            return
         comm.dispatch(ids, n, payloads, tpr, stats, mask, views=False)
         if experts:
             comm.combine_experts(wts, y, out)
+        elif scaled:
+            comm.combine_scaled(codes, row_scales, out)
         else:
             comm.combine(comb_in, out)
 
@@ -367,7 +390,11 @@ def run_ours(args):
         alive = np.array([r not in w.masked_ranks for r in range(w.ep_size)] + [False])
         exists = (np.arange(tpr)[None, :] < n[:, None]) & alive[:w.ep_size, None]
         live_slots = int((alive[owner] & exists[:, :, None]).sum())
-    by = algorithmic_bytes(w, n_tok, sum_d, live, fp8, live_slots)
+    if dense:       # every existing token goes to, and is summed over, every live rank
+        sum_d = n_tok * live
+    by = algorithmic_bytes(w, n_tok, sum_d, live, fp8 or scaled, live_slots)
+    if scaled:      # the row scales travel with the codes
+        by = dataclasses.replace(by, combine=by.combine + sum_d * 4, step=by.step + sum_d * 4)
 
     clocks = ClockSampler(local)
     flush_buf = None
@@ -381,9 +408,17 @@ def run_ours(args):
             if flush_buf is not None:
                 flush_buf.zero_()
             step()
-        run_timed(flushed_step, args.steps, args.warmup, CudaTimer(stream), dist, device,
-                  on_start=lambda: ep_a2a.ep_a2a_profile_start(comm.handle, 4 * args.steps + 8))
-        kt = ep_a2a.ep_a2a_profile_stop(comm.handle)
+        if dense:
+            for _ in range(args.warmup):
+                flushed_step()
+            kt = dense_call_times(dense_calls, args.steps, stream,
+                                  flush=(lambda: flush_buf.zero_()) if flush_buf is not None
+                                  else None)
+        else:
+            run_timed(flushed_step, args.steps, args.warmup, CudaTimer(stream), dist, device,
+                      on_start=lambda: ep_a2a.ep_a2a_profile_start(comm.handle,
+                                                                   4 * args.steps + 8))
+            kt = ep_a2a.ep_a2a_profile_stop(comm.handle)
         timed_step = step
         if args.graph:
             graph = torch.cuda.CUDAGraph()
@@ -401,6 +436,10 @@ def run_ours(args):
         else:
             ms = run_timed(timed_step, args.steps, args.warmup, CudaTimer(stream), dist, device,
                            during=clocks)
+    elif dense:
+        ms = run_timed(step, args.steps, args.warmup, CudaTimer(stream), dist, device,
+                       during=clocks)
+        kt = dense_call_times(dense_calls, args.steps, stream)
     else:
         # the headline: K steps with nothing recorded between the kernels (an
         # event between two kernels would stop them from overlapping)
@@ -423,7 +462,8 @@ def run_ours(args):
         if cnt:
             per_kernel[name] = {"launches": cnt, "avg_ms": tot / cnt}
     kbytes = {"route_plan": by.route, "copy_bulk": by.copy, "copy_vec": by.copy,
-              "copy_staged": by.copy, "combine": by.combine, "combine_experts": by.combine}
+              "copy_staged": by.copy, "combine": by.combine, "combine_experts": by.combine,
+              "allgather": by.copy, "reduce_scatter": by.combine}
     for name, e in per_kernel.items():
         e["algorithmic_bytes"] = kbytes[name]
         e["achieved_gbs"] = kbytes[name] / (e["avg_ms"] / 1e3) / 1e9
@@ -434,7 +474,7 @@ def run_ours(args):
 
     # FP8 combine, timed alone on the same plan (context, not the headline)
     fp8_ctx = None
-    if not fp8 and not experts and args.fp8_steps > 0:
+    if not fp8 and not experts and not scaled and not dense and args.fp8_steps > 0:
         comm.dispatch(ids, n, payloads, tpr, stats, mask)
         t8 = run_timed(lambda: comm.combine(xo8, out), args.fp8_steps, 3, CudaTimer(stream),
                        dist, device, on_start=lambda: ep_a2a.ep_a2a_profile_start(
@@ -448,8 +488,8 @@ def run_ours(args):
 
     e2e = None
     if args.e2e_steps > 0:
-        e2e = run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws,
-                      y_dev=y if experts else None)
+        e2e = None if (scaled or dense) else run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws,
+                                          y_dev=y if experts else None)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -466,7 +506,7 @@ def run_ours(args):
                             f"extra {w.extra_bytes} B/token, EPLB stats, "
                             + ("combine of per-expert outputs (weighted local reduction "
                                "fused, fp32 accumulate)" if experts else
-                               f"{'FP8 E4M3' if fp8 else 'BF16'} combine (fp32 accumulate)"),
+                               f"{'FP8 E4M3 with a per-row fp32 scale' if scaled else 'FP8 E4M3' if fp8 else 'BF16'} combine (fp32 accumulate)"),
                 "tokens_per_step_per_gpu": n_tok, "mean_distinct_ranks": sum_d / n_tok,
                 "l2": ("512 MB L2 flush before every step, each step timed alone"
                        if args.l2_flush else "inputs larger than L2 (no flush)"),
@@ -475,6 +515,8 @@ def run_ours(args):
                 "kernel_times": "CUDA events around each launch, in a second timed region of "
                                 "the same K steps (events between kernels stop them overlapping)",
                 "parallelism": f"{ws} independent replicas" if ws > 1 else "1 GPU, virtual ranks",
+                "variant": ("dense: all-gather dispatch + reduce-scatter combine (vllm AgRs)"
+                            if dense else "rank-major dispatch + combine"),
             },
             "hbm": {"step_algorithmic_bytes": by.step, "achieved_gbs": step_gbs,
                     "peak_gbs": peak, "peak_kind": peak_kind, "frac": step_gbs / peak},
@@ -495,6 +537,24 @@ def run_ours(args):
     comm.destroy()
     if dist is not None:
         dist.destroy_process_group()
+
+
+def dense_call_times(calls, steps, stream, flush=None):
+    """{name: (launches, total ms)} of the dense variant's two calls, each
+    bracketed by CUDA events on the stream (they have no handle to profile)."""
+    import torch
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(steps)] for _ in calls]
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        for c, call in enumerate(calls):
+            evs[c][i][0].record(stream)
+            call()
+            evs[c][i][1].record(stream)
+    torch.cuda.synchronize()
+    return {name: (steps, sum(a.elapsed_time(b) for a, b in ev))
+            for name, ev in zip(("allgather", "reduce_scatter"), evs)}
 
 
 def run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws, y_dev=None):
@@ -634,9 +694,10 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--tokens-per-rank", type=int, default=0,
                     help="run the workload with this many tokens per rank (small profiling cases)")
-    ap.add_argument("--combine", choices=["bf16", "fp8", "experts"], default="bf16",
-                    help="combine input: bf16 or fp8 rows per rank, or bf16 outputs per "
-                         "(token, slot) reduced with topk_weights inside the combine")
+    ap.add_argument("--combine", choices=["bf16", "fp8", "fp8s", "experts"], default="bf16",
+                    help="combine input: bf16 / fp8 / fp8 with a per-row scale rows per rank, "
+                         "or bf16 outputs per (token, slot) reduced with topk_weights inside "
+                         "the combine")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--fp8-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -646,6 +707,9 @@ def main(argv=None):
                     help="time CUDA-graph replays of the step (small workloads)")
     ap.add_argument("--l2-flush", action="store_true",
                     help="flush L2 before every step and time steps alone (small workloads)")
+    ap.add_argument("--variant", choices=["rank-major", "agrs"], default="rank-major",
+                    help="agrs: the dense all-gather / reduce-scatter formulation of the same "
+                         "step, for comparison")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch")
     args = ap.parse_args(argv)

@@ -321,6 +321,166 @@ __global__ void __launch_bounds__(512) combine_experts_any_kernel(const CombineE
   }
 }
 
+// FP8 combine with one fp32 scale per row: acc = fmaf(decode(q), scale_d, acc)
+// over the token's destination ranks in ascending order.
+template <bool kVec>
+__global__ void __launch_bounds__(512) combine_scaled_kernel(const CombineArgs a,
+                                                             const float* __restrict__ scales) {
+  pdl_wait();
+  const int words = a.plan_stride / 8;
+  const int nvec = kVec ? a.H / 16 : 0;
+  if (kVec && a.prefetch && threadIdx.x == 0) prefetch_token_rows<1>(a, blockIdx.x);
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    if (kVec && a.prefetch && threadIdx.x == 0) prefetch_token_rows<1>(a, tok + gridDim.x);
+    const int nd = a.plan_nd[tok];
+    if (nd == kNoToken) continue;
+    const uint64_t* row = reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    const uint64_t w0 = row[0];
+    const uint64_t w1 = words > 1 ? row[1] : 0;
+    const uint64_t w2 = words > 2 ? row[2] : 0;
+    const uint64_t w3 = words > 3 ? row[3] : 0;
+    uint16_t* out = a.out + tok * (int64_t)a.H;
+    if (kVec) {
+      const uint8_t* xt = a.x + tok * (int64_t)a.H;
+      const int64_t rank_stride = a.ntok * (int64_t)a.H;
+      for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+        float acc[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
+        for (int c0 = 0; c0 < nd; c0 += 8) {
+          uint4 raw[8];
+          float sc[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (c0 + i < nd) {
+              const int d = dst_rank(w0, w1, w2, w3, c0 + i);
+              raw[i] = ld_stream_v4(xt + (int64_t)d * rank_stride + (int64_t)v * 16);
+              sc[i] = scales[(int64_t)d * a.ntok + tok];
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (c0 + i >= nd) continue;
+            const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+                    (__nv_fp8x2_storage_t)((w[q] >> (16 * h)) & 0xFFFFu), __NV_E4M3);
+                __half_raw lo, hi;
+                lo.x = hr.x;
+                hi.x = hr.y;
+                float& a0 = acc[4 * q + 2 * h];
+                float& a1 = acc[4 * q + 2 * h + 1];
+                a0 = __fmaf_rn(__half2float(__half(lo)), sc[i], a0);
+                a1 = __fmaf_rn(__half2float(__half(hi)), sc[i], a1);
+              }
+            }
+          }
+        }
+        uint4* o = reinterpret_cast<uint4*>(out + (int64_t)v * 16);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint4 pk;
+          pk.x = pack_bf16x2(acc[8 * q + 0], acc[8 * q + 1]);
+          pk.y = pack_bf16x2(acc[8 * q + 2], acc[8 * q + 3]);
+          pk.z = pack_bf16x2(acc[8 * q + 4], acc[8 * q + 5]);
+          pk.w = pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]);
+          o[q] = pk;
+        }
+      }
+    } else {
+      for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
+        float acc = 0.0f;
+        for (int i = 0; i < nd; ++i) {
+          const int d = dst_rank(w0, w1, w2, w3, i);
+          const int64_t r = (int64_t)d * a.ntok + tok;
+          const __half_raw hr =
+              __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)a.x[r * a.H + h], __NV_E4M3);
+          acc = __fmaf_rn(__half2float(__half(hr)), scales[r], acc);
+        }
+        out[h] = (uint16_t)f32_to_bf16_bits(acc);
+      }
+    }
+  }
+}
+
+// One scale per row: amax = max |x|, scale = amax / 448, inv = 448 / amax
+// (each rounded to nearest; 1 and 1 for a zero row), code = E4M3(x * inv),
+// nearest even, saturating.  One CTA per row; the row stays in registers
+// between the amax pass and the encode pass when it fits (kVec), else it is
+// read twice.
+template <bool kVec>
+__global__ void __launch_bounds__(256) quantize_e4m3_rows_kernel(const uint16_t* __restrict__ in,
+                                                                 uint8_t* __restrict__ out,
+                                                                 float* __restrict__ scales,
+                                                                 int64_t rows, int hidden) {
+  constexpr int kMaxV = 4;            // 16-byte vectors per thread held in registers
+  __shared__ float s_amax[8];
+  __shared__ float s_scale, s_inv;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const uint16_t* x = in + r * hidden;
+    float amax = 0.0f;
+    uint4 v[kMaxV];
+    if (kVec) {
+#pragma unroll
+      for (int i = 0; i < kMaxV; ++i) {
+        const int c = threadIdx.x + i * 256;
+        if (c * 8 < hidden) {
+          v[i] = reinterpret_cast<const uint4*>(x)[c];
+          const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            amax = fmaxf(amax, fabsf(bf16_bits_to_f32(w[q] & 0xFFFFu)));
+            amax = fmaxf(amax, fabsf(bf16_bits_to_f32(w[q] >> 16)));
+          }
+        }
+      }
+    } else {
+      for (int h = threadIdx.x; h < hidden; h += 256)
+        amax = fmaxf(amax, fabsf(bf16_bits_to_f32(x[h])));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    if ((threadIdx.x & 31) == 0) s_amax[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float m = 0.0f;
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, s_amax[i]);
+      s_scale = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
+      s_inv = m > 0.0f ? __fdiv_rn(448.0f, m) : 1.0f;
+      scales[r] = s_scale;
+    }
+    __syncthreads();
+    const float inv = s_inv;
+    uint8_t* o = out + r * hidden;
+    if (kVec) {
+#pragma unroll
+      for (int i = 0; i < kMaxV; ++i) {
+        const int c = threadIdx.x + i * 256;
+        if (c * 8 < hidden) {
+          const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+          uint32_t pk[2] = {0u, 0u};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = make_float2(__fmul_rn(bf16_bits_to_f32(w[q] & 0xFFFFu), inv),
+                                         __fmul_rn(bf16_bits_to_f32(w[q] >> 16), inv));
+            const uint32_t pair = (uint32_t)__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+            pk[q >> 1] |= pair << (16 * (q & 1));
+          }
+          reinterpret_cast<uint2*>(o)[c] = make_uint2(pk[0], pk[1]);
+        }
+      }
+    } else {
+      for (int h = threadIdx.x; h < hidden; h += 256)
+        o[h] = (uint8_t)__nv_cvt_float_to_fp8(__fmul_rn(bf16_bits_to_f32(x[h]), inv),
+                                              __NV_SATFINITE, __NV_E4M3);
+    }
+    __syncthreads();   // s_amax / s_inv are rewritten for the next row
+  }
+}
+
 // bf16 -> E4M3, round to nearest even, saturating (satfinite).
 __global__ void quantize_e4m3_kernel(const uint16_t* __restrict__ in, uint8_t* __restrict__ out,
                                      int64_t n, bool vec) {
@@ -370,6 +530,27 @@ cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, int threads
   }
   if (fp8) return launch_kernel(combine_scalar_kernel<true>, g, b, 0, stream, pdl, a);
   return launch_kernel(combine_scalar_kernel<false>, g, b, 0, stream, pdl, a);
+}
+
+cudaError_t launch_combine_scaled(const CombineArgs& a, const float* scales, bool vec,
+                                  int threads, int grid, cudaStream_t stream, bool pdl) {
+  const dim3 g(grid), b(threads);
+  if (vec) return launch_kernel(combine_scaled_kernel<true>, g, b, 0, stream, pdl, a, scales);
+  return launch_kernel(combine_scaled_kernel<false>, g, b, 0, stream, pdl, a, scales);
+}
+
+cudaError_t launch_quantize_e4m3_rows(const uint16_t* in, uint8_t* out, float* scales,
+                                      int64_t rows, int hidden, cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  const bool vec = hidden % 8 == 0 && hidden <= 4 * 256 * 8 &&
+                   reinterpret_cast<uintptr_t>(in) % 16 == 0 &&
+                   reinterpret_cast<uintptr_t>(out) % 8 == 0;
+  const int grid = (int)std::min<int64_t>(rows, 148 * 8);
+  if (vec)
+    quantize_e4m3_rows_kernel<true><<<grid, 256, 0, stream>>>(in, out, scales, rows, hidden);
+  else
+    quantize_e4m3_rows_kernel<false><<<grid, 256, 0, stream>>>(in, out, scales, rows, hidden);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, int threads, int grid,

@@ -640,6 +640,48 @@ EP_API ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle h, const float* topk_w
   return EP_A2A_OK;
 }
 
+EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_output_e4m3,
+                                           const float* row_scales, void* output,
+                                           void* stream_v) {
+  ep_a2a_status st = check_handle(h);
+  if (st != EP_A2A_OK) return st;
+  if (!h->have_plan) return fail(EP_A2A_ERR_NO_PLAN, "combine needs a preceding dispatch");
+  if (!expert_output_e4m3 || !row_scales || !output)
+    return fail(EP_A2A_ERR_INVALID_ARG, "expert_output / row_scales / output is NULL");
+  CombineArgs a;
+  a.plan_nd = h->ws + h->L.off_plan_nd;
+  a.plan_dst = h->ws + h->L.off_plan_dst;
+  a.x = static_cast<const uint8_t*>(expert_output_e4m3);
+  a.out = static_cast<uint16_t*>(output);
+  a.ntok = (int64_t)h->p.ep_size * h->last_tpr;
+  a.H = h->p.hidden_size;
+  a.plan_stride = h->L.plan_stride;
+  a.prefetch = h->combine_prefetch != 0 ? 1 : 0;   // default: on, as for the FP8 combine
+  const bool vec = a.H % 16 == 0 && aligned(expert_output_e4m3, 16) && aligned(output, 16);
+  const int grid = (int)std::max<int64_t>(
+      1, std::min<int64_t>(a.ntok, (int64_t)h->num_sms * h->combine_ctas_per_sm));
+  const int threads = h->combine_threads > 0 ? h->combine_threads : 64;
+  const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);
+  cudaError_t e = launch_combine_scaled(a, row_scales, vec, threads, grid,
+                                        (cudaStream_t)stream_v, h->pdl != 0);
+  prof_end(h, slot, (cudaStream_t)stream_v);
+  if (e != cudaSuccess) return cuda_fail(e, "scaled combine kernel launch");
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_quantize_e4m3_rows(const void* bf16_in, void* e4m3_out,
+                                               float* row_scales, int64_t rows, int32_t hidden,
+                                               void* stream) {
+  if (rows < 0 || hidden < 1) return fail(EP_A2A_ERR_INVALID_ARG, "rows < 0 or hidden < 1");
+  if (rows > 0 && (!bf16_in || !e4m3_out || !row_scales))
+    return fail(EP_A2A_ERR_INVALID_ARG, "NULL buffer");
+  cudaError_t e = launch_quantize_e4m3_rows(static_cast<const uint16_t*>(bf16_in),
+                                            static_cast<uint8_t*>(e4m3_out), row_scales, rows,
+                                            hidden, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "row quantize kernel launch");
+  return EP_A2A_OK;
+}
+
 EP_API ep_a2a_status ep_a2a_quantize_e4m3(const void* bf16_in, void* e4m3_out, int64_t n,
                                           void* stream) {
   if (n < 0) return fail(EP_A2A_ERR_INVALID_ARG, "n < 0");

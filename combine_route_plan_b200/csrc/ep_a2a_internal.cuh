@@ -122,6 +122,11 @@ struct CombineExpertsArgs {
 cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, int threads, int grid,
                                    cudaStream_t stream, bool pdl);
 cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n, cudaStream_t stream);
+cudaError_t launch_quantize_e4m3_rows(const uint16_t* in, uint8_t* out, float* scales,
+                                      int64_t rows, int hidden, cudaStream_t stream);
+// FP8 combine with one fp32 scale per row (scales [ep, ep*tpr]).
+cudaError_t launch_combine_scaled(const CombineArgs& a, const float* scales, bool vec,
+                                  int threads, int grid, cudaStream_t stream, bool pdl);
 cudaError_t launch_wait_timeout_probe(uint32_t* err, unsigned long long limit_ns,
                                       cudaStream_t stream);
 

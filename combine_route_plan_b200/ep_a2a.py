@@ -97,6 +97,10 @@ def _load():
         "ep_a2a_combine": (st, [VP, VP, ctypes.c_int, VP, VP]),
         "ep_a2a_quantize_e4m3": (st, [VP, VP, I64, VP]),
         "ep_a2a_combine_experts": (st, [VP, VP, VP, VP, VP]),
+        "ep_a2a_combine_scaled": (st, [VP, VP, VP, VP, VP]),
+        "ep_a2a_quantize_e4m3_rows": (st, [VP, VP, VP, I64, I32, VP]),
+        "ep_a2a_allgather": (st, [I32, I32, VP, VP, P(VP), P(I64), I32, P(VP), I64, VP]),
+        "ep_a2a_reduce_scatter": (st, [I32, I32, I32, VP, VP, VP, VP, VP]),
         "ep_a2a_get_status": (st, [VP, VP]),
         "ep_a2a_debug_wait_probe": (st, [VP, I64, VP]),
         "ep_a2a_set_option": (st, [VP, ctypes.c_int, I64]),
@@ -179,6 +183,56 @@ def ep_a2a_combine_experts(handle: int, topk_weights_ptr: int, expert_out_ptr: i
     _check(lib.ep_a2a_combine_experts(ctypes.c_void_p(handle), ctypes.c_void_p(topk_weights_ptr),
                                       ctypes.c_void_p(expert_out_ptr), ctypes.c_void_p(output_ptr),
                                       ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def ep_a2a_combine_scaled(handle: int, e4m3_ptr: int, scales_ptr: int, output_ptr: int,
+                          stream=None):
+    _check(lib.ep_a2a_combine_scaled(ctypes.c_void_p(handle), ctypes.c_void_p(e4m3_ptr),
+                                     ctypes.c_void_p(scales_ptr), ctypes.c_void_p(output_ptr),
+                                     ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def ep_a2a_quantize_e4m3_rows(bf16_ptr: int, e4m3_ptr: int, scales_ptr: int, rows: int,
+                              hidden: int, stream=None):
+    _check(lib.ep_a2a_quantize_e4m3_rows(ctypes.c_void_p(bf16_ptr), ctypes.c_void_p(e4m3_ptr),
+                                         ctypes.c_void_p(scales_ptr), int(rows), int(hidden),
+                                         ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def _host_i32(values):
+    arr = (ctypes.c_int32 * len(values))(*[int(v) for v in values])
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def _host_mask(active_rank_mask):
+    if active_rank_mask is None:
+        return None, None
+    words = [int(w) for w in np.asarray(active_rank_mask, dtype=np.uint64)] + [0] * RANK_MASK_WORDS
+    arr = (ctypes.c_uint64 * RANK_MASK_WORDS)(*words[:RANK_MASK_WORDS])
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def ep_a2a_allgather(ep_size: int, tokens_per_rank: int, local_num_tokens, payload_ptrs,
+                     payload_row_bytes, recv_ptrs, recv_rank_stride_bytes: int,
+                     active_rank_mask=None, stream=None):
+    n_ptr, n_keep = _host_i32(local_num_tokens)
+    m_ptr, m_keep = _host_mask(active_rank_mask)
+    k = max(1, len(payload_ptrs))
+    src = (ctypes.c_void_p * k)(*[ctypes.c_void_p(p) for p in payload_ptrs])
+    dst = (ctypes.c_void_p * k)(*[ctypes.c_void_p(p) for p in recv_ptrs])
+    rb = (ctypes.c_int64 * k)(*[int(b) for b in payload_row_bytes])
+    _check(lib.ep_a2a_allgather(ep_size, tokens_per_rank, n_ptr, m_ptr, src, rb,
+                                len(payload_ptrs), dst, int(recv_rank_stride_bytes),
+                                ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def ep_a2a_reduce_scatter(ep_size: int, tokens_per_rank: int, hidden: int, local_num_tokens,
+                          x_ptr: int, out_ptr: int, active_rank_mask=None, stream=None):
+    n_ptr, n_keep = _host_i32(local_num_tokens)
+    m_ptr, m_keep = _host_mask(active_rank_mask)
+    _check(lib.ep_a2a_reduce_scatter(ep_size, tokens_per_rank, hidden, n_ptr, m_ptr,
+                                     ctypes.c_void_p(x_ptr), ctypes.c_void_p(out_ptr),
+                                     ctypes.c_void_p(_stream_ptr(stream))))
 
 
 def ep_a2a_quantize_e4m3(bf16_ptr: int, e4m3_ptr: int, n: int, stream=None):
@@ -382,6 +436,25 @@ class EpA2A:
         ep_a2a_combine_experts(self.handle, w.data_ptr(), y.data_ptr(), output.data_ptr(), stream)
         return output
 
+    def combine_scaled(self, codes: torch.Tensor, row_scales: torch.Tensor,
+                       output: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """codes E4M3 [ep, ep*tpr, hidden]; row_scales fp32 [ep, ep*tpr]; bf16 out."""
+        tpr = self.last_tokens_per_rank
+        assert tpr is not None, "combine needs a preceding dispatch"
+        rows = self.ep_size * self.ep_size * tpr
+        assert codes.is_cuda and codes.is_contiguous() and codes.element_size() == 1
+        assert codes.numel() == rows * self.hidden_size, codes.shape
+        assert row_scales.is_cuda and row_scales.dtype == torch.float32
+        assert row_scales.is_contiguous() and row_scales.numel() == rows, row_scales.shape
+        if output is None:
+            output = torch.empty((self.ep_size, tpr, self.hidden_size), dtype=torch.bfloat16,
+                                 device=codes.device)
+        assert output.is_cuda and output.dtype == torch.bfloat16 and output.is_contiguous()
+        assert output.numel() == self.ep_size * tpr * self.hidden_size, output.shape
+        ep_a2a_combine_scaled(self.handle, codes.data_ptr(), row_scales.data_ptr(),
+                              output.data_ptr(), stream)
+        return output
+
     def get_status(self, stream=None) -> int:
         return ep_a2a_get_status(self.handle, stream)
 
@@ -394,6 +467,18 @@ class EpA2A:
                 lib.ep_a2a_destroy(ctypes.byref(self._h))
         except Exception:
             pass
+
+
+def quantize_e4m3_rows(x_bf16: torch.Tensor, stream=None):
+    """bf16 [..., hidden] -> (E4M3 codes as torch.float8_e4m3fn, fp32 scales [...])."""
+    assert x_bf16.is_cuda and x_bf16.dtype == torch.bfloat16 and x_bf16.is_contiguous()
+    hidden = x_bf16.shape[-1]
+    rows = x_bf16.numel() // hidden
+    codes = torch.empty(x_bf16.shape, dtype=torch.float8_e4m3fn, device=x_bf16.device)
+    scales = torch.empty(x_bf16.shape[:-1], dtype=torch.float32, device=x_bf16.device)
+    ep_a2a_quantize_e4m3_rows(x_bf16.data_ptr(), codes.data_ptr(), scales.data_ptr(), rows,
+                              hidden, stream)
+    return codes, scales
 
 
 def quantize_e4m3(x_bf16: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None):

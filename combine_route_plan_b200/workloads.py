@@ -12,7 +12,8 @@ dispatch formats; an extra per-token payload; EPLB statistics; a rank mask):
   c1  ep 4,  E 8,   k 2, 16 tokens/rank, hidden 128 BF16          (tiny, exhaustive)
   c2  ep 8,  E 256, k 8, 128 tokens/rank, hidden 7168 BF16        (decode step)
   c3  ep 16, E 256, k 8, 512 tokens/rank, Zipf(1.2) routing,
-      hidden 7168 as NVFP4 (run "nvfp4") or MXFP8 (run "mxfp8")   (quantized dispatch)
+      hidden 7168 as NVFP4 (run "nvfp4"), MXFP8 (run "mxfp8") or
+      DeepSeekFp8 (run "dsfp8")                                   (quantized dispatch)
   c4  ep 8,  E 256, k 8, 4096 tokens/rank, hidden 7168 BF16, extra 64 B,
       EPLB stats, BF16 and FP8-E4M3 combine                        (prefill step)
   c5  ep 64, E 256, k 8, runtime max 64, local_num_tokens ~ U[1, 64],
@@ -40,7 +41,7 @@ class Workload:
     top_k: int
     tokens_per_rank: int          # the step's runtime_max_tokens_per_rank
     hidden: int
-    dispatch_format: str          # "bf16" | "nvfp4" | "mxfp8"
+    dispatch_format: str          # "bf16" | "nvfp4" | "mxfp8" | "dsfp8"
     routing: str = "uniform"      # "uniform" | "zipf"
     zipf_s: float = 1.2
     ragged_tokens: bool = False   # local_num_tokens ~ U[1, tokens_per_rank]
@@ -75,6 +76,8 @@ class Workload:
             rows += [self.hidden // 2, self.hidden // 16]
         elif self.dispatch_format == "mxfp8":
             rows += [self.hidden, self.hidden // 32]
+        elif self.dispatch_format == "dsfp8":
+            rows += [self.hidden, self.hidden // 128 * 4]
         else:
             raise ValueError(self.dispatch_format)
         if self.extra_bytes:
@@ -96,12 +99,13 @@ C1 = Workload("c1_ep4_tiny", 1, 4, 8, 2, 16, 128, "bf16")
 C2 = Workload("c2_ep8_decode", 2, 8, 256, 8, 128, 7168, "bf16")
 C3_NVFP4 = Workload("c3_ep16_zipf_nvfp4", 3, 16, 256, 8, 512, 7168, "nvfp4", routing="zipf")
 C3_MXFP8 = Workload("c3_ep16_zipf_mxfp8", 3, 16, 256, 8, 512, 7168, "mxfp8", routing="zipf")
+C3_DSFP8 = Workload("c3_ep16_zipf_dsfp8", 3, 16, 256, 8, 512, 7168, "dsfp8", routing="zipf")
 C4 = Workload("c4_ep8_prefill", 4, 8, 256, 8, 4096, 7168, "bf16", extra_bytes=64,
               eplb=True, fp8_combine=True)
 C5 = Workload("c5_ep64_wide_masked", 5, 64, 256, 8, 64, 7168, "bf16", ragged_tokens=True,
               masked_ranks=(5, 17, 42))
 
-ALL = [C1, C2, C3_NVFP4, C3_MXFP8, C4, C5]
+ALL = [C1, C2, C3_NVFP4, C3_MXFP8, C4, C5, C3_DSFP8]
 BY_NAME = {w.name: w for w in ALL}
 
 
@@ -181,6 +185,18 @@ def _encode_mxfp8(x: torch.Tensor):
     return y.view(torch.uint8).view(ntok, H).contiguous(), scales.contiguous()
 
 
+def _encode_dsfp8(x: torch.Tensor):
+    """[ntok, H] fp32 -> (E4M3 elements [ntok, H] u8, fp32 block-128 scales [ntok, H/128 * 4] u8).
+
+    DeepSeek-style FP8: one fp32 scale per 128 consecutive elements, amax / 448."""
+    ntok, H = x.shape
+    blk = x.view(ntok, H // 128, 128)
+    scale = (blk.abs().amax(dim=2, keepdim=True) / 448.0).clamp_min(1e-30)
+    y = (blk / scale).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+    scales = scale.to(torch.float32).view(ntok, H // 128).contiguous()
+    return y.view(torch.uint8).view(ntok, H).contiguous(), scales.view(torch.uint8)
+
+
 def make_inputs(w: Workload, with_expert_output: bool = True) -> Inputs:
     """Draw every input of one step of workload ``w``."""
     gen = torch.Generator().manual_seed(w.seed)
@@ -203,6 +219,9 @@ def make_inputs(w: Workload, with_expert_output: bool = True) -> Inputs:
         payloads += [q.view(ep, tpr, -1), s.view(ep, tpr, -1)]
     elif w.dispatch_format == "mxfp8":
         q, s = _encode_mxfp8(hid)
+        payloads += [q.view(ep, tpr, -1), s.view(ep, tpr, -1)]
+    elif w.dispatch_format == "dsfp8":
+        q, s = _encode_dsfp8(hid)
         payloads += [q.view(ep, tpr, -1), s.view(ep, tpr, -1)]
     del hid
     if w.extra_bytes:

@@ -226,6 +226,57 @@ ep_a2a_status ep_a2a_quantize_e4m3(const void* bf16_in, void* e4m3_out, int64_t 
                                    void* stream);
 
 /*
+ * FP8 combine with one scale per row (flashinfer.moe_ep.NVLinkOneSidedConfig,
+ * use_low_precision_combine; the pages fix no scale convention, this is one):
+ * as ep_a2a_combine with E4M3 rows, each row (d, s) also carrying an fp32 scale:
+ *   out[src][t] = bf16( acc ),  acc = fmaf(decode(q[d][s]), row_scales[d][s], acc)
+ * over the token's destination ranks d in ascending order, from +0.0f.
+ *   expert_output_e4m3  device [ep, ep*tpr, hidden_size] E4M3 codes
+ *   row_scales          device fp32 [ep, ep*tpr] (only valid rows are read)
+ *   output              device bf16 [ep, tpr, hidden_size]
+ */
+ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle handle, const void* expert_output_e4m3,
+                                    const float* row_scales, void* output, void* stream);
+
+/*
+ * Rows to E4M3 with one scale per row, the sender side of the scaled FP8
+ * combine: per row of `hidden` bf16 values, amax = max |x|, scale = amax / 448
+ * and inv = 448 / amax (fp32, rounded to nearest; 1 and 1 for an all-zero row),
+ * code = E4M3(x * inv) rounded to nearest even and saturating.  Device
+ * pointers: bf16_in [rows, hidden], e4m3_out [rows, hidden], row_scales [rows].
+ */
+ep_a2a_status ep_a2a_quantize_e4m3_rows(const void* bf16_in, void* e4m3_out, float* row_scales,
+                                        int64_t rows, int32_t hidden, void* stream);
+
+/*
+ * Dense variant (vllm.distributed.device_communicators.all2all,
+ * AgRsAll2AllManager: dispatch by all-gather, combine by reduce-scatter), for
+ * comparison with the rank-major path on the same arrays; no handle, no plan.
+ *
+ * ep_a2a_allgather: every live rank receives every token of every live rank,
+ * recv_payloads[i] + d * recv_rank_stride_bytes + (src * tpr + t) * row_bytes[i]
+ * = payloads[i] + (src * tpr + t) * row_bytes[i] for live d, live src and
+ * t < local_num_tokens[src].  local_num_tokens and active_rank_mask (NULL = all
+ * live) are host arrays; payloads and recv_payloads are host arrays of device
+ * pointers (rank 0's receive array per payload); other rows are not written.
+ *
+ * ep_a2a_reduce_scatter: out[src][t] = bf16( fp32 sum over live ranks d,
+ * ascending, from +0.0f, of x[d][src * tpr + t] ) for live src and
+ * t < local_num_tokens[src]; x is device bf16 [ep, ep*tpr, hidden], out device
+ * bf16 [ep, tpr, hidden]; other rows are not written.
+ */
+ep_a2a_status ep_a2a_allgather(int32_t ep_size, int32_t tokens_per_rank,
+                               const int32_t* local_num_tokens,
+                               const uint64_t* active_rank_mask, const void* const* payloads,
+                               const int64_t* payload_row_bytes, int32_t num_payloads,
+                               void* const* recv_payloads, int64_t recv_rank_stride_bytes,
+                               void* stream);
+ep_a2a_status ep_a2a_reduce_scatter(int32_t ep_size, int32_t tokens_per_rank, int32_t hidden,
+                                    const int32_t* local_num_tokens,
+                                    const uint64_t* active_rank_mask, const void* x, void* out,
+                                    void* stream);
+
+/*
  * Synchronise `stream`, then read and clear the handle's device error word.
  * DEVICE_TIMEOUT if a kernel's bounded wait ran out since the last check.
  */

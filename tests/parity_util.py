@@ -20,6 +20,10 @@ def to_np(t: torch.Tensor) -> np.ndarray:
     return t.numpy()
 
 
+def bits_f32(bits_u16: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits_u16, np.uint32) << 16).view(np.float32)
+
+
 def assert_equal(gpu: torch.Tensor, want: np.ndarray, what: str):
     """Bit-exact comparison on the GPU (large arrays), with the first mismatches."""
     g = gpu.contiguous().view(-1)

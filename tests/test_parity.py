@@ -516,3 +516,112 @@ def test_combine_experts_with_masks_and_invalid_ids():
     wts = torch.randn((ep, tpr, k), generator=g)
     y = torch.randn((ep, tpr, k, H), generator=g).to(torch.bfloat16)
     _check_combine_experts(w, x, y, wts)
+
+
+# --------------------------------------------------------------------------- #
+# FP8 combine with one scale per row
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("hidden,rows", [(7168, 4096), (100, 333), (16, 7), (8192, 64)])
+def test_quantize_rows_matches_oracle(hidden, rows):
+    from combine_route_plan_b200 import ep_a2a
+    g = torch.Generator().manual_seed(hidden + rows)
+    x = torch.randn((rows, hidden), generator=g) * torch.exp(torch.randn((rows, 1), generator=g) * 3)
+    x[rows // 2] = 0.0
+    xb = x.to(torch.bfloat16)
+    codes, scales = ep_a2a.quantize_e4m3_rows(xb.cuda())
+    torch.cuda.synchronize()
+    oc, osc = U.oracle.quantize_e4m3_rows(U.to_np(xb), hidden)
+    U.assert_equal(codes.view(torch.uint8), oc, "row codes")
+    U.assert_equal(scales, osc, "row scales")
+
+
+@pytest.mark.parametrize("name", ["c2_ep8_decode", "c5_ep64_wide_masked", "c1_ep4_tiny"])
+def test_combine_scaled_bit_exact(name):
+    from combine_route_plan_b200 import ep_a2a
+    w = W.BY_NAME[name]
+    x = _inputs(w.name)
+    run = U.Run(w, W.Inputs(w, x.token_selected_experts, x.local_num_tokens, x.payloads,
+                            x.eplb_local_stats, x.active_rank_mask, None))
+    xo = x.expert_output
+    codes, scales = ep_a2a.quantize_e4m3_rows(xo.cuda())
+    out = torch.full((w.ep_size, w.tokens_per_rank, w.hidden), U.OUT_CANARY, dtype=torch.int16,
+                     device="cuda").view(torch.bfloat16)
+    run.comm.combine_scaled(codes, scales, out)
+    torch.cuda.synchronize()
+    assert run.comm.get_status() == ep_a2a.OK
+    oc, osc = U.oracle.quantize_e4m3_rows(U.to_np(xo), w.hidden)
+    plan = U.oracle_plan(w, x)
+    want = U.oracle.combine_scaled(plan, oc, osc, w.hidden, out_init=U.oracle_out_init(w))
+    U.assert_equal(out, want, "scaled fp8 combine")
+    # against the unquantized bf16 combine: E4M3 keeps 3 mantissa bits per term
+    ref = U.oracle.combine(plan, U.to_np(xo), w.hidden)
+    exists = plan.num_dst >= 0
+    got = U.bits_f32(U.to_np(out)[exists]).astype(np.float64)
+    exact = U.bits_f32(ref[exists]).astype(np.float64)
+    absx = np.abs(U.bits_f32(U.to_np(xo))).max()
+    assert np.max(np.abs(got - exact)) <= 8 * 2.0 ** -4 * absx
+
+
+def test_combine_scaled_odd_hidden():
+    from combine_route_plan_b200 import ep_a2a
+    ep, E, k, tpr, H = 4, 16, 4, 30, 40
+    w, x = _custom(ep, E, k, tpr, H, [16], seed=31)
+    run = U.Run(w, W.Inputs(w, x.token_selected_experts, x.local_num_tokens, x.payloads, None,
+                            None, None))
+    codes, scales = ep_a2a.quantize_e4m3_rows(x.expert_output.cuda())
+    out = run.comm.combine_scaled(codes, scales)
+    torch.cuda.synchronize()
+    oc, osc = U.oracle.quantize_e4m3_rows(U.to_np(x.expert_output), H)
+    plan = U.oracle_plan(w, x)
+    want = U.oracle.combine_scaled(plan, oc, osc, H)
+    exists = plan.num_dst >= 0
+    assert np.array_equal(U.to_np(out)[exists], want[exists])
+
+
+# --------------------------------------------------------------------------- #
+# Dense variant: all-gather dispatch, reduce-scatter combine
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("name", ["c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked"])
+def test_dense_allgather_and_reduce_scatter(name):
+    from combine_route_plan_b200 import ep_a2a
+    w = W.BY_NAME[name]
+    x = _inputs(w.name)
+    ep, tpr, H = w.ep_size, w.tokens_per_rank, w.hidden
+    rows = w.payload_row_bytes()
+    offs, off = [], 0
+    for rb in rows:
+        offs.append(off)
+        off += (ep * tpr * rb + 255) // 256 * 256
+    stride = off
+    recv = torch.full((ep, stride), U.CANARY, dtype=torch.uint8, device="cuda")
+    pays = [p.cuda() for p in x.payloads]
+    ep_a2a.ep_a2a_allgather(ep, tpr, x.local_num_tokens, [p.data_ptr() for p in pays], rows,
+                            [recv.data_ptr() + o for o in offs], stride, x.active_rank_mask)
+    xo = x.expert_output.cuda()
+    out = torch.full((ep, tpr, H), U.OUT_CANARY, dtype=torch.int16, device="cuda") \
+        .view(torch.bfloat16)
+    ep_a2a.ep_a2a_reduce_scatter(ep, tpr, H, x.local_num_tokens, xo.data_ptr(), out.data_ptr(),
+                                 x.active_rank_mask)
+    torch.cuda.synchronize()
+    for i, (p, rb) in enumerate(zip(x.payloads, rows)):
+        want = U.oracle.allgather(ep, tpr, x.local_num_tokens, p.numpy(), x.active_rank_mask)
+        got = recv[:, offs[i]:offs[i] + ep * tpr * rb]
+        U.assert_equal(got, want, f"allgather payload {i}")
+    want = U.oracle.reduce_scatter(ep, tpr, H, x.local_num_tokens, U.to_np(x.expert_output),
+                                   x.active_rank_mask)
+    U.assert_equal(out, want, "reduce_scatter")
+
+
+def test_reduce_scatter_element_path():
+    from combine_route_plan_b200 import ep_a2a
+    ep, tpr, H = 3, 10, 100
+    g = torch.Generator().manual_seed(3)
+    xo = torch.randn((ep, ep * tpr, H), generator=g).to(torch.bfloat16)
+    n = [10, 4, 0]
+    out = torch.full((ep, tpr, H), U.OUT_CANARY, dtype=torch.int16, device="cuda") \
+        .view(torch.bfloat16)
+    ep_a2a.ep_a2a_reduce_scatter(ep, tpr, H, n, xo.cuda().data_ptr(), out.data_ptr())
+    torch.cuda.synchronize()
+    U.assert_equal(out, U.oracle.reduce_scatter(ep, tpr, H, n, U.to_np(xo)), "reduce_scatter")
