@@ -130,6 +130,7 @@ struct ep_a2a_handle_s {
   int max_smem_optin;
   bool have_plan;
   int last_tpr;
+  int combine_hidden;     // row length of the combines, 1..p.hidden_size
   // tuning
   int copy_path;          // 0 staged, 1 vector only, 2 bulk loads + bulk stores
   int copy_consumer_warps;
@@ -268,6 +269,7 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   h->max_smem_optin = smem;
   h->have_plan = false;
   h->last_tpr = 0;
+  h->combine_hidden = params->hidden_size;
   // Defaults measured on the prefill workload (ep 8, 4096 tokens/rank, 14.4 KB
   // rows): the vector copy with 4 vectors per lane in flight, 32 CTAs per SM
   // requested and evict-first stores moved the rows fastest (487 us, against
@@ -586,7 +588,7 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   a.x = static_cast<const uint8_t*>(expert_output);
   a.out = static_cast<uint16_t*>(output);
   a.ntok = (int64_t)h->p.ep_size * h->last_tpr;
-  a.H = h->p.hidden_size;
+  a.H = h->combine_hidden;
   a.plan_stride = h->L.plan_stride;
   a.prefetch = h->combine_prefetch < 0 ? (fp8 ? 1 : 0) : h->combine_prefetch;
   const int elems = fp8 ? 16 : 8;
@@ -621,7 +623,7 @@ EP_API ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle h, const float* topk_w
   a.y = static_cast<const uint16_t*>(expert_output_per_slot);
   a.out = static_cast<uint16_t*>(output);
   a.ntok = (int64_t)h->p.ep_size * h->last_tpr;
-  a.H = h->p.hidden_size;
+  a.H = h->combine_hidden;
   a.k = h->p.top_k;
   a.E = h->p.num_experts;
   a.epr = h->p.num_experts / h->p.ep_size;
@@ -654,7 +656,7 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
   a.x = static_cast<const uint8_t*>(expert_output_e4m3);
   a.out = static_cast<uint16_t*>(output);
   a.ntok = (int64_t)h->p.ep_size * h->last_tpr;
-  a.H = h->p.hidden_size;
+  a.H = h->combine_hidden;
   a.plan_stride = h->L.plan_stride;
   a.prefetch = h->combine_prefetch != 0 ? 1 : 0;   // default: on, as for the FP8 combine
   const bool vec = a.H % 16 == 0 && aligned(expert_output_e4m3, 16) && aligned(output, 16);
@@ -762,6 +764,61 @@ EP_API ep_a2a_status ep_a2a_profile_stop(ep_a2a_handle h, ep_a2a_kernel_times* t
   }
   prof_free(h);
   if (times) *times = t;
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_grow_params(const ep_a2a_params* cur, const ep_a2a_params* req,
+                                        ep_a2a_params* out, int32_t* grown) {
+  ep_a2a_status st = check_params(cur);
+  if (st != EP_A2A_OK) return st;
+  if ((st = check_params(req)) != EP_A2A_OK) return st;
+  if (!out || !grown) return fail(EP_A2A_ERR_INVALID_ARG, "out / grown is NULL");
+  if (cur->ep_size != req->ep_size || cur->num_experts != req->num_experts ||
+      cur->top_k != req->top_k)
+    return fail(EP_A2A_ERR_INVALID_ARG,
+                "ep_size / num_experts / top_k differ (%d/%d/%d vs %d/%d/%d): one handle "
+                "serves one of each",
+                cur->ep_size, cur->num_experts, cur->top_k, req->ep_size, req->num_experts,
+                req->top_k);
+  const int32_t inv_cur = cur->invalid_expert_id < 0 ? cur->num_experts : cur->invalid_expert_id;
+  const int32_t inv_req = req->invalid_expert_id < 0 ? req->num_experts : req->invalid_expert_id;
+  if (inv_cur != inv_req)
+    return fail(EP_A2A_ERR_INVALID_ARG, "invalid_expert_id differs (%d vs %d)", inv_cur, inv_req);
+  ep_a2a_params g = *cur;
+  g.invalid_expert_id = inv_cur;
+  g.max_tokens_per_rank = std::max(cur->max_tokens_per_rank, req->max_tokens_per_rank);
+  g.hidden_size = std::max(cur->hidden_size, req->hidden_size);
+  g.num_payloads = std::max(cur->num_payloads, req->num_payloads);
+  for (int i = 0; i < kMaxPayloads; ++i) {
+    const int64_t a = i < cur->num_payloads ? cur->payload_row_bytes[i] : 0;
+    const int64_t b = i < req->num_payloads ? req->payload_row_bytes[i] : 0;
+    g.payload_row_bytes[i] = i < g.num_payloads ? std::max(a, b) : 0;
+  }
+  g.eplb_stats_num_experts =
+      (cur->eplb_stats_num_experts != 0 || req->eplb_stats_num_experts != 0) ? cur->num_experts
+                                                                               : 0;
+  g.enable_rank_mask = (cur->enable_rank_mask | req->enable_rank_mask) ? 1 : 0;
+  if ((int64_t)g.ep_size * g.max_tokens_per_rank > (int64_t)1 << 30)
+    return fail(EP_A2A_ERR_UNSUPPORTED, "grown ep_size * max_tokens_per_rank too large");
+  bool differs = g.max_tokens_per_rank != cur->max_tokens_per_rank ||
+                 g.hidden_size != cur->hidden_size || g.num_payloads != cur->num_payloads ||
+                 g.eplb_stats_num_experts != cur->eplb_stats_num_experts ||
+                 g.enable_rank_mask != cur->enable_rank_mask;
+  for (int i = 0; i < g.num_payloads; ++i)
+    differs |= g.payload_row_bytes[i] != cur->payload_row_bytes[i];
+  *out = g;
+  *grown = differs ? 1 : 0;
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_set_combine_hidden(ep_a2a_handle h, int32_t hidden) {
+  ep_a2a_status st = check_handle(h);
+  if (st != EP_A2A_OK) return st;
+  if (hidden < 1) return fail(EP_A2A_ERR_INVALID_ARG, "hidden %d must be >= 1", hidden);
+  if (hidden > h->p.hidden_size)
+    return fail(EP_A2A_ERR_CAPACITY, "hidden %d exceeds the handle's hidden_size %d", hidden,
+                h->p.hidden_size);
+  h->combine_hidden = hidden;
   return EP_A2A_OK;
 }
 

@@ -105,6 +105,8 @@ def _load():
         "ep_a2a_debug_wait_probe": (st, [VP, I64, VP]),
         "ep_a2a_set_option": (st, [VP, ctypes.c_int, I64]),
         "ep_a2a_destroy": (st, [P(VP)]),
+        "ep_a2a_grow_params": (st, [P(Params), P(Params), P(Params), P(I32)]),
+        "ep_a2a_set_combine_hidden": (st, [VP, I32]),
         "ep_a2a_profile_start": (st, [VP, I32]),
         "ep_a2a_profile_stop": (st, [VP, P(KernelTimes)]),
         "ep_a2a_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -269,6 +271,35 @@ def ep_a2a_destroy(handle_box: ctypes.c_void_p):
     _check(lib.ep_a2a_destroy(ctypes.byref(handle_box)))
 
 
+def ep_a2a_grow_params(current: Params, request: Params):
+    """(parameters serving both, True if they differ from ``current``)."""
+    out, grown = Params(), ctypes.c_int32(0)
+    _check(lib.ep_a2a_grow_params(ctypes.byref(current), ctypes.byref(request),
+                                  ctypes.byref(out), ctypes.byref(grown)))
+    return out, bool(grown.value)
+
+
+def ep_a2a_set_combine_hidden(handle: int, hidden: int):
+    _check(lib.ep_a2a_set_combine_hidden(ctypes.c_void_p(handle), int(hidden)))
+
+
+def make_params(ep_size: int, num_experts: int, top_k: int, max_tokens_per_rank: int,
+                hidden_size: int, payload_row_bytes: Sequence[int],
+                eplb_stats_num_experts: int = 0, enable_rank_mask: bool = False,
+                invalid_expert_id: int = -1) -> Params:
+    p = Params()
+    p.ep_size, p.num_experts, p.top_k = ep_size, num_experts, top_k
+    p.max_tokens_per_rank, p.hidden_size = max_tokens_per_rank, hidden_size
+    p.num_payloads = len(payload_row_bytes)
+    for i, rb in enumerate(payload_row_bytes):
+        p.payload_row_bytes[i] = int(rb)
+    p.eplb_stats_num_experts = eplb_stats_num_experts
+    p.enable_rank_mask = int(bool(enable_rank_mask))
+    p.invalid_expert_id = invalid_expert_id
+    p.reserved = 0
+    return p
+
+
 def ep_a2a_status_string(status: int) -> str:
     return lib.ep_a2a_status_string(int(status)).decode()
 
@@ -326,29 +357,60 @@ class EpA2A:
                  eplb_stats_num_experts: int = 0, enable_rank_mask: bool = False,
                  invalid_expert_id: int = -1, device=None, stream=None,
                  workspace_fill: Optional[int] = None):
-        p = Params()
-        p.ep_size, p.num_experts, p.top_k = ep_size, num_experts, top_k
-        p.max_tokens_per_rank, p.hidden_size = max_tokens_per_rank, hidden_size
-        p.num_payloads = len(payload_row_bytes)
-        for i, rb in enumerate(payload_row_bytes):
-            p.payload_row_bytes[i] = int(rb)
-        p.eplb_stats_num_experts = eplb_stats_num_experts
-        p.enable_rank_mask = int(bool(enable_rank_mask))
-        p.invalid_expert_id = invalid_expert_id
-        p.reserved = 0
-        self.params = p
-        self.ep_size, self.num_experts, self.top_k = ep_size, num_experts, top_k
-        self.hidden_size = hidden_size
-        self.payload_row_bytes = [int(x) for x in payload_row_bytes]
-        self.eplb_stats_num_experts = eplb_stats_num_experts
+        p = make_params(ep_size, num_experts, top_k, max_tokens_per_rank, hidden_size,
+                        payload_row_bytes, eplb_stats_num_experts, enable_rank_mask,
+                        invalid_expert_id)
         self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
             else torch.device(device)
+        self._workspace_fill = workspace_fill
+        self._options = {}
+        self._h = ctypes.c_void_p(0)
+        self._create(p, stream)
+
+    def _create(self, p: Params, stream):
+        self.params = p
+        self.ep_size, self.num_experts, self.top_k = p.ep_size, p.num_experts, p.top_k
+        self.hidden_size = p.hidden_size
+        self.payload_row_bytes = [int(p.payload_row_bytes[i]) for i in range(p.num_payloads)]
+        self.eplb_stats_num_experts = p.eplb_stats_num_experts
         nbytes = ep_a2a_workspace_size(p)
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
-        if workspace_fill is not None:
-            self.workspace.fill_(workspace_fill)
+        if self._workspace_fill is not None:
+            self.workspace.fill_(self._workspace_fill)
         self._h = ctypes.c_void_p(ep_a2a_init(p, self.workspace.data_ptr(), nbytes, stream))
+        for option, value in self._options.items():
+            ep_a2a_set_option(self._h.value, option, value)
+        self.combine_hidden = p.hidden_size
         self.last_tokens_per_rank = None
+
+    def ensure_capacity(self, max_tokens_per_rank: Optional[int] = None,
+                        hidden_size: Optional[int] = None,
+                        payload_row_bytes: Optional[Sequence[int]] = None,
+                        eplb_stats_num_experts: int = 0, enable_rank_mask: bool = False,
+                        stream=None) -> bool:
+        """Grow the handle to also serve this request (ep_a2a_grow_params); True if
+        it was replaced.  Replacing synchronises the device, destroys the old handle
+        and allocates a new workspace: earlier views and the plan are gone."""
+        cur = self.params
+        req = make_params(cur.ep_size, cur.num_experts, cur.top_k,
+                          max_tokens_per_rank or cur.max_tokens_per_rank,
+                          hidden_size or cur.hidden_size,
+                          self.payload_row_bytes if payload_row_bytes is None
+                          else payload_row_bytes,
+                          eplb_stats_num_experts, enable_rank_mask, cur.invalid_expert_id)
+        grown_params, grown = ep_a2a_grow_params(cur, req)
+        if not grown:
+            return False
+        torch.cuda.synchronize(self.device)
+        ep_a2a_destroy(self._h)
+        self.workspace = None
+        self._create(grown_params, stream)
+        return True
+
+    def _use_hidden(self, hidden: int):
+        if hidden != self.combine_hidden:
+            ep_a2a_set_combine_hidden(self.handle, hidden)
+            self.combine_hidden = hidden
 
     @property
     def handle(self) -> int:
@@ -358,6 +420,7 @@ class EpA2A:
 
     def set_option(self, option: int, value: int):
         ep_a2a_set_option(self.handle, option, value)
+        self._options[option] = value
 
     def dispatch(self, token_selected_experts: torch.Tensor, local_num_tokens: Sequence[int],
                  payloads: Sequence[torch.Tensor], runtime_max_tokens_per_rank: Optional[int] = None,
@@ -404,16 +467,18 @@ class EpA2A:
         else:
             raise TypeError(f"combine input must be bf16 or float8_e4m3fn, got {x.dtype}")
         tpr = self.last_tokens_per_rank
+        hidden = x.shape[-1] if x.dim() >= 2 else self.hidden_size
         if tpr is not None:
-            assert x.numel() == self.ep_size * self.ep_size * tpr * self.hidden_size, x.shape
+            assert x.numel() == self.ep_size * self.ep_size * tpr * hidden, x.shape
+            self._use_hidden(hidden)
         if output is None:
             if tpr is None:
                 tpr = tokens_per_rank if tokens_per_rank is not None else 1
-            output = torch.empty((self.ep_size, tpr, self.hidden_size), dtype=torch.bfloat16,
+            output = torch.empty((self.ep_size, tpr, hidden), dtype=torch.bfloat16,
                                  device=x.device)
         assert output.is_cuda and output.dtype == torch.bfloat16 and output.is_contiguous()
         if tpr is not None:
-            assert output.numel() == self.ep_size * tpr * self.hidden_size, output.shape
+            assert output.numel() == self.ep_size * tpr * hidden, output.shape
         ep_a2a_combine(self.handle, x.data_ptr(), dt, output.data_ptr(), stream)
         return output
 
@@ -427,12 +492,14 @@ class EpA2A:
         assert w.is_cuda and w.dtype == torch.float32 and w.is_contiguous()
         assert w.numel() == self.ep_size * tpr * self.top_k, w.shape
         assert y.is_cuda and y.dtype == torch.bfloat16 and y.is_contiguous()
-        assert y.numel() == self.ep_size * tpr * self.top_k * self.hidden_size, y.shape
+        hidden = y.shape[-1]
+        assert y.numel() == self.ep_size * tpr * self.top_k * hidden, y.shape
         if output is None:
-            output = torch.empty((self.ep_size, tpr, self.hidden_size), dtype=torch.bfloat16,
+            output = torch.empty((self.ep_size, tpr, hidden), dtype=torch.bfloat16,
                                  device=y.device)
         assert output.is_cuda and output.dtype == torch.bfloat16 and output.is_contiguous()
-        assert output.numel() == self.ep_size * tpr * self.hidden_size, output.shape
+        assert output.numel() == self.ep_size * tpr * hidden, output.shape
+        self._use_hidden(hidden)
         ep_a2a_combine_experts(self.handle, w.data_ptr(), y.data_ptr(), output.data_ptr(), stream)
         return output
 
@@ -443,14 +510,16 @@ class EpA2A:
         assert tpr is not None, "combine needs a preceding dispatch"
         rows = self.ep_size * self.ep_size * tpr
         assert codes.is_cuda and codes.is_contiguous() and codes.element_size() == 1
-        assert codes.numel() == rows * self.hidden_size, codes.shape
+        hidden = codes.shape[-1]
+        assert codes.numel() == rows * hidden, codes.shape
         assert row_scales.is_cuda and row_scales.dtype == torch.float32
         assert row_scales.is_contiguous() and row_scales.numel() == rows, row_scales.shape
         if output is None:
-            output = torch.empty((self.ep_size, tpr, self.hidden_size), dtype=torch.bfloat16,
+            output = torch.empty((self.ep_size, tpr, hidden), dtype=torch.bfloat16,
                                  device=codes.device)
         assert output.is_cuda and output.dtype == torch.bfloat16 and output.is_contiguous()
-        assert output.numel() == self.ep_size * tpr * self.hidden_size, output.shape
+        assert output.numel() == self.ep_size * tpr * hidden, output.shape
+        self._use_hidden(hidden)
         ep_a2a_combine_scaled(self.handle, codes.data_ptr(), row_scales.data_ptr(),
                               output.data_ptr(), stream)
         return output

@@ -362,6 +362,45 @@ ep_a2a_status ep_a2a_profile_stop(ep_a2a_handle handle, ep_a2a_kernel_times* tim
  */
 ep_a2a_status ep_a2a_destroy(ep_a2a_handle* handle);
 
+/*
+ * Capacity growth (vllm.distributed.device_communicators.all2all,
+ * FlashInferNVLinkOneSidedManager.initialize): the MoE layers of a model share
+ * one handle, sized for the largest of them, and a layer whose request does not
+ * fit replaces it with a larger one.  Given the parameters of the current handle
+ * and of a new request, writes to *out the parameters that serve both and to
+ * *grown 1 if they differ from `current` (a new handle is needed), else 0
+ * (*out = *current with invalid_expert_id resolved).
+ *   ep_size, num_experts, top_k   must be equal (INVALID_ARG otherwise: a handle
+ *                                 serves one top_k and one expert count)
+ *   max_tokens_per_rank,
+ *   hidden_size                   the larger of the two
+ *   payload_row_bytes[i]          the larger of the two, a payload that one side
+ *                                 lacks counting as 0; num_payloads the larger
+ *   eplb_stats_num_experts        num_experts if either side gathers, else 0
+ *   enable_rank_mask              1 if either side is 1
+ *   invalid_expert_id             must resolve (< 0 = num_experts) to the same id
+ * Both inputs are checked as by ep_a2a_init.  Host only: no CUDA call.  To
+ * grow, the caller synchronises the streams that use the old handle, destroys
+ * it, allocates a workspace of ep_a2a_workspace_size(out) bytes and calls
+ * ep_a2a_init on it; the old workspace's views and plan are gone, so the next
+ * combine needs a new dispatch.
+ */
+ep_a2a_status ep_a2a_grow_params(const ep_a2a_params* current, const ep_a2a_params* request,
+                                 ep_a2a_params* out, int32_t* grown);
+
+/*
+ * Row length of this handle's combines.  A handle grown to the largest hidden
+ * size also serves layers with smaller ones, whose combine reads and writes rows
+ * of their own length (the combine takes it from its payload in
+ * vllm.distributed.device_communicators.all2all,
+ * FlashInferNVLinkOneSidedManager.initialize).  ep_a2a_combine,
+ * ep_a2a_combine_experts and ep_a2a_combine_scaled called after this returns use
+ * rows of `hidden` elements: 1..params.hidden_size, which init sets.  Host state
+ * only, nothing is enqueued.  INVALID_ARG for hidden < 1, CAPACITY above
+ * params.hidden_size.
+ */
+ep_a2a_status ep_a2a_set_combine_hidden(ep_a2a_handle handle, int32_t hidden);
+
 const char* ep_a2a_status_string(ep_a2a_status status);
 const char* ep_a2a_last_error(void);
 

@@ -345,6 +345,97 @@ def test_runtime_max_below_capacity_and_redispatch():
                 U.assert_equal(g[torch.from_numpy(valid).cuda()], pw[valid], f"p{i} d{dst}")
 
 
+def _check_valid_rows(d, plan, x, ep):
+    """Plan arrays in full; payload rows where the plan says received."""
+    nd = plan.num_dst.copy()
+    nd[nd < 0] = 0xFF
+    U.assert_equal(d.plan_num_dst, nd.astype(np.uint8), "plan_num_dst")
+    U.assert_equal(d.recv_valid, plan.recv_valid, "recv_valid")
+    U.assert_equal(d.recv_topk_ids, plan.recv_topk_ids, "recv_topk_ids")
+    U.assert_equal(d.send_counts, plan.send_counts, "send_counts")
+    for i, p in enumerate(x.payloads):
+        for dst in range(ep):
+            pw = U.oracle.dispatch_payload(plan, p.numpy(), only_dst=dst)[0]
+            valid = plan.recv_valid[dst] == 1
+            U.assert_equal(d.recv_payloads[i][dst][torch.from_numpy(valid).cuda()], pw[valid],
+                           f"p{i} d{dst}")
+
+
+def test_capacity_growth_serves_every_layer():
+    """Layers of different sizes share one handle, grown on demand
+    (vllm.distributed.device_communicators.all2all,
+    FlashInferNVLinkOneSidedManager.initialize); every layer's dispatch and
+    combine on the grown handle match the oracle, and options survive growth."""
+    from combine_route_plan_b200 import ep_a2a
+    ep, E, k = 4, 16, 4
+    layers = [(24, 64, [128, 16]),
+              (40, 32, [64, 16, 8]),      # more tokens, a smaller hidden, one more payload
+              (16, 96, [256, 16]),        # a larger hidden and rows, fewer payloads
+              (40, 64, [128, 16, 8])]     # fits
+    comm = ep_a2a.EpA2A(ep, E, k, 24, 64, [128, 16], workspace_fill=U.CANARY)
+    comm.set_option(ep_a2a.OPT_COMBINE_THREADS, 128)
+    grew = []
+    for i, (tpr, H, rows) in enumerate(layers):
+        grew.append(comm.ensure_capacity(tpr, H, rows))
+        w, x = _custom(ep, E, k, tpr, H, rows, n=[tpr, tpr - 3, 1, tpr], seed=40 + i)
+        d = comm.dispatch(x.token_selected_experts.cuda(), x.local_num_tokens,
+                          [p.cuda() for p in x.payloads], tpr)
+        out = torch.full((ep, tpr, H), U.OUT_CANARY, dtype=torch.int16,
+                         device="cuda").view(torch.bfloat16)
+        comm.combine(x.expert_output.cuda(), out)
+        torch.cuda.synchronize()
+        assert comm.get_status() == ep_a2a.OK
+        plan = U.oracle_plan(w, x)
+        _check_valid_rows(d, plan, x, ep)
+        U.assert_equal(out, U.oracle.combine(plan, U.to_np(x.expert_output), H,
+                                             out_init=U.oracle_out_init(w)), f"combine {i}")
+    assert grew == [False, True, True, False]
+    assert (comm.params.max_tokens_per_rank, comm.params.hidden_size) == (40, 96)
+    assert comm.payload_row_bytes == [256, 16, 8]
+    assert comm._options[ep_a2a.OPT_COMBINE_THREADS] == 128
+
+
+def test_combine_rows_shorter_than_the_handle_hidden():
+    """A handle sized for hidden 128 combines rows of 64, 40 and 128 elements
+    (BF16, FP8, expert outputs and scaled FP8), each matching the oracle."""
+    from combine_route_plan_b200 import ep_a2a
+    ep, E, k, tpr, Hcap = 4, 16, 4, 30, 128
+    comm = ep_a2a.EpA2A(ep, E, k, tpr, Hcap, [32], workspace_fill=U.CANARY)
+    for H in (64, 40, 128, 16):
+        w, x = _custom(ep, E, k, tpr, H, [32], n=[30, 0, 17, 29], seed=60 + H)
+        comm.dispatch(x.token_selected_experts.cuda(), x.local_num_tokens,
+                      [p.cuda() for p in x.payloads], tpr)
+        plan = U.oracle_plan(w, x)
+        xo = x.expert_output
+        out = comm.combine(xo.cuda())
+        q = ep_a2a.quantize_e4m3(xo.cuda())
+        out8 = comm.combine(q)
+        g = torch.Generator().manual_seed(H)
+        wts = torch.randn((ep, tpr, k), generator=g)
+        y = torch.randn((ep, tpr, k, H), generator=g).to(torch.bfloat16)
+        oute = comm.combine_experts(wts.cuda(), y.cuda())
+        codes, scales = ep_a2a.quantize_e4m3_rows(xo.cuda())
+        outs = comm.combine_scaled(codes, scales)
+        torch.cuda.synchronize()
+        assert comm.get_status() == ep_a2a.OK
+        exists = plan.num_dst >= 0
+        xq = U.oracle_quantize_big(U.to_np(xo), U.oracle_e4m3_table())
+        oc, osc = U.oracle.quantize_e4m3_rows(U.to_np(xo), H)
+        for got, want, what in [
+                (out, U.oracle.combine(plan, U.to_np(xo), H), "bf16"),
+                (out8, U.oracle.combine(plan, xq, H, input_is_e4m3=True), "fp8"),
+                (oute, U.oracle.combine_experts(plan, E, x.token_selected_experts.numpy(),
+                                                wts.numpy(), U.to_np(y), H), "experts"),
+                (outs, U.oracle.combine_scaled(plan, oc, osc, H), "scaled")]:
+            assert np.array_equal(U.to_np(got)[exists], want[exists]), (H, what)
+    with pytest.raises(ep_a2a.EpA2AError) as e:
+        ep_a2a.ep_a2a_set_combine_hidden(comm.handle, Hcap + 1)
+    assert e.value.status == ep_a2a.ERR_CAPACITY
+    with pytest.raises(ep_a2a.EpA2AError) as e:
+        ep_a2a.ep_a2a_set_combine_hidden(comm.handle, 0)
+    assert e.value.status == ep_a2a.ERR_INVALID_ARG
+
+
 def test_counts_scratch_resets_between_calls():
     w = W.scaled(W.C2, 64)
     x = W.make_inputs(w, with_expert_output=False)
