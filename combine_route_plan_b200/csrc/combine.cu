@@ -89,7 +89,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // Thread 0 asks for the rows of token `tok` (if it exists) to be brought into
-// L2, so that this CTA's loads of it hit L2 when it gets there.
+// L2, so that this CTA's loads of it hit L2 when it gets there.  The combines
+// call it for the token a.prefetch grid strides ahead of the current one.
 template <int kElemBytes>
 __device__ __forceinline__ void prefetch_token_rows(const CombineArgs& a, int64_t tok) {
   if (tok >= a.ntok) return;
@@ -113,9 +114,12 @@ __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
   constexpr int kElemBytes = kFp8 ? 1 : 2;
   const int nvec = a.H / kElems;
   const int words = a.plan_stride / 8;
-  if (a.prefetch && threadIdx.x == 0) prefetch_token_rows<kElemBytes>(a, blockIdx.x);
+  if (a.prefetch && threadIdx.x == 0)
+    for (int p = 0; p < a.prefetch; ++p)
+      prefetch_token_rows<kElemBytes>(a, blockIdx.x + (int64_t)p * gridDim.x);
   for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
-    if (a.prefetch && threadIdx.x == 0) prefetch_token_rows<kElemBytes>(a, tok + gridDim.x);
+    if (a.prefetch && threadIdx.x == 0)
+      prefetch_token_rows<kElemBytes>(a, tok + (int64_t)a.prefetch * gridDim.x);
     const int nd = a.plan_nd[tok];
     if (nd == kNoToken) continue;
     const uint64_t* row = reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
@@ -157,6 +161,125 @@ __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
         pk.w = pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]);
         o[q] = pk;
       }
+    }
+  }
+}
+
+enum CombineMode { kCombineBf16 = 0, kCombineFp8 = 1, kCombineFp8Scaled = 2 };
+
+// acc[0..16) = fmaf(widen(code), scale, acc) for the 16 E4M3 codes of v.
+__device__ __forceinline__ void fma_e4m3x16(float* acc, const uint4& v, float scale) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+          (__nv_fp8x2_storage_t)((w[q] >> (16 * h)) & 0xFFFFu), __NV_E4M3);
+      __half_raw lo, hi;
+      lo.x = hr.x;
+      hi.x = hr.y;
+      float& a0 = acc[4 * q + 2 * h];
+      float& a1 = acc[4 * q + 2 * h + 1];
+      a0 = __fmaf_rn(__half2float(__half(lo)), scale, a0);
+      a1 = __fmaf_rn(__half2float(__half(hi)), scale, a1);
+    }
+  }
+}
+
+// Loads of one 16-byte column vector (at byte offset `off`) of each of the
+// token's first nd (<= 8) destination rows.
+__device__ __forceinline__ void load_rows(uint4 (&r)[8], const uint8_t* const (&src)[8], int nd,
+                                          int64_t off) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (i < nd) r[i] = ld_stream_v4(src[i] + off);
+}
+
+// Sum one column vector over the rows in ascending destination order and store
+// it as bf16.
+template <int kMode>
+__device__ __forceinline__ void reduce_store(const uint4 (&r)[8], const float (&sc)[8], int nd,
+                                             uint16_t* o) {
+  constexpr int kElems = kMode == kCombineBf16 ? 8 : 16;
+  float acc[kElems];
+#pragma unroll
+  for (int e = 0; e < kElems; ++e) acc[e] = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (i < nd) {
+      if (kMode == kCombineBf16)
+        add_bf16x8(acc, r[i]);
+      else if (kMode == kCombineFp8)
+        add_e4m3x16(acc, r[i]);
+      else
+        fma_e4m3x16(acc, r[i], sc[i]);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < kElems / 8; ++q) {
+    uint4 pk;
+    pk.x = pack_bf16x2(acc[8 * q + 0], acc[8 * q + 1]);
+    pk.y = pack_bf16x2(acc[8 * q + 2], acc[8 * q + 3]);
+    pk.z = pack_bf16x2(acc[8 * q + 4], acc[8 * q + 5]);
+    pk.w = pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]);
+    reinterpret_cast<uint4*>(o)[q] = pk;
+  }
+}
+
+// The combines for tokens with at most 8 destination ranks (top_k or ep_size
+// <= 8), 16-byte vectors: the same sums as combine_vec_kernel and
+// combine_scaled_kernel<true>, with each thread's loads pipelined two deep --
+// the rows of its next column vector are in flight while it adds the current
+// one, so a thread never waits on memory with its adds still to do.
+template <int kMode>
+__global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
+                                                           const float* __restrict__ scales) {
+  pdl_wait();
+  constexpr int kElems = kMode == kCombineBf16 ? 8 : 16;
+  constexpr int kElemBytes = kMode == kCombineBf16 ? 2 : 1;
+  const int nvec = a.H / kElems;
+  const int64_t rank_stride = a.ntok * (int64_t)a.H * kElemBytes;
+  const int64_t step = (int64_t)blockDim.x * 16;       // bytes between a thread's vectors
+  if (a.prefetch && threadIdx.x == 0)
+    for (int p = 0; p < a.prefetch; ++p)
+      prefetch_token_rows<kElemBytes>(a, blockIdx.x + (int64_t)p * gridDim.x);
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    if (a.prefetch && threadIdx.x == 0)
+      prefetch_token_rows<kElemBytes>(a, tok + (int64_t)a.prefetch * gridDim.x);
+    const int nd = a.plan_nd[tok];
+    if (nd == kNoToken || (int)threadIdx.x >= nvec) continue;
+    const uint64_t w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    const uint8_t* xt = a.x + tok * (int64_t)a.H * kElemBytes + (int64_t)threadIdx.x * 16;
+    const uint8_t* src[8];
+    float sc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int d = (int)((w0 >> (8 * i)) & 0xFFu);
+      src[i] = xt + (int64_t)(i < nd ? d : 0) * rank_stride;
+      sc[i] = 1.0f;
+      if (kMode == kCombineFp8Scaled && i < nd) sc[i] = scales[(int64_t)d * a.ntok + tok];
+    }
+    uint16_t* o = a.out + tok * (int64_t)a.H + (int64_t)threadIdx.x * kElems;
+    const int64_t ostep = (int64_t)blockDim.x * kElems;
+    uint4 ra[8], rb[8];
+    load_rows(ra, src, nd, 0);
+    int64_t off = 0;
+    for (int v = threadIdx.x;;) {
+      const bool more_b = v + (int)blockDim.x < nvec;
+      if (more_b) load_rows(rb, src, nd, off + step);
+      reduce_store<kMode>(ra, sc, nd, o);
+      if (!more_b) break;
+      v += blockDim.x;
+      off += step;
+      o += ostep;
+      const bool more_a = v + (int)blockDim.x < nvec;
+      if (more_a) load_rows(ra, src, nd, off + step);
+      reduce_store<kMode>(rb, sc, nd, o);
+      if (!more_a) break;
+      v += blockDim.x;
+      off += step;
+      o += ostep;
     }
   }
 }
@@ -231,11 +354,16 @@ __global__ void __launch_bounds__(512) combine_experts_vec_kernel(const CombineE
   const int words = a.plan_stride / 8;
   // the k slot rows of a token are contiguous: one prefetch per token
   const uint32_t tok_bytes = (uint32_t)a.k * a.H * 2;
-  if (a.prefetch && threadIdx.x == 0 && blockIdx.x < a.ntok)
-    prefetch_l2(a.y + (int64_t)blockIdx.x * a.k * a.H, tok_bytes);
+  if (a.prefetch && threadIdx.x == 0)
+    for (int p = 0; p < a.prefetch; ++p) {
+      const int64_t t = blockIdx.x + (int64_t)p * gridDim.x;
+      if (t < a.ntok) prefetch_l2(a.y + t * a.k * a.H, tok_bytes);
+    }
   for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
-    if (a.prefetch && threadIdx.x == 0 && tok + gridDim.x < a.ntok)
-      prefetch_l2(a.y + (tok + gridDim.x) * a.k * a.H, tok_bytes);
+    if (a.prefetch && threadIdx.x == 0) {
+      const int64_t t = tok + (int64_t)a.prefetch * gridDim.x;
+      if (t < a.ntok) prefetch_l2(a.y + t * a.k * a.H, tok_bytes);
+    }
     const int nd = a.plan_nd[tok];
     if (nd == kNoToken) continue;
     uint16_t* out = a.out + tok * (int64_t)a.H;
@@ -289,6 +417,102 @@ __global__ void __launch_bounds__(512) combine_experts_vec_kernel(const CombineE
   }
 }
 
+// Loads of one 16-byte column vector of each slot row that takes part.
+__device__ __forceinline__ void expert_rows_load(uint4 (&r)[8], const uint16_t* yv,
+                                                 const int (&own)[8], int H) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (own[j] >= 0) r[j] = ld_stream_v4(yv + (int64_t)j * H);
+}
+
+// For each destination rank d in ascending order: z = fp32 fused multiply-add
+// over the slots d owns (ascending), rounded to bf16, added to the sum; the sum
+// is stored as bf16.
+__device__ __forceinline__ void expert_rows_reduce_store(const uint4 (&raw)[8],
+                                                         const int (&own)[8],
+                                                         const float (&wt)[8], int nd,
+                                                         uint64_t w0, uint16_t* o) {
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+  for (int q = 0; q < nd; ++q) {
+    const int d = (int)((w0 >> (8 * q)) & 0xFFu);
+    float z[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) z[e] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (own[j] != d) continue;
+      const uint32_t wv[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        z[2 * i] = __fmaf_rn(wt[j], bf16_bits_to_f32(wv[i] & 0xFFFFu), z[2 * i]);
+        z[2 * i + 1] = __fmaf_rn(wt[j], bf16_bits_to_f32(wv[i] >> 16), z[2 * i + 1]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], bf16_round(z[e]));
+  }
+  uint4 pk;
+  pk.x = pack_bf16x2(acc[0], acc[1]);
+  pk.y = pack_bf16x2(acc[2], acc[3]);
+  pk.z = pack_bf16x2(acc[4], acc[5]);
+  pk.w = pack_bf16x2(acc[6], acc[7]);
+  *reinterpret_cast<uint4*>(o) = pk;
+}
+
+// combine_experts_vec_kernel with each thread's loads pipelined two deep: the
+// slot rows of its next column vector are in flight while it reduces the
+// current one.  top_k <= 8, so a token has at most 8 destinations.
+__global__ void __launch_bounds__(512) combine_experts_pipe_kernel(const CombineExpertsArgs a) {
+  pdl_wait();
+  const int nvec = a.H / 8;
+  const uint32_t tok_bytes = (uint32_t)a.k * a.H * 2;
+  if (a.prefetch && threadIdx.x == 0)
+    for (int p = 0; p < a.prefetch; ++p) {
+      const int64_t t = blockIdx.x + (int64_t)p * gridDim.x;
+      if (t < a.ntok) prefetch_l2(a.y + t * a.k * a.H, tok_bytes);
+    }
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    if (a.prefetch && threadIdx.x == 0) {
+      const int64_t t = tok + (int64_t)a.prefetch * gridDim.x;
+      if (t < a.ntok) prefetch_l2(a.y + t * a.k * a.H, tok_bytes);
+    }
+    const int nd = a.plan_nd[tok];
+    if (nd == kNoToken || (int)threadIdx.x >= nvec) continue;
+    uint16_t* o = a.out + tok * (int64_t)a.H + (int64_t)threadIdx.x * 8;
+    const int64_t step = (int64_t)blockDim.x * 8;      // elements between a thread's vectors
+    if (nd == 0) {           // every owner masked off: the sum is empty
+      for (int v = threadIdx.x; v < nvec; v += blockDim.x, o += step)
+        *reinterpret_cast<uint4*>(o) = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const uint64_t w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    int own[8];
+    float wt[8];
+    slot_owners<8>(a, tok, nd, w0, 0, 0, 0, own, wt);
+    const uint16_t* yv = a.y + tok * (int64_t)a.k * a.H + (int64_t)threadIdx.x * 8;
+    uint4 ra[8], rb[8];
+    expert_rows_load(ra, yv, own, a.H);
+    for (int v = threadIdx.x;;) {
+      const bool more_b = v + (int)blockDim.x < nvec;
+      if (more_b) expert_rows_load(rb, yv + step, own, a.H);
+      expert_rows_reduce_store(ra, own, wt, nd, w0, o);
+      if (!more_b) break;
+      v += blockDim.x;
+      yv += step;
+      o += step;
+      const bool more_a = v + (int)blockDim.x < nvec;
+      if (more_a) expert_rows_load(ra, yv + step, own, a.H);
+      expert_rows_reduce_store(rb, own, wt, nd, w0, o);
+      if (!more_a) break;
+      v += blockDim.x;
+      yv += step;
+      o += step;
+    }
+  }
+}
+
 // Any top_k (<= 32) and hidden size: one element per thread step.
 __global__ void __launch_bounds__(512) combine_experts_any_kernel(const CombineExpertsArgs a) {
   pdl_wait();
@@ -329,9 +553,12 @@ __global__ void __launch_bounds__(512) combine_scaled_kernel(const CombineArgs a
   pdl_wait();
   const int words = a.plan_stride / 8;
   const int nvec = kVec ? a.H / 16 : 0;
-  if (kVec && a.prefetch && threadIdx.x == 0) prefetch_token_rows<1>(a, blockIdx.x);
+  if (kVec && a.prefetch && threadIdx.x == 0)
+    for (int p = 0; p < a.prefetch; ++p)
+      prefetch_token_rows<1>(a, blockIdx.x + (int64_t)p * gridDim.x);
   for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
-    if (kVec && a.prefetch && threadIdx.x == 0) prefetch_token_rows<1>(a, tok + gridDim.x);
+    if (kVec && a.prefetch && threadIdx.x == 0)
+      prefetch_token_rows<1>(a, tok + (int64_t)a.prefetch * gridDim.x);
     const int nd = a.plan_nd[tok];
     if (nd == kNoToken) continue;
     const uint64_t* row = reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
@@ -521,9 +748,15 @@ __global__ void wait_timeout_probe_kernel(uint32_t* err, unsigned long long limi
 
 }  // namespace
 
-cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, int threads, int grid,
-                           cudaStream_t stream, bool pdl) {
+cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, bool pipe, int threads,
+                           int grid, cudaStream_t stream, bool pdl) {
   const dim3 g(grid), b(threads);
+  const float* no_scales = nullptr;
+  if (vec && pipe) {
+    if (fp8) return launch_kernel(combine_pipe_kernel<kCombineFp8>, g, b, 0, stream, pdl, a,
+                                  no_scales);
+    return launch_kernel(combine_pipe_kernel<kCombineBf16>, g, b, 0, stream, pdl, a, no_scales);
+  }
   if (vec) {
     if (fp8) return launch_kernel(combine_vec_kernel<true>, g, b, 0, stream, pdl, a);
     return launch_kernel(combine_vec_kernel<false>, g, b, 0, stream, pdl, a);
@@ -532,9 +765,11 @@ cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, int threads
   return launch_kernel(combine_scalar_kernel<false>, g, b, 0, stream, pdl, a);
 }
 
-cudaError_t launch_combine_scaled(const CombineArgs& a, const float* scales, bool vec,
+cudaError_t launch_combine_scaled(const CombineArgs& a, const float* scales, bool vec, bool pipe,
                                   int threads, int grid, cudaStream_t stream, bool pdl) {
   const dim3 g(grid), b(threads);
+  if (vec && pipe)
+    return launch_kernel(combine_pipe_kernel<kCombineFp8Scaled>, g, b, 0, stream, pdl, a, scales);
   if (vec) return launch_kernel(combine_scaled_kernel<true>, g, b, 0, stream, pdl, a, scales);
   return launch_kernel(combine_scaled_kernel<false>, g, b, 0, stream, pdl, a, scales);
 }
@@ -553,9 +788,10 @@ cudaError_t launch_quantize_e4m3_rows(const uint16_t* in, uint8_t* out, float* s
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, int threads, int grid,
-                                   cudaStream_t stream, bool pdl) {
+cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, bool pipe, int threads,
+                                   int grid, cudaStream_t stream, bool pdl) {
   const dim3 g(grid), b(threads);
+  if (vec && pipe) return launch_kernel(combine_experts_pipe_kernel, g, b, 0, stream, pdl, a);
   if (vec) return launch_kernel(combine_experts_vec_kernel, g, b, 0, stream, pdl, a);
   return launch_kernel(combine_experts_any_kernel, g, b, 0, stream, pdl, a);
 }

@@ -140,9 +140,10 @@ struct ep_a2a_handle_s {
   int store_streaming;
   int pdl;                // programmatic dependent launch for the path's kernels
   int vec_threads_per_token;  // 0 = from the token count
-  int combine_prefetch;       // prefetch the next token's rows into L2 (combines);
-                              // -1 = for the FP8 combine only
-  int copy_prefetch;          // the same for the vector copy
+  // combine launch shape; -1 / 0 = automatic (combine_launch)
+  int combine_prefetch;       // tokens ahead (grid strides) whose rows go to L2
+  int copy_prefetch;          // vector copy: prefetch the next token's rows
+  int combine_pipeline;       // 1: the two-deep pipelined kernels
   int copy_ctas_per_sm;
   int copy_stages;        // 0 = choose from the row size
   int combine_threads;
@@ -190,6 +191,40 @@ void prof_free(ep_a2a_handle h) {
 int copy_threads_per_token(int64_t tokens) { return tokens >= 8192 ? 32 : 256; }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+enum CombineKind { kKindBf16, kKindFp8, kKindExperts };
+
+struct CombineLaunch {
+  bool pipe;
+  int threads, grid, prefetch;
+};
+
+// Launch shape of a combine: the options where set, else the defaults measured
+// on the decode (1024 token slots), wide-EP (4096), Zipf (8192) and prefill
+// (32768) workloads at hidden 7168:
+//  * BF16: one vector at a time, 64 threads, 128 CTAs per SM requested, no
+//    prefetch (pipelining and prefetch were 1-12 % slower);
+//  * FP8 and scaled FP8: pipelined (27-54 % faster); 64 threads below 16384
+//    token slots and 128 from there; from 8192 slots on, prefetch one token
+//    ahead (faster by 5-10 %, slower by 5-10 % on the small steps); 16 CTAs per
+//    SM requested from 16384 slots on (scaled: 291 against 310 us), else 128;
+//  * expert outputs: pipelined (24-28 % faster), 64 threads, no prefetch.
+// The pipelined kernels hold at most 8 destination rows per token, and a token
+// has at most min(top_k, ep_size) destinations.
+CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
+  const bool fits = std::min(h->p.top_k, h->p.ep_size) <= 8;
+  const bool big = ntok >= 16384;
+  CombineLaunch c;
+  c.pipe = fits && (h->combine_pipeline < 0 ? kind != kKindBf16 : h->combine_pipeline > 0);
+  c.threads = h->combine_threads > 0 ? h->combine_threads
+                                     : (kind == kKindFp8 && big ? 128 : 64);
+  const int cps = h->combine_ctas_per_sm > 0 ? h->combine_ctas_per_sm
+                                             : (kind == kKindFp8 && big ? 16 : 128);
+  c.grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntok, (int64_t)h->num_sms * cps));
+  c.prefetch = h->combine_prefetch >= 0 ? h->combine_prefetch
+                                        : (kind == kKindFp8 && ntok >= 8192 ? 1 : 0);
+  return c;
+}
 
 uint32_t vec_bytes(const void* src, const void* dst_base, int64_t rank_stride, int64_t rb) {
   for (uint32_t v : {16u, 8u, 4u, 2u}) {
@@ -282,16 +317,14 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   h->store_streaming = 1;
   h->pdl = 1;
   h->vec_threads_per_token = 0;
-  // Measured on the prefill and wide-EP workloads: the prefetch speeds up the
-  // FP8 combine (446 -> 372 us, 74 -> 64 us) and slows the BF16 and expert
-  // combines (their next-token rows, 14-115 KB per CTA, crowd L2).
-  h->combine_prefetch = -1;
+  h->combine_prefetch = -1;       // automatic (combine_launch)
   h->copy_prefetch = 0;
+  h->combine_pipeline = -1;
   h->copy_ctas_per_sm = 1;
   h->copy_stages = 4;
   h->combine_threads = 0;
   h->bulk_min_row = 0;
-  h->combine_ctas_per_sm = 128;
+  h->combine_ctas_per_sm = 0;
   h->profiling = false;
   h->prof_max = 0;
   *out_handle = h;
@@ -350,9 +383,14 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       h->vec_threads_per_token = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_COMBINE_PREFETCH:
-      if (value < -1 || value > 1)
-        return fail(EP_A2A_ERR_INVALID_ARG, "prefetch must be -1 (FP8 only), 0 or 1");
+      if (value < -1 || value > 4)
+        return fail(EP_A2A_ERR_INVALID_ARG, "prefetch must be -1 (FP8 only), 0 or 1..4");
       h->combine_prefetch = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_COMBINE_PIPELINE:
+      if (value < -1 || value > 1)
+        return fail(EP_A2A_ERR_INVALID_ARG, "combine pipeline must be -1 (automatic), 0 or 1");
+      h->combine_pipeline = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_COPY_PREFETCH:
       if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "prefetch must be 0 or 1");
@@ -370,7 +408,7 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
     case EP_A2A_OPT_COMBINE_CTAS_PER_SM:
       if (value < 0 || value > 1024)
         return fail(EP_A2A_ERR_INVALID_ARG, "combine CTAs per SM must be 0..1024");
-      h->combine_ctas_per_sm = value == 0 ? 128 : (int)value;
+      h->combine_ctas_per_sm = (int)value;
       return EP_A2A_OK;
   }
   return fail(EP_A2A_ERR_INVALID_ARG, "unknown option %d", (int)option);
@@ -590,16 +628,12 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   a.ntok = (int64_t)h->p.ep_size * h->last_tpr;
   a.H = h->combine_hidden;
   a.plan_stride = h->L.plan_stride;
-  a.prefetch = h->combine_prefetch < 0 ? (fp8 ? 1 : 0) : h->combine_prefetch;
+  const CombineLaunch c = combine_launch(h, fp8 ? kKindFp8 : kKindBf16, a.ntok);
+  a.prefetch = c.prefetch;
   const int elems = fp8 ? 16 : 8;
   const bool vec = a.H % elems == 0 && aligned(expert_output, 16) && aligned(output, 16);
-  const int grid = (int)std::max<int64_t>(
-      1, std::min<int64_t>(a.ntok, (int64_t)h->num_sms * h->combine_ctas_per_sm));
-  // 64-thread CTAs measured best for every token count (16-1024 CTAs per SM,
-  // 64-512 threads swept on the decode, wide-EP and prefill workloads)
-  const int threads = h->combine_threads > 0 ? h->combine_threads : 64;
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);
-  cudaError_t e = launch_combine(a, fp8, vec, threads, grid, (cudaStream_t)stream_v,
+  cudaError_t e = launch_combine(a, fp8, vec, c.pipe, c.threads, c.grid, (cudaStream_t)stream_v,
                                  h->pdl != 0);
   prof_end(h, slot, (cudaStream_t)stream_v);
   if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
@@ -628,15 +662,13 @@ EP_API ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle h, const float* topk_w
   a.E = h->p.num_experts;
   a.epr = h->p.num_experts / h->p.ep_size;
   a.plan_stride = h->L.plan_stride;
-  a.prefetch = h->combine_prefetch > 0 ? 1 : 0;
+  const CombineLaunch c = combine_launch(h, kKindExperts, a.ntok);
+  a.prefetch = c.prefetch;
   const bool vec = a.k <= 8 && a.H % 8 == 0 && aligned(expert_output_per_slot, 16) &&
                    aligned(output, 16);
-  const int grid = (int)std::max<int64_t>(
-      1, std::min<int64_t>(a.ntok, (int64_t)h->num_sms * h->combine_ctas_per_sm));
-  const int threads = h->combine_threads > 0 ? h->combine_threads : 64;
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE_EXPERTS, (cudaStream_t)stream_v);
-  cudaError_t e = launch_combine_experts(a, vec, threads, grid, (cudaStream_t)stream_v,
-                                         h->pdl != 0);
+  cudaError_t e = launch_combine_experts(a, vec, c.pipe, c.threads, c.grid,
+                                         (cudaStream_t)stream_v, h->pdl != 0);
   prof_end(h, slot, (cudaStream_t)stream_v);
   if (e != cudaSuccess) return cuda_fail(e, "expert combine kernel launch");
   return EP_A2A_OK;
@@ -658,13 +690,11 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
   a.ntok = (int64_t)h->p.ep_size * h->last_tpr;
   a.H = h->combine_hidden;
   a.plan_stride = h->L.plan_stride;
-  a.prefetch = h->combine_prefetch != 0 ? 1 : 0;   // default: on, as for the FP8 combine
+  const CombineLaunch c = combine_launch(h, kKindFp8, a.ntok);
+  a.prefetch = c.prefetch;
   const bool vec = a.H % 16 == 0 && aligned(expert_output_e4m3, 16) && aligned(output, 16);
-  const int grid = (int)std::max<int64_t>(
-      1, std::min<int64_t>(a.ntok, (int64_t)h->num_sms * h->combine_ctas_per_sm));
-  const int threads = h->combine_threads > 0 ? h->combine_threads : 64;
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);
-  cudaError_t e = launch_combine_scaled(a, row_scales, vec, threads, grid,
+  cudaError_t e = launch_combine_scaled(a, row_scales, vec, c.pipe, c.threads, c.grid,
                                         (cudaStream_t)stream_v, h->pdl != 0);
   prof_end(h, slot, (cudaStream_t)stream_v);
   if (e != cudaSuccess) return cuda_fail(e, "scaled combine kernel launch");

@@ -98,11 +98,13 @@ struct CombineArgs {
   int64_t ntok;                // ep * tpr
   int H;
   int plan_stride;
-  int prefetch;                // 1: prefetch the CTA's next token's rows into L2
+  int prefetch;                // p > 0: prefetch the rows of the CTA's token p
+                               // grid strides ahead into L2
 };
 
-cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, int threads, int grid,
-                           cudaStream_t stream, bool pdl);
+// pipe: the two-deep pipelined kernel (needs at most 8 destinations per token)
+cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, bool pipe, int threads,
+                           int grid, cudaStream_t stream, bool pdl);
 
 // Combine of per-(token, slot) expert outputs: the weighted reduction over each
 // destination's local experts fused into the combine.
@@ -116,16 +118,17 @@ struct CombineExpertsArgs {
   uint16_t* out;               // bf16 [ep*tpr, H]
   int64_t ntok;
   int H, k, E, epr, plan_stride;
-  int prefetch;                // 1: prefetch the CTA's next token's rows into L2
+  int prefetch;                // p > 0: prefetch the slot rows of the CTA's token p
+                               // grid strides ahead into L2
 };
 
-cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, int threads, int grid,
-                                   cudaStream_t stream, bool pdl);
+cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, bool pipe, int threads,
+                                   int grid, cudaStream_t stream, bool pdl);
 cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n, cudaStream_t stream);
 cudaError_t launch_quantize_e4m3_rows(const uint16_t* in, uint8_t* out, float* scales,
                                       int64_t rows, int hidden, cudaStream_t stream);
 // FP8 combine with one fp32 scale per row (scales [ep, ep*tpr]).
-cudaError_t launch_combine_scaled(const CombineArgs& a, const float* scales, bool vec,
+cudaError_t launch_combine_scaled(const CombineArgs& a, const float* scales, bool vec, bool pipe,
                                   int threads, int grid, cudaStream_t stream, bool pdl);
 cudaError_t launch_wait_timeout_probe(uint32_t* err, unsigned long long limit_ns,
                                       cudaStream_t stream);

@@ -303,11 +303,13 @@ typedef enum {
   EP_A2A_OPT_COPY_CTAS_PER_SM = 1,/* CTAs per SM of the bulk copy kernel (1..8) */
   EP_A2A_OPT_COPY_STAGES = 2,     /* shared-memory row stages per copy CTA (2..32; 0 = as
                                      many as fit, up to 8 / 16) */
-  EP_A2A_OPT_COMBINE_THREADS = 3, /* threads per CTA of the combine kernel (64..512);
-                                     0 (default) = 64 */
+  EP_A2A_OPT_COMBINE_THREADS = 3, /* threads per CTA of the combine kernels (64..512);
+                                     0 (default) = automatic: 128 for the FP8 combines of
+                                     16384 or more token slots, else 64 */
   EP_A2A_OPT_BULK_MIN_ROW_BYTES = 4, /* rows shorter than this take the vector copy (0..2^24) */
   EP_A2A_OPT_COMBINE_CTAS_PER_SM = 5, /* combine grid = min(tokens, SMs x this) (1..1024);
-                                       0 = 128 */
+                                       0 (default) = automatic: 16 for the FP8 combines
+                                       of 16384 or more token slots, else 128 */
   EP_A2A_OPT_COPY_CONSUMER_WARPS = 6, /* store warps per CTA of copy path 0 (4, 8 or 16) */
   EP_A2A_OPT_COPY_INTERLEAVE = 7, /* paths 0 and 2: 1 = CTA b copies tokens b, b + grid, ...
                                      (default); 0 = each CTA copies a contiguous chunk */
@@ -322,11 +324,19 @@ typedef enum {
                                      touches memory, so results do not change */
   EP_A2A_OPT_VEC_THREADS_PER_TOKEN = 12,/* vector copy: threads per token (32, 64, 128,
                                      256); 0 (default) = from the token count */
-  EP_A2A_OPT_COMBINE_PREFETCH = 13,/* combines: 1 = each CTA asks for its next token's rows
-                                     to be brought into L2 (cp.async.bulk.prefetch.L2)
-                                     while it sums the current one; 0 = never; -1
-                                     (default) = for the FP8 combine only */
-  EP_A2A_OPT_COPY_PREFETCH = 14   /* vector copy: the same for the next token's rows */
+  EP_A2A_OPT_COMBINE_PREFETCH = 13,/* combines: p in 1..4 = each CTA asks for the rows of
+                                     its token p grid strides ahead to be brought into L2
+                                     (cp.async.bulk.prefetch.L2) while it sums the current
+                                     one; 0 = never; -1 (default) = 1 for the FP8 combines
+                                     of 8192 or more token slots, else 0 */
+  EP_A2A_OPT_COPY_PREFETCH = 14,  /* vector copy: 1 = the same for the next token's rows */
+  EP_A2A_OPT_COMBINE_PIPELINE = 15/* BF16 / FP8 / scaled FP8 combines of 16-byte vectors
+                                     with at most 8 destinations per token (top_k or
+                                     ep_size <= 8): 1 = each thread keeps the loads of its
+                                     next column vector in flight while it adds the
+                                     current one; 0 = one vector at a time; -1 (default) =
+                                     on for the FP8, scaled FP8 and expert-output
+                                     combines, off for BF16 */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

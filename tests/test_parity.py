@@ -177,6 +177,64 @@ def test_combine_launch_shape_does_not_change_results(threads, ctas):
     U.check_combine(run, U.oracle_plan(w, x), w, x)
 
 
+@pytest.mark.parametrize("case", [
+    ("c2_ep8_decode", None),
+    ("c5_ep64_wide_masked", None),
+    ("c1_ep4_tiny", None),
+    ("mask", [0b10100101, 0, 0, 0]),       # tokens whose owners are all masked: +0
+    ("odd", None),                          # hidden 40: FP8 rows take the element kernels
+    ("wide_k", None),                       # top_k 16 over 16 ranks: not pipelined
+])
+@pytest.mark.parametrize("prefetch,threads", [(-1, 0), (2, 128), (0, 64)])
+def test_pipelined_combines_match_the_oracle(case, prefetch, threads):
+    """BF16, FP8, scaled-FP8 and expert-output combines with the two-deep
+    pipelined kernels."""
+    from combine_route_plan_b200 import ep_a2a
+    name, mask = case
+    if name in W.BY_NAME:
+        w = W.BY_NAME[name]
+        x = _inputs(w.name)
+    elif name == "mask":
+        w, x = _custom(8, 64, 6, 40, 64, [32], n=[40, 1, 0, 39, 17, 40, 2, 33], mask=mask, seed=8)
+    elif name == "odd":
+        w, x = _custom(4, 16, 4, 30, 40, [32], seed=19)
+    else:
+        w, x = _custom(16, 64, 16, 20, 64, [32], seed=23)
+    opts = {ep_a2a.OPT_COMBINE_PIPELINE: 1, ep_a2a.OPT_COMBINE_PREFETCH: prefetch,
+            ep_a2a.OPT_COMBINE_THREADS: threads}
+    run = U.Run(w, W.Inputs(w, x.token_selected_experts, x.local_num_tokens, x.payloads,
+                            x.eplb_local_stats, x.active_rank_mask, None), options=opts)
+    plan = U.oracle_plan(w, x)
+    xo = x.expert_output
+    H = w.hidden
+
+    def fresh():
+        return torch.full((w.ep_size, w.tokens_per_rank, H), U.OUT_CANARY, dtype=torch.int16,
+                          device="cuda").view(torch.bfloat16)
+    out, out8, outs = fresh(), fresh(), fresh()
+    run.comm.combine(xo.cuda(), out)
+    run.comm.combine(ep_a2a.quantize_e4m3(xo.cuda()), out8)
+    codes, scales = ep_a2a.quantize_e4m3_rows(xo.cuda())
+    run.comm.combine_scaled(codes, scales, outs)
+    torch.cuda.synchronize()
+    assert run.comm.get_status() == ep_a2a.OK
+    init = U.oracle_out_init(w)
+    xq = U.oracle_quantize_big(U.to_np(xo), U.oracle_e4m3_table())
+    oc, osc = U.oracle.quantize_e4m3_rows(U.to_np(xo), H)
+    U.assert_equal(out, U.oracle.combine(plan, U.to_np(xo), H, out_init=init), "bf16")
+    U.assert_equal(out8, U.oracle.combine(plan, xq, H, input_is_e4m3=True, out_init=init), "fp8")
+    U.assert_equal(outs, U.oracle.combine_scaled(plan, oc, osc, H, out_init=init), "scaled")
+    g = torch.Generator().manual_seed(w.top_k + H)
+    wts = torch.randn((w.ep_size, w.tokens_per_rank, w.top_k), generator=g)
+    y = torch.randn((w.ep_size, w.tokens_per_rank, w.top_k, H), generator=g).to(torch.bfloat16)
+    oute = fresh()
+    run.comm.combine_experts(wts.cuda(), y.cuda(), oute)
+    torch.cuda.synchronize()
+    U.assert_equal(oute, U.oracle.combine_experts(plan, w.num_experts,
+                                                  x.token_selected_experts.numpy(), wts.numpy(),
+                                                  U.to_np(y), H, out_init=init), "experts")
+
+
 def test_fp8_quantize_all_bf16_patterns():
     from combine_route_plan_b200 import ep_a2a
     table = U.oracle_e4m3_table()
