@@ -197,10 +197,11 @@ __device__ __forceinline__ void load_rows(uint4 (&r)[8], const uint8_t* const (&
 }
 
 // Sum one column vector over the rows in ascending destination order and store
-// it as bf16.
+// it as bf16 (the 32 output bytes of an E4M3 vector as one 256-bit store when
+// `wide`, i.e. the output is 32-byte aligned).
 template <int kMode>
 __device__ __forceinline__ void reduce_store(const uint4 (&r)[8], const float (&sc)[8], int nd,
-                                             uint16_t* o) {
+                                             uint16_t* o, bool wide) {
   constexpr int kElems = kMode == kCombineBf16 ? 8 : 16;
   float acc[kElems];
 #pragma unroll
@@ -216,15 +217,20 @@ __device__ __forceinline__ void reduce_store(const uint4 (&r)[8], const float (&
         fma_e4m3x16(acc, r[i], sc[i]);
     }
   }
+  uint32_t pk[kElems / 2];
 #pragma unroll
-  for (int q = 0; q < kElems / 8; ++q) {
-    uint4 pk;
-    pk.x = pack_bf16x2(acc[8 * q + 0], acc[8 * q + 1]);
-    pk.y = pack_bf16x2(acc[8 * q + 2], acc[8 * q + 3]);
-    pk.z = pack_bf16x2(acc[8 * q + 4], acc[8 * q + 5]);
-    pk.w = pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]);
-    reinterpret_cast<uint4*>(o)[q] = pk;
+  for (int i = 0; i < kElems / 2; ++i) pk[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+  if (kElems == 16 && wide) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(o),
+                 "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[kElems / 2 - 4]),
+                 "r"(pk[kElems / 2 - 3]), "r"(pk[kElems / 2 - 2]), "r"(pk[kElems / 2 - 1])
+                 : "memory");
+    return;
   }
+#pragma unroll
+  for (int q = 0; q < kElems / 8; ++q)
+    reinterpret_cast<uint4*>(o)[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
+                                                pk[4 * q + 3]);
 }
 
 // The combines for tokens with at most 8 destination ranks (top_k or ep_size
@@ -268,14 +274,14 @@ __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
     for (int v = threadIdx.x;;) {
       const bool more_b = v + (int)blockDim.x < nvec;
       if (more_b) load_rows(rb, src, nd, off + step);
-      reduce_store<kMode>(ra, sc, nd, o);
+      reduce_store<kMode>(ra, sc, nd, o, a.out32 != 0);
       if (!more_b) break;
       v += blockDim.x;
       off += step;
       o += ostep;
       const bool more_a = v + (int)blockDim.x < nvec;
       if (more_a) load_rows(ra, src, nd, off + step);
-      reduce_store<kMode>(rb, sc, nd, o);
+      reduce_store<kMode>(rb, sc, nd, o, a.out32 != 0);
       if (!more_a) break;
       v += blockDim.x;
       off += step;

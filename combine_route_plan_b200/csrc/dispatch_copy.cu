@@ -242,6 +242,33 @@ __device__ __forceinline__ void store_dst<uint4>(uint4* p, const uint4& v, bool 
     *p = v;
 }
 
+// 32-byte accesses (sm_100 256-bit loads and stores), the same hints.
+struct alignas(32) Vec32 {
+  uint32_t w[8];
+};
+template <>
+__device__ __forceinline__ Vec32 load_src<Vec32>(const Vec32* p) {
+  Vec32 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]),
+                 "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
+               : "l"(p));
+  return v;
+}
+template <>
+__device__ __forceinline__ void store_dst<Vec32>(Vec32* p, const Vec32& v, bool streaming) {
+  if (streaming)
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+                 "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]),
+                 "r"(v.w[6]), "r"(v.w[7])
+                 : "memory");
+  else
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+                 "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]),
+                 "r"(v.w[6]), "r"(v.w[7])
+                 : "memory");
+}
+
 // Copy one payload row of a token to its nd destinations: the TPT threads of a
 // token group each take vectors gl, gl + TPT, ... (U of them in flight).
 template <typename T, int U, int TPT>
@@ -315,18 +342,19 @@ __device__ __forceinline__ int token_destinations(const CopyArgs& a, int64_t tok
 // destinations from the routing ids itself, so the kernel does not depend on
 // the routing kernel's plan and may run alongside it (programmatic dependent
 // launch); it waits for the preceding grid only before it exits, so that work
-// after it sees the plan complete.  kAll16: every payload of the launch moves
-// in 16-byte vectors (one code path, fewer registers); otherwise each payload
-// picks its own vector width.
-template <int U, bool kAll16, bool kStreaming, int TPT>
+// after it sees the plan complete.  kAll = 16 or 32: every payload of the
+// launch moves in vectors of that many bytes (one code path, fewer registers);
+// kAll = 0: each payload picks its own vector width.
+template <int U, int kAll, bool kStreaming, int TPT>
 __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArgs a) {
+  constexpr bool kUniform = kAll != 0;
   constexpr int kGroups = kVecThreads / TPT;
   const int gl = threadIdx.x % TPT;
   const int group = threadIdx.x / TPT;
   const int lane = threadIdx.x & 31;
   const int64_t tok_step = (int64_t)gridDim.x * kGroups;
   for (int64_t tok = (int64_t)blockIdx.x * kGroups + group; tok < a.ntok; tok += tok_step) {
-    if (kAll16 && a.prefetch && gl == 0 && tok + tok_step < a.ntok) {
+    if (kUniform && a.prefetch && gl == 0 && tok + tok_step < a.ntok) {
       // the group's next token: its rows into L2 while this one is copied
       for (int p = 0; p < a.np; ++p)
         prefetch_l2(a.src[p] + (tok + tok_step) * a.rb[p], (uint32_t)a.rb[p]);
@@ -337,12 +365,21 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
     for (int p = 0; p < a.np; ++p) {
       const uint8_t* src = a.src[p] + tok * a.rb[p];
       const int64_t off = a.dst_off[p] + tok * a.rb[p];
-      if (kAll16) {
+      if (kAll == 32) {
+        copy_row<Vec32, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
+                                gl, kStreaming);
+        continue;
+      }
+      if (kAll == 16) {
         copy_row<uint4, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
                                 gl, kStreaming);
         continue;
       }
       switch (a.vec[p]) {
+        case 32:
+          copy_row<Vec32, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
+                                  gl, kStreaming);
+          break;
         case 16:
           copy_row<uint4, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
                                   gl, kStreaming);
@@ -556,17 +593,25 @@ cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t strea
 template <int U, int TPT>
 cudaError_t launch_vec_ut(const CopyArgs& a, int grid, bool streaming, cudaStream_t stream,
                           bool pdl) {
-  bool all16 = true;
-  for (int p = 0; p < a.np; ++p) all16 &= a.vec[p] == 16;
+  bool all16 = true, all32 = true;
+  for (int p = 0; p < a.np; ++p) {
+    all16 &= a.vec[p] == 16;
+    all32 &= a.vec[p] == 32;
+  }
   const dim3 g(grid), b(kVecThreads);
+  if (all32) {
+    if (streaming)
+      return launch_kernel(dispatch_vec_kernel<U, 32, true, TPT>, g, b, 0, stream, pdl, a);
+    return launch_kernel(dispatch_vec_kernel<U, 32, false, TPT>, g, b, 0, stream, pdl, a);
+  }
   if (all16) {
     if (streaming)
-      return launch_kernel(dispatch_vec_kernel<U, true, true, TPT>, g, b, 0, stream, pdl, a);
-    return launch_kernel(dispatch_vec_kernel<U, true, false, TPT>, g, b, 0, stream, pdl, a);
+      return launch_kernel(dispatch_vec_kernel<U, 16, true, TPT>, g, b, 0, stream, pdl, a);
+    return launch_kernel(dispatch_vec_kernel<U, 16, false, TPT>, g, b, 0, stream, pdl, a);
   }
   if (streaming)
-    return launch_kernel(dispatch_vec_kernel<U, false, true, TPT>, g, b, 0, stream, pdl, a);
-  return launch_kernel(dispatch_vec_kernel<U, false, false, TPT>, g, b, 0, stream, pdl, a);
+    return launch_kernel(dispatch_vec_kernel<U, 0, true, TPT>, g, b, 0, stream, pdl, a);
+  return launch_kernel(dispatch_vec_kernel<U, 0, false, TPT>, g, b, 0, stream, pdl, a);
 }
 
 template <int U>

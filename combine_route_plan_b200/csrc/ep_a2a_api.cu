@@ -143,6 +143,7 @@ struct ep_a2a_handle_s {
   // combine launch shape; -1 / 0 = automatic (combine_launch)
   int combine_prefetch;       // tokens ahead (grid strides) whose rows go to L2
   int copy_prefetch;          // vector copy: prefetch the next token's rows
+  int copy_vec_bytes;         // vector copy: widest access, 16 or 32 bytes
   int combine_pipeline;       // 1: the two-deep pipelined kernels
   int copy_ctas_per_sm;
   int copy_stages;        // 0 = choose from the row size
@@ -226,8 +227,25 @@ CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
   return c;
 }
 
-uint32_t vec_bytes(const void* src, const void* dst_base, int64_t rank_stride, int64_t rb) {
-  for (uint32_t v : {16u, 8u, 4u, 2u}) {
+// Vectors per thread in flight in the vector copy: the fewest of 2, 4, 8 with
+// which a token group moves its largest row in at most two rounds (measured:
+// 8 for the prefill rows of 448 32-byte vectors over a warp, 2 for the
+// 3.5-14 KB rows of the decode, Zipf and wide-EP steps; a group with more
+// vectors in flight than its row has only ties up registers).
+int copy_unroll(const CopyArgs& c, int tpt) {
+  int64_t most = 0;
+  for (int p = 0; p < c.np; ++p) most = std::max<int64_t>(most, c.rb[p] / (int64_t)c.vec[p]);
+  const int64_t per_thread = (most + tpt - 1) / tpt;
+  if (per_thread <= 4) return 2;
+  if (per_thread <= 8) return 4;
+  return 8;
+}
+
+// Widest access (up to `widest` bytes) that every row of a payload allows.
+uint32_t vec_bytes(const void* src, const void* dst_base, int64_t rank_stride, int64_t rb,
+                   uint32_t widest) {
+  for (uint32_t v : {32u, 16u, 8u, 4u, 2u}) {
+    if (v > widest) continue;
     if (rb % v == 0 && aligned(src, v) && aligned(dst_base, v) && rank_stride % v == 0) return v;
   }
   return 1u;
@@ -306,19 +324,21 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   h->last_tpr = 0;
   h->combine_hidden = params->hidden_size;
   // Defaults measured on the prefill workload (ep 8, 4096 tokens/rank, 14.4 KB
-  // rows): the vector copy with 4 vectors per lane in flight, 32 CTAs per SM
-  // requested and evict-first stores moved the rows fastest (487 us, against
-  // 527 us for the staged bulk-load path and 539 us for bulk loads + stores).
+  // rows): the vector copy with 32 CTAs per SM requested and evict-first stores
+  // moved the rows fastest (487 us with 16-byte vectors, against 527 us for the
+  // staged bulk-load path and 539 us for bulk loads + stores); 32-byte vectors
+  // took it to 475 us (decode, Zipf and wide-EP workloads: 1-4 % faster too).
   h->copy_path = 1;
   h->copy_consumer_warps = 4;
   h->copy_interleave = 1;
-  h->vec_unroll = 4;
+  h->vec_unroll = 0;
   h->vec_ctas_per_sm = 32;
   h->store_streaming = 1;
   h->pdl = 1;
   h->vec_threads_per_token = 0;
   h->combine_prefetch = -1;       // automatic (combine_launch)
   h->copy_prefetch = 0;
+  h->copy_vec_bytes = 32;
   h->combine_pipeline = -1;
   h->copy_ctas_per_sm = 1;
   h->copy_stages = 4;
@@ -364,8 +384,8 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       h->copy_interleave = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_VEC_UNROLL:
-      if (value != 2 && value != 4 && value != 8)
-        return fail(EP_A2A_ERR_INVALID_ARG, "vector unroll must be 2, 4 or 8");
+      if (value != 0 && value != 2 && value != 4 && value != 8)
+        return fail(EP_A2A_ERR_INVALID_ARG, "vector unroll must be 0 (automatic), 2, 4 or 8");
       h->vec_unroll = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_VEC_CTAS_PER_SM:
@@ -386,6 +406,11 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       if (value < -1 || value > 4)
         return fail(EP_A2A_ERR_INVALID_ARG, "prefetch must be -1 (FP8 only), 0 or 1..4");
       h->combine_prefetch = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_COPY_VEC_BYTES:
+      if (value != 16 && value != 32)
+        return fail(EP_A2A_ERR_INVALID_ARG, "vector copy width must be 16 or 32 bytes");
+      h->copy_vec_bytes = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_COMBINE_PIPELINE:
       if (value < -1 || value > 1)
@@ -537,7 +562,8 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
       c.smem_off[j] = stage;
       stage += (uint32_t)rb[i];
     } else {
-      c.vec[j] = vec_bytes(src, rank0 + L.off_payload[i], L.rank_stride, rb[i]);
+      c.vec[j] = vec_bytes(src, rank0 + L.off_payload[i], L.rank_stride, rb[i],
+                           (uint32_t)h->copy_vec_bytes);
     }
   }
   if (bulk.np > 0) {
@@ -561,7 +587,8 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
         vec.src[k] = bulk.src[j];
         vec.rb[k] = bulk.rb[j];
         vec.dst_off[k] = bulk.dst_off[j];
-        vec.vec[k] = vec_bytes(bulk.src[j], rank0 + bulk.dst_off[j], L.rank_stride, bulk.rb[j]);
+        vec.vec[k] = vec_bytes(bulk.src[j], rank0 + bulk.dst_off[j], L.rank_stride, bulk.rb[j],
+                               (uint32_t)h->copy_vec_bytes);
       }
       bulk.np = 0;
     } else {
@@ -586,8 +613,9 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
     const int grid = (int)std::max<int64_t>(
         1, std::min<int64_t>((ntok + groups_per_cta - 1) / groups_per_cta,
                              (int64_t)h->num_sms * h->vec_ctas_per_sm));
+    const int unroll = h->vec_unroll > 0 ? h->vec_unroll : copy_unroll(vec, tpt);
     slot = prof_begin(h, EP_A2A_KERNEL_COPY_VEC, stream);
-    e = launch_dispatch_vec(vec, grid, h->vec_unroll, tpt, h->store_streaming != 0, stream, pdl);
+    e = launch_dispatch_vec(vec, grid, unroll, tpt, h->store_streaming != 0, stream, pdl);
     prof_end(h, slot, stream);
     if (e != cudaSuccess) return cuda_fail(e, "vector copy kernel launch");
   }
@@ -630,6 +658,7 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   a.plan_stride = h->L.plan_stride;
   const CombineLaunch c = combine_launch(h, fp8 ? kKindFp8 : kKindBf16, a.ntok);
   a.prefetch = c.prefetch;
+  a.out32 = aligned(output, 32) ? 1 : 0;
   const int elems = fp8 ? 16 : 8;
   const bool vec = a.H % elems == 0 && aligned(expert_output, 16) && aligned(output, 16);
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);
@@ -692,6 +721,7 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
   a.plan_stride = h->L.plan_stride;
   const CombineLaunch c = combine_launch(h, kKindFp8, a.ntok);
   a.prefetch = c.prefetch;
+  a.out32 = aligned(output, 32) ? 1 : 0;
   const bool vec = a.H % 16 == 0 && aligned(expert_output_e4m3, 16) && aligned(output, 16);
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);
   cudaError_t e = launch_combine_scaled(a, row_scales, vec, c.pipe, c.threads, c.grid,

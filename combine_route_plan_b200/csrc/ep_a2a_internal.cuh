@@ -100,6 +100,8 @@ struct CombineArgs {
   int plan_stride;
   int prefetch;                // p > 0: prefetch the rows of the CTA's token p
                                // grid strides ahead into L2
+  int out32;                   // pipelined E4M3 combines: one 32-byte store per
+                               // vector (output 32-byte aligned)
 };
 
 // pipe: the two-deep pipelined kernel (needs at most 8 destinations per token)

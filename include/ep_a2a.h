@@ -313,7 +313,9 @@ typedef enum {
   EP_A2A_OPT_COPY_CONSUMER_WARPS = 6, /* store warps per CTA of copy path 0 (4, 8 or 16) */
   EP_A2A_OPT_COPY_INTERLEAVE = 7, /* paths 0 and 2: 1 = CTA b copies tokens b, b + grid, ...
                                      (default); 0 = each CTA copies a contiguous chunk */
-  EP_A2A_OPT_VEC_UNROLL = 8,      /* vector copy: vectors per lane in flight (2, 4 = default, 8) */
+  EP_A2A_OPT_VEC_UNROLL = 8,      /* vector copy: vectors per lane in flight (2, 4, 8; 0 =
+                                     default: the fewest that move the largest row in
+                                     two rounds) */
   EP_A2A_OPT_VEC_CTAS_PER_SM = 9, /* vector copy grid = SMs x this (1..64; default 32) */
   EP_A2A_OPT_STORE_STREAMING = 10,/* vector copy: 1 = evict-first (.cs) 16-byte stores
                                      (default), 0 = plain stores */
@@ -330,13 +332,16 @@ typedef enum {
                                      one; 0 = never; -1 (default) = 1 for the FP8 combines
                                      of 8192 or more token slots, else 0 */
   EP_A2A_OPT_COPY_PREFETCH = 14,  /* vector copy: 1 = the same for the next token's rows */
-  EP_A2A_OPT_COMBINE_PIPELINE = 15/* BF16 / FP8 / scaled FP8 combines of 16-byte vectors
+  EP_A2A_OPT_COMBINE_PIPELINE = 15,/* BF16 / FP8 / scaled FP8 combines of 16-byte vectors
                                      with at most 8 destinations per token (top_k or
                                      ep_size <= 8): 1 = each thread keeps the loads of its
                                      next column vector in flight while it adds the
                                      current one; 0 = one vector at a time; -1 (default) =
                                      on for the FP8, scaled FP8 and expert-output
                                      combines, off for BF16 */
+  EP_A2A_OPT_COPY_VEC_BYTES = 16  /* vector copy: widest access per thread, 16 or 32
+                                     (default) bytes (sm_100 256-bit loads and stores,
+                                     for rows and addresses that are 32-byte multiples) */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

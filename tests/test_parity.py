@@ -93,6 +93,73 @@ def test_vector_copy_variants(unroll, ctas, streaming, tpt, rows):
     U.check_payloads(run, plan, w, x)
 
 
+@pytest.mark.parametrize("name", ["c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked",
+                                  "c3_ep16_zipf_nvfp4", "c3_ep16_zipf_mxfp8"])
+def test_vector_copy_32_byte_accesses(name):
+    """256-bit loads and stores where every row allows them (all-32 kernel),
+    per-payload widths otherwise."""
+    from combine_route_plan_b200 import ep_a2a
+    _full_check(W.BY_NAME[name], options={ep_a2a.OPT_COPY_VEC_BYTES: 32})
+
+
+@pytest.mark.parametrize("rows,shift", [([14336, 64, 32], 0), ([14336, 48], 0),
+                                        ([4096 + 16, 32], 16), ([7, 96, 224], 0)])
+def test_vector_copy_32_byte_mixed_rows(rows, shift):
+    """Rows that are 32-byte multiples next to rows that are not, and sources
+    that are only 16-byte aligned."""
+    from combine_route_plan_b200 import ep_a2a
+    ep, E, k, tpr, H = 8, 64, 8, 50, 32
+    w, x = _custom(ep, E, k, tpr, H, rows, seed=sum(rows) % 1000 + shift)
+    comm = ep_a2a.EpA2A(ep, E, k, tpr, H, rows, workspace_fill=U.CANARY)
+    comm.set_option(ep_a2a.OPT_COPY_VEC_BYTES, 32)
+    for tpt in (32, 256):
+        comm.set_option(ep_a2a.OPT_VEC_THREADS_PER_TOKEN, tpt)
+        srcs = []
+        for p in x.payloads:
+            buf = torch.empty(p.numel() + 64, dtype=torch.uint8, device="cuda")
+            v = buf[shift: shift + p.numel()].view(p.shape)
+            v.copy_(p.cuda())
+            srcs.append(v)
+        d = comm.dispatch(x.token_selected_experts.cuda(), x.local_num_tokens, srcs, tpr)
+        torch.cuda.synchronize()
+        plan = U.oracle_plan(w, x)
+        for i, p in enumerate(x.payloads):
+            for dst in range(ep):
+                want = U.oracle.dispatch_payload(plan, p.numpy(), only_dst=dst, recv_init=np.full(
+                    (1, ep * tpr, p.shape[2]), U.CANARY, np.uint8))
+                U.assert_equal(d.recv_payloads[i][dst], want, f"payload {i} rank {dst} tpt {tpt}")
+
+
+@pytest.mark.parametrize("name", ["c2_ep8_decode", "c5_ep64_wide_masked"])
+def test_fp8_combines_with_16_byte_aligned_output(name):
+    """The pipelined E4M3 combines store 32 bytes at once only into 32-byte
+    aligned outputs; a 16-byte aligned output takes two 16-byte stores."""
+    from combine_route_plan_b200 import ep_a2a
+    w = W.BY_NAME[name]
+    x = _inputs(w.name)
+    run = U.Run(w, W.Inputs(w, x.token_selected_experts, x.local_num_tokens, x.payloads,
+                            x.eplb_local_stats, x.active_rank_mask, None))
+    plan = U.oracle_plan(w, x)
+    n = w.ep_size * w.tokens_per_rank * w.hidden
+    xo = x.expert_output
+    init = U.oracle_out_init(w)
+    for shift in (8, 0):       # in bf16 elements: 16 and 0 bytes
+        buf = torch.full((n + 16,), U.OUT_CANARY, dtype=torch.int16, device="cuda")
+        out = buf[shift: shift + n].view(torch.bfloat16).view(w.ep_size, w.tokens_per_rank, w.hidden)
+        run.comm.combine(ep_a2a.quantize_e4m3(xo.cuda()), out)
+        torch.cuda.synchronize()
+        xq = U.oracle_quantize_big(U.to_np(xo), U.oracle_e4m3_table())
+        U.assert_equal(out, U.oracle.combine(plan, xq, w.hidden, input_is_e4m3=True,
+                                             out_init=init), f"fp8 shift {shift}")
+        buf.fill_(U.OUT_CANARY)
+        codes, scales = ep_a2a.quantize_e4m3_rows(xo.cuda())
+        run.comm.combine_scaled(codes, scales, out)
+        torch.cuda.synchronize()
+        oc, osc = U.oracle.quantize_e4m3_rows(U.to_np(xo), w.hidden)
+        U.assert_equal(out, U.oracle.combine_scaled(plan, oc, osc, w.hidden, out_init=init),
+                       f"scaled shift {shift}")
+
+
 @pytest.mark.parametrize("rows", [[16], [4096 + 16, 32], [65536 + 16, 48]])
 def test_staged_copy_row_sizes(rows):
     """Rows from one vector per token up to more than the staged kernel holds in
