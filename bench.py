@@ -491,9 +491,11 @@ def run_ours(args):
         e2e = None if (scaled or dense) else run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws,
                                           y_dev=y if experts else None)
 
-    cpu = None
+    cpu = cpu_all = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_seconds)
+        if args.cpu_all_cores_seconds > 0:
+            cpu_all = cpu_baseline_all_cores(w, args.cpu_all_cores_seconds)
 
     if rank == 0:
         rec = {
@@ -529,6 +531,7 @@ def run_ours(args):
             "clocks": clocks.record(),
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "cpu_baseline_all_cores": cpu_all,
             "kernel_sources": kernel_sources_hash(),
         }
         if fp8_ctx:
@@ -577,23 +580,42 @@ def run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws, y_dev=None):
         (h_stats.nbytes if h_stats is not None else 0)
     d2h = h_out.nbytes
 
+    # Three streams: the inputs go up on s_in once the previous step's kernels
+    # are done with the device buffers, the result comes down on s_out, so a
+    # step's result download overlaps the next step's upload (separate copy
+    # engines, PCIe is full duplex); the kernels run on `stream`.
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+
     def step():
-        d_ids.copy_(h_ids, non_blocking=True)
-        for d, h in zip(d_pay, h_pay):
-            d.copy_(h, non_blocking=True)
-        if d_stats is not None:
-            d_stats.copy_(h_stats, non_blocking=True)
-        d_xo.copy_(h_xo, non_blocking=True)
+        s_in.wait_stream(stream)
+        with torch.cuda.stream(s_in):
+            d_ids.copy_(h_ids, non_blocking=True)
+            for d, h in zip(d_pay, h_pay):
+                d.copy_(h, non_blocking=True)
+            if d_stats is not None:
+                d_stats.copy_(h_stats, non_blocking=True)
+            d_xo.copy_(h_xo, non_blocking=True)
+        stream.wait_stream(s_in)
         comm.dispatch(d_ids, x.local_num_tokens, d_pay, w.tokens_per_rank, d_stats,
-                      x.active_rank_mask, views=False)
+                      x.active_rank_mask, stream=stream, views=False)
+        stream.wait_stream(s_out)        # d_out: the previous download is done
         if y_dev is not None:
             wts = d_pay[-1].view(torch.float32).view(w.ep_size, w.tokens_per_rank, w.top_k)
-            comm.combine_experts(wts, d_xo, d_out)
+            comm.combine_experts(wts, d_xo, d_out, stream=stream)
         else:
-            comm.combine(d_xo, d_out)
-        h_out.copy_(d_out, non_blocking=True)
+            comm.combine(d_xo, d_out, stream=stream)
+        s_out.wait_stream(stream)
+        with torch.cuda.stream(s_out):
+            h_out.copy_(d_out, non_blocking=True)
 
-    ms = run_timed(step, args.e2e_steps, 2, CudaTimer(stream), dist, device)
+    class JoinTimer(CudaTimer):
+        """Stops only after the last step's download."""
+
+        def stop(self) -> float:
+            self.stream.wait_stream(s_out)
+            return super().stop()
+
+    ms = run_timed(step, args.e2e_steps, 2, JoinTimer(stream), dist, device)
     return {"value": ws * n_tok * args.e2e_steps / (ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "steps": args.e2e_steps, "ms_per_step": ms / args.e2e_steps}
@@ -641,6 +663,58 @@ def cpu_baseline(w, seconds: float, tokens_per_rank: int = 1024):
                       f"({toks // reps} tokens) x {reps} steps, route + dispatch + EPLB + "
                       f"BF16 combine, {dt:.1f} s, single thread",
             "host_cpus": os.cpu_count()}
+
+
+def _oracle_worker(name: str, tokens_per_rank: int, seconds: float, barrier_, results):
+    """One process of the all-cores baseline: the oracle, single-threaded, on
+    its own copy of the sample, from the moment every process is ready."""
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import torch
+    torch.set_num_threads(1)
+    from combine_route_plan_b200 import workloads as W
+    ws = W.scaled(W.BY_NAME[name], tokens_per_rank)
+    xs = W.make_inputs(ws)
+    oracle_step(ws, xs)            # untimed: page in buffers
+    barrier_.wait()
+    t0 = time.perf_counter()
+    toks = reps = 0
+    while True:
+        toks += oracle_step(ws, xs)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    results.put((toks, time.perf_counter() - t0, reps))
+
+
+def cpu_baseline_all_cores(w, seconds: float, tokens_per_rank: int = 128, procs: int = 0):
+    """The oracle as it stands on every host core: one single-threaded process
+    per core, each on its own copy of a bounded sample (the same shapes with
+    fewer tokens per rank), started together; tokens of all processes over
+    the slowest one's time.  Processes are spawned (never forked after CUDA
+    work)."""
+    import multiprocessing as mp
+    import oracle
+    oracle.build()
+    n = procs or len(os.sched_getaffinity(0))
+    ctx = mp.get_context("spawn")
+    barrier_ = ctx.Barrier(n)
+    results = ctx.Queue()
+    tpr = min(tokens_per_rank, w.tokens_per_rank)
+    ps = [ctx.Process(target=_oracle_worker, args=(w.name, tpr, seconds, barrier_, results))
+          for _ in range(n)]
+    for p in ps:
+        p.start()
+    got = [results.get(timeout=600) for _ in ps]
+    for p in ps:
+        p.join(timeout=60)
+    toks = sum(g[0] for g in got)
+    dt = max(g[1] for g in got)
+    reps = min(g[2] for g in got)
+    return {"value": toks / dt, "unit": UNIT, "cores": n, "kind": "oracle",
+            "sample": f"{w.name} at {tpr} tokens/rank: {n} single-threaded processes, each on "
+                      f"its own copy, >= {reps} steps of route + dispatch + EPLB + BF16 combine "
+                      f"in {dt:.1f} s"}
 
 
 def run_reference(args):
@@ -702,6 +776,8 @@ def main(argv=None):
     ap.add_argument("--fp8-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-all-cores-seconds", type=float, default=10.0,
+                    help="also time the oracle on every host core (one process each); 0 = skip")
     ap.add_argument("--ref-budget-s", type=float, default=120.0)
     ap.add_argument("--graph", action="store_true",
                     help="time CUDA-graph replays of the step (small workloads)")

@@ -411,7 +411,8 @@ __global__ void __launch_bounds__(512) combine_experts_vec_kernel(const CombineE
           }
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], bf16_round(z[e]));
+        for (int e = 0; e < 4; ++e)       // z_d to bf16 in pairs, then added exactly widened
+          add_bf16x2(acc[2 * e], acc[2 * e + 1], pack_bf16x2(z[2 * e], z[2 * e + 1]));
       }
       uint4 pk;
       pk.x = pack_bf16x2(acc[0], acc[1]);
@@ -457,7 +458,8 @@ __device__ __forceinline__ void expert_rows_reduce_store(const uint4 (&raw)[8],
       }
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], bf16_round(z[e]));
+    for (int e = 0; e < 4; ++e)           // z_d to bf16 in pairs, then added exactly widened
+      add_bf16x2(acc[2 * e], acc[2 * e + 1], pack_bf16x2(z[2 * e], z[2 * e + 1]));
   }
   uint4 pk;
   pk.x = pack_bf16x2(acc[0], acc[1]);

@@ -76,3 +76,12 @@ def test_algorithmic_bytes_of_the_prefill_step():
     assert b.combine == sum_d * 7168 * 2 + n_tok * 7168 * 2
     b8 = bench.algorithmic_bytes(w, n_tok, sum_d, live=8, fp8=True)
     assert b8.combine == sum_d * 7168 + n_tok * 7168 * 2
+
+
+def test_all_cores_oracle_baseline_runs_spawned_processes():
+    sys.path.insert(0, ROOT)
+    import bench
+    from combine_route_plan_b200 import workloads as W
+    rec = bench.cpu_baseline_all_cores(W.C1, 0.5, tokens_per_rank=16, procs=2)
+    assert rec["cores"] == 2 and rec["kind"] == "oracle" and rec["value"] > 0
+    assert "2 single-threaded processes" in rec["sample"]

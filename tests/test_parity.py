@@ -385,6 +385,60 @@ def test_edge_shapes(ep, E, k, tpr, H, rows):
     U.check_combine(run, plan, w, x)
 
 
+def _mask_of(ep, live):
+    words = [0, 0, 0, 0]
+    for r in live:
+        words[r // 64] |= 1 << (r % 64)
+    return words
+
+
+@pytest.mark.parametrize("case", [
+    # the largest ep_size and top_k, one expert per rank
+    dict(ep=256, E=256, k=32, tpr=4, H=64, rows=[32, 16]),
+    # a mask spanning all four mask words, k 8 over 512 experts
+    dict(ep=256, E=512, k=8, tpr=3, H=16, rows=[8],
+         live=[0, 1, 63, 64, 100, 127, 128, 200, 254, 255]),
+    # one token slot per rank, hidden 1 (element kernels), one-byte rows
+    dict(ep=7, E=28, k=4, tpr=1, H=1, rows=[1]),
+    # no rank has a token
+    dict(ep=8, E=64, k=8, tpr=16, H=32, rows=[16], n=[0] * 8),
+    # one live rank with tokens, the others empty or masked off
+    dict(ep=8, E=64, k=8, tpr=16, H=32, rows=[16], n=[0, 0, 16, 0, 5, 0, 0, 0],
+         live=[2, 5, 6]),
+])
+def test_extreme_shapes(case):
+    """Maximum and degenerate sizes: every plan array, payload and the BF16,
+    FP8 and expert-output combines against the oracle."""
+    from combine_route_plan_b200 import ep_a2a
+    ep, E, k, tpr, H, rows = (case[key] for key in ("ep", "E", "k", "tpr", "H", "rows"))
+    mask = _mask_of(ep, case["live"]) if "live" in case else None
+    w, x = _custom(ep, E, k, tpr, H, rows, n=case.get("n"), mask=mask, seed=ep + k + tpr)
+    run = U.Run(w, x)
+    plan = U.oracle_plan(w, x)
+    U.check_plan(run, plan, w)
+    U.check_payloads(run, plan, w, x)
+    U.check_combine(run, plan, w, x)
+    init = U.oracle_out_init(w)
+    out8 = torch.full((ep, tpr, H), U.OUT_CANARY, dtype=torch.int16,
+                      device="cuda").view(torch.bfloat16)
+    run.comm.combine(ep_a2a.quantize_e4m3(x.expert_output.cuda()), out8)
+    g = torch.Generator().manual_seed(ep * k)
+    wts = torch.randn((ep, tpr, k), generator=g)
+    y = torch.randn((ep, tpr, k, H), generator=g).to(torch.bfloat16)
+    oute = torch.full((ep, tpr, H), U.OUT_CANARY, dtype=torch.int16,
+                      device="cuda").view(torch.bfloat16)
+    run.comm.combine_experts(wts.cuda(), y.cuda(), oute)
+    torch.cuda.synchronize()
+    assert run.comm.get_status() == ep_a2a.OK
+    xq = U.oracle_quantize_big(U.to_np(x.expert_output), U.oracle_e4m3_table())
+    U.assert_equal(out8, U.oracle.combine(plan, xq, H, input_is_e4m3=True, out_init=init), "fp8")
+    U.assert_equal(oute, U.oracle.combine_experts(plan, E, x.token_selected_experts.numpy(),
+                                                  wts.numpy(), U.to_np(y), H, out_init=init),
+                   "experts")
+    if "n" in case and not any(case["n"]):
+        assert int(run.d.send_counts.sum()) == 0 and int(run.d.recv_valid.sum()) == 0
+
+
 def test_misaligned_payload_pointers():
     ep, E, k, tpr, H = 4, 16, 4, 25, 64
     w, x = _custom(ep, E, k, tpr, H, [64, 32], seed=5)
