@@ -270,16 +270,26 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and blank space, so that editing a comment
+    does not count as changing a kernel (the sources hold no string literals
+    with comment markers)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_sources_hash() -> str:
-    """Hash of the CUDA sources, to tell whether committed ncu counters still
-    describe the kernels that run."""
+    """Hash of the CUDA sources' code (comments and spacing ignored), to tell
+    whether committed ncu counters still describe the kernels that run."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "combine_route_plan_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
                 h.update(name.encode())
-                h.update(f.read())
+                h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -5,29 +5,32 @@
 // Bytes are moved verbatim, so every bit pattern arrives unchanged.
 //
 // Three kernels:
-//   * dispatch_staged_kernel (default) — for payloads whose rows are 16-byte
-//     multiples at 16-byte-aligned addresses.  A producer warp streams each
-//     token's rows from HBM into a ring of shared-memory stages with bulk-async
-//     loads (completion counted on a "full" mbarrier per stage); consumer warps
-//     copy the token from shared memory into registers, release the stage
-//     ("empty" mbarrier), and write the rows to every destination with 16-byte
-//     vector stores, all threads of the CTA sharing each token.  Loads run as
-//     far ahead as the ring allows and cost no registers; the SM's threads only
+//   * dispatch_vec_kernel (default) — any row size and alignment.  A group of
+//     32..256 threads per token finds the token's destinations from its routing
+//     ids (the routing kernel's rule, so it need not wait for the plan), loads
+//     each row once in the widest aligned vectors (32 bytes with sm_100 256-bit
+//     accesses, else 16 down to 1) into registers, and stores them to every
+//     destination with evict-first stores.
+//   * dispatch_staged_kernel — for payloads whose rows are 16-byte multiples at
+//     16-byte-aligned addresses.  A producer warp streams each token's rows
+//     from HBM into a ring of shared-memory stages with bulk-async loads
+//     (completion counted on a "full" mbarrier per stage); consumer warps copy
+//     the token from shared memory into registers, release the stage ("empty"
+//     mbarrier), and write the rows to every destination with 16-byte vector
+//     stores, all threads of the CTA sharing each token.  Loads run as far
+//     ahead as the ring allows and cost no registers; the SM's threads only
 //     issue stores.
 //   * dispatch_bulk_kernel — the same staging, but the copy engine also does
-//     the stores (one bulk-async store per destination and payload).  For rows
-//     that are 16-byte multiples at
-//     16-byte-aligned addresses.  One warp per CTA; lane 0 drives a ring of
-//     shared-memory stages: a bulk-async load (cp.async.bulk, completion on an
-//     mbarrier) brings one token's rows of all such payloads into a stage, then
-//     one bulk-async store per (destination, payload) writes the stage out.
-//     Loads run `L = stages - Q` tokens ahead of the stores, and at most Q
-//     tokens' store groups are still reading shared memory when a stage is
-//     refilled.  The copy engine generates the addresses; the SM only issues.
-//   * dispatch_vec_kernel (default) — any row size and alignment.  A group of
-//     32..256 threads per token loads the row in the widest aligned vectors
-//     into registers once and stores them to each destination.
-// Both read the plan (plan_nd / plan_dst) the routing kernel wrote just before.
+//     the stores (one bulk-async store per destination and payload).  One warp
+//     per CTA; lane 0 drives a ring of shared-memory stages: a bulk-async load
+//     (cp.async.bulk, completion on an mbarrier) brings one token's rows of all
+//     such payloads into a stage, then one bulk-async store per (destination,
+//     payload) writes the stage out.  Loads run `L = stages - Q` tokens ahead of
+//     the stores, and at most Q tokens' store groups are still reading shared
+//     memory when a stage is refilled.  The copy engine generates the
+//     addresses; the SM only issues.
+// The two staged kernels read the plan (plan_nd / plan_dst) the routing kernel
+// wrote just before them.
 #include "ep_a2a_internal.cuh"
 
 namespace ep_a2a {
