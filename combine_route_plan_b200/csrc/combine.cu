@@ -12,7 +12,10 @@
 // destination rows before the adds, so one thread keeps up to 128 bytes in
 // flight.  Loads bypass L1 (each row is read exactly once).  The widening and
 // the add are one sm_100 mixed-precision instruction per element
-// (add.rn.f32.bf16 / add.rn.f32.f16).
+// (add.rn.f32.bf16 / add.rn.f32.f16).  The E4M3 combines and the combine of
+// per-slot expert outputs do more arithmetic per loaded byte, so their
+// kernels (combine_pipe_kernel, combine_experts_pipe_kernel) keep a second
+// vector's loads in flight while they reduce the first.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>

@@ -64,7 +64,7 @@ struct CopyArgs {
   int64_t rb[kMaxPayloads];              // row bytes
   int64_t dst_off[kMaxPayloads];         // receive array offset inside a rank region
   uint32_t smem_off[kMaxPayloads];       // bulk path: offset of the row in a stage
-  uint32_t vec[kMaxPayloads];            // vector path: bytes per access (16/8/4/2/1)
+  uint32_t vec[kMaxPayloads];            // vector path: bytes per access (32/16/8/4/2/1)
   uint32_t stage_bytes;                  // bulk path: bytes of one stage
   uint32_t tx_bytes;                     // bulk path: bytes one token brings in
   int stages;                            // bulk path
