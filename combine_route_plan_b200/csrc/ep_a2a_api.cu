@@ -185,11 +185,26 @@ void prof_free(ep_a2a_handle h) {
   h->profiling = false;
 }
 
-// Threads per token of the vector copy.  Measured on the workloads: with
-// 8192 or more token slots a warp per token is fastest (enough tokens to fill
-// the GPU; 32 beat 64-256 by 2-30 %), below that a whole 256-thread CTA per
-// token is (fewer tokens, each spread over more threads).
-int copy_threads_per_token(int64_t tokens) { return tokens >= 8192 ? 32 : 256; }
+// Threads per token of the vector copy, given the vectors in the largest row.
+// Measured on the workloads: with 16384 or more token slots a warp per token
+// is fastest (enough tokens to fill the GPU; 32 beat 64-256 by 2-30 % at
+// prefill); with fewer, the fewest threads (32..256) that hold the row in
+// about two vectors each (Zipf step, 8192 slots: 224-vector MXFP8 rows 7 %
+// faster on 128 threads than on a warp, 112-vector NVFP4 rows 1 % on 64;
+// decode and wide-EP steps: 448-vector rows on 256).
+int copy_threads_per_token(int64_t tokens, int64_t row_vectors) {
+  if (tokens >= 16384) return 32;
+  int t = 32;
+  while (t < 256 && 2 * t < row_vectors) t *= 2;
+  return t;
+}
+
+// Vectors in the largest row of a vector-copy launch.
+int64_t largest_row_vectors(const CopyArgs& c) {
+  int64_t most = 0;
+  for (int p = 0; p < c.np; ++p) most = std::max<int64_t>(most, c.rb[p] / (int64_t)c.vec[p]);
+  return most;
+}
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -203,8 +218,11 @@ struct CombineLaunch {
 // Launch shape of a combine: the options where set, else the defaults measured
 // on the decode (1024 token slots), wide-EP (4096), Zipf (8192) and prefill
 // (32768) workloads at hidden 7168:
-//  * BF16: one vector at a time, 64 threads, 128 CTAs per SM requested, no
-//    prefetch (pipelining and prefetch were 1-12 % slower);
+//  * BF16: one vector at a time (pipelining was 1-12 % slower); from 16384
+//    token slots 64 threads, 128 CTAs per SM requested, no prefetch; from 8192
+//    128 threads and a one-token prefetch (Zipf step: 98 against 103 us);
+//    below that 256 threads and 16 CTAs per SM (wide-EP step: 51 against
+//    55 us; decode 26.1 against 26.7 us), no prefetch;
 //  * FP8 and scaled FP8: pipelined (27-54 % faster); 64 threads below 16384
 //    token slots and 128 from there; from 8192 slots on, prefetch one token
 //    ahead (faster by 5-10 %, slower by 5-10 % on the small steps); 16 CTAs per
@@ -217,13 +235,21 @@ CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
   const bool big = ntok >= 16384;
   CombineLaunch c;
   c.pipe = fits && (h->combine_pipeline < 0 ? kind != kKindBf16 : h->combine_pipeline > 0);
-  c.threads = h->combine_threads > 0 ? h->combine_threads
-                                     : (kind == kKindFp8 && big ? 128 : 64);
-  const int cps = h->combine_ctas_per_sm > 0 ? h->combine_ctas_per_sm
-                                             : (kind == kKindFp8 && big ? 16 : 128);
+  const bool mid = !big && ntok >= 8192;
+  int threads = 64, cps = 128, prefetch = 0;
+  if (kind == kKindFp8) {
+    threads = big ? 128 : 64;
+    cps = big ? 16 : 128;
+    prefetch = ntok >= 8192 ? 1 : 0;
+  } else if (kind == kKindBf16) {
+    threads = big ? 64 : (mid ? 128 : 256);
+    cps = (big || mid) ? 128 : 16;
+    prefetch = mid ? 1 : 0;
+  }
+  c.threads = h->combine_threads > 0 ? h->combine_threads : threads;
+  if (h->combine_ctas_per_sm > 0) cps = h->combine_ctas_per_sm;
   c.grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntok, (int64_t)h->num_sms * cps));
-  c.prefetch = h->combine_prefetch >= 0 ? h->combine_prefetch
-                                        : (kind == kKindFp8 && ntok >= 8192 ? 1 : 0);
+  c.prefetch = h->combine_prefetch >= 0 ? h->combine_prefetch : prefetch;
   return c;
 }
 
@@ -232,10 +258,8 @@ CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
 // 8 for the prefill rows of 448 32-byte vectors over a warp, 2 for the
 // 3.5-14 KB rows of the decode, Zipf and wide-EP steps; a group with more
 // vectors in flight than its row has only ties up registers).
-int copy_unroll(const CopyArgs& c, int tpt) {
-  int64_t most = 0;
-  for (int p = 0; p < c.np; ++p) most = std::max<int64_t>(most, c.rb[p] / (int64_t)c.vec[p]);
-  const int64_t per_thread = (most + tpt - 1) / tpt;
+int copy_unroll(int64_t row_vectors, int tpt) {
+  const int64_t per_thread = (row_vectors + tpt - 1) / tpt;
   if (per_thread <= 4) return 2;
   if (per_thread <= 8) return 4;
   return 8;
@@ -607,13 +631,14 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
     }
   }
   if (vec.np > 0) {
+    const int64_t row_vectors = largest_row_vectors(vec);
     const int tpt = h->vec_threads_per_token > 0 ? h->vec_threads_per_token
-                                                 : copy_threads_per_token(ntok);
+                                                 : copy_threads_per_token(ntok, row_vectors);
     const int64_t groups_per_cta = 256 / tpt;
     const int grid = (int)std::max<int64_t>(
         1, std::min<int64_t>((ntok + groups_per_cta - 1) / groups_per_cta,
                              (int64_t)h->num_sms * h->vec_ctas_per_sm));
-    const int unroll = h->vec_unroll > 0 ? h->vec_unroll : copy_unroll(vec, tpt);
+    const int unroll = h->vec_unroll > 0 ? h->vec_unroll : copy_unroll(row_vectors, tpt);
     slot = prof_begin(h, EP_A2A_KERNEL_COPY_VEC, stream);
     e = launch_dispatch_vec(vec, grid, unroll, tpt, h->store_streaming != 0, stream, pdl);
     prof_end(h, slot, stream);

@@ -304,12 +304,11 @@ typedef enum {
   EP_A2A_OPT_COPY_STAGES = 2,     /* shared-memory row stages per copy CTA (2..32; 0 = as
                                      many as fit, up to 8 / 16) */
   EP_A2A_OPT_COMBINE_THREADS = 3, /* threads per CTA of the combine kernels (64..512);
-                                     0 (default) = automatic: 128 for the FP8 combines of
-                                     16384 or more token slots, else 64 */
+                                     0 (default) = automatic, from the combine kind and
+                                     the token slots (64, 128 or 256) */
   EP_A2A_OPT_BULK_MIN_ROW_BYTES = 4, /* rows shorter than this take the vector copy (0..2^24) */
   EP_A2A_OPT_COMBINE_CTAS_PER_SM = 5, /* combine grid = min(tokens, SMs x this) (1..1024);
-                                       0 (default) = automatic: 16 for the FP8 combines
-                                       of 16384 or more token slots, else 128 */
+                                       0 (default) = automatic (16 or 128) */
   EP_A2A_OPT_COPY_CONSUMER_WARPS = 6, /* store warps per CTA of copy path 0 (4, 8 or 16) */
   EP_A2A_OPT_COPY_INTERLEAVE = 7, /* paths 0 and 2: 1 = CTA b copies tokens b, b + grid, ...
                                      (default); 0 = each CTA copies a contiguous chunk */
@@ -325,12 +324,14 @@ typedef enum {
                                      each kernel waits for the previous one before it
                                      touches memory, so results do not change */
   EP_A2A_OPT_VEC_THREADS_PER_TOKEN = 12,/* vector copy: threads per token (32, 64, 128,
-                                     256); 0 (default) = from the token count */
+                                     256); 0 (default) = from the token count and the
+                                     largest row */
   EP_A2A_OPT_COMBINE_PREFETCH = 13,/* combines: p in 1..4 = each CTA asks for the rows of
                                      its token p grid strides ahead to be brought into L2
                                      (cp.async.bulk.prefetch.L2) while it sums the current
-                                     one; 0 = never; -1 (default) = 1 for the FP8 combines
-                                     of 8192 or more token slots, else 0 */
+                                     one; 0 = never; -1 (default) = automatic: 1 for the
+                                     FP8 combines from 8192 token slots and the BF16
+                                     combine from 8192 to 16383, else 0 */
   EP_A2A_OPT_COPY_PREFETCH = 14,  /* vector copy: 1 = the same for the next token's rows */
   EP_A2A_OPT_COMBINE_PIPELINE = 15,/* BF16 / FP8 / scaled FP8 combines of 16-byte vectors
                                      with at most 8 destinations per token (top_k or
