@@ -329,6 +329,15 @@ def run_ours(args):
     if args.tokens_per_rank:
         w = W.scaled(w, args.tokens_per_rank)
     x = W.make_inputs(w)
+    if args.e2e_steps > 0:
+        # the end-to-end leg copies from pinned host memory: pin the inputs once
+        # (in place of the pageable copies, so the host holds one copy)
+        x = dataclasses.replace(
+            x, token_selected_experts=x.token_selected_experts.pin_memory(),
+            payloads=[p.pin_memory() for p in x.payloads],
+            eplb_local_stats=(x.eplb_local_stats.pin_memory()
+                              if x.eplb_local_stats is not None else None),
+            expert_output=x.expert_output.pin_memory())
     stream = torch.cuda.current_stream()
 
     ids = x.token_selected_experts.to(device)
