@@ -1,10 +1,13 @@
 """Build libep_a2a.so (sm_100a) in-tree with nvcc.
 
-    python -m combine_route_plan_b200.build [--force] [--verbose]
+    python -m combine_route_plan_b200.build [--force] [--verbose] [--checked]
 
 Every .cu under csrc/ is compiled for sm_100a only and linked into one shared
 library next to this file.  No fast-math: the combine relies on IEEE fp32 adds
-with subnormals kept.
+with subnormals kept.  --checked builds libep_a2a_checked.so instead, the same
+ABI with the device index checks compiled in (EP_A2A_CHECKS=1): kernels test
+indices read from device memory before using them and report a bad one
+through ep_a2a_get_status (EP_A2A_ERR_DEVICE_BOUNDS) instead of touching it.
 """
 from __future__ import annotations
 
@@ -20,6 +23,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libep_a2a.so")
+LIB_CHECKED = os.path.join(HERE, "libep_a2a_checked.so")
 BUILD_DIR = os.path.join(HERE, "_build")
 
 NVCC_FLAGS = [
@@ -45,22 +49,25 @@ def _deps():
         [os.path.join(INCLUDE, "ep_a2a.h"), os.path.abspath(__file__)]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD_DIR, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB
+    if not force and up_to_date(lib):
+        return lib
+    build_dir = os.path.join(BUILD_DIR, "checked") if checked else BUILD_DIR
+    os.makedirs(build_dir, exist_ok=True)
     nvcc = _nvcc()
+    flags = NVCC_FLAGS + (["-DEP_A2A_CHECKS=1"] if checked else [])
     objs = []
     for src in _sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src)[:-3] + ".o")
-        cmd = [nvcc, *NVCC_FLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
+        cmd = [nvcc, *flags, "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -69,19 +76,20 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {os.path.basename(src)}")
         objs.append(obj)
-    tmp = LIB + f".{os.getpid()}.{time.time_ns()}.tmp"
+    tmp = lib + f".{os.getpid()}.{time.time_ns()}.tmp"
     r = subprocess.run([nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
                         "-o", tmp, *objs], capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
         raise RuntimeError("nvcc link failed")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--checked", action="store_true")
     args = ap.parse_args()
-    print(build(force=args.force, verbose=args.verbose))
+    print(build(force=args.force, verbose=args.verbose, checked=args.checked))

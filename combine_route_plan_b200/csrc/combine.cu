@@ -101,6 +101,9 @@ __device__ __forceinline__ void prefetch_token_rows(const CombineArgs& a, int64_
   if (nd == kNoToken || nd == 0) return;
   const uint64_t* row = reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
   const int words = a.plan_stride / 8;
+  if (EP_A2A_CHECKS && !plan_row_ok(nd, row[0], words > 1 ? row[1] : 0, words > 2 ? row[2] : 0,
+                                    words > 3 ? row[3] : 0, a.ep, a.plan_stride, nullptr))
+    return;
   const uint32_t bytes = (uint32_t)a.H * kElemBytes;
   const int64_t rank_stride = a.ntok * (int64_t)a.H * kElemBytes;
   for (int q = 0; q < nd; ++q) {
@@ -130,6 +133,7 @@ __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
     const uint64_t w1 = words > 1 ? row[1] : 0;
     const uint64_t w2 = words > 2 ? row[2] : 0;
     const uint64_t w3 = words > 3 ? row[3] : 0;
+    if (!plan_row_ok(nd, w0, w1, w2, w3, a.ep, a.plan_stride, a.err)) continue;
     const uint8_t* xt = a.x + tok * (int64_t)a.H * kElemBytes;           // rank 0's row
     const int64_t rank_stride = a.ntok * (int64_t)a.H * kElemBytes;      // bytes per rank
     uint16_t* out = a.out + tok * (int64_t)a.H;
@@ -259,6 +263,7 @@ __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
     const int nd = a.plan_nd[tok];
     if (nd == kNoToken || (int)threadIdx.x >= nvec) continue;
     const uint64_t w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    if (!plan_row_ok(nd, w0, 0, 0, 0, a.ep, 8, a.err)) continue;
     const uint8_t* xt = a.x + tok * (int64_t)a.H * kElemBytes + (int64_t)threadIdx.x * 16;
     const uint8_t* src[8];
     float sc[8];
@@ -306,6 +311,7 @@ __global__ void __launch_bounds__(512) combine_scalar_kernel(const CombineArgs a
     const uint64_t w1 = words > 1 ? row[1] : 0;
     const uint64_t w2 = words > 2 ? row[2] : 0;
     const uint64_t w3 = words > 3 ? row[3] : 0;
+    if (!plan_row_ok(nd, w0, w1, w2, w3, a.ep, a.plan_stride, a.err)) continue;
     for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
       float acc = 0.0f;
       for (int i = 0; i < nd; ++i) {
@@ -386,6 +392,7 @@ __global__ void __launch_bounds__(512) combine_experts_vec_kernel(const CombineE
     const uint64_t w1 = words > 1 ? row[1] : 0;
     const uint64_t w2 = words > 2 ? row[2] : 0;
     const uint64_t w3 = words > 3 ? row[3] : 0;
+    if (!plan_row_ok(nd, w0, w1, w2, w3, a.ep, a.plan_stride, a.err)) continue;
     int own[KMAX];
     float wt[KMAX];
     slot_owners<KMAX>(a, tok, nd, w0, w1, w2, w3, own, wt);
@@ -499,6 +506,7 @@ __global__ void __launch_bounds__(512) combine_experts_pipe_kernel(const Combine
       continue;
     }
     const uint64_t w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    if (!plan_row_ok(nd, w0, 0, 0, 0, a.ep, 8, a.err)) continue;
     int own[8];
     float wt[8];
     slot_owners<8>(a, tok, nd, w0, 0, 0, 0, own, wt);
@@ -538,6 +546,7 @@ __global__ void __launch_bounds__(512) combine_experts_any_kernel(const CombineE
     const uint64_t w1 = words > 1 ? row[1] : 0;
     const uint64_t w2 = words > 2 ? row[2] : 0;
     const uint64_t w3 = words > 3 ? row[3] : 0;
+    if (!plan_row_ok(nd, w0, w1, w2, w3, a.ep, a.plan_stride, a.err)) continue;
     int own[KMAX];
     float wt[KMAX];
     if (nd > 0) slot_owners<KMAX>(a, tok, nd, w0, w1, w2, w3, own, wt);
@@ -577,6 +586,7 @@ __global__ void __launch_bounds__(512) combine_scaled_kernel(const CombineArgs a
     const uint64_t w1 = words > 1 ? row[1] : 0;
     const uint64_t w2 = words > 2 ? row[2] : 0;
     const uint64_t w3 = words > 3 ? row[3] : 0;
+    if (!plan_row_ok(nd, w0, w1, w2, w3, a.ep, a.plan_stride, a.err)) continue;
     uint16_t* out = a.out + tok * (int64_t)a.H;
     if (kVec) {
       const uint8_t* xt = a.x + tok * (int64_t)a.H;

@@ -287,6 +287,7 @@ EP_API const char* ep_a2a_status_string(ep_a2a_status s) {
     case EP_A2A_ERR_NOT_INITIALIZED: return "handle not initialised";
     case EP_A2A_ERR_NO_PLAN: return "combine called before any dispatch";
     case EP_A2A_ERR_DEVICE_TIMEOUT: return "a bounded device wait ran out";
+    case EP_A2A_ERR_DEVICE_BOUNDS: return "a device index check failed (checked build)";
   }
   return "unknown status";
 }
@@ -681,6 +682,8 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   a.ntok = (int64_t)h->p.ep_size * h->last_tpr;
   a.H = h->combine_hidden;
   a.plan_stride = h->L.plan_stride;
+  a.ep = h->p.ep_size;
+  a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
   const CombineLaunch c = combine_launch(h, fp8 ? kKindFp8 : kKindBf16, a.ntok);
   a.prefetch = c.prefetch;
   a.out32 = aligned(output, 32) ? 1 : 0;
@@ -716,6 +719,8 @@ EP_API ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle h, const float* topk_w
   a.E = h->p.num_experts;
   a.epr = h->p.num_experts / h->p.ep_size;
   a.plan_stride = h->L.plan_stride;
+  a.ep = h->p.ep_size;
+  a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
   const CombineLaunch c = combine_launch(h, kKindExperts, a.ntok);
   a.prefetch = c.prefetch;
   const bool vec = a.k <= 8 && a.H % 8 == 0 && aligned(expert_output_per_slot, 16) &&
@@ -744,6 +749,8 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
   a.ntok = (int64_t)h->p.ep_size * h->last_tpr;
   a.H = h->combine_hidden;
   a.plan_stride = h->L.plan_stride;
+  a.ep = h->p.ep_size;
+  a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
   const CombineLaunch c = combine_launch(h, kKindFp8, a.ntok);
   a.prefetch = c.prefetch;
   a.out32 = aligned(output, 32) ? 1 : 0;
@@ -794,6 +801,9 @@ EP_API ep_a2a_status ep_a2a_get_status(ep_a2a_handle h, void* stream) {
     if (word & kErrWaitTimeout)
       return fail(EP_A2A_ERR_DEVICE_TIMEOUT, "a bounded wait in a kernel ran out (word 0x%x)",
                   word);
+    if (word & kErrBounds)
+      return fail(EP_A2A_ERR_DEVICE_BOUNDS,
+                  "a kernel found a plan entry out of range and skipped it (word 0x%x)", word);
   }
   return EP_A2A_OK;
 }

@@ -19,7 +19,30 @@ constexpr uint8_t kPad = 0xFF;           // plan_dst_ranks entries past the coun
 constexpr int kMaxStages = 32;           // shared-memory row stages per bulk-copy CTA
 
 // Bits of the device error word.
-enum : uint32_t { kErrWaitTimeout = 1u };
+enum : uint32_t { kErrWaitTimeout = 1u, kErrBounds = 2u };
+
+// Checked builds (-DEP_A2A_CHECKS=1, libep_a2a_checked.so) test indices that
+// come from device memory (the plan another kernel or the caller left in the
+// workspace) before using them; a bad one sets kErrBounds and the access is
+// skipped.  In the default build the checks compile to nothing.
+#ifndef EP_A2A_CHECKS
+#define EP_A2A_CHECKS 0
+#endif
+
+// Whether a token's plan row is usable: at most plan_stride destinations, each
+// one a rank below ep.  Always true unless checks are compiled in.
+__device__ __forceinline__ bool plan_row_ok(int nd, uint64_t w0, uint64_t w1, uint64_t w2,
+                                            uint64_t w3, int ep, int plan_stride,
+                                            uint32_t* err) {
+  if (!EP_A2A_CHECKS) return true;
+  bool ok = nd <= plan_stride && nd <= 32;
+  for (int q = 0; ok && q < nd; ++q) {
+    const uint64_t w = q < 8 ? w0 : (q < 16 ? w1 : (q < 24 ? w2 : w3));
+    ok = (int)((w >> ((q & 7) * 8)) & 0xFFu) < ep;
+  }
+  if (!ok && err) atomicOr(err, kErrBounds);
+  return ok;
+}
 
 // Bounded waits give up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -100,6 +123,8 @@ struct CombineArgs {
   int plan_stride;
   int prefetch;                // p > 0: prefetch the rows of the CTA's token p
                                // grid strides ahead into L2
+  int ep;
+  uint32_t* err;               // device error word (checked builds)
   int out32;                   // pipelined E4M3 combines: one 32-byte store per
                                // vector (output 32-byte aligned)
 };
@@ -122,6 +147,8 @@ struct CombineExpertsArgs {
   int H, k, E, epr, plan_stride;
   int prefetch;                // p > 0: prefetch the slot rows of the CTA's token p
                                // grid strides ahead into L2
+  int ep;
+  uint32_t* err;               // device error word (checked builds)
 };
 
 cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, bool pipe, int threads,

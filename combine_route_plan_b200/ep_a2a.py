@@ -19,7 +19,9 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libep_a2a.so")
+# EP_A2A_LIBRARY selects another build of the same ABI, e.g. the checked build
+# libep_a2a_checked.so (index checks compiled in); default: libep_a2a.so.
+LIB_PATH = os.environ.get("EP_A2A_LIBRARY") or os.path.join(_HERE, "libep_a2a.so")
 
 MAX_RANKS = 256
 RANK_MASK_WORDS = 4
@@ -28,7 +30,7 @@ MAX_TOP_K = 32
 
 # ep_a2a_status
 OK, ERR_INVALID_ARG, ERR_CAPACITY, ERR_UNSUPPORTED, ERR_CUDA, ERR_NOT_INITIALIZED, \
-    ERR_NO_PLAN, ERR_DEVICE_TIMEOUT = range(8)
+    ERR_NO_PLAN, ERR_DEVICE_TIMEOUT, ERR_DEVICE_BOUNDS = range(9)
 COMBINE_BF16, COMBINE_FP8_E4M3 = 0, 1
 OPT_COPY_PATH, OPT_COPY_CTAS_PER_SM, OPT_COPY_STAGES, OPT_COMBINE_THREADS, \
     OPT_BULK_MIN_ROW_BYTES, OPT_COMBINE_CTAS_PER_SM, OPT_COPY_CONSUMER_WARPS, \

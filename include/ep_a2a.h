@@ -56,7 +56,12 @@ typedef enum {
   EP_A2A_ERR_CUDA = 4,            /* a CUDA runtime call failed (launch, device query) */
   EP_A2A_ERR_NOT_INITIALIZED = 5, /* NULL or destroyed handle */
   EP_A2A_ERR_NO_PLAN = 6,         /* combine without a preceding dispatch */
-  EP_A2A_ERR_DEVICE_TIMEOUT = 7   /* a bounded wait inside a kernel ran out */
+  EP_A2A_ERR_DEVICE_TIMEOUT = 7,  /* a bounded wait inside a kernel ran out */
+  EP_A2A_ERR_DEVICE_BOUNDS = 8    /* checked build (libep_a2a_checked.so, compiled with
+                                     EP_A2A_CHECKS=1) only: a combine kernel found a
+                                     plan entry in the workspace out of range (a
+                                     destination rank >= ep_size or more destinations
+                                     than the plan holds) and skipped that token */
 } ep_a2a_status;
 
 typedef enum {
@@ -278,7 +283,8 @@ ep_a2a_status ep_a2a_reduce_scatter(int32_t ep_size, int32_t tokens_per_rank, in
 
 /*
  * Synchronise `stream`, then read and clear the handle's device error word.
- * DEVICE_TIMEOUT if a kernel's bounded wait ran out since the last check.
+ * DEVICE_TIMEOUT if a kernel's bounded wait ran out since the last check;
+ * DEVICE_BOUNDS (checked build only) if a kernel skipped an out-of-range index.
  */
 ep_a2a_status ep_a2a_get_status(ep_a2a_handle handle, void* stream);
 

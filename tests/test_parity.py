@@ -217,6 +217,54 @@ def test_cuda_graph_capture_and_replay():
     assert comm.get_status() == ep_a2a.OK
 
 
+def test_cuda_graph_with_pipelined_combines():
+    """Dispatch, the FP8 combine and the expert-output combine (pipelined
+    kernels, L2 prefetch on) captured into one CUDA graph."""
+    from combine_route_plan_b200 import ep_a2a
+    w = W.C2
+    x = _inputs(w.name)
+    comm = ep_a2a.EpA2A(w.ep_size, w.num_experts, w.top_k, w.tokens_per_rank, w.hidden,
+                        w.payload_row_bytes(), workspace_fill=U.CANARY)
+    comm.set_option(ep_a2a.OPT_COMBINE_PREFETCH, 1)
+    ids = x.token_selected_experts.cuda()
+    pays = [p.cuda() for p in x.payloads]
+    xq = ep_a2a.quantize_e4m3(x.expert_output.cuda())
+    g_ = torch.Generator().manual_seed(12)
+    wts = torch.randn((w.ep_size, w.tokens_per_rank, w.top_k), generator=g_)
+    y = torch.randn((w.ep_size, w.tokens_per_rank, w.top_k, w.hidden), generator=g_) \
+        .to(torch.bfloat16)
+    wts_d, y_d = wts.cuda(), y.cuda()
+    out8 = torch.empty((w.ep_size, w.tokens_per_rank, w.hidden), dtype=torch.bfloat16,
+                       device="cuda")
+    oute = torch.empty_like(out8)
+
+    def step():
+        comm.dispatch(ids, x.local_num_tokens, pays, w.tokens_per_rank, views=False)
+        comm.combine(xq, out8)
+        comm.combine_experts(wts_d, y_d, oute)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    plan = U.oracle_plan(w, x)
+    want8 = U.oracle.combine(plan, U.to_np(xq), w.hidden, input_is_e4m3=True)
+    wante = U.oracle.combine_experts(plan, w.num_experts, x.token_selected_experts.numpy(),
+                                     wts.numpy(), U.to_np(y), w.hidden)
+    for _ in range(2):
+        out8.fill_(0)
+        oute.fill_(0)
+        g.replay()
+        torch.cuda.synchronize()
+        U.assert_equal(out8, want8, "fp8 combine in a graph")
+        U.assert_equal(oute, wante, "expert combine in a graph")
+    assert comm.get_status() == ep_a2a.OK
+
+
 @pytest.mark.parametrize("prefetch,ctas", [(1, 4), (1, 12), (1, 128), (0, 8)])
 def test_prefetch_options_do_not_change_results(prefetch, ctas):
     from combine_route_plan_b200 import ep_a2a
