@@ -139,7 +139,7 @@ struct ep_a2a_handle_s {
   int vec_ctas_per_sm;
   int store_streaming;
   int pdl;                // programmatic dependent launch for the path's kernels
-  int vec_threads_per_token;  // 0 = from the token count
+  int vec_threads_per_token;  // 0 = from the token count and the largest row
   // combine launch shape; -1 / 0 = automatic (combine_launch)
   int combine_prefetch;       // tokens ahead (grid strides) whose rows go to L2
   int copy_prefetch;          // vector copy: prefetch the next token's rows
