@@ -84,3 +84,37 @@ def test_all_cores_oracle_baseline_runs_spawned_processes():
     rec = bench.cpu_baseline_all_cores(W.C1, 0.5, tokens_per_rank=16, procs=2)
     assert rec["cores"] == 2 and rec["kind"] == "oracle" and rec["value"] > 0
     assert "2 single-threaded processes" in rec["sample"]
+
+
+def test_algorithmic_bytes_of_the_expert_output_combine():
+    sys.path.insert(0, ROOT)
+    import bench
+    from combine_route_plan_b200 import workloads as W
+    w = W.C4
+    n_tok, sum_d, slots = 32768, 173434, 32768 * 8
+    b = bench.algorithmic_bytes(w, n_tok, sum_d, live=8, fp8=False, live_slots=slots)
+    # one bf16 row per (token, slot), the ids and weights, one bf16 output row
+    assert b.combine == slots * 7168 * 2 + n_tok * 8 * 8 + n_tok * 7168 * 2
+    assert b.step == b.copy + b.combine + b.route
+
+
+def test_kernel_sources_hash_ignores_comments_only():
+    sys.path.insert(0, ROOT)
+    import bench
+    code = "__global__ void k(int* p) { p[0] = 1; }\n"
+    commented = ("// a comment\n/* a block\n   comment */\n__global__ void k(int* p) {\n"
+                 "  p[0] = 1;  // trailing\n}\n")
+    assert bench._code_only(code) == bench._code_only(commented)
+    assert bench._code_only(code) != bench._code_only(code.replace("1;", "2;"))
+
+
+def test_committed_traffic_only_for_the_sources_it_was_taken_on(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    rec = json.load(open(os.path.join(ROOT, "profiles", "dram_traffic.json")))
+    assert bench.committed_traffic("copy_vec", "c4_ep8_prefill") == (
+        rec["kernels"]["copy_vec"]["dram_bytes_per_launch"]
+        if rec["sources_hash"] == bench.kernel_sources_hash() else None)
+    monkeypatch.setattr(bench, "kernel_sources_hash", lambda: "0" * 16)
+    assert bench.committed_traffic("copy_vec", "c4_ep8_prefill") is None
+    assert bench.committed_traffic("copy_vec", "c2_ep8_decode") is None
