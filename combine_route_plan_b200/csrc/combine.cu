@@ -1,7 +1,7 @@
 // Combine of rank-major MoE dispatch (flashinfer.moe_ep.NVLinkTwoSidedAlltoAll,
 // combine()): each existing token (src, t) gets the sum of the rows its
-// destination ranks return, already weighted and reduced over each rank's local
-// experts.  The sum is an fp32 accumulator that starts at +0.0f and adds the
+// destination ranks return, each row being that rank's experts' outputs for the
+// token with the routing weights applied and summed.  The sum is an fp32 accumulator that starts at +0.0f and adds the
 // rows in ascending destination-rank order with round-to-nearest adds, then is
 // rounded once to bf16 (nearest-even).  With the low-precision combine
 // (flashinfer.moe_ep.NVLinkOneSidedConfig, use_low_precision_combine) the rows

@@ -93,8 +93,8 @@ typedef struct {
 } ep_a2a_params;
 
 /*
- * Everything dispatch produced, as device pointers into the workspace (the
- * pages' "workspace-backed views").  They stay valid, and keep their contents,
+ * Everything dispatch produced, as device pointers into the workspace (views of
+ * the workspace, as the pages return them).  They stay valid, and keep their contents,
  * until the next dispatch on the same handle or its destruction.  Every
  * per-rank array of rank d sits at (rank-0 pointer + d * rank_stride_bytes).
  * Let tpr = tokens_per_rank and slot s = src * tpr + t.
@@ -184,9 +184,12 @@ ep_a2a_status ep_a2a_dispatch(ep_a2a_handle handle, const int32_t* token_selecte
  * over the token's destination ranks d; one round-to-nearest-even at the end.
  * A token whose destinations were all masked off gets +0.0.
  *
- *   expert_output   device [ep, ep*tpr, hidden_size] of `dtype` (bf16 or E4M3),
- *                   each rank's rows already weighted and reduced over its local
- *                   experts.  Only rows of valid slots are read.
+ *   expert_output   device [ep, ep*tpr, hidden_size] of `dtype` (bf16 or E4M3):
+ *                   row (d, s) is rank d's result for the token in slot s, its
+ *                   experts' outputs with the routing weights applied and summed
+ *                   on that rank.  Only rows of valid slots are read.  (hidden_size
+ *                   is the handle's combine row length, see
+ *                   ep_a2a_set_combine_hidden.)
  *   output          device bf16 [ep, tpr, hidden_size].  Rows of tokens that do
  *                   not exist (t >= local_num_tokens[src], masked-off src) are not
  *                   written.
@@ -197,9 +200,9 @@ ep_a2a_status ep_a2a_combine(ep_a2a_handle handle, const void* expert_output,
 
 /*
  * Combine of per-expert outputs: the step that makes the combine's input
- * (NVLinkTwoSidedAlltoAll.combine(): rows "already weighted and reduced over
- * this rank's local experts") fused into the combine, so the per-rank rows are
- * never written to memory.  For each existing token (src, t) of the last
+ * (NVLinkTwoSidedAlltoAll.combine(): each rank's row is its own experts'
+ * outputs, weighted and summed) fused into the combine, so the per-rank rows
+ * are never written to memory.  For each existing token (src, t) of the last
  * dispatch:
  *   z_d = bf16( fp32 sum over the token's slots j whose expert rank d owns,
  *               ascending j, of topk_weights[j] * y[j] (one fused multiply-add

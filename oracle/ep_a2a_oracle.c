@@ -24,8 +24,8 @@
  *   [TSD]  flashinfer.moe_ep.NVLinkTwoSidedAlltoAll, dispatch(): each token is
  *          sent to the ranks that own its selected experts; topk_ids are global
  *          expert ids; weights and scales travel row-aligned with the token.
- *   [TSC]  same page, combine(): each token's expert outputs, already weighted
- *          and reduced over the receiving rank's local experts, summed over ranks.
+ *   [TSC]  same page, combine(): each rank returns one row per token, its own
+ *          experts' outputs weighted and summed; the rows are summed over ranks.
  *   [A2A]  flashinfer.comm.moe_a2a_dispatch, Parameters (active_rank_mask,
  *          eplb_local_stats) and Returns (eplb_gathered_stats row r = rank r).
  *   [V2S]  vllm.distributed.device_communicators.all2all,
@@ -37,8 +37,8 @@
  *          dispatch as an all-gather of every rank's rows, combine as a
  *          reduce-scatter (each rank gets its own rows summed over all ranks).
  *   [TSCi] flashinfer.moe_ep.NVLinkTwoSidedAlltoAll, combine(): its input rows
- *          are "already weighted and reduced over this rank's local experts";
- *          oracle_expert_reduce states that step.
+ *          come out of a per-rank weighting and summing over the rank's own
+ *          experts; oracle_expert_reduce states that step.
  *
  * Readings where the pages are silent (each is one deliberate choice):
  *   - expert e is owned by rank e / (E / ep_size) (contiguous blocks);
