@@ -20,8 +20,8 @@
  *     (extra_payload_bytes_per_token, eplb_stats_num_experts, enable_rank_mask,
  *     use_low_precision_combine) and the `lamport` paragraph (slot
  *     src * tokens_per_rank + t; tokens_per_rank = runtime_max_tokens_per_rank).
- *   flashinfer.moe_ep.NVLinkTwoSidedAlltoAll — class constraints (num_experts
- *     divisible by 4; EPLB statistics cover all experts), dispatch(), combine(),
+ *   flashinfer.moe_ep.NVLinkTwoSidedAlltoAll — class constraints (num_experts a
+ *     multiple of 4; the EPLB stats span every expert), dispatch(), combine(),
  *     destroy().
  *   flashinfer.comm.moe_a2a_dispatch — Parameters (token_selected_experts,
  *     input_payloads, workspace, runtime_max_tokens_per_rank, eplb_local_stats,
@@ -325,13 +325,13 @@ typedef enum {
                                      default: the fewest that move the largest row in
                                      two rounds) */
   EP_A2A_OPT_VEC_CTAS_PER_SM = 9, /* vector copy grid = SMs x this (1..64; default 32) */
-  EP_A2A_OPT_STORE_STREAMING = 10,/* vector copy: 1 = evict-first (.cs) 16-byte stores
+  EP_A2A_OPT_STORE_STREAMING = 10,/* vector copy: 1 = evict-first (.cs) stores
                                      (default), 0 = plain stores */
-  EP_A2A_OPT_PDL = 11,            /* 1 (default): launch the routing, copy and combine
-                                     kernels with programmatic dependent launch
-                                     (flashinfer.moe_ep.NVLinkOneSidedConfig, enable_pdl);
-                                     each kernel waits for the previous one before it
-                                     touches memory, so results do not change */
+  EP_A2A_OPT_PDL = 11,            /* 1 (default): each kernel of the path may start while
+                                     the one before it finishes (programmatic dependent
+                                     launch; flashinfer.moe_ep.NVLinkOneSidedConfig,
+                                     enable_pdl); each waits for its predecessor before
+                                     it touches memory, so results do not change */
   EP_A2A_OPT_VEC_THREADS_PER_TOKEN = 12,/* vector copy: threads per token (32, 64, 128,
                                      256); 0 (default) = from the token count and the
                                      largest row */

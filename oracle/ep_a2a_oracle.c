@@ -21,16 +21,16 @@
  *   [OSC]  flashinfer.moe_ep.NVLinkOneSidedConfig, `lamport` paragraph: rows a
  *          rank receives from rank src for token t land at
  *          src * tokens_per_rank + t.
- *   [TSD]  flashinfer.moe_ep.NVLinkTwoSidedAlltoAll, dispatch(): each token is
- *          sent to the ranks that own its selected experts; topk_ids are global
- *          expert ids; weights and scales travel row-aligned with the token.
+ *   [TSD]  flashinfer.moe_ep.NVLinkTwoSidedAlltoAll, dispatch(): a token goes to
+ *          every rank owning one of the experts chosen for it; topk_ids hold
+ *          global expert ids; weights and scales move in the token's row slot.
  *   [TSC]  same page, combine(): each rank returns one row per token, its own
  *          experts' outputs weighted and summed; the rows are summed over ranks.
  *   [A2A]  flashinfer.comm.moe_a2a_dispatch, Parameters (active_rank_mask,
  *          eplb_local_stats) and Returns (eplb_gathered_stats row r = rank r).
  *   [V2S]  vllm.distributed.device_communicators.all2all,
- *          FlashInferNVLinkTwoSidedManager.get_communication: received rows
- *          past a source's token count keep expert id num_experts.
+ *          FlashInferNVLinkTwoSidedManager.get_communication: a received row
+ *          beyond a source's tokens carries the id num_experts.
  *   [OSCu] flashinfer.moe_ep.NVLinkOneSidedConfig, `use_low_precision_combine`:
  *          combine payloads travel as FP8.
  *   [AGRS] vllm.distributed.device_communicators.all2all, AgRsAll2AllManager:
@@ -441,7 +441,7 @@ void oracle_combine_scaled(int ep_size, int top_k, int tokens_per_rank, int hidd
 }
 
 /* ------------------------------------------------------------------------- */
-/* Dense variant: all-gather dispatch and reduce-scatter combine [AGRS].      */
+/* Dense variant [AGRS]: every rank gets every token; every rank's row sums.  */
 /* ------------------------------------------------------------------------- */
 
 /*
