@@ -257,3 +257,11 @@ def test_grow_properties_on_random_requests(ep):
             assert st == ep.OK and again == 0
         wa, wb, wg = (_ws_status(ep, p)[1] for p in (a, b, ab))
         assert wg >= max(wa, wb)
+
+
+def test_checked_build_compiles_and_exports_every_symbol():
+    """The checked build (device index checks compiled in) is the same ABI."""
+    from combine_route_plan_b200 import build
+    lib = ctypes.CDLL(build.build(checked=True))
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
