@@ -260,6 +260,17 @@ def algorithmic_bytes(w, n_tok: int, sum_d: int, live: int, fp8: bool,
     return Bytes(copy, combine, route, copy + combine + route)
 
 
+def l2_note(flushed: bool, step_bytes: int, l2_bytes: int) -> str:
+    """How the timed steps meet the L2 rule, for the JSON line's config."""
+    if flushed:
+        return "512 MB L2 flush before every step, each step timed alone"
+    mb, l2 = step_bytes / 1e6, l2_bytes / 1e6
+    if step_bytes > 4 * l2_bytes:
+        return f"inputs larger than L2 (no flush): each step moves {mb:.0f} MB, L2 holds {l2:.0f} MB"
+    return (f"no flush, warm L2: each step moves {mb:.0f} MB and part of it stays in the "
+            f"{l2:.0f} MB L2 between steps")
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -529,8 +540,9 @@ def run_ours(args):
                                "fused, fp32 accumulate)" if experts else
                                f"{'FP8 E4M3 with a per-row fp32 scale' if scaled else 'FP8 E4M3' if fp8 else 'BF16'} combine (fp32 accumulate)"),
                 "tokens_per_step_per_gpu": n_tok, "mean_distinct_ranks": sum_d / n_tok,
-                "l2": ("512 MB L2 flush before every step, each step timed alone"
-                       if args.l2_flush else "inputs larger than L2 (no flush)"),
+                "l2": l2_note(args.l2_flush, by.step,
+                              getattr(torch.cuda.get_device_properties(device),
+                                      "L2_cache_size", 0) or (126 << 20)),
                 "launch": ("CUDA graph replay" if args.graph else "eager") +
                           (", programmatic dependent launch" if not args.no_pdl else ""),
                 "kernel_times": "CUDA events around each launch, in a second timed region of "

@@ -118,3 +118,12 @@ def test_committed_traffic_only_for_the_sources_it_was_taken_on(monkeypatch):
     monkeypatch.setattr(bench, "kernel_sources_hash", lambda: "0" * 16)
     assert bench.committed_traffic("copy_vec", "c4_ep8_prefill") is None
     assert bench.committed_traffic("copy_vec", "c2_ep8_decode") is None
+
+
+def test_l2_note_says_which_rule_the_timing_meets():
+    sys.path.insert(0, ROOT)
+    import bench
+    l2 = 126 << 20
+    assert bench.l2_note(True, 10 ** 8, l2).startswith("512 MB L2 flush")
+    assert bench.l2_note(False, 5_938_896_128, l2).startswith("inputs larger than L2")
+    assert bench.l2_note(False, 185_000_000, l2).startswith("no flush, warm L2")
