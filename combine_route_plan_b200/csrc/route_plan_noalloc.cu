@@ -13,11 +13,14 @@
 //
 // Limits and sharing: the array holds the scratch of at most
 // EP_A2A_NOALLOC_MAX_RANKS ranks (16,640 bytes), and every GPU that loads the
-// library keeps it until the process exits.  All calls share it: each call
+// library keeps it until the process exits.  Its device address is looked up
+// once per CUDA context (again after a device reset).  All calls share it: each call
 // clears the part it uses on its stream before the kernel, so calls that
 // follow one another in stream order are independent, but calls whose work
 // overlaps on the GPU (different streams, or different host threads on the
 // same device) race on the array.
+#include <cuda.h>
+
 #include <cstring>
 #include <mutex>
 
@@ -37,26 +40,71 @@ namespace {
 constexpr int kNoAllocMaxRanks = EP_A2A_NOALLOC_MAX_RANKS;
 constexpr int kMaxDevices = 64;
 
+// The array's device address is only valid in the CUDA context it was looked
+// up in.  A device reset (or a primary context released and created again)
+// gives the device a new context, where the array has a new address, so the
+// cache holds the address together with the context's id (cuCtxGetId: unique
+// for the life of the process) and looks it up again when the id changes.
+struct ScratchEntry {
+  unsigned long long ctx_id;   // 0 = not looked up yet
+  void* addr;
+};
+
 std::mutex g_setup_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+ScratchEntry g_scratch[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
 
 ep_a2a_status noalloc_fail(ep_a2a_status st, const char* msg) {
   record_last_error(msg);
   return st;
 }
 
-// Device address of the array on `dev` (the current device).  The host-side
-// symbol is only a stand-in, so the address is looked up once per device with
-// that device current and cached.
+// Id of the calling thread's current context (the runtime has made one
+// current: callers run cudaGetDevice first, and the lookups below go through
+// the driver entry points the runtime hands out, so no driver library is
+// linked).
+cudaError_t current_context_id(unsigned long long* id) {
+  if (g_ctx_get_current == nullptr || g_ctx_get_id == nullptr) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1);
+    if (e != cudaSuccess) return e;
+    e = cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2);
+    if (e != cudaSuccess) return e;
+    if (q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || !f1 || !f2)
+      return cudaErrorNotSupported;
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
+  if (g_ctx_get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  return cudaSuccess;
+}
+
+// Device address of the array on `dev` (the current device) in the current
+// context.  The host-side symbol is only a stand-in, so the address is looked
+// up (cudaGetSymbolAddress) with that device current, once per context, and
+// cached with the context's id.
 cudaError_t scratch_address(int dev, void** out) {
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
+  unsigned long long ctx_id = 0;
+  cudaError_t e = current_context_id(&ctx_id);
+  if (e != cudaSuccess) return e;
+  ScratchEntry& c = g_scratch[dev];
+  if (c.ctx_id != ctx_id || c.addr == nullptr) {
     void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+    e = cudaGetSymbolAddress(&p, g_route_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
+    c.ctx_id = ctx_id;
+    c.addr = p;
   }
-  *out = g_scratch_addr[dev];
+  *out = c.addr;
   return cudaSuccess;
 }
 
@@ -88,8 +136,23 @@ EP_API ep_a2a_status ep_a2a_route_plan_noalloc(
     return noalloc_fail(EP_A2A_ERR_INVALID_ARG,
                         "recv_topk_ids and recv_rank_stride_bytes must be 4-byte aligned");
   const int64_t slots = (int64_t)ep_size * tokens_per_rank;
-  if (ep_size > 1 && recv_rank_stride_bytes < slots * top_k * 4)
-    return noalloc_fail(EP_A2A_ERR_INVALID_ARG, "recv_rank_stride_bytes too small");
+  // Each rank's two receive arrays: ids [0, ids_bytes) and valid bytes
+  // [off_valid, off_valid + slots), relative to its recv_topk_ids.  They must
+  // not overlap, and with more than one rank both must fit inside one stride,
+  // so that no rank's writes land on another array or another rank's.
+  const int64_t ids_bytes = slots * top_k * 4;
+  const int64_t off_valid =
+      (int64_t)(reinterpret_cast<intptr_t>(recv_valid) - reinterpret_cast<intptr_t>(recv_topk_ids));
+  if (off_valid < ids_bytes && off_valid + slots > 0)
+    return noalloc_fail(EP_A2A_ERR_INVALID_ARG, "recv_valid overlaps recv_topk_ids");
+  if (ep_size > 1) {
+    const int64_t lo = off_valid < 0 ? off_valid : 0;
+    const int64_t hi = off_valid + slots > ids_bytes ? off_valid + slots : ids_bytes;
+    if (recv_rank_stride_bytes < hi - lo)
+      return noalloc_fail(EP_A2A_ERR_INVALID_ARG,
+                          "recv_rank_stride_bytes is smaller than one rank's recv_topk_ids and "
+                          "recv_valid together");
+  }
 
   RouteArgs ra;
   std::memset(&ra, 0, sizeof(ra));
@@ -131,7 +194,7 @@ EP_API ep_a2a_status ep_a2a_route_plan_noalloc(
   ra.rank0 = reinterpret_cast<uint8_t*>(recv_topk_ids);
   ra.rank_stride = recv_rank_stride_bytes;
   ra.off_ids = 0;
-  ra.off_valid = reinterpret_cast<intptr_t>(recv_valid) - reinterpret_cast<intptr_t>(recv_topk_ids);
+  ra.off_valid = off_valid;
   ra.off_eplb = 0;
   ra.ep = ep_size;
   ra.E = num_experts;

@@ -122,8 +122,11 @@ typedef struct {
 } ep_a2a_dispatch_result;
 
 /*
- * Bytes of device workspace needed for `params`.  Host only; no CUDA call.
- * INVALID_ARG / UNSUPPORTED when params break the rules of ep_a2a_params.
+ * Bytes of device workspace needed for `params` (flashinfer.comm.moe_a2a_dispatch,
+ * Parameters, `workspace`: one workspace of [ep_size, size_per_rank] bytes; here
+ * a control region followed by ep_size rank regions, each holding that rank's
+ * receive arrays for ep_size * max_tokens_per_rank slots).  Host only; no CUDA
+ * call.  INVALID_ARG / UNSUPPORTED when params break the rules of ep_a2a_params.
  */
 ep_a2a_status ep_a2a_workspace_size(const ep_a2a_params* params, size_t* bytes);
 
@@ -456,13 +459,20 @@ const char* ep_a2a_last_error(void);
  *   recv_rank_stride_bytes  bytes from rank d's recv_topk_ids / recv_valid to rank
  *                           d+1's (the same for both arrays; a multiple of 4)
  *
+ * recv_valid must not overlap recv_topk_ids, and with ep_size > 1 the two
+ * arrays of one rank must fit together inside recv_rank_stride_bytes
+ * (INVALID_ARG otherwise), so that no write lands on another array or rank.
+ *
  * Limit: ep_size <= EP_A2A_NOALLOC_MAX_RANKS (64); larger sizes return
  * EP_A2A_ERR_UNSUPPORTED.  The array takes 16,640 bytes on every GPU that loads
- * the library, until the process exits.  The first call on each device looks up
- * the array's device address with that device current (cudaGetSymbolAddress);
- * make that first call before any stream capture.  Every call shares the array
- * and clears the part it uses on `stream` before its kernel, so calls in stream
- * order are independent; calls whose work overlaps on the GPU race on the array.
+ * the library, until the process exits.  The first call in each CUDA context of
+ * a device looks up the array's device address with that device current
+ * (cudaGetSymbolAddress) and caches it with the context's id; after a device
+ * reset the device has a new context, and the next call looks the address up
+ * again.  Make that first call before any stream capture.  Every call shares
+ * the array and clears the part it uses on `stream` before its kernel, so calls
+ * in stream order are independent; calls whose work overlaps on the GPU race
+ * on the array.
  */
 #define EP_A2A_NOALLOC_MAX_RANKS 64
 ep_a2a_status ep_a2a_route_plan_noalloc(

@@ -368,8 +368,11 @@ def test_fp8_quantize_all_bf16_patterns():
         assert np.all((got[nan] & 0x7F) == 0x7F)      # NaN stays NaN (its sign is not fixed)
 
 
-@pytest.mark.parametrize("name", ["c4_ep8_prefill", "c2_ep8_decode"])
+@pytest.mark.parametrize("name", ["c4_ep8_prefill", "c2_ep8_decode", "c3_ep16_zipf_nvfp4",
+                                  "c1_ep4_tiny", "c5_ep64_wide_masked"])
 def test_fp8_combine(name):
+    """The low-precision combine on every workload, at the library's default
+    launch shape for its token count (8192 slots for the Zipf workload)."""
     w = W.BY_NAME[name]
     x = _inputs(w.name)
     run = U.Run(w, x, fp8=True)
@@ -799,7 +802,7 @@ def _check_combine_experts(w, x, y, wts, options=None):
 
 
 @pytest.mark.parametrize("name", ["c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked",
-                                  "c4_ep8_prefill"])
+                                  "c4_ep8_prefill", "c3_ep16_zipf_nvfp4"])
 def test_combine_experts_bit_exact(name):
     w = W.BY_NAME[name]
     x = _inputs(w.name)
@@ -854,7 +857,8 @@ def test_quantize_rows_matches_oracle(hidden, rows):
     U.assert_equal(scales, osc, "row scales")
 
 
-@pytest.mark.parametrize("name", ["c2_ep8_decode", "c5_ep64_wide_masked", "c1_ep4_tiny"])
+@pytest.mark.parametrize("name", ["c2_ep8_decode", "c5_ep64_wide_masked", "c1_ep4_tiny",
+                                  "c3_ep16_zipf_nvfp4", "c4_ep8_prefill"])
 def test_combine_scaled_bit_exact(name):
     from combine_route_plan_b200 import ep_a2a
     w = W.BY_NAME[name]

@@ -1,5 +1,5 @@
 """The allocation-free routing plan (ep_a2a_route_plan_noalloc) against the
-workspace-based ep_a2a_dispatch.
+CPU oracle and the workspace-based ep_a2a_dispatch.
 
 Some callers cannot allocate device memory: their HBM is owned by an outer
 allocator (a serving engine that reserves almost all of it for its own pools,
@@ -8,9 +8,11 @@ They cannot give ep_a2a_init a workspace holding the routing kernel's scratch,
 so ep_a2a_route_plan_noalloc keeps that scratch in a fixed device array of the
 library and takes only inputs and outputs.  This test calls it through the C
 ABI, twice in a row on the same inputs and once more on another shape, and
-checks every output against what ep_a2a_dispatch wrote (all integers, so the
-comparison is exact).  It lives in its own file, collected last, and passes
-alone in a fresh process as well as after the other tests.
+checks every output against the oracle's routing plan and against what
+ep_a2a_dispatch wrote (all integers, so the comparisons are exact); it also
+checks that warm calls leave the device's allocated and free memory unchanged.
+It lives in its own file, collected last, and passes alone in a fresh process
+as well as after the other tests.
 """
 import ctypes
 
@@ -19,6 +21,7 @@ import pytest
 import torch
 
 from combine_route_plan_b200 import workloads as W
+import parity_util as U
 
 pytestmark = pytest.mark.gpu
 
@@ -102,16 +105,47 @@ def _compare(w, o, d):
     assert torch.equal(o.recv_ids(w), d.recv_topk_ids)
 
 
-def test_noalloc_plan_matches_workspace_plan(ep):
+def _compare_oracle(w, x, o):
+    """Every output against the oracle's plan of the same step: plan rows, send
+    counts, and each rank's valid bytes and received ids (the oracle leaves the
+    rows of masked-off ranks at the canary, as the kernel does)."""
+    torch.cuda.synchronize()
+    plan = U.oracle_plan(w, x)
+    k = w.top_k
+    nd = plan.num_dst.copy()
+    nd[nd < 0] = 0xFF
+    U.assert_equal(o.plan_nd, nd.astype(np.uint8), "plan_num_dst")
+    want = np.full(tuple(o.plan_dst.shape), 0xFF, np.uint8)
+    ranks = plan.dst_ranks.copy()
+    ranks[ranks < 0] = 0xFF
+    want[:, :, :k] = ranks.astype(np.uint8)
+    U.assert_equal(o.plan_dst, want, "plan_dst_ranks")
+    U.assert_equal(o.counts, plan.send_counts, "send_counts")
+    U.assert_equal(o.recv_valid(w), plan.recv_valid, "recv_valid")
+    U.assert_equal(o.recv_ids(w), plan.recv_topk_ids, "recv_topk_ids")
+
+
+def _device_memory():
+    free, _ = torch.cuda.mem_get_info()
+    return torch.cuda.memory_allocated(), torch.cuda.memory_reserved(), free
+
+
+def test_noalloc_plan_matches_oracle_and_workspace_plan(ep):
     # wide EP with a rank mask and ragged token counts, at the full size
     w = W.C5
     x = W.make_inputs(w, with_expert_output=False)
     comm, d = _reference(ep, w, x)
     ids_dev = x.token_selected_experts.cuda()
     o = Outputs(w)
+    _call_noalloc(ep, w, x, o, ids_dev)         # warm: the kernel's code is loaded
     for _ in range(2):                          # two calls in a row share the array
+        torch.cuda.synchronize()
+        before = _device_memory()
         _call_noalloc(ep, w, x, o, ids_dev)
+        torch.cuda.synchronize()
+        assert _device_memory() == before       # allocated, reserved and free bytes
         _compare(w, o, d)
+        _compare_oracle(w, x, o)
     # a different shape after it: the array keeps the last call's contents
     w2 = W.scaled(W.C2, 100)
     x2 = W.make_inputs(w2, with_expert_output=False)
@@ -119,6 +153,7 @@ def test_noalloc_plan_matches_workspace_plan(ep):
     o2 = Outputs(w2)
     _call_noalloc(ep, w2, x2, o2, x2.token_selected_experts.cuda())
     _compare(w2, o2, d2)
+    _compare_oracle(w2, x2, o2)
     comm.destroy()
     comm2.destroy()
 
@@ -130,3 +165,20 @@ def test_noalloc_rejects_too_many_ranks(ep):
                                           None, dummy, dummy, dummy, dummy, dummy, 4096, None)
     assert st == ep.ERR_UNSUPPORTED
     assert b"64" in ep.lib.ep_a2a_last_error()
+
+
+@pytest.mark.parametrize("valid_off,stride", [
+    (0, 4096),            # recv_valid on top of recv_topk_ids
+    (64, 4096),           # starts inside recv_topk_ids
+    (-8, 4096),           # ends inside recv_topk_ids
+    (2048, 2100),         # both fit, but not inside one stride
+])
+def test_noalloc_rejects_overlapping_outputs(ep, valid_off, stride):
+    # ep 4, 16 tokens per rank, top_k 8: 2048 id bytes and 64 valid bytes per rank
+    n = (ctypes.c_int32 * 4)(*([16] * 4))
+    dummy = ctypes.c_void_p(1 << 20)
+    ids = 1 << 24
+    st = ep.lib.ep_a2a_route_plan_noalloc(4, 16, 8, 16, -1, dummy, ctypes.cast(n, ctypes.c_void_p),
+                                          None, dummy, dummy, dummy, ctypes.c_void_p(ids),
+                                          ctypes.c_void_p(ids + valid_off), stride, None)
+    assert st == ep.ERR_INVALID_ARG
