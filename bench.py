@@ -322,6 +322,187 @@ def committed_traffic(kernel: str, workload: str):
 
 
 # --------------------------------------------------------------------------- #
+# Every workload on the record: one measurement per (workload, combine input)
+# --------------------------------------------------------------------------- #
+
+# (workload, combine inputs) measured for the `workloads` record of the
+# default line, besides the headline's prefill step: bf16 rows, E4M3 rows,
+# E4M3 rows with a per-row scale, per-(token, slot) expert outputs.
+RECORD_CASES = [
+    ("c1_ep4_tiny", ("bf16", "fp8", "fp8s", "experts")),
+    ("c2_ep8_decode", ("bf16", "fp8", "fp8s", "experts")),
+    ("c3_ep16_zipf_nvfp4", ("bf16", "fp8", "fp8s", "experts")),
+    ("c3_ep16_zipf_mxfp8", ("bf16",)),
+    ("c3_ep16_zipf_dsfp8", ("bf16",)),
+    ("c5_ep64_wide_masked", ("bf16", "fp8", "fp8s", "experts")),
+]
+COMBINE_KINDS = {"bf16": "BF16 rows", "fp8": "FP8 E4M3 rows",
+                 "fp8s": "FP8 E4M3 rows + per-row fp32 scale",
+                 "experts": "per-(token, slot) BF16 expert outputs, weighted reduction fused"}
+
+
+def live_slot_count(w, x) -> int:
+    """(token, slot) pairs of existing tokens whose expert a live rank owns: the
+    rows the combine of per-slot expert outputs reads."""
+    idn = x.token_selected_experts.numpy()
+    n = x.local_num_tokens
+    owner = np.where((idn >= 0) & (idn < w.num_experts), idn // w.experts_per_rank, -1)
+    alive = np.array([r not in w.masked_ranks for r in range(w.ep_size)] + [False])
+    exists = (np.arange(w.tokens_per_rank)[None, :] < n[:, None]) & alive[:w.ep_size, None]
+    return int((alive[owner] & exists[:, :, None]).sum())
+
+
+class DeviceCase:
+    """One workload's inputs on the device and a handle, with the step of each
+    combine input.  Combine inputs are drawn on the device from a seeded CUDA
+    generator (their values do not change the work), unless given."""
+
+    def __init__(self, w, x, device, kinds, xo=None):
+        import torch
+        from combine_route_plan_b200 import ep_a2a
+        self.w, self.x = w, x
+        self.ids = x.token_selected_experts.to(device)
+        self.payloads = [p.to(device) for p in x.payloads]
+        self.stats = x.eplb_local_stats.to(device) if x.eplb_local_stats is not None else None
+        self.n, self.mask = x.local_num_tokens, x.active_rank_mask
+        ep, tpr, k, H = w.ep_size, w.tokens_per_rank, w.top_k, w.hidden
+        gen = torch.Generator(device=device).manual_seed(w.seed + 55)
+        if xo is None and set(kinds) & {"bf16", "fp8", "fp8s"}:
+            xo = torch.randn((ep, ep * tpr, H), generator=gen, device=device,
+                             dtype=torch.bfloat16)
+        self.xo = xo
+        self.xo8 = ep_a2a.quantize_e4m3(xo) if "fp8" in kinds else None
+        self.codes = self.row_scales = None
+        if "fp8s" in kinds:
+            self.codes, self.row_scales = ep_a2a.quantize_e4m3_rows(xo)
+        self.y = self.wts = None
+        if "experts" in kinds:
+            self.y = torch.randn((ep, tpr, k, H), generator=gen, device=device,
+                                 dtype=torch.bfloat16)
+            self.wts = self.payloads[-1].view(torch.float32).view(ep, tpr, k)
+        self.out = torch.empty((ep, tpr, H), dtype=torch.bfloat16, device=device)
+        self.comm = ep_a2a.EpA2A(ep, w.num_experts, k, tpr, H, w.payload_row_bytes(),
+                                 eplb_stats_num_experts=w.num_experts if w.eplb else 0,
+                                 enable_rank_mask=self.mask is not None)
+        d = self.comm.dispatch(self.ids, self.n, self.payloads, tpr, self.stats, self.mask)
+        torch.cuda.synchronize()
+        self.sum_d = int(d.send_counts.sum().item())
+        self.live = ep - len(w.masked_ranks)
+        self.n_tok = int(sum(int(self.n[r]) for r in range(ep) if r not in w.masked_ranks))
+        self.live_slots = live_slot_count(w, x) if "experts" in kinds else 0
+
+    def step(self, kind):
+        c, tpr = self.comm, self.w.tokens_per_rank
+
+        def dispatch():
+            c.dispatch(self.ids, self.n, self.payloads, tpr, self.stats, self.mask, views=False)
+        if kind == "bf16":
+            return lambda: (dispatch(), c.combine(self.xo, self.out))
+        if kind == "fp8":
+            return lambda: (dispatch(), c.combine(self.xo8, self.out))
+        if kind == "fp8s":
+            return lambda: (dispatch(), c.combine_scaled(self.codes, self.row_scales, self.out))
+        return lambda: (dispatch(), c.combine_experts(self.wts, self.y, self.out))
+
+    def bytes(self, kind) -> "Bytes":
+        by = algorithmic_bytes(self.w, self.n_tok, self.sum_d, self.live, kind in ("fp8", "fp8s"),
+                               self.live_slots if kind == "experts" else 0)
+        if kind == "fp8s":        # the row scales travel with the codes
+            by = dataclasses.replace(by, combine=by.combine + self.sum_d * 4,
+                                     step=by.step + self.sum_d * 4)
+        return by
+
+    def destroy(self):
+        self.comm.destroy()
+
+
+def measure_case(case, kind, steps, warmup, stream, flush_buf, graph, peak):
+    """Step time (CUDA events; with flush_buf, L2 is flushed before every step
+    and each step is timed alone), per-kernel times from an eager pass with
+    events around each launch, and the roofline figures of both."""
+    import torch
+    from combine_route_plan_b200 import ep_a2a
+    step = case.step(kind)
+
+    def flushed():
+        if flush_buf is not None:
+            flush_buf.zero_()
+        step()
+    for _ in range(warmup):
+        flushed()
+    torch.cuda.synchronize()
+    ep_a2a.ep_a2a_profile_start(case.comm.handle, 4 * steps + 8)
+    for _ in range(steps):
+        flushed()
+    kt = ep_a2a.ep_a2a_profile_stop(case.comm.handle)
+    timed = step
+    g = None
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.current_stream().wait_stream(side)
+        with torch.cuda.graph(g):
+            step()
+        timed = g.replay
+    if flush_buf is not None:
+        ms = run_timed_flushed(timed, lambda: flush_buf.zero_(), steps, warmup, stream, None)
+    else:
+        ms = run_timed(timed, steps, warmup, CudaTimer(stream), None)
+    torch.cuda.synchronize()
+    del g
+    if case.comm.get_status() != ep_a2a.OK:
+        raise RuntimeError("device error word set")
+    by = case.bytes(kind)
+    step_s = ms / steps / 1e3
+    kbytes = {"route_plan": by.route, "copy_vec": by.copy, "copy_bulk": by.copy,
+              "copy_staged": by.copy, "combine": by.combine, "combine_experts": by.combine}
+    kernels = {}
+    for name, (cnt, tot) in kt.items():
+        if cnt:
+            avg_s = tot / cnt / 1e3
+            kernels[name] = {"avg_us": avg_s * 1e6, "algorithmic_bytes": kbytes[name],
+                             "gbs": kbytes[name] / avg_s / 1e9,
+                             "frac": kbytes[name] / avg_s / 1e9 / peak}
+    return {"workload": case.w.name, "combine": kind, "step_us": step_s * 1e6,
+            "tokens_per_s": case.n_tok / step_s, "step_algorithmic_bytes": by.step,
+            "step_gbs": by.step / step_s / 1e9, "step_frac": by.step / step_s / 1e9 / peak,
+            "tokens": case.n_tok, "mean_distinct_ranks": case.sum_d / max(case.n_tok, 1),
+            "kernels": kernels}
+
+
+def workloads_record(args, device, stream, peak, prefill_case=None):
+    """The `workloads` record: every other workload with every combine input
+    (L2 flushed before each step, CUDA-graph replay of the step), and the
+    prefill step with the other combine inputs (eager, inputs larger than L2)."""
+    import gc
+    import torch
+    from combine_route_plan_b200 import workloads as W
+    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    out = []
+    for name, kinds in RECORD_CASES:
+        w = W.BY_NAME[name]
+        case = DeviceCase(w, W.make_inputs(w, with_expert_output=False), device, kinds)
+        for kind in kinds:
+            r = measure_case(case, kind, args.workload_steps, 5, stream, flush_buf, True, peak)
+            r["timing"] = "CUDA-graph replay, 512 MB L2 flush before each step, steps timed alone"
+            out.append(r)
+        case.destroy()
+        del case
+        gc.collect()
+        torch.cuda.empty_cache()
+    del flush_buf
+    if prefill_case is not None:
+        for kind in ("fp8", "fp8s", "experts"):
+            r = measure_case(prefill_case, kind, args.workload_steps, 5, stream, None, False, peak)
+            r["timing"] = "eager, inputs larger than L2 (no flush)"
+            out.append(r)
+    return out
+
+
+# --------------------------------------------------------------------------- #
 # Our arm
 # --------------------------------------------------------------------------- #
 
@@ -413,13 +594,7 @@ def run_ours(args):
     sum_d = int(d.send_counts.sum().item())
     live = w.ep_size - len(w.masked_ranks)
     n_tok = int(sum(int(n[r]) for r in range(w.ep_size) if r not in w.masked_ranks))
-    live_slots = 0
-    if experts:
-        idn = x.token_selected_experts.numpy()
-        owner = np.where((idn >= 0) & (idn < w.num_experts), idn // w.experts_per_rank, -1)
-        alive = np.array([r not in w.masked_ranks for r in range(w.ep_size)] + [False])
-        exists = (np.arange(tpr)[None, :] < n[:, None]) & alive[:w.ep_size, None]
-        live_slots = int((alive[owner] & exists[:, :, None]).sum())
+    live_slots = live_slot_count(w, x) if experts else 0
     if dense:       # every existing token goes to, and is summed over, every live rank
         sum_d = n_tok * live
     by = algorithmic_bytes(w, n_tok, sum_d, live, fp8 or scaled, live_slots)
@@ -521,6 +696,17 @@ def run_ours(args):
         e2e = None if (scaled or dense) else run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws,
                                           y_dev=y if experts else None)
 
+    # every other workload and combine input on the record (one GPU only; the
+    # headline above is unaffected: it was timed before any of this ran)
+    records = None
+    if (rank == 0 and ws == 1 and args.workload_steps > 0 and not dense and not experts
+            and not scaled and not fp8 and args.workload == DEFAULT_WORKLOAD
+            and not args.tokens_per_rank):
+        pc = DeviceCase(w, x, device, ("fp8", "fp8s", "experts"), xo=xo)
+        records = workloads_record(args, device, stream, peak, pc)
+        pc.destroy()
+        del pc
+
     cpu = cpu_all = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_seconds)
@@ -567,6 +753,8 @@ def run_ours(args):
         }
         if fp8_ctx:
             rec["fp8_combine"] = fp8_ctx
+        if records is not None:
+            rec["workloads"] = records
         print(json.dumps(rec), flush=True)
     comm.destroy()
     if dist is not None:
@@ -805,6 +993,9 @@ def main(argv=None):
                          "the combine")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--fp8-steps", type=int, default=100)
+    ap.add_argument("--workload-steps", type=int, default=30,
+                    help="steps per entry of the `workloads` record (every other workload "
+                         "and combine input, measured after the headline); 0 = skip")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-all-cores-seconds", type=float, default=10.0,
