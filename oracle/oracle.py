@@ -259,6 +259,23 @@ def combine_scaled(plan: RoutePlan, codes, row_scales, hidden, out_init=None):
     return out
 
 
+def combine_experts_fp8(plan: RoutePlan, num_experts, token_selected_experts, topk_weights,
+                        expert_out, hidden, out_init=None):
+    """The low-precision combine of per-expert outputs with the quantisation on
+    the sending side (flashinfer.moe_ep.NVLinkOneSidedConfig,
+    use_low_precision_combine; flashinfer.moe_ep.NVLinkTwoSidedAlltoAll,
+    combine()): each destination rank forms its row z_d from its own experts'
+    weighted outputs (``expert_reduce``), quantises it to E4M3 with one fp32
+    scale per row (``quantize_e4m3_rows``), and the rows are summed as decoded
+    codes times their scales in ascending rank order (``combine_scaled``).
+    The three steps in that order; nothing else."""
+    z = expert_reduce(plan, num_experts, token_selected_experts, topk_weights, expert_out,
+                      hidden)
+    codes, scales = quantize_e4m3_rows(z, hidden)
+    return combine_scaled(plan, codes.reshape(z.shape), scales.reshape(z.shape[:2]), hidden,
+                          out_init=out_init)
+
+
 def allgather(ep_size, tokens_per_rank, local_num_tokens, payload, active_rank_mask=None,
               recv_init=None):
     """Dense dispatch: uint8 ``[ep, ep*tpr, row_bytes]`` (see ``oracle_allgather``)."""
@@ -318,7 +335,8 @@ def e4m3_to_f32(b: int) -> float:
 
 
 __all__ = ["build", "route", "dispatch_payload", "eplb_gather", "combine", "expert_reduce",
-           "combine_experts", "quantize_e4m3_rows", "combine_scaled", "allgather",
+           "combine_experts", "quantize_e4m3_rows", "combine_scaled", "combine_experts_fp8",
+           "allgather",
            "reduce_scatter",
            "quantize_e4m3", "bf16_from_f32", "bf16_to_f32", "e4m3_from_f32",
            "e4m3_to_f32", "RoutePlan"]

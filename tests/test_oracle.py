@@ -656,3 +656,65 @@ def test_reduce_scatter_hand_example(oracle_mod):
     assert bits_to_f32(out[0, 0]).tolist() == [101.0, 1.0]
     assert bits_to_f32(out[2, 0]).tolist() == [101.0, 5.0]
     assert np.all(out[1, 0] == 0xEEEE)
+
+
+def test_combine_experts_fp8_hand_example(oracle_mod):
+    """The sender-side FP8 combine of per-expert outputs, worked by hand.
+
+    ep 2, E 4 (rank 0 owns experts 0-1, rank 1 owns 2-3), top_k 2, one token of
+    rank 0 with ids [0, 3] and weights [1, 0.5], hidden 2:
+      y0 = [224, -3]       -> z_0 = bf16(1 * y0)   = [224, -3]
+      y1 = [14, 1.1875]    -> z_1 = bf16(0.5 * y1) = [7, 0.59375]
+    Row quantisation (one scale per row, amax / 448):
+      z_0: amax 224, scale 0.5, inv 2   -> codes E4M3([448, -6]) = [448, -6]
+      z_1: amax 7, scale 2^-6, inv 64   -> codes E4M3([448, 38]) = [448, 40]
+           (38 lies halfway between 36 and 40; nearest-even picks 40)
+    Combine, ascending rank, fma(decode, scale, acc) from +0:
+      column 0: 448 * 0.5 = 224, then 224 + 448 * 2^-6 = 231
+      column 1: -6 * 0.5 = -3,   then -3 + 40 * 2^-6 = -2.375
+    The unquantised combine gives -2.40625 in column 1: the quantisation shows."""
+    ids = np.array([[[0, 3]], [[0, 0]]], np.int32)
+    n = np.array([1, 0], np.int32)
+    plan = oracle_mod.route(2, 4, 2, 1, ids, n)
+    w = np.array([[[1.0, 0.5]], [[0.0, 0.0]]], np.float32)
+    y = np.zeros((2, 1, 2, 2), np.uint16)
+    y[0, 0, 0] = bf16_bits([224.0, -3.0])
+    y[0, 0, 1] = bf16_bits([14.0, 1.1875])
+    out = oracle_mod.combine_experts_fp8(plan, 4, ids, w, y, 2)
+    assert list(bits_to_f32(out[0, 0])) == [231.0, -2.375]
+    plain = oracle_mod.combine_experts(plan, 4, ids, w, y, 2)
+    assert list(bits_to_f32(plain[0, 0])) == [231.0, -2.40625]
+    assert np.all(out[1] == 0xEEEE)          # rank 1 has no token: its row is untouched
+
+
+def test_combine_experts_fp8_error_bound(oracle_mod):
+    """Against the unquantised combine of the same expert outputs: each rank's
+    row loses at most half an E4M3 step (2^-4 relative, or 2^-10 of its scale
+    near zero) before the sum, so the result differs by at most the sum of those
+    bounds plus the final bf16 rounding."""
+    w = W.scaled(W.C2, 8)
+    x = W.make_inputs(w, with_expert_output=False)
+    ids = x.token_selected_experts.numpy()
+    plan = oracle_mod.route(w.ep_size, w.num_experts, w.top_k, w.tokens_per_rank, ids,
+                            x.local_num_tokens)
+    rng = np.random.default_rng(12)
+    H = 64
+    wts = rng.standard_normal((w.ep_size, w.tokens_per_rank, w.top_k)).astype(np.float32)
+    y = bf16_bits(rng.standard_normal(w.ep_size * w.tokens_per_rank * w.top_k * H)
+                  .astype(np.float32)).reshape(w.ep_size, w.tokens_per_rank, w.top_k, H)
+    got = bits_to_f32(oracle_mod.combine_experts_fp8(plan, w.num_experts, ids, wts, y, H))
+    z = oracle_mod.expert_reduce(plan, w.num_experts, ids, wts, y, H)
+    zf = bits_to_f32(z).astype(np.float64)
+    exact = np.zeros((w.ep_size, w.tokens_per_rank, H))
+    bound = np.zeros_like(exact)
+    tpr = w.tokens_per_rank
+    for s in range(w.ep_size * tpr):
+        r, t = divmod(s, tpr)
+        for i in range(plan.num_dst[r, t]):
+            d = plan.dst_ranks[r, t, i]
+            row = zf[d, s]
+            scale = np.abs(row).max() / 448.0
+            exact[r, t] += row
+            bound[r, t] += np.maximum(2.0 ** -4 * np.abs(row), 2.0 ** -10 * scale)
+    bound = bound * (1 + 2.0 ** -10) + 2.0 ** -8 * np.abs(exact) + 1e-30
+    assert np.all(np.abs(got - exact) <= bound)
