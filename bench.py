@@ -329,16 +329,18 @@ def committed_traffic(kernel: str, workload: str):
 # default line, besides the headline's prefill step: bf16 rows, E4M3 rows,
 # E4M3 rows with a per-row scale, per-(token, slot) expert outputs.
 RECORD_CASES = [
-    ("c1_ep4_tiny", ("bf16", "fp8", "fp8s", "experts")),
-    ("c2_ep8_decode", ("bf16", "fp8", "fp8s", "experts")),
-    ("c3_ep16_zipf_nvfp4", ("bf16", "fp8", "fp8s", "experts")),
+    ("c1_ep4_tiny", ("bf16", "fp8", "fp8s", "experts", "experts_fp8")),
+    ("c2_ep8_decode", ("bf16", "fp8", "fp8s", "experts", "experts_fp8")),
+    ("c3_ep16_zipf_nvfp4", ("bf16", "fp8", "fp8s", "experts", "experts_fp8")),
     ("c3_ep16_zipf_mxfp8", ("bf16",)),
     ("c3_ep16_zipf_dsfp8", ("bf16",)),
-    ("c5_ep64_wide_masked", ("bf16", "fp8", "fp8s", "experts")),
+    ("c5_ep64_wide_masked", ("bf16", "fp8", "fp8s", "experts", "experts_fp8")),
 ]
 COMBINE_KINDS = {"bf16": "BF16 rows", "fp8": "FP8 E4M3 rows",
                  "fp8s": "FP8 E4M3 rows + per-row fp32 scale",
-                 "experts": "per-(token, slot) BF16 expert outputs, weighted reduction fused"}
+                 "experts": "per-(token, slot) BF16 expert outputs, weighted reduction fused",
+                 "experts_fp8": "per-(token, slot) BF16 expert outputs, weighted reduction and "
+                                "per-row E4M3 quantisation fused (sender-side FP8)"}
 
 
 def live_slot_count(w, x) -> int:
@@ -376,7 +378,7 @@ class DeviceCase:
         if "fp8s" in kinds:
             self.codes, self.row_scales = ep_a2a.quantize_e4m3_rows(xo)
         self.y = self.wts = None
-        if "experts" in kinds:
+        if "experts" in kinds or "experts_fp8" in kinds:
             self.y = torch.randn((ep, tpr, k, H), generator=gen, device=device,
                                  dtype=torch.bfloat16)
             self.wts = self.payloads[-1].view(torch.float32).view(ep, tpr, k)
@@ -389,7 +391,8 @@ class DeviceCase:
         self.sum_d = int(d.send_counts.sum().item())
         self.live = ep - len(w.masked_ranks)
         self.n_tok = int(sum(int(self.n[r]) for r in range(ep) if r not in w.masked_ranks))
-        self.live_slots = live_slot_count(w, x) if "experts" in kinds else 0
+        self.live_slots = live_slot_count(w, x) if ("experts" in kinds or
+                                                    "experts_fp8" in kinds) else 0
 
     def step(self, kind):
         c, tpr = self.comm, self.w.tokens_per_rank
@@ -402,11 +405,13 @@ class DeviceCase:
             return lambda: (dispatch(), c.combine(self.xo8, self.out))
         if kind == "fp8s":
             return lambda: (dispatch(), c.combine_scaled(self.codes, self.row_scales, self.out))
+        if kind == "experts_fp8":
+            return lambda: (dispatch(), c.combine_experts_fp8(self.wts, self.y, self.out))
         return lambda: (dispatch(), c.combine_experts(self.wts, self.y, self.out))
 
     def bytes(self, kind) -> "Bytes":
         by = algorithmic_bytes(self.w, self.n_tok, self.sum_d, self.live, kind in ("fp8", "fp8s"),
-                               self.live_slots if kind == "experts" else 0)
+                               self.live_slots if kind in ("experts", "experts_fp8") else 0)
         if kind == "fp8s":        # the row scales travel with the codes
             by = dataclasses.replace(by, combine=by.combine + self.sum_d * 4,
                                      step=by.step + self.sum_d * 4)
@@ -458,7 +463,10 @@ def measure_case(case, kind, steps, warmup, stream, flush_buf, graph, peak):
     by = case.bytes(kind)
     step_s = ms / steps / 1e3
     kbytes = {"route_plan": by.route, "copy_vec": by.copy, "copy_bulk": by.copy,
-              "copy_staged": by.copy, "combine": by.combine, "combine_experts": by.combine}
+              "copy_staged": by.copy, "combine": by.combine, "combine_experts": by.combine,
+              "combine_experts_fp8": by.combine}
+    if not kt["route_plan"][0]:     # the copy kernel routed the tokens itself
+        kbytes["copy_vec"] = by.copy + by.route
     kernels = {}
     for name, (cnt, tot) in kt.items():
         if cnt:
@@ -495,7 +503,7 @@ def workloads_record(args, device, stream, peak, prefill_case=None):
         torch.cuda.empty_cache()
     del flush_buf
     if prefill_case is not None:
-        for kind in ("fp8", "fp8s", "experts"):
+        for kind in ("fp8", "fp8s", "experts", "experts_fp8"):
             r = measure_case(prefill_case, kind, args.workload_steps, 5, stream, None, False, peak)
             r["timing"] = "eager, inputs larger than L2 (no flush)"
             out.append(r)
@@ -537,7 +545,8 @@ def run_ours(args):
     stats = x.eplb_local_stats.to(device) if x.eplb_local_stats is not None else None
     xo = x.expert_output.to(device)
     xo8 = ep_a2a.quantize_e4m3(xo)
-    experts = args.combine == "experts"
+    experts = args.combine in ("experts", "experts_fp8")
+    experts_fp8 = args.combine == "experts_fp8"
     scaled = args.combine == "fp8s"
     if scaled:
         codes, row_scales = ep_a2a.quantize_e4m3_rows(xo)
@@ -579,7 +588,9 @@ def run_ours(args):
                 call()
             return
         comm.dispatch(ids, n, payloads, tpr, stats, mask, views=False)
-        if experts:
+        if experts_fp8:
+            comm.combine_experts_fp8(wts, y, out)
+        elif experts:
             comm.combine_experts(wts, y, out)
         elif scaled:
             comm.combine_scaled(codes, row_scales, out)
@@ -668,7 +679,10 @@ def run_ours(args):
             per_kernel[name] = {"launches": cnt, "avg_ms": tot / cnt}
     kbytes = {"route_plan": by.route, "copy_bulk": by.copy, "copy_vec": by.copy,
               "copy_staged": by.copy, "combine": by.combine, "combine_experts": by.combine,
+              "combine_experts_fp8": by.combine,
               "allgather": by.copy, "reduce_scatter": by.combine}
+    if "copy_vec" in per_kernel and "route_plan" not in per_kernel:
+        kbytes["copy_vec"] = by.copy + by.route     # the copy kernel routed the tokens itself
     for name, e in per_kernel.items():
         e["algorithmic_bytes"] = kbytes[name]
         e["achieved_gbs"] = kbytes[name] / (e["avg_ms"] / 1e3) / 1e9
@@ -694,7 +708,8 @@ def run_ours(args):
     e2e = None
     if args.e2e_steps > 0:
         e2e = None if (scaled or dense) else run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws,
-                                          y_dev=y if experts else None)
+                                          y_dev=y if experts else None,
+                                          experts_fp8=experts_fp8)
 
     # every other workload and combine input on the record (one GPU only; the
     # headline above is unaffected: it was timed before any of this ran)
@@ -702,7 +717,7 @@ def run_ours(args):
     if (rank == 0 and ws == 1 and args.workload_steps > 0 and not dense and not experts
             and not scaled and not fp8 and args.workload == DEFAULT_WORKLOAD
             and not args.tokens_per_rank):
-        pc = DeviceCase(w, x, device, ("fp8", "fp8s", "experts"), xo=xo)
+        pc = DeviceCase(w, x, device, ("fp8", "fp8s", "experts", "experts_fp8"), xo=xo)
         records = workloads_record(args, device, stream, peak, pc)
         pc.destroy()
         del pc
@@ -723,6 +738,9 @@ def run_ours(args):
                             f"top_k {w.top_k}, {tpr} tokens/rank, hidden {w.hidden} BF16, "
                             f"extra {w.extra_bytes} B/token, EPLB stats, "
                             + ("combine of per-expert outputs (weighted local reduction "
+                               "and per-row E4M3 quantisation fused, fp32 accumulate)"
+                               if experts_fp8 else
+                               "combine of per-expert outputs (weighted local reduction "
                                "fused, fp32 accumulate)" if experts else
                                f"{'FP8 E4M3 with a per-row fp32 scale' if scaled else 'FP8 E4M3' if fp8 else 'BF16'} combine (fp32 accumulate)"),
                 "tokens_per_step_per_gpu": n_tok, "mean_distinct_ranks": sum_d / n_tok,
@@ -779,7 +797,7 @@ def dense_call_times(calls, steps, stream, flush=None):
             for name, ev in zip(("allgather", "reduce_scatter"), evs)}
 
 
-def run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws, y_dev=None):
+def run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws, y_dev=None, experts_fp8=False):
     """Same step through the public API with the inputs in pinned host memory:
     every step copies the inputs host->device and the result device->host.
     With y_dev (the combine of per-expert outputs) the combine input is the
@@ -820,7 +838,10 @@ def run_e2e(args, w, x, comm, device, stream, dist, n_tok, ws, y_dev=None):
         stream.wait_stream(s_out)        # d_out: the previous download is done
         if y_dev is not None:
             wts = d_pay[-1].view(torch.float32).view(w.ep_size, w.tokens_per_rank, w.top_k)
-            comm.combine_experts(wts, d_xo, d_out, stream=stream)
+            if experts_fp8:
+                comm.combine_experts_fp8(wts, d_xo, d_out, stream=stream)
+            else:
+                comm.combine_experts(wts, d_xo, d_out, stream=stream)
         else:
             comm.combine(d_xo, d_out, stream=stream)
         s_out.wait_stream(stream)
@@ -987,10 +1008,12 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--tokens-per-rank", type=int, default=0,
                     help="run the workload with this many tokens per rank (small profiling cases)")
-    ap.add_argument("--combine", choices=["bf16", "fp8", "fp8s", "experts"], default="bf16",
+    ap.add_argument("--combine", choices=["bf16", "fp8", "fp8s", "experts", "experts_fp8"],
+                    default="bf16",
                     help="combine input: bf16 / fp8 / fp8 with a per-row scale rows per rank, "
                          "or bf16 outputs per (token, slot) reduced with topk_weights inside "
-                         "the combine")
+                         "the combine (experts_fp8: and each rank's row quantised to E4M3 "
+                         "with one scale before the sum)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--fp8-steps", type=int, default=100)
     ap.add_argument("--workload-steps", type=int, default=30,

@@ -532,6 +532,218 @@ __global__ void __launch_bounds__(512) combine_experts_pipe_kernel(const Combine
   }
 }
 
+// ---------------------------------------------------------------------------
+// Low-precision combine of per-expert outputs, quantised on the sending side
+// (flashinfer.moe_ep.NVLinkOneSidedConfig, use_low_precision_combine, with the
+// per-row scale convention of the scaled FP8 combine): for each destination d
+// of a token, z_d = bf16(sum over d's slots of w_j * y_j) as in the expert
+// combine; amax_d = max |z_d|, scale_d = amax_d / 448, inv_d = 448 / amax_d
+// (fp32, rounded to nearest; 1 and 1 for a zero row); code = E4M3(z_d * inv_d)
+// nearest-even, saturating; out = bf16(sum over d ascending of
+// fmaf(decode(code), scale_d, acc)) from +0.0f.  Neither the rows z_d nor the
+// codes and scales are written to memory.
+// ---------------------------------------------------------------------------
+
+// E4M3 round trip of 8 values scaled by inv: code = E4M3(z * inv) (product
+// rounded to fp32, nearest-even, saturating), then acc = fmaf(decode, scale, acc).
+__device__ __forceinline__ void fp8_roundtrip_acc(float* acc, const uint4& zb, float inv,
+                                                  float scale) {
+  const uint32_t w[4] = {zb.x, zb.y, zb.z, zb.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = make_float2(__fmul_rn(bf16_bits_to_f32(w[i] & 0xFFFFu), inv),
+                                 __fmul_rn(bf16_bits_to_f32(w[i] >> 16), inv));
+    const __nv_fp8x2_storage_t code = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(code, __NV_E4M3);
+    __half_raw lo, hi;
+    lo.x = hr.x;
+    hi.x = hr.y;
+    acc[2 * i] = __fmaf_rn(__half2float(__half(lo)), scale, acc[2 * i]);
+    acc[2 * i + 1] = __fmaf_rn(__half2float(__half(hi)), scale, acc[2 * i + 1]);
+  }
+}
+
+// The same for one value.
+__device__ __forceinline__ float fp8_roundtrip(float z, float inv, float scale, float acc) {
+  const __nv_fp8_storage_t code =
+      __nv_cvt_float_to_fp8(__fmul_rn(z, inv), __NV_SATFINITE, __NV_E4M3);
+  const __half_raw hr = __nv_cvt_fp8_to_halfraw(code, __NV_E4M3);
+  return __fmaf_rn(__half2float(__half(hr)), scale, acc);
+}
+
+// Per-destination scale and inverse from amax (the row quantiser's rule).
+__device__ __forceinline__ void row_scale_of(float amax, float& scale, float& inv) {
+  scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  inv = amax > 0.0f ? __fdiv_rn(448.0f, amax) : 1.0f;
+}
+
+constexpr int kFp8ExpertsMaxWarps = 32;
+
+// top_k <= 8, hidden a multiple of 8, 16-byte aligned rows, and the token's
+// rows z_d (at most min(top_k, ep) of them, bf16) fit in shared memory; at
+// most 448 threads, so that two CTAs share an SM without spilling.  One
+// token per CTA at a time: phase 1 loads each 16-byte column vector of every
+// participating slot row once, forms every destination's z_d for it, stores
+// it to shared memory and keeps a per-destination running max; the CTA
+// reduces the maxima to the scales; phase 2 reads z_d back, takes each value
+// through E4M3 and sums in ascending rank order.
+__global__ void __launch_bounds__(448, 2) combine_experts_fp8_kernel(const CombineExpertsArgs a) {
+  pdl_wait();
+  extern __shared__ __align__(16) uint8_t z_mem[];       // [rows][H] bf16
+  __shared__ float s_max[kFp8ExpertsMaxWarps][8];
+  __shared__ float s_scale[8], s_inv[8];
+  uint16_t* zs = reinterpret_cast<uint16_t*>(z_mem);
+  const int nvec = a.H / 8;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    const int nd = a.plan_nd[tok];
+    if (nd == kNoToken) continue;
+    uint16_t* out = a.out + tok * (int64_t)a.H;
+    if (nd == 0) {           // every owner masked off: the sum is empty
+      for (int v = threadIdx.x; v < nvec; v += blockDim.x)
+        reinterpret_cast<uint4*>(out)[v] = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const uint64_t w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    if (!plan_row_ok(nd, w0, 0, 0, 0, a.ep, 8, a.err)) continue;
+    int own[8];
+    float wt[8];
+    slot_owners<8>(a, tok, nd, w0, 0, 0, 0, own, wt);
+    // phase 1: z rows into shared memory and the per-destination maxima
+    float amax[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) amax[q] = 0.0f;
+    const uint16_t* yt = a.y + tok * (int64_t)a.k * a.H;
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      uint4 raw[8];
+      expert_rows_load(raw, yt + (int64_t)v * 8, own, a.H);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q >= nd) break;
+        const int d = (int)((w0 >> (8 * q)) & 0xFFu);
+        float z[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) z[e] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (own[j] != d) continue;
+          const uint32_t wv[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            z[2 * i] = __fmaf_rn(wt[j], bf16_bits_to_f32(wv[i] & 0xFFFFu), z[2 * i]);
+            z[2 * i + 1] = __fmaf_rn(wt[j], bf16_bits_to_f32(wv[i] >> 16), z[2 * i + 1]);
+          }
+        }
+        uint4 pk;
+        pk.x = pack_bf16x2(z[0], z[1]);
+        pk.y = pack_bf16x2(z[2], z[3]);
+        pk.z = pack_bf16x2(z[4], z[5]);
+        pk.w = pack_bf16x2(z[6], z[7]);
+        const uint32_t pw[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          amax[q] = fmaxf(amax[q], fabsf(bf16_bits_to_f32(pw[i] & 0xFFFFu)));
+          amax[q] = fmaxf(amax[q], fabsf(bf16_bits_to_f32(pw[i] >> 16)));
+        }
+        *reinterpret_cast<uint4*>(zs + (int64_t)q * a.H + (int64_t)v * 8) = pk;
+      }
+    }
+    // the CTA's maxima -> scales
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+        amax[q] = fmaxf(amax[q], __shfl_xor_sync(0xFFFFFFFFu, amax[q], o));
+      if (lane == 0) s_max[warp][q] = amax[q];
+    }
+    __syncthreads();
+    if (threadIdx.x < 8) {
+      float m = 0.0f;
+      for (int i = 0; i < nwarps; ++i) m = fmaxf(m, s_max[i][threadIdx.x]);
+      row_scale_of(m, s_scale[threadIdx.x], s_inv[threadIdx.x]);
+    }
+    __syncthreads();
+    // phase 2: through E4M3 and summed in ascending rank order
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q >= nd) break;
+        const uint4 zb = *reinterpret_cast<const uint4*>(zs + (int64_t)q * a.H + (int64_t)v * 8);
+        fp8_roundtrip_acc(acc, zb, s_inv[q], s_scale[q]);
+      }
+      uint4 pk;
+      pk.x = pack_bf16x2(acc[0], acc[1]);
+      pk.y = pack_bf16x2(acc[2], acc[3]);
+      pk.z = pack_bf16x2(acc[4], acc[5]);
+      pk.w = pack_bf16x2(acc[6], acc[7]);
+      reinterpret_cast<uint4*>(out)[v] = pk;
+    }
+    __syncthreads();         // z rows and scales are rewritten for the next token
+  }
+}
+
+// Any top_k (<= 32) and hidden size, no shared-memory rows: for each
+// destination a first pass recomputes z_d over the row to find its maximum;
+// a second pass recomputes z_d, takes it through E4M3 and sums.
+__global__ void __launch_bounds__(256) combine_experts_fp8_any_kernel(const CombineExpertsArgs a) {
+  pdl_wait();
+  constexpr int KMAX = kMaxTopK;
+  __shared__ float s_max[8];
+  __shared__ float s_scale[KMAX], s_inv[KMAX];
+  const int words = a.plan_stride / 8;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    const int nd = a.plan_nd[tok];
+    if (nd == kNoToken) continue;
+    uint16_t* out = a.out + tok * (int64_t)a.H;
+    const uint64_t* row = reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    const uint64_t w0 = row[0];
+    const uint64_t w1 = words > 1 ? row[1] : 0;
+    const uint64_t w2 = words > 2 ? row[2] : 0;
+    const uint64_t w3 = words > 3 ? row[3] : 0;
+    if (!plan_row_ok(nd, w0, w1, w2, w3, a.ep, a.plan_stride, a.err)) continue;
+    int own[KMAX];
+    float wt[KMAX];
+    if (nd > 0) slot_owners<KMAX>(a, tok, nd, w0, w1, w2, w3, own, wt);
+    const uint16_t* yt = a.y + tok * (int64_t)a.k * a.H;
+    auto z_of = [&](int d, int h) {
+      float z = 0.0f;
+      for (int j = 0; j < a.k; ++j)
+        if (own[j] == d) z = __fmaf_rn(wt[j], bf16_bits_to_f32(yt[(int64_t)j * a.H + h]), z);
+      return bf16_round(z);
+    };
+    for (int q = 0; q < nd; ++q) {
+      const int d = dst_rank(w0, w1, w2, w3, q);
+      float m = 0.0f;
+      for (int h = threadIdx.x; h < a.H; h += blockDim.x) m = fmaxf(m, fabsf(z_of(d, h)));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      if (lane == 0) s_max[warp] = m;
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        float mm = 0.0f;
+        for (int i = 0; i < nwarps; ++i) mm = fmaxf(mm, s_max[i]);
+        row_scale_of(mm, s_scale[q], s_inv[q]);
+      }
+      __syncthreads();
+    }
+    for (int h = threadIdx.x; h < a.H; h += blockDim.x) {
+      float acc = 0.0f;
+      for (int q = 0; q < nd; ++q)
+        acc = fp8_roundtrip(z_of(dst_rank(w0, w1, w2, w3, q), h), s_inv[q], s_scale[q], acc);
+      out[h] = (uint16_t)f32_to_bf16_bits(acc);
+    }
+    __syncthreads();         // scales are rewritten for the next token
+  }
+}
+
 // Any top_k (<= 32) and hidden size: one element per thread step.
 __global__ void __launch_bounds__(512) combine_experts_any_kernel(const CombineExpertsArgs a) {
   pdl_wait();
@@ -815,6 +1027,18 @@ cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, bool p
   if (vec && pipe) return launch_kernel(combine_experts_pipe_kernel, g, b, 0, stream, pdl, a);
   if (vec) return launch_kernel(combine_experts_vec_kernel, g, b, 0, stream, pdl, a);
   return launch_kernel(combine_experts_any_kernel, g, b, 0, stream, pdl, a);
+}
+
+cudaError_t launch_combine_experts_fp8(const CombineExpertsArgs& a, bool smem_rows, int threads,
+                                       int grid, size_t smem, cudaStream_t stream, bool pdl) {
+  const dim3 g(grid), b(threads);
+  if (smem_rows) {
+    cudaError_t e = cudaFuncSetAttribute(combine_experts_fp8_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_kernel(combine_experts_fp8_kernel, g, b, smem, stream, pdl, a);
+  }
+  return launch_kernel(combine_experts_fp8_any_kernel, g, b, 0, stream, pdl, a);
 }
 
 cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n,

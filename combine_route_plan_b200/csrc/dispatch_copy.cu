@@ -340,6 +340,107 @@ __device__ __forceinline__ int token_destinations(const CopyArgs& a, int64_t tok
   return nd;
 }
 
+__device__ __forceinline__ bool rank_is_live(const CopyArgs& a, int r) {
+  return !a.use_mask || ((a.live[r >> 6] >> (r & 63)) & 1ull);
+}
+
+// The routing outputs of token slot `tok` (one warp, all 32 lanes), the same
+// as the routing kernel writes for it: plan_nd / plan_dst (destinations in
+// ascending rank order), the send counts, and for every live rank d its valid
+// byte and received ids (the token's ids if d is a destination, else
+// invalid_id).  Lane j < k holds expert slot j; owners are de-duplicated with
+// a warp match; a leader's position in the ascending list is the number of
+// leaders with a smaller rank; lane w < 8 holds bits 32w..32w+31 of the
+// destination set, which the lanes writing rank d's row read by shuffle.
+__device__ __forceinline__ void route_token(const CopyArgs& a, int64_t tok, int lane) {
+  const int r = (int)(tok / a.tpr);
+  const int t = (int)(tok - (int64_t)r * a.tpr);
+  const bool exists = t < a.n[r];          // n[r] is 0 for masked-off ranks
+  int32_t e = 0;
+  int d = -1;
+  if (exists && lane < a.k) {
+    e = a.ids[tok * a.k + lane];
+    if (e >= 0 && e < a.E) {
+      const int owner = e / a.epr;
+      if (rank_is_live(a, owner)) d = owner;
+    }
+  }
+  const unsigned peers = __match_any_sync(kFull, d);
+  const bool leader = d >= 0 && (__ffs(peers) - 1) == lane;
+  const unsigned leaders = __ballot_sync(kFull, leader);
+  const int nd = __popc(leaders);
+  int pos = 0;
+  uint32_t word = 0;                       // lane w: set bits 32w..32w+31
+  for (int i = 0; i < a.k; ++i) {
+    const int other = __shfl_sync(kFull, d, i);
+    pos += (((leaders >> i) & 1u) != 0u) && other < d;
+    if (other >= 0 && (other >> 5) == lane) word |= 1u << (other & 31);
+  }
+  uint8_t* row = const_cast<uint8_t*>(a.plan_dst) + tok * a.plan_stride;
+  if (lane == 0) const_cast<uint8_t*>(a.plan_nd)[tok] = exists ? (uint8_t)nd : kNoToken;
+  if (leader) {
+    row[pos] = (uint8_t)d;
+    atomicAdd(&a.count_acc[r * a.ep + d], 1);
+  }
+  if (lane < a.plan_stride && lane >= nd) row[lane] = kPad;
+  // received ids of every live rank: lane handles (rank idx / k, slot idx % k)
+  const int total = a.ep * a.k;
+  for (int base = 0; base < total; base += 32) {
+    const int idx = base + lane;
+    const int dd = idx / a.k;
+    const int j = idx - dd * a.k;
+    const int32_t ej = __shfl_sync(kFull, e, j & 31);
+    const uint32_t wd = __shfl_sync(kFull, word, (dd >> 5) & 7);
+    if (idx < total && rank_is_live(a, dd)) {
+      int32_t* ids = reinterpret_cast<int32_t*>(a.rank0 + (int64_t)dd * a.rank_stride + a.off_ids);
+      ids[tok * a.k + j] = ((wd >> (dd & 31)) & 1u) ? ej : a.invalid_id;
+    }
+  }
+  for (int base = 0; base < a.ep; base += 32) {
+    const int dd = base + lane;
+    const uint32_t wd = __shfl_sync(kFull, word, (dd >> 5) & 7);
+    if (dd < a.ep && rank_is_live(a, dd))
+      a.rank0[(int64_t)dd * a.rank_stride + a.off_valid + tok] = (uint8_t)((wd >> (dd & 31)) & 1u);
+  }
+}
+
+// EPLB gather: gathered[d][r][:] = live(r) ? stats[r][:] : 0 for live d, as
+// int4 (E % 4 == 0; rank regions and offsets are 256-byte aligned).
+__device__ __forceinline__ void eplb_gather_rows(const CopyArgs& a) {
+  const int e4 = a.eplb_n / 4;
+  const int64_t total = (int64_t)a.ep * a.ep * e4;
+  const int4* src = reinterpret_cast<const int4*>(a.eplb_stats);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int d = (int)(i / ((int64_t)a.ep * e4));
+    const int64_t rem = i - (int64_t)d * a.ep * e4;
+    const int r = (int)(rem / e4);
+    const int c = (int)(rem - (int64_t)r * e4);
+    if (!rank_is_live(a, d)) continue;
+    int4 v = make_int4(0, 0, 0, 0);
+    if (rank_is_live(a, r)) v = src[(int64_t)r * e4 + c];
+    reinterpret_cast<int4*>(a.rank0 + d * a.rank_stride + a.off_eplb)[(int64_t)r * e4 + c] = v;
+  }
+}
+
+// send_counts = the accumulators, once every CTA has added its tokens: the
+// last CTA to take a ticket copies them and resets the scratch to zero, so no
+// clearing is needed per call.
+__device__ __forceinline__ void finish_counts(const CopyArgs& a) {
+  __shared__ bool s_last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(a.count_ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int i = threadIdx.x; i < a.ep * a.ep; i += blockDim.x)
+    a.send_counts[i] = atomicExch(&a.count_acc[i], 0);
+  if (threadIdx.x == 0) atomicExch(a.count_ticket, 0u);
+}
+
 // TPT threads per token (a warp for many tokens, up to the whole CTA for few,
 // so that short steps still fill the GPU).  Each warp finds its token's
 // destinations from the routing ids itself, so the kernel does not depend on
@@ -356,12 +457,20 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
   const int group = threadIdx.x / TPT;
   const int lane = threadIdx.x & 31;
   const int64_t tok_step = (int64_t)gridDim.x * kGroups;
+  if (a.route) {
+    // this launch is the whole dispatch: it reads the caller's ids and rows and
+    // rewrites the plan the previous combine read, so it waits for the
+    // preceding grid first
+    pdl_wait();
+    if (a.eplb_stats != nullptr) eplb_gather_rows(a);
+  }
   for (int64_t tok = (int64_t)blockIdx.x * kGroups + group; tok < a.ntok; tok += tok_step) {
     if (kUniform && a.prefetch && gl == 0 && tok + tok_step < a.ntok) {
       // the group's next token: its rows into L2 while this one is copied
       for (int p = 0; p < a.np; ++p)
         prefetch_l2(a.src[p] + (tok + tok_step) * a.rb[p], (uint32_t)a.rb[p]);
     }
+    if (a.route && gl < 32) route_token(a, tok, lane);   // the group's first warp
     uint64_t w0, w1, w2, w3;
     const int nd = token_destinations(a, tok, lane, w0, w1, w2, w3);
     if (nd == 0) continue;
@@ -406,7 +515,10 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
       }
     }
   }
-  pdl_wait();
+  if (a.route)
+    finish_counts(a);
+  else
+    pdl_wait();
 }
 
 template <int NCW, int MAXV>

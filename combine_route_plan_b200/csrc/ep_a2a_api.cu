@@ -146,6 +146,7 @@ struct ep_a2a_handle_s {
   int copy_vec_bytes;         // vector copy: widest access, 16 or 32 bytes
   int combine_pipeline;       // 1: the two-deep pipelined kernels
   int copy_ctas_per_sm;
+  int route_in_copy;      // vector copy path: 1 = the copy kernel also routes (one launch)
   int copy_stages;        // 0 = choose from the row size
   int combine_threads;
   int64_t bulk_min_row;   // rows below this go to the vector copy
@@ -366,6 +367,7 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   h->copy_vec_bytes = 32;
   h->combine_pipeline = -1;
   h->copy_ctas_per_sm = 1;
+  h->route_in_copy = 1;
   h->copy_stages = 4;
   h->combine_threads = 0;
   h->bulk_min_row = 0;
@@ -460,6 +462,10 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
         return fail(EP_A2A_ERR_INVALID_ARG, "combine CTAs per SM must be 0..1024");
       h->combine_ctas_per_sm = (int)value;
       return EP_A2A_OK;
+    case EP_A2A_OPT_ROUTE_IN_COPY:
+      if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "route in copy must be 0 or 1");
+      h->route_in_copy = (int)value;
+      return EP_A2A_OK;
   }
   return fail(EP_A2A_ERR_INVALID_ARG, "unknown option %d", (int)option);
 }
@@ -546,11 +552,19 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
   ra.plan_stride = L.plan_stride;
   ra.eplb_n = p.eplb_stats_num_experts;
   ra.invalid_id = p.invalid_expert_id;
-  int slot = prof_begin(h, EP_A2A_KERNEL_ROUTE_PLAN, stream);
+  // On the vector copy path the copy kernel routes each token itself and writes
+  // everything the routing kernel would (one launch per dispatch); the bulk
+  // paths read the plan, so they run after the routing kernel.
+  const bool fused = h->copy_path == 1 && h->route_in_copy != 0;
+  int slot = -1;
   const bool pdl = h->pdl != 0;
-  cudaError_t e = launch_route_plan(ra, active_rank_mask != nullptr, stream, pdl);
-  prof_end(h, slot, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "routing-plan kernel launch");
+  cudaError_t e = cudaSuccess;
+  if (!fused) {
+    slot = prof_begin(h, EP_A2A_KERNEL_ROUTE_PLAN, stream);
+    e = launch_route_plan(ra, active_rank_mask != nullptr, stream, pdl);
+    prof_end(h, slot, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "routing-plan kernel launch");
+  }
 
   // split payloads between the bulk-async copy and the vector copy
   CopyArgs bulk, vec;
@@ -572,7 +586,20 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
   bulk.prefetch = h->copy_prefetch;
   std::memcpy(bulk.n, ra.n, sizeof(bulk.n));
   std::memcpy(bulk.live, ra.live, sizeof(bulk.live));
+  bulk.ep = ep;
   vec = bulk;
+  if (fused) {
+    vec.route = 1;
+    vec.invalid_id = ra.invalid_id;
+    vec.count_acc = ra.count_acc;
+    vec.count_ticket = ra.count_ticket;
+    vec.send_counts = ra.send_counts;
+    vec.off_ids = ra.off_ids;
+    vec.off_valid = ra.off_valid;
+    vec.off_eplb = ra.off_eplb;
+    vec.eplb_stats = ra.eplb_stats;
+    vec.eplb_n = ra.eplb_n;
+  }
   uint32_t stage = 0;
   for (int i = 0; i < num_payloads; ++i) {
     const uint8_t* src = static_cast<const uint8_t*>(payloads[i]);
@@ -631,7 +658,7 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
       if (e != cudaSuccess) return cuda_fail(e, "bulk copy kernel launch");
     }
   }
-  if (vec.np > 0) {
+  if (vec.np > 0 || fused) {
     const int64_t row_vectors = largest_row_vectors(vec);
     const int tpt = h->vec_threads_per_token > 0 ? h->vec_threads_per_token
                                                  : copy_threads_per_token(ntok, row_vectors);
@@ -730,6 +757,58 @@ EP_API ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle h, const float* topk_w
                                          (cudaStream_t)stream_v, h->pdl != 0);
   prof_end(h, slot, (cudaStream_t)stream_v);
   if (e != cudaSuccess) return cuda_fail(e, "expert combine kernel launch");
+  return EP_A2A_OK;
+}
+
+EP_API ep_a2a_status ep_a2a_combine_experts_fp8(ep_a2a_handle h, const float* topk_weights,
+                                                const void* expert_output_per_slot, void* output,
+                                                void* stream_v) {
+  ep_a2a_status st = check_handle(h);
+  if (st != EP_A2A_OK) return st;
+  if (!h->have_plan) return fail(EP_A2A_ERR_NO_PLAN, "combine needs a preceding dispatch");
+  if (!topk_weights || !expert_output_per_slot || !output)
+    return fail(EP_A2A_ERR_INVALID_ARG, "topk_weights / expert output / output is NULL");
+  CombineExpertsArgs a;
+  a.plan_nd = h->ws + h->L.off_plan_nd;
+  a.plan_dst = h->ws + h->L.off_plan_dst;
+  a.recv_ids0 = h->ws + h->L.rank_base + h->L.off_ids;
+  a.rank_stride = h->L.rank_stride;
+  a.w = topk_weights;
+  a.y = static_cast<const uint16_t*>(expert_output_per_slot);
+  a.out = static_cast<uint16_t*>(output);
+  a.ntok = (int64_t)h->p.ep_size * h->last_tpr;
+  a.H = h->combine_hidden;
+  a.k = h->p.top_k;
+  a.E = h->p.num_experts;
+  a.epr = h->p.num_experts / h->p.ep_size;
+  a.plan_stride = h->L.plan_stride;
+  a.ep = h->p.ep_size;
+  a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
+  a.prefetch = 0;
+  // The shared-memory kernel keeps a token's rows z_d (one per destination, at
+  // most min(top_k, ep_size)) as bf16; two CTAs of at most 448 threads share an
+  // SM when the rows take at most half of its shared memory.
+  const int rows = std::min(h->p.top_k, h->p.ep_size);
+  const size_t smem = (size_t)rows * a.H * 2;
+  const bool smem_rows = a.k <= 8 && a.H % 8 == 0 && aligned(expert_output_per_slot, 16) &&
+                         aligned(output, 16) && (int64_t)smem <= h->max_smem_optin - 2048;
+  int threads, cps;
+  if (smem_rows) {
+    const int nvec = a.H / 8;
+    threads = std::min(448, std::max(32, ((nvec + 1) / 2 + 31) / 32 * 32));
+    cps = 2;
+  } else {
+    threads = 256;
+    cps = 8;
+  }
+  if (h->combine_threads > 0) threads = std::min(h->combine_threads, smem_rows ? 448 : 256);
+  if (h->combine_ctas_per_sm > 0) cps = h->combine_ctas_per_sm;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(a.ntok, (int64_t)h->num_sms * cps));
+  const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE_EXPERTS_FP8, (cudaStream_t)stream_v);
+  cudaError_t e = launch_combine_experts_fp8(a, smem_rows, threads, grid, smem_rows ? smem : 0,
+                                             (cudaStream_t)stream_v, h->pdl != 0);
+  prof_end(h, slot, (cudaStream_t)stream_v);
+  if (e != cudaSuccess) return cuda_fail(e, "FP8 expert combine kernel launch");
   return EP_A2A_OK;
 }
 

@@ -98,6 +98,18 @@ struct CopyArgs {
   const int32_t* ids;                    // [ep, tpr, k]
   int E, k, epr, tpr, use_mask;
   int prefetch;                          // vector path: prefetch the next token's rows into L2
+  // vector path with `route` set: the kernel also writes the routing plan,
+  // the per-destination valid bytes and received ids, the send counts and the
+  // EPLB gather (what launch_route_plan writes), so a dispatch is one launch
+  int route;
+  int ep;
+  int32_t invalid_id;
+  int32_t* count_acc;                    // [ep*ep] scratch; zero between calls
+  uint32_t* count_ticket;                // [1] scratch; zero between calls
+  int32_t* send_counts;                  // [ep*ep]
+  int64_t off_ids, off_valid, off_eplb;  // inside a rank region
+  const int32_t* eplb_stats;             // [ep, eplb_n] or nullptr
+  int eplb_n;
   int32_t n[kMaxRanks];                  // local_num_tokens (0 for masked-off ranks)
   uint64_t live[kMaskWords];
 };
@@ -153,6 +165,12 @@ struct CombineExpertsArgs {
 
 cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, bool pipe, int threads,
                                    int grid, cudaStream_t stream, bool pdl);
+// The same with each destination's row quantised to E4M3 with one scale per row
+// before the sum.  smem_rows: the kernel that keeps the token's rows in `smem`
+// bytes of shared memory (top_k <= 8, hidden % 8 == 0, 16-byte aligned rows);
+// else the element kernel (threads <= 256).
+cudaError_t launch_combine_experts_fp8(const CombineExpertsArgs& a, bool smem_rows, int threads,
+                                       int grid, size_t smem, cudaStream_t stream, bool pdl);
 cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n, cudaStream_t stream);
 cudaError_t launch_quantize_e4m3_rows(const uint16_t* in, uint8_t* out, float* scales,
                                       int64_t rows, int hidden, cudaStream_t stream);

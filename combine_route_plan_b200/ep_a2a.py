@@ -36,7 +36,7 @@ OPT_COPY_PATH, OPT_COPY_CTAS_PER_SM, OPT_COPY_STAGES, OPT_COMBINE_THREADS, \
     OPT_BULK_MIN_ROW_BYTES, OPT_COMBINE_CTAS_PER_SM, OPT_COPY_CONSUMER_WARPS, \
     OPT_COPY_INTERLEAVE, OPT_VEC_UNROLL, OPT_VEC_CTAS_PER_SM, OPT_STORE_STREAMING, \
     OPT_PDL, OPT_VEC_THREADS_PER_TOKEN, OPT_COMBINE_PREFETCH, OPT_COPY_PREFETCH, \
-    OPT_COMBINE_PIPELINE, OPT_COPY_VEC_BYTES = range(17)
+    OPT_COMBINE_PIPELINE, OPT_COPY_VEC_BYTES, OPT_ROUTE_IN_COPY = range(18)
 
 
 class EpA2AError(RuntimeError):
@@ -79,11 +79,11 @@ class DispatchResult(ctypes.Structure):
 
 
 KERNEL_NAMES = ["route_plan", "copy_bulk", "copy_vec", "combine", "copy_staged",
-                "combine_experts"]
+                "combine_experts", "combine_experts_fp8"]
 
 
 class KernelTimes(ctypes.Structure):
-    _fields_ = [("launches", ctypes.c_int64 * 6), ("total_ms", ctypes.c_double * 6)]
+    _fields_ = [("launches", ctypes.c_int64 * 7), ("total_ms", ctypes.c_double * 7)]
 
 
 def _load():
@@ -100,6 +100,7 @@ def _load():
         "ep_a2a_combine": (st, [VP, VP, ctypes.c_int, VP, VP]),
         "ep_a2a_quantize_e4m3": (st, [VP, VP, I64, VP]),
         "ep_a2a_combine_experts": (st, [VP, VP, VP, VP, VP]),
+        "ep_a2a_combine_experts_fp8": (st, [VP, VP, VP, VP, VP]),
         "ep_a2a_combine_scaled": (st, [VP, VP, VP, VP, VP]),
         "ep_a2a_quantize_e4m3_rows": (st, [VP, VP, VP, I64, I32, VP]),
         "ep_a2a_allgather": (st, [I32, I32, VP, VP, P(VP), P(I64), I32, P(VP), I64, VP]),
@@ -188,6 +189,15 @@ def ep_a2a_combine_experts(handle: int, topk_weights_ptr: int, expert_out_ptr: i
     _check(lib.ep_a2a_combine_experts(ctypes.c_void_p(handle), ctypes.c_void_p(topk_weights_ptr),
                                       ctypes.c_void_p(expert_out_ptr), ctypes.c_void_p(output_ptr),
                                       ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def ep_a2a_combine_experts_fp8(handle: int, topk_weights_ptr: int, expert_out_ptr: int,
+                               output_ptr: int, stream=None):
+    _check(lib.ep_a2a_combine_experts_fp8(ctypes.c_void_p(handle),
+                                          ctypes.c_void_p(topk_weights_ptr),
+                                          ctypes.c_void_p(expert_out_ptr),
+                                          ctypes.c_void_p(output_ptr),
+                                          ctypes.c_void_p(_stream_ptr(stream))))
 
 
 def ep_a2a_combine_scaled(handle: int, e4m3_ptr: int, scales_ptr: int, output_ptr: int,
@@ -504,6 +514,28 @@ class EpA2A:
         assert output.numel() == self.ep_size * tpr * hidden, output.shape
         self._use_hidden(hidden)
         ep_a2a_combine_experts(self.handle, w.data_ptr(), y.data_ptr(), output.data_ptr(), stream)
+        return output
+
+    def combine_experts_fp8(self, topk_weights: torch.Tensor, expert_output_per_slot: torch.Tensor,
+                            output: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """As :meth:`combine_experts`, with each destination's row quantised to E4M3
+        with one fp32 scale per row before the sum (ep_a2a_combine_experts_fp8)."""
+        tpr = self.last_tokens_per_rank
+        assert tpr is not None, "combine needs a preceding dispatch"
+        w, y = topk_weights, expert_output_per_slot
+        assert w.is_cuda and w.dtype == torch.float32 and w.is_contiguous()
+        assert w.numel() == self.ep_size * tpr * self.top_k, w.shape
+        assert y.is_cuda and y.dtype == torch.bfloat16 and y.is_contiguous()
+        hidden = y.shape[-1]
+        assert y.numel() == self.ep_size * tpr * self.top_k * hidden, y.shape
+        if output is None:
+            output = torch.empty((self.ep_size, tpr, hidden), dtype=torch.bfloat16,
+                                 device=y.device)
+        assert output.is_cuda and output.dtype == torch.bfloat16 and output.is_contiguous()
+        assert output.numel() == self.ep_size * tpr * hidden, output.shape
+        self._use_hidden(hidden)
+        ep_a2a_combine_experts_fp8(self.handle, w.data_ptr(), y.data_ptr(), output.data_ptr(),
+                                   stream)
         return output
 
     def combine_scaled(self, codes: torch.Tensor, row_scales: torch.Tensor,

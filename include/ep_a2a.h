@@ -229,6 +229,26 @@ ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle handle, const float* topk_wei
                                      void* stream);
 
 /*
+ * Low-precision combine of per-expert outputs with the quantisation on the
+ * sending side (flashinfer.moe_ep.NVLinkOneSidedConfig, use_low_precision_combine:
+ * the combine rows travel as FP8; NVLinkTwoSidedAlltoAll.combine(): each rank's
+ * row is its own experts' weighted outputs, summed).  For each existing token
+ * (src, t) of the last dispatch and each destination rank d, in one kernel:
+ *   z_d     = the row of ep_a2a_combine_experts (bf16, one fma per term)
+ *   amax_d  = max |z_d|; scale_d = amax_d / 448, inv_d = 448 / amax_d (fp32,
+ *             rounded to nearest; 1 and 1 for an all-zero row)
+ *   q_d     = E4M3(z_d * inv_d), nearest even, saturating
+ *   out[src][t] = bf16( acc ),  acc = fmaf(decode(q_d), scale_d, acc) over the
+ *             token's destination ranks in ascending order, from +0.0f
+ * which equals ep_a2a_quantize_e4m3_rows applied to the rows z_d followed by
+ * ep_a2a_combine_scaled.  The rows, codes and scales are never written to
+ * memory.  Arguments, layouts and errors as ep_a2a_combine_experts.
+ */
+ep_a2a_status ep_a2a_combine_experts_fp8(ep_a2a_handle handle, const float* topk_weights,
+                                         const void* expert_output_per_slot, void* output,
+                                         void* stream);
+
+/*
  * FP8 helper (flashinfer.moe_ep.NVLinkOneSidedConfig, use_low_precision_combine):
  * e4m3_out[i] = E4M3(bf16_in[i]), round to nearest even, saturating to +-448.
  * Device pointers; n elements.  Not part of a dispatch / combine step.
@@ -352,9 +372,15 @@ typedef enum {
                                      current one; 0 = one vector at a time; -1 (default) =
                                      on for the FP8, scaled FP8 and expert-output
                                      combines, off for BF16 */
-  EP_A2A_OPT_COPY_VEC_BYTES = 16  /* vector copy: widest access per thread, 16 or 32
+  EP_A2A_OPT_COPY_VEC_BYTES = 16, /* vector copy: widest access per thread, 16 or 32
                                      (default) bytes (sm_100 256-bit loads and stores,
                                      for rows and addresses that are 32-byte multiples) */
+  EP_A2A_OPT_ROUTE_IN_COPY = 17   /* vector copy path (COPY_PATH 1): 1 (default) = the
+                                     copy kernel also writes the routing plan, valid
+                                     bytes, received ids, send counts and EPLB gather,
+                                     so a dispatch is one kernel; 0 = a separate
+                                     routing kernel runs first (the bulk paths always
+                                     use it) */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 
@@ -374,7 +400,8 @@ typedef enum {
   EP_A2A_KERNEL_COMBINE = 3,
   EP_A2A_KERNEL_COPY_STAGED = 4,  /* dispatch rows, bulk-async loads + vector stores */
   EP_A2A_KERNEL_COMBINE_EXPERTS = 5, /* combine of per-expert outputs */
-  EP_A2A_KERNEL_COUNT = 6
+  EP_A2A_KERNEL_COMBINE_EXPERTS_FP8 = 6, /* the same, quantised on the sending side */
+  EP_A2A_KERNEL_COUNT = 7
 } ep_a2a_kernel;
 typedef struct {
   int64_t launches[EP_A2A_KERNEL_COUNT];
