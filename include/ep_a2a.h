@@ -509,6 +509,126 @@ ep_a2a_status ep_a2a_route_plan_noalloc(
     uint8_t* plan_dst_ranks, int32_t* send_counts, int32_t* recv_topk_ids, uint8_t* recv_valid,
     int64_t recv_rank_stride_bytes, void* stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * Expert parallelism between real ranks: one process per EP rank.
+ *
+ * The same dispatch and combine as above (flashinfer.moe_ep.NVLinkTwoSidedAlltoAll,
+ * dispatch() / combine(); slots src * tokens_per_rank + t, OneSidedConfig
+ * `lamport`), with each EP rank a process that owns one device "window" for
+ * what its peers send it.  Windows are exported with CUDA IPC handles and
+ * mapped by every peer; senders write rows into peer windows with plain
+ * stores (no rank ever loads from a peer's memory) and then set one flag per
+ * (source, destination) pair with a release store at system scope.
+ * Receivers check those flags with acquire loads in a bounded wait
+ * (NVLinkOneSidedConfig, `timeout_sec`: there a kernel traps on expiry; here
+ * the wait gives up, sets the handle's error word and ep_mp_get_status returns
+ * EP_A2A_ERR_DEVICE_TIMEOUT, leaving the context usable).
+ *
+ * The library does no host communication.  The caller exchanges the IPC
+ * handles (ep_mp_export on every rank, then all-gather) and separates the
+ * phases with a host barrier after synchronising its stream:
+ *   init (every rank) | barrier | dispatch | barrier | dispatch_wait,
+ *   experts, combine_send | barrier | combine_finish
+ * so that no kernel ever waits for a kernel of another process to run: the
+ * flags are already set when a wait starts, unless a rank skipped its send.
+ * Every live rank must make the same calls in the same order with the same
+ * active_rank_mask; a masked-off rank makes none of the step's calls.
+ * ---------------------------------------------------------------------------
+ */
+typedef struct ep_mp_handle_s* ep_mp_handle;   /* opaque, library-owned host object */
+
+typedef struct {
+  uint8_t handle[64];             /* cudaIpcMemHandle_t of the window's allocation */
+  int64_t offset;                 /* window start minus allocation start (bytes) */
+} ep_mp_ipc_handle;
+
+/*
+ * Bytes of one rank's window for `params` (the same params on every rank; the
+ * rules of ep_a2a_params).  It holds the rank's own plan and counters, the
+ * flags, the receive arrays [ep*cap] of every payload, ids and valid bytes,
+ * the EPLB rows [ep, E], and the combine landing rows [ep, cap, hidden] of
+ * 2-byte elements.  Host only.
+ */
+ep_a2a_status ep_mp_window_size(const ep_a2a_params* params, size_t* bytes);
+
+/*
+ * IPC handle of `window` (device memory from cudaMalloc, e.g. a torch
+ * tensor; not from a stream-ordered pool or a virtual-memory mapping) for the
+ * peers' ep_mp_init.  Host only, no device work.
+ */
+ep_a2a_status ep_mp_export(void* window, ep_mp_ipc_handle* out);
+
+/*
+ * Create rank `rank`'s handle: `window` (>= ep_mp_window_size bytes, 256-byte
+ * aligned, caller-owned, kept alive until ep_mp_destroy on every rank) is
+ * this rank's; peers[r] (r != rank) are the other ranks' exported handles
+ * (peers[rank] is ignored).  Opens every peer window, clears this window's
+ * control region and flags, and synchronises `stream`.  Every rank must
+ * finish init before any rank dispatches (a host barrier).
+ */
+ep_a2a_status ep_mp_init(const ep_a2a_params* params, int32_t rank, void* window,
+                         size_t window_bytes, const ep_mp_ipc_handle* peers, void* stream,
+                         ep_mp_handle* out_handle);
+
+/*
+ * Send this rank's tokens (as ep_a2a_dispatch for source rank `rank`):
+ *   token_selected_experts  device int32 [tpr, top_k] (this rank's tokens)
+ *   local_num_tokens        this rank's token count, 0..tpr
+ *   payloads                host array of device pointers, each [tpr, row_bytes_i]
+ *   eplb_local_stats        device int32 [E] or NULL
+ *   active_rank_mask        host uint64 [EP_A2A_RANK_MASK_WORDS] or NULL; this rank
+ *                           must be live in it
+ * Fills `result` with views of this rank's window: recv_payloads[i] [ep*tpr, rb_i],
+ * recv_topk_ids [ep*tpr, k], recv_valid [ep*tpr], eplb_gathered_stats [ep, E]
+ * (what peers sent this rank, complete once every live rank has dispatched and
+ * ep_mp_dispatch_wait has succeeded), send_counts [ep] (tokens this rank sent to
+ * each rank), plan_num_dst [tpr] and plan_dst_ranks [tpr, plan_stride] (this
+ * rank's plan); rank_stride_bytes is 0.
+ */
+ep_a2a_status ep_mp_dispatch(ep_mp_handle handle, const int32_t* token_selected_experts,
+                             int32_t local_num_tokens, int32_t runtime_max_tokens_per_rank,
+                             const void* const* payloads, const int64_t* payload_row_bytes,
+                             int32_t num_payloads, const int32_t* eplb_local_stats,
+                             const uint64_t* active_rank_mask, void* stream,
+                             ep_a2a_dispatch_result* result);
+
+/*
+ * Receive side of the dispatch: wait (bounded by timeout_ns, 1..1e10, of GPU
+ * time) until every live rank's flag of this step has arrived.  On expiry the
+ * handle's error word is set (ep_mp_get_status: EP_A2A_ERR_DEVICE_TIMEOUT).
+ */
+ep_a2a_status ep_mp_dispatch_wait(ep_mp_handle handle, int64_t timeout_ns, void* stream);
+
+/*
+ * Return rows: expert_output device [ep*tpr, hidden] of `dtype` holds this
+ * rank's row for each slot it received (rank src's token t at src*tpr + t: its
+ * own experts' outputs, weighted and summed); each valid slot's row is written
+ * to source src's landing rows, then one flag per live rank.
+ */
+ep_a2a_status ep_mp_combine_send(ep_mp_handle handle, const void* expert_output,
+                                 ep_a2a_combine_dtype dtype, void* stream);
+
+/*
+ * Wait (bounded, as ep_mp_dispatch_wait) for every live rank's combine flag,
+ * then output device bf16 [tpr, hidden] = for each of this rank's tokens, the
+ * fp32 sum in ascending destination-rank order, from +0.0f, of the rows its
+ * destinations returned, rounded once to bf16 (the arithmetic of
+ * ep_a2a_combine).  Rows of tokens t >= local_num_tokens are not written.
+ */
+ep_a2a_status ep_mp_combine_finish(ep_mp_handle handle, void* output, ep_a2a_combine_dtype dtype,
+                                   int64_t timeout_ns, void* stream);
+
+/* Synchronise `stream`, then read and clear the handle's error word. */
+ep_a2a_status ep_mp_get_status(ep_mp_handle handle, void* stream);
+
+/*
+ * Close the peer mappings and free the handle (idempotent, NULL ok).  Every
+ * rank's kernels that write into this rank's window must have completed, and
+ * every rank must destroy before any rank frees its window (host barriers).
+ */
+ep_a2a_status ep_mp_destroy(ep_mp_handle* handle);
+
 #ifdef __cplusplus
 }
 #endif
