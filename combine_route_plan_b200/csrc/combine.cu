@@ -298,6 +298,134 @@ __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
   }
 }
 
+// The combines with their rows staged in shared memory by bulk-async copies
+// (cp.async.bulk, completion counted on an mbarrier): a work item is one
+// chunk of kChunk bytes of a token's row; the producer warp's lane 0 loads the
+// chunk of every destination row of the item into a stage of a ring, and the
+// consumer warps sum it in ascending rank order from shared memory, store the
+// output and release the stage.  The loads cost no registers, so an SM keeps
+// stages x destinations x kChunk bytes in flight whatever the token count.
+// At most 8 destinations per token; rows of 16-byte multiples at 16-byte
+// aligned addresses.
+constexpr int kStageChunk = 4096;                 // bytes of one row per item
+constexpr int kCombineMaxStages = 8;
+
+template <int kMode, int NCW>
+__global__ void __launch_bounds__(32 * (NCW + 1)) combine_staged_kernel(
+    const CombineArgs a, const float* __restrict__ scales, int stages, int stage_rows) {
+  pdl_wait();
+  extern __shared__ __align__(128) uint8_t cs_mem[];
+  __shared__ __align__(8) uint64_t full_bar[kCombineMaxStages];
+  __shared__ __align__(8) uint64_t empty_bar[kCombineMaxStages];
+  __shared__ int64_t st_item[kCombineMaxStages];
+  __shared__ int st_nd[kCombineMaxStages];
+  __shared__ uint64_t st_w0[kCombineMaxStages];
+  constexpr int kElemBytes = kMode == kCombineBf16 ? 2 : 1;
+  constexpr int kElems = 16 / kElemBytes;          // elements per 16-byte vector
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t row_bytes = (int64_t)a.H * kElemBytes;
+  const int chunks = (int)((row_bytes + kStageChunk - 1) / kStageChunk);
+  const int64_t items = a.ntok * chunks;
+  const int64_t rank_stride = a.ntok * row_bytes;
+  const uint32_t stage_bytes = (uint32_t)stage_rows * kStageChunk;
+  const uint32_t smem0 = smem_addr(cs_mem);
+  const uint32_t full0 = smem_addr(full_bar);
+  const uint32_t empty0 = smem_addr(empty_bar);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, NCW);
+    }
+    mbar_init_fence();
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // producer: items blockIdx.x, blockIdx.x + gridDim.x, ...; after the last
+    // one a sentinel (item -1) tells the consumers to stop
+    if (lane != 0) return;
+    int64_t n = 0;
+    for (int64_t it = blockIdx.x;; it += gridDim.x) {
+      int nd = 0;
+      uint64_t w0 = 0;
+      if (it < items) {
+        const int64_t tok = it / chunks;
+        nd = a.plan_nd[tok];
+        if (nd == kNoToken) continue;
+        w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+        if (!plan_row_ok(nd, w0, 0, 0, 0, a.ep, 8, a.err)) continue;
+      }
+      const int s = (int)(n % stages);
+      const uint32_t use = (uint32_t)(n / stages);
+      if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1u, kWaitLimitNs)) {
+        atomicOr(a.err, kErrWaitTimeout);
+        return;
+      }
+      ++n;
+      st_item[s] = it < items ? it : -1;
+      st_nd[s] = nd;
+      st_w0[s] = w0;
+      if (it >= items || nd == 0) {
+        mbar_arrive(full0 + 8 * s);
+        if (it >= items) return;
+        continue;
+      }
+      const int64_t tok = it / chunks;
+      const int c = (int)(it - tok * chunks);
+      const int64_t off = (int64_t)c * kStageChunk;
+      const int64_t left = row_bytes - off;
+      const uint32_t cb = (uint32_t)(left < kStageChunk ? left : kStageChunk);
+      mbar_arrive_expect_tx(full0 + 8 * s, cb * (uint32_t)nd);
+      const uint8_t* src = a.x + tok * row_bytes + off;
+      for (int q = 0; q < nd; ++q) {
+        const int d = (int)((w0 >> (8 * q)) & 0xFFu);
+        bulk_load(smem0 + (uint32_t)s * stage_bytes + (uint32_t)q * kStageChunk,
+                  src + (int64_t)d * rank_stride, cb, full0 + 8 * s);
+      }
+    }
+  }
+
+  // consumers: thread c sums the 16-byte column vectors c, c + 32*NCW, ...
+  constexpr int kCons = 32 * NCW;
+  const int ct = threadIdx.x - 32;
+  for (int64_t n = 0;; ++n) {
+    const int s = (int)(n % stages);
+    if (!mbar_wait_bounded(full0 + 8 * s, (uint32_t)((n / stages) & 1), kWaitLimitNs)) {
+      atomicOr(a.err, kErrWaitTimeout);
+      break;
+    }
+    const int64_t it = st_item[s];
+    if (it < 0) break;
+    const int nd = st_nd[s];
+    const uint64_t w0 = st_w0[s];
+    const int64_t tok = it / chunks;
+    const int c = (int)(it - tok * chunks);
+    const int64_t off = (int64_t)c * kStageChunk;
+    const int64_t left = row_bytes - off;
+    const int nvec = (int)((left < kStageChunk ? left : kStageChunk) / 16);
+    float sc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      sc[q] = 1.0f;
+      if (kMode == kCombineFp8Scaled && q < nd)
+        sc[q] = scales[(int64_t)((w0 >> (8 * q)) & 0xFFu) * a.ntok + tok];
+    }
+    const uint8_t* stage = cs_mem + (size_t)s * stage_bytes;
+    uint16_t* o = a.out + tok * (int64_t)a.H + off / kElemBytes;
+    for (int v = ct; v < nvec; v += kCons) {
+      uint4 r[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q < nd)
+          r[q] = *reinterpret_cast<const uint4*>(stage + q * kStageChunk + v * 16);
+      reduce_store<kMode>(r, sc, nd, o + (int64_t)v * kElems, false);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * s);      // this warp is done with the stage
+  }
+}
+
 // Any hidden size and alignment: one element per thread step.
 template <bool kFp8>
 __global__ void __launch_bounds__(512) combine_scalar_kernel(const CombineArgs a) {
@@ -996,6 +1124,42 @@ cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, bool pipe, 
   }
   if (fp8) return launch_kernel(combine_scalar_kernel<true>, g, b, 0, stream, pdl, a);
   return launch_kernel(combine_scalar_kernel<false>, g, b, 0, stream, pdl, a);
+}
+
+cudaError_t launch_combine_staged(const CombineArgs& a, int mode, const float* scales,
+                                  int grid, int ctas_per_sm, int max_smem, cudaStream_t stream,
+                                  bool pdl) {
+  constexpr int NCW = 8;
+  const int rows = 8;
+  const int stage_bytes = rows * kStageChunk;
+  // shared memory per CTA when `ctas_per_sm` share an SM (1 KB per CTA is
+  // reserved; 1 KB covers the static arrays)
+  const int per_cta = std::min(max_smem, 228 * 1024 / std::max(1, ctas_per_sm) - 1024) - 1024;
+  const int stages = std::min(kCombineMaxStages, per_cta / stage_bytes);
+  if (stages < 2) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)stages * stage_bytes;
+  const dim3 g(grid), b(32 * (NCW + 1));
+  cudaError_t e;
+  switch (mode) {
+    case kCombineBf16:
+      e = cudaFuncSetAttribute(combine_staged_kernel<kCombineBf16, NCW>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      return launch_kernel(combine_staged_kernel<kCombineBf16, NCW>, g, b, smem, stream, pdl, a,
+                           scales, stages, rows);
+    case kCombineFp8:
+      e = cudaFuncSetAttribute(combine_staged_kernel<kCombineFp8, NCW>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      return launch_kernel(combine_staged_kernel<kCombineFp8, NCW>, g, b, smem, stream, pdl, a,
+                           scales, stages, rows);
+    default:
+      e = cudaFuncSetAttribute(combine_staged_kernel<kCombineFp8Scaled, NCW>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      return launch_kernel(combine_staged_kernel<kCombineFp8Scaled, NCW>, g, b, smem, stream, pdl,
+                           a, scales, stages, rows);
+  }
 }
 
 cudaError_t launch_combine_scaled(const CombineArgs& a, const float* scales, bool vec, bool pipe,

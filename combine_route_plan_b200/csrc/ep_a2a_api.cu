@@ -213,7 +213,9 @@ enum CombineKind { kKindBf16, kKindFp8, kKindExperts };
 
 struct CombineLaunch {
   bool pipe;
+  bool staged;               // rows staged in shared memory by bulk-async copies
   int threads, grid, prefetch;
+  int staged_ctas_per_sm;
 };
 
 // Launch shape of a combine: the options where set, else the defaults measured
@@ -235,7 +237,11 @@ CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
   const bool fits = std::min(h->p.top_k, h->p.ep_size) <= 8;
   const bool big = ntok >= 16384;
   CombineLaunch c;
-  c.pipe = fits && (h->combine_pipeline < 0 ? kind != kKindBf16 : h->combine_pipeline > 0);
+  c.pipe = fits && (h->combine_pipeline < 0 ? kind != kKindBf16
+                                             : h->combine_pipeline == 1 ||
+                                                   (h->combine_pipeline == 2 && kind == kKindExperts));
+  c.staged = fits && kind != kKindExperts && h->combine_pipeline == 2;
+  c.staged_ctas_per_sm = h->combine_ctas_per_sm > 0 ? std::min(h->combine_ctas_per_sm, 4) : 2;
   const bool mid = !big && ntok >= 8192;
   int threads = 64, cps = 128, prefetch = 0;
   if (kind == kKindFp8) {
@@ -440,8 +446,9 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       h->copy_vec_bytes = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_COMBINE_PIPELINE:
-      if (value < -1 || value > 1)
-        return fail(EP_A2A_ERR_INVALID_ARG, "combine pipeline must be -1 (automatic), 0 or 1");
+      if (value < -1 || value > 2)
+        return fail(EP_A2A_ERR_INVALID_ARG,
+                    "combine pipeline must be -1 (automatic), 0, 1 or 2 (staged)");
       h->combine_pipeline = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_COPY_PREFETCH:
@@ -717,8 +724,14 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   const int elems = fp8 ? 16 : 8;
   const bool vec = a.H % elems == 0 && aligned(expert_output, 16) && aligned(output, 16);
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);
-  cudaError_t e = launch_combine(a, fp8, vec, c.pipe, c.threads, c.grid, (cudaStream_t)stream_v,
-                                 h->pdl != 0);
+  cudaError_t e;
+  if (vec && c.staged)
+    e = launch_combine_staged(a, fp8 ? 1 : 0, nullptr, h->num_sms * c.staged_ctas_per_sm,
+                              c.staged_ctas_per_sm, h->max_smem_optin, (cudaStream_t)stream_v,
+                              h->pdl != 0);
+  else
+    e = launch_combine(a, fp8, vec, c.pipe, c.threads, c.grid, (cudaStream_t)stream_v,
+                       h->pdl != 0);
   prof_end(h, slot, (cudaStream_t)stream_v);
   if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
   return EP_A2A_OK;
@@ -835,8 +848,14 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
   a.out32 = aligned(output, 32) ? 1 : 0;
   const bool vec = a.H % 16 == 0 && aligned(expert_output_e4m3, 16) && aligned(output, 16);
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);
-  cudaError_t e = launch_combine_scaled(a, row_scales, vec, c.pipe, c.threads, c.grid,
-                                        (cudaStream_t)stream_v, h->pdl != 0);
+  cudaError_t e;
+  if (vec && c.staged)
+    e = launch_combine_staged(a, 2, row_scales, h->num_sms * c.staged_ctas_per_sm,
+                              c.staged_ctas_per_sm, h->max_smem_optin, (cudaStream_t)stream_v,
+                              h->pdl != 0);
+  else
+    e = launch_combine_scaled(a, row_scales, vec, c.pipe, c.threads, c.grid,
+                              (cudaStream_t)stream_v, h->pdl != 0);
   prof_end(h, slot, (cudaStream_t)stream_v);
   if (e != cudaSuccess) return cuda_fail(e, "scaled combine kernel launch");
   return EP_A2A_OK;

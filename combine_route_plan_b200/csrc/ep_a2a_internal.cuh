@@ -174,6 +174,12 @@ cudaError_t launch_combine_experts_fp8(const CombineExpertsArgs& a, bool smem_ro
 cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n, cudaStream_t stream);
 cudaError_t launch_quantize_e4m3_rows(const uint16_t* in, uint8_t* out, float* scales,
                                       int64_t rows, int hidden, cudaStream_t stream);
+// The BF16 (mode 0), FP8 (1) or scaled FP8 (2, scales [ep, ep*tpr]) combine with
+// the rows staged in shared memory by bulk-async copies; at most 8 destinations
+// per token, rows of 16-byte multiples at 16-byte aligned addresses.
+cudaError_t launch_combine_staged(const CombineArgs& a, int mode, const float* scales,
+                                  int grid, int ctas_per_sm, int max_smem, cudaStream_t stream,
+                                  bool pdl);
 // FP8 combine with one fp32 scale per row (scales [ep, ep*tpr]).
 cudaError_t launch_combine_scaled(const CombineArgs& a, const float* scales, bool vec, bool pipe,
                                   int threads, int grid, cudaStream_t stream, bool pdl);

@@ -369,9 +369,12 @@ typedef enum {
                                      with at most 8 destinations per token (top_k or
                                      ep_size <= 8): 1 = each thread keeps the loads of its
                                      next column vector in flight while it adds the
-                                     current one; 0 = one vector at a time; -1 (default) =
-                                     on for the FP8, scaled FP8 and expert-output
-                                     combines, off for BF16 */
+                                     current one; 2 = the rows are staged in shared
+                                     memory by bulk-async copies (4 KB chunks of every
+                                     destination row per stage) and summed from there
+                                     (not the expert-output combine); 0 = one vector at
+                                     a time; -1 (default) = 1 for the FP8, scaled FP8
+                                     and expert-output combines, 0 for BF16 */
   EP_A2A_OPT_COPY_VEC_BYTES = 16, /* vector copy: widest access per thread, 16 or 32
                                      (default) bytes (sm_100 256-bit loads and stores,
                                      for rows and addresses that are 32-byte multiples) */

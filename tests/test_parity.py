@@ -359,6 +359,54 @@ def test_pipelined_combines_match_the_oracle(case, prefetch, threads):
                                                   U.to_np(y), H, out_init=init), "experts")
 
 
+@pytest.mark.parametrize("case,ctas", [
+    (("c2_ep8_decode", None), 0),
+    (("c2_ep8_decode", None), 3),
+    (("c5_ep64_wide_masked", None), 0),
+    (("c1_ep4_tiny", None), 1),
+    (("c3_ep16_zipf_nvfp4", None), 0),
+    (("mask", [0b10100101, 0, 0, 0]), 0),   # tokens whose owners are all masked: +0
+    (("mask", [0b10100101, 0, 0, 0]), 1),
+    (("short", None), 0),                   # hidden 40: rows shorter than a chunk
+    (("short", None), 3),
+])
+def test_staged_combines_match_the_oracle(case, ctas):
+    """BF16, FP8 and scaled-FP8 combines with the rows staged in shared memory by
+    bulk-async copies (combine pipeline option 2), at 1 to 3 CTAs per SM."""
+    from combine_route_plan_b200 import ep_a2a
+    name, mask = case
+    if name in W.BY_NAME:
+        w = W.BY_NAME[name]
+        x = _inputs(w.name)
+    elif name == "mask":
+        w, x = _custom(8, 64, 6, 40, 64, [32], n=[40, 1, 0, 39, 17, 40, 2, 33], mask=mask, seed=8)
+    else:
+        w, x = _custom(4, 16, 4, 30, 40, [32], seed=19)
+    opts = {ep_a2a.OPT_COMBINE_PIPELINE: 2, ep_a2a.OPT_COMBINE_CTAS_PER_SM: ctas}
+    run = U.Run(w, W.Inputs(w, x.token_selected_experts, x.local_num_tokens, x.payloads,
+                            x.eplb_local_stats, x.active_rank_mask, None), options=opts)
+    plan = U.oracle_plan(w, x)
+    xo = x.expert_output
+    H = w.hidden
+
+    def fresh():
+        return torch.full((w.ep_size, w.tokens_per_rank, H), U.OUT_CANARY, dtype=torch.int16,
+                          device="cuda").view(torch.bfloat16)
+    out, out8, outs = fresh(), fresh(), fresh()
+    run.comm.combine(xo.cuda(), out)
+    run.comm.combine(ep_a2a.quantize_e4m3(xo.cuda()), out8)
+    codes, scales = ep_a2a.quantize_e4m3_rows(xo.cuda())
+    run.comm.combine_scaled(codes, scales, outs)
+    torch.cuda.synchronize()
+    assert run.comm.get_status() == ep_a2a.OK
+    init = U.oracle_out_init(w)
+    xq = U.oracle_quantize_big(U.to_np(xo), U.oracle_e4m3_table())
+    oc, osc = U.oracle.quantize_e4m3_rows(U.to_np(xo), H)
+    U.assert_equal(out, U.oracle.combine(plan, U.to_np(xo), H, out_init=init), "bf16")
+    U.assert_equal(out8, U.oracle.combine(plan, xq, H, input_is_e4m3=True, out_init=init), "fp8")
+    U.assert_equal(outs, U.oracle.combine_scaled(plan, oc, osc, H, out_init=init), "scaled")
+
+
 def test_fp8_quantize_all_bf16_patterns():
     from combine_route_plan_b200 import ep_a2a
     table = U.oracle_e4m3_table()
