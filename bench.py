@@ -260,6 +260,15 @@ def algorithmic_bytes(w, n_tok: int, sum_d: int, live: int, fp8: bool,
     return Bytes(copy, combine, route, copy + combine + route)
 
 
+def parse_options(items):
+    """[("COMBINE_PIPELINE", 2), ...] from NAME=VALUE strings."""
+    out = []
+    for it in items or []:
+        name, _, value = it.partition("=")
+        out.append((name.strip().upper(), int(value)))
+    return out
+
+
 def l2_note(flushed: bool, step_bytes: int, l2_bytes: int) -> str:
     """How the timed steps meet the L2 rule, for the JSON line's config."""
     if flushed:
@@ -563,6 +572,8 @@ def run_ours(args):
                         enable_rank_mask=mask is not None)
     if args.no_pdl:
         comm.set_option(ep_a2a.OPT_PDL, 0)
+    for name, value in parse_options(args.opt):
+        comm.set_option(getattr(ep_a2a, "OPT_" + name), value)
     out = torch.empty((w.ep_size, w.tokens_per_rank, w.hidden), dtype=torch.bfloat16, device=device)
     tpr = w.tokens_per_rank
     fp8 = args.combine == "fp8"
@@ -754,6 +765,7 @@ def run_ours(args):
                 "parallelism": f"{ws} independent replicas" if ws > 1 else "1 GPU, virtual ranks",
                 "variant": ("dense: all-gather dispatch + reduce-scatter combine (vllm AgRs)"
                             if dense else "rank-major dispatch + combine"),
+                "options": dict(parse_options(args.opt)) or "library defaults",
             },
             "hbm": {"step_algorithmic_bytes": by.step, "achieved_gbs": step_gbs,
                     "peak_gbs": peak, "peak_kind": peak_kind, "frac": step_gbs / peak},
@@ -1033,6 +1045,9 @@ def main(argv=None):
                          "step, for comparison")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch")
+    ap.add_argument("--opt", action="append", default=[],
+                    help="library tuning option NAME=VALUE (ep_a2a_option without the "
+                         "EP_A2A_OPT_ prefix, e.g. COMBINE_PIPELINE=2); repeatable")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         raise SystemExit("--warmup must be >= 3")
