@@ -52,6 +52,29 @@ def _global_inputs(ep, E, k, tpr, H, rows, n, seed):
     return ids, payloads, stats, xo
 
 
+def _agree(ok: bool) -> bool:
+    """Whether every rank's checks passed (gloo all-reduce).  Ranks agree before
+    any rank starts the next phase, so that no rank leaves while a peer could
+    still be writing into its window."""
+    import torch.distributed as dist
+    t = torch.tensor([0 if ok else 1], dtype=torch.int64)
+    dist.all_reduce(t)
+    return int(t.item()) == 0
+
+
+def _checked(comm, fn):
+    """Run the checks `fn`; if any rank's fail, every rank tears down cleanly
+    (no kernel in flight, peer mappings closed) and this rank re-raises."""
+    err = None
+    try:
+        fn()
+    except Exception:
+        err = traceback.format_exc()
+    if not _agree(err is None):
+        comm.destroy()
+        raise AssertionError(err or "another rank's checks failed")
+
+
 def _rank_main(rank, world, case):
     import oracle
     from combine_route_plan_b200 import ep_a2a, ep_mp
@@ -73,26 +96,55 @@ def _rank_main(rank, world, case):
         d = comm.dispatch(ids[rank].to(dev), int(n[rank]), [p[rank].to(dev) for p in payloads],
                           tpr, stats[rank].to(dev), mask, timeout_ns=50_000_000,
                           send=rank != 1, wait=rank == 0)
-        if rank == 0:
+        def check_timeout():
+            if rank != 0:
+                return
             st = comm.get_status()
             assert st == ep_a2a.ERR_DEVICE_TIMEOUT, st
             assert comm.get_status() == ep_a2a.OK           # read and cleared
             y = torch.arange(1024, device=dev, dtype=torch.float32).sum()   # context usable
             assert float(y.item()) == 1023 * 1024 / 2
-        comm.barrier()
+        _checked(comm, check_timeout)
         comm.destroy()
         return "timeout seen" if rank == 0 else "skipped"
 
     d = comm.dispatch(ids[rank].to(dev), int(n[rank]), [p[rank].to(dev) for p in payloads], tpr,
                       stats[rank].to(dev), mask)
-    st = comm.get_status()
-    assert st == ep_a2a.OK, (st, ep_a2a.lib.ep_a2a_last_error())
-
     # the oracle of the whole step, this rank's slice
     plan = oracle.route(ep, E, k, tpr, ids.numpy(), n, mask,
                         recv_valid_init=np.full((ep, ep * tpr), CANARY, np.uint8),
                         recv_topk_ids_init=np.full((ep, ep * tpr, 4 * k), CANARY, np.uint8)
                         .view(np.int32))
+    _checked(comm, lambda: _check_dispatch(comm, d, plan, live, rank, ep, tpr, k, rows, payloads,
+                                           stats, mask))
+
+    # combine: this rank returns its rows for the slots it received
+    fp8 = case == "fp8"
+    x = xo[rank].to(dev)
+    if fp8:
+        x = ep_a2a.quantize_e4m3(x)
+    out = torch.full((tpr, H), OUT_CANARY, dtype=torch.int16, device=dev).view(torch.bfloat16)
+    out = comm.combine(x, out, mask)
+
+    def check_combine():
+        if not live:
+            return
+        assert comm.get_status() == ep_a2a.OK
+        bits = xo.view(torch.int16).numpy().view(np.uint16)
+        if fp8:
+            bits = oracle.quantize_e4m3(bits)
+        want = oracle.combine(plan, bits, H, input_is_e4m3=fp8)
+        assert np.array_equal(out.cpu().view(torch.int16).numpy().view(np.uint16), want[rank])
+    _checked(comm, check_combine)
+    comm.destroy()
+    return "ok"
+
+
+def _check_dispatch(comm, d, plan, live, rank, ep, tpr, k, rows, payloads, stats, mask):
+    import oracle
+    from combine_route_plan_b200 import ep_a2a
+    st = comm.get_status()
+    assert st == ep_a2a.OK, (st, ep_a2a.lib.ep_a2a_last_error())
     if live:
         assert np.array_equal(d.recv_valid.cpu().numpy(), plan.recv_valid[rank])
         assert np.array_equal(d.recv_topk_ids.cpu().numpy(), plan.recv_topk_ids[rank])
@@ -107,23 +159,6 @@ def _rank_main(rank, world, case):
             assert np.array_equal(d.recv_payloads[i].cpu().numpy(), want.reshape(ep * tpr, -1)), i
         want_eplb = oracle.eplb_gather(ep, stats.numpy(), mask)
         assert np.array_equal(d.eplb_gathered_stats.cpu().numpy(), want_eplb[rank])
-
-    # combine: this rank returns its rows for the slots it received
-    fp8 = case == "fp8"
-    x = xo[rank].to(dev)
-    if fp8:
-        x = ep_a2a.quantize_e4m3(x)
-    out = torch.full((tpr, H), OUT_CANARY, dtype=torch.int16, device=dev).view(torch.bfloat16)
-    out = comm.combine(x, out, mask)
-    if live:
-        assert comm.get_status() == ep_a2a.OK
-        bits = xo.view(torch.int16).numpy().view(np.uint16)
-        if fp8:
-            bits = oracle.quantize_e4m3(bits)
-        want = oracle.combine(plan, bits, H, input_is_e4m3=fp8)
-        assert np.array_equal(out.cpu().view(torch.int16).numpy().view(np.uint16), want[rank])
-    comm.destroy()
-    return "ok"
 
 
 def _worker(rank, world, port, case, q):
