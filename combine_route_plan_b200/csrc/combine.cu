@@ -872,6 +872,136 @@ __global__ void __launch_bounds__(256) combine_experts_fp8_any_kernel(const Comb
   }
 }
 
+// combine_experts_pipe_kernel with the slot rows staged in shared memory by
+// bulk-async copies, as combine_staged_kernel does for the per-rank rows: a
+// work item is one kStageChunk-byte chunk of a token's slot rows; the
+// producer lane finds the slots' owners and weights, loads the chunk of every
+// participating slot row into a stage, and the consumer warps form each
+// destination's z_d and the ordered sum from shared memory.  top_k <= 8,
+// hidden a multiple of 8, 16-byte aligned rows.
+template <int NCW>
+__global__ void __launch_bounds__(32 * (NCW + 1)) combine_experts_staged_kernel(
+    const CombineExpertsArgs a, int stages) {
+  pdl_wait();
+  extern __shared__ __align__(128) uint8_t es_mem[];
+  __shared__ __align__(8) uint64_t full_bar[kCombineMaxStages];
+  __shared__ __align__(8) uint64_t empty_bar[kCombineMaxStages];
+  __shared__ int64_t st_item[kCombineMaxStages];
+  __shared__ int st_nd[kCombineMaxStages];
+  __shared__ uint64_t st_w0[kCombineMaxStages];
+  __shared__ int st_own[kCombineMaxStages][8];
+  __shared__ float st_wt[kCombineMaxStages][8];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t row_bytes = (int64_t)a.H * 2;
+  const int chunks = (int)((row_bytes + kStageChunk - 1) / kStageChunk);
+  const int64_t items = a.ntok * chunks;
+  const uint32_t stage_bytes = 8u * kStageChunk;
+  const uint32_t smem0 = smem_addr(es_mem);
+  const uint32_t full0 = smem_addr(full_bar);
+  const uint32_t empty0 = smem_addr(empty_bar);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, NCW);
+    }
+    mbar_init_fence();
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    if (lane != 0) return;
+    int64_t n = 0;
+    for (int64_t it = blockIdx.x;; it += gridDim.x) {
+      int nd = 0;
+      uint64_t w0 = 0;
+      int own[8];
+      float wt[8];
+      const int64_t tok = it < items ? it / chunks : 0;
+      if (it < items) {
+        nd = a.plan_nd[tok];
+        if (nd == kNoToken) continue;
+        w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+        if (!plan_row_ok(nd, w0, 0, 0, 0, a.ep, 8, a.err)) continue;
+        if (nd > 0) slot_owners<8>(a, tok, nd, w0, 0, 0, 0, own, wt);
+      }
+      const int s = (int)(n % stages);
+      const uint32_t use = (uint32_t)(n / stages);
+      if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1u, kWaitLimitNs)) {
+        atomicOr(a.err, kErrWaitTimeout);
+        return;
+      }
+      ++n;
+      st_item[s] = it < items ? it : -1;
+      st_nd[s] = nd;
+      st_w0[s] = w0;
+      if (it >= items || nd == 0) {
+        mbar_arrive(full0 + 8 * s);
+        if (it >= items) return;
+        continue;
+      }
+      const int c = (int)(it - tok * chunks);
+      const int64_t off = (int64_t)c * kStageChunk;
+      const int64_t left = row_bytes - off;
+      const uint32_t cb = (uint32_t)(left < kStageChunk ? left : kStageChunk);
+      uint32_t tx = 0;
+      for (int j = 0; j < 8; ++j) {
+        st_own[s][j] = own[j];
+        st_wt[s][j] = wt[j];
+        if (own[j] >= 0) tx += cb;
+      }
+      mbar_arrive_expect_tx(full0 + 8 * s, tx);
+      const uint8_t* yt = reinterpret_cast<const uint8_t*>(a.y) + tok * a.k * row_bytes + off;
+      for (int j = 0; j < 8; ++j)
+        if (own[j] >= 0)
+          bulk_load(smem0 + (uint32_t)s * stage_bytes + (uint32_t)j * kStageChunk,
+                    yt + (int64_t)j * row_bytes, cb, full0 + 8 * s);
+    }
+  }
+
+  constexpr int kCons = 32 * NCW;
+  const int ct = threadIdx.x - 32;
+  for (int64_t n = 0;; ++n) {
+    const int s = (int)(n % stages);
+    if (!mbar_wait_bounded(full0 + 8 * s, (uint32_t)((n / stages) & 1), kWaitLimitNs)) {
+      atomicOr(a.err, kErrWaitTimeout);
+      break;
+    }
+    const int64_t it = st_item[s];
+    if (it < 0) break;
+    const int nd = st_nd[s];
+    const uint64_t w0 = st_w0[s];
+    const int64_t tok = it / chunks;
+    const int c = (int)(it - tok * chunks);
+    const int64_t off = (int64_t)c * kStageChunk;
+    const int64_t left = row_bytes - off;
+    const int nvec = (int)((left < kStageChunk ? left : kStageChunk) / 16);
+    uint16_t* o = a.out + tok * (int64_t)a.H + off / 2;
+    if (nd == 0) {
+      for (int v = ct; v < nvec; v += kCons)
+        reinterpret_cast<uint4*>(o)[v] = make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      int own[8];
+      float wt[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        own[j] = st_own[s][j];
+        wt[j] = st_wt[s][j];
+      }
+      const uint8_t* stage = es_mem + (size_t)s * stage_bytes;
+      for (int v = ct; v < nvec; v += kCons) {
+        uint4 r[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (own[j] >= 0) r[j] = *reinterpret_cast<const uint4*>(stage + j * kStageChunk + v * 16);
+        expert_rows_reduce_store(r, own, wt, nd, w0, o + (int64_t)v * 8);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * s);
+  }
+}
+
 // Any top_k (<= 32) and hidden size: one element per thread step.
 __global__ void __launch_bounds__(512) combine_experts_any_kernel(const CombineExpertsArgs a) {
   pdl_wait();
@@ -1191,6 +1321,21 @@ cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, bool p
   if (vec && pipe) return launch_kernel(combine_experts_pipe_kernel, g, b, 0, stream, pdl, a);
   if (vec) return launch_kernel(combine_experts_vec_kernel, g, b, 0, stream, pdl, a);
   return launch_kernel(combine_experts_any_kernel, g, b, 0, stream, pdl, a);
+}
+
+cudaError_t launch_combine_experts_staged(const CombineExpertsArgs& a, int grid, int ctas_per_sm,
+                                          int max_smem, cudaStream_t stream, bool pdl) {
+  constexpr int NCW = 8;
+  const int stage_bytes = 8 * kStageChunk;
+  const int per_cta = std::min(max_smem, 228 * 1024 / std::max(1, ctas_per_sm) - 1024) - 1024;
+  const int stages = std::min(kCombineMaxStages, per_cta / stage_bytes);
+  if (stages < 2) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)stages * stage_bytes;
+  cudaError_t e = cudaFuncSetAttribute(combine_experts_staged_kernel<NCW>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(combine_experts_staged_kernel<NCW>, dim3(grid), dim3(32 * (NCW + 1)), smem,
+                       stream, pdl, a, stages);
 }
 
 cudaError_t launch_combine_experts_fp8(const CombineExpertsArgs& a, bool smem_rows, int threads,

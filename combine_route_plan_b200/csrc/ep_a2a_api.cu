@@ -237,10 +237,8 @@ CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
   const bool fits = std::min(h->p.top_k, h->p.ep_size) <= 8;
   const bool big = ntok >= 16384;
   CombineLaunch c;
-  c.pipe = fits && (h->combine_pipeline < 0 ? kind != kKindBf16
-                                             : h->combine_pipeline == 1 ||
-                                                   (h->combine_pipeline == 2 && kind == kKindExperts));
-  c.staged = fits && kind != kKindExperts && h->combine_pipeline == 2;
+  c.pipe = fits && (h->combine_pipeline < 0 ? kind != kKindBf16 : h->combine_pipeline == 1);
+  c.staged = fits && h->combine_pipeline == 2;
   c.staged_ctas_per_sm = h->combine_ctas_per_sm > 0 ? std::min(h->combine_ctas_per_sm, 4) : 2;
   const bool mid = !big && ntok >= 8192;
   int threads = 64, cps = 128, prefetch = 0;
@@ -766,8 +764,13 @@ EP_API ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle h, const float* topk_w
   const bool vec = a.k <= 8 && a.H % 8 == 0 && aligned(expert_output_per_slot, 16) &&
                    aligned(output, 16);
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE_EXPERTS, (cudaStream_t)stream_v);
-  cudaError_t e = launch_combine_experts(a, vec, c.pipe, c.threads, c.grid,
-                                         (cudaStream_t)stream_v, h->pdl != 0);
+  cudaError_t e;
+  if (vec && c.staged)
+    e = launch_combine_experts_staged(a, h->num_sms * c.staged_ctas_per_sm, c.staged_ctas_per_sm,
+                                      h->max_smem_optin, (cudaStream_t)stream_v, h->pdl != 0);
+  else
+    e = launch_combine_experts(a, vec, c.pipe, c.threads, c.grid, (cudaStream_t)stream_v,
+                               h->pdl != 0);
   prof_end(h, slot, (cudaStream_t)stream_v);
   if (e != cudaSuccess) return cuda_fail(e, "expert combine kernel launch");
   return EP_A2A_OK;

@@ -165,6 +165,10 @@ struct CombineExpertsArgs {
 
 cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, bool pipe, int threads,
                                    int grid, cudaStream_t stream, bool pdl);
+// The same with the slot rows staged in shared memory by bulk-async copies
+// (top_k <= 8, hidden % 8 == 0, 16-byte aligned rows).
+cudaError_t launch_combine_experts_staged(const CombineExpertsArgs& a, int grid, int ctas_per_sm,
+                                          int max_smem, cudaStream_t stream, bool pdl);
 // The same with each destination's row quantised to E4M3 with one scale per row
 // before the sum.  smem_rows: the kernel that keeps the token's rows in `smem`
 // bytes of shared memory (top_k <= 8, hidden % 8 == 0, 16-byte aligned rows);

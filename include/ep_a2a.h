@@ -371,8 +371,9 @@ typedef enum {
                                      next column vector in flight while it adds the
                                      current one; 2 = the rows are staged in shared
                                      memory by bulk-async copies (4 KB chunks of every
-                                     destination row per stage) and summed from there
-                                     (not the expert-output combine); 0 = one vector at
+                                     destination row, or slot row for the expert-output
+                                     combine, per stage) and summed from there; 0 = one
+                                     vector at
                                      a time; -1 (default) = 1 for the FP8, scaled FP8
                                      and expert-output combines, 0 for BF16 */
   EP_A2A_OPT_COPY_VEC_BYTES = 16, /* vector copy: widest access per thread, 16 or 32

@@ -391,8 +391,9 @@ def test_pipelined_combines_match_the_oracle(case, prefetch, threads):
     (("short", None), 3),
 ])
 def test_staged_combines_match_the_oracle(case, ctas):
-    """BF16, FP8 and scaled-FP8 combines with the rows staged in shared memory by
-    bulk-async copies (combine pipeline option 2), at 1 to 3 CTAs per SM."""
+    """BF16, FP8, scaled-FP8 and expert-output combines with the rows staged in
+    shared memory by bulk-async copies (combine pipeline option 2), at 1 to 3
+    CTAs per SM."""
     from combine_route_plan_b200 import ep_a2a
     name, mask = case
     if name in W.BY_NAME:
@@ -425,6 +426,16 @@ def test_staged_combines_match_the_oracle(case, ctas):
     U.assert_equal(out, U.oracle.combine(plan, U.to_np(xo), H, out_init=init), "bf16")
     U.assert_equal(out8, U.oracle.combine(plan, xq, H, input_is_e4m3=True, out_init=init), "fp8")
     U.assert_equal(outs, U.oracle.combine_scaled(plan, oc, osc, H, out_init=init), "scaled")
+    g = torch.Generator().manual_seed(w.top_k + H + 1)
+    wts = torch.randn((w.ep_size, w.tokens_per_rank, w.top_k), generator=g)
+    y = torch.randn((w.ep_size, w.tokens_per_rank, w.top_k, H), generator=g).to(torch.bfloat16)
+    oute = fresh()
+    run.comm.combine_experts(wts.cuda(), y.cuda(), oute)
+    torch.cuda.synchronize()
+    assert run.comm.get_status() == ep_a2a.OK
+    U.assert_equal(oute, U.oracle.combine_experts(plan, w.num_experts,
+                                                  x.token_selected_experts.numpy(), wts.numpy(),
+                                                  U.to_np(y), H, out_init=init), "experts")
 
 
 def test_fp8_quantize_all_bf16_patterns():
