@@ -344,15 +344,18 @@ __device__ __forceinline__ bool rank_is_live(const CopyArgs& a, int r) {
   return !a.use_mask || ((a.live[r >> 6] >> (r & 63)) & 1ull);
 }
 
-// The routing outputs of token slot `tok` (one warp, all 32 lanes), the same
-// as the routing kernel writes for it: plan_nd / plan_dst (destinations in
-// ascending rank order), the send counts, and for every live rank d its valid
-// byte and received ids (the token's ids if d is a destination, else
-// invalid_id).  Lane j < k holds expert slot j; owners are de-duplicated with
-// a warp match; a leader's position in the ascending list is the number of
+// The routing outputs of token slot `tok`, the same as the routing kernel
+// writes for it: plan_nd / plan_dst (destinations in ascending rank order),
+// the send counts, and for every live rank d its valid byte and received ids
+// (the token's ids if d is a destination, else invalid_id).  Every warp of
+// the token's group calls it (all 32 lanes); warp gw of nw writes the plan
+// row and counts if gw == 0, and its share of the per-rank ids and valid
+// bytes.  Lane j < k holds expert slot j; owners are de-duplicated with a
+// warp match; a leader's position in the ascending list is the number of
 // leaders with a smaller rank; lane w < 8 holds bits 32w..32w+31 of the
 // destination set, which the lanes writing rank d's row read by shuffle.
-__device__ __forceinline__ void route_token(const CopyArgs& a, int64_t tok, int lane) {
+__device__ __forceinline__ void route_token(const CopyArgs& a, int64_t tok, int lane, int gw,
+                                            int nw) {
   const int r = (int)(tok / a.tpr);
   const int t = (int)(tok - (int64_t)r * a.tpr);
   const bool exists = t < a.n[r];          // n[r] is 0 for masked-off ranks
@@ -376,16 +379,18 @@ __device__ __forceinline__ void route_token(const CopyArgs& a, int64_t tok, int 
     pos += (((leaders >> i) & 1u) != 0u) && other < d;
     if (other >= 0 && (other >> 5) == lane) word |= 1u << (other & 31);
   }
-  uint8_t* row = const_cast<uint8_t*>(a.plan_dst) + tok * a.plan_stride;
-  if (lane == 0) const_cast<uint8_t*>(a.plan_nd)[tok] = exists ? (uint8_t)nd : kNoToken;
-  if (leader) {
-    row[pos] = (uint8_t)d;
-    atomicAdd(&a.count_acc[r * a.ep + d], 1);
+  if (gw == 0) {
+    uint8_t* row = const_cast<uint8_t*>(a.plan_dst) + tok * a.plan_stride;
+    if (lane == 0) const_cast<uint8_t*>(a.plan_nd)[tok] = exists ? (uint8_t)nd : kNoToken;
+    if (leader) {
+      row[pos] = (uint8_t)d;
+      atomicAdd(&a.count_acc[r * a.ep + d], 1);
+    }
+    if (lane < a.plan_stride && lane >= nd) row[lane] = kPad;
   }
-  if (lane < a.plan_stride && lane >= nd) row[lane] = kPad;
   // received ids of every live rank: lane handles (rank idx / k, slot idx % k)
   const int total = a.ep * a.k;
-  for (int base = 0; base < total; base += 32) {
+  for (int base = gw * 32; base < total; base += nw * 32) {
     const int idx = base + lane;
     const int dd = idx / a.k;
     const int j = idx - dd * a.k;
@@ -396,7 +401,7 @@ __device__ __forceinline__ void route_token(const CopyArgs& a, int64_t tok, int 
       ids[tok * a.k + j] = ((wd >> (dd & 31)) & 1u) ? ej : a.invalid_id;
     }
   }
-  for (int base = 0; base < a.ep; base += 32) {
+  for (int base = gw * 32; base < a.ep; base += nw * 32) {
     const int dd = base + lane;
     const uint32_t wd = __shfl_sync(kFull, word, (dd >> 5) & 7);
     if (dd < a.ep && rank_is_live(a, dd))
@@ -470,7 +475,7 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
       for (int p = 0; p < a.np; ++p)
         prefetch_l2(a.src[p] + (tok + tok_step) * a.rb[p], (uint32_t)a.rb[p]);
     }
-    if (a.route && gl < 32) route_token(a, tok, lane);   // the group's first warp
+    if (a.route) route_token(a, tok, lane, gl >> 5, TPT / 32);
     uint64_t w0, w1, w2, w3;
     const int nd = token_destinations(a, tok, lane, w0, w1, w2, w3);
     if (nd == 0) continue;

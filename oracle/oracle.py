@@ -271,7 +271,16 @@ def combine_experts_fp8(plan: RoutePlan, num_experts, token_selected_experts, to
     The three steps in that order; nothing else."""
     z = expert_reduce(plan, num_experts, token_selected_experts, topk_weights, expert_out,
                       hidden)
-    codes, scales = quantize_e4m3_rows(z, hidden)
+    # the rows a destination sends are those of the tokens it received; only
+    # they are quantised (rows are independent) and read by the combine
+    rows = np.nonzero((np.asarray(plan.recv_valid) == 1).reshape(-1))[0]
+    flat = z.reshape(-1, hidden)
+    codes = np.zeros(flat.shape, np.uint8)
+    scales = np.ones(flat.shape[0], np.float32)
+    if rows.size:
+        c, sc = quantize_e4m3_rows(np.ascontiguousarray(flat[rows]), hidden)
+        codes[rows] = c
+        scales[rows] = sc
     return combine_scaled(plan, codes.reshape(z.shape), scales.reshape(z.shape[:2]), hidden,
                           out_init=out_init)
 

@@ -144,3 +144,34 @@ def oracle_quantize_big(bf16_bits: np.ndarray, table: np.ndarray) -> np.ndarray:
     for s in range(0, flat.size, step):
         out[s:s + step] = table[flat[s:s + step]]
     return out.reshape(bf16_bits.shape)
+
+
+def valid_rows(plan) -> np.ndarray:
+    """Flat indices d * (ep * tpr) + s of the receive rows a combine reads: rank
+    d's row for slot s where d received the token (recv_valid == 1)."""
+    return np.nonzero((np.asarray(plan.recv_valid) == 1).reshape(-1))[0]
+
+
+def oracle_e4m3_rows_read(bf16_bits: np.ndarray, plan, table: np.ndarray) -> np.ndarray:
+    """The oracle's E4M3 codes (through its table of every bf16 input) of the rows
+    a combine reads; the other rows are 0 and never read."""
+    H = bf16_bits.shape[-1]
+    flat = bf16_bits.reshape(-1, H)
+    idx = valid_rows(plan)
+    out = np.zeros(flat.shape, np.uint8)
+    out[idx] = table[flat[idx]]
+    return out.reshape(bf16_bits.shape)
+
+
+def oracle_row_quantize_read(bf16_bits: np.ndarray, plan, hidden: int):
+    """oracle.quantize_e4m3_rows applied to the rows a combine reads (rows are
+    independent); the other rows get codes 0 and scale 1 and are never read."""
+    flat = bf16_bits.reshape(-1, hidden)
+    idx = valid_rows(plan)
+    codes = np.zeros(flat.shape, np.uint8)
+    scales = np.ones(flat.shape[0], np.float32)
+    if idx.size:
+        c, sc = oracle.quantize_e4m3_rows(np.ascontiguousarray(flat[idx]), hidden)
+        codes[idx] = c
+        scales[idx] = sc
+    return codes.reshape(bf16_bits.shape), scales.reshape(bf16_bits.shape[:-1])
