@@ -815,6 +815,140 @@ __global__ void __launch_bounds__(448, 2) combine_experts_fp8_kernel(const Combi
   }
 }
 
+// The same with a thread-block cluster of C CTAs per token, each CTA owning a
+// slice of the row's 16-byte column vectors, one per thread, so that every
+// z_d stays in registers: phase 1 loads the thread's vector of each
+// participating slot row once and forms every destination's z_d (bf16) and
+// its partial max; each CTA reduces its maxima, the cluster exchanges them
+// through distributed shared memory (one cluster barrier per token; the
+// exchange slots alternate between tokens so that one barrier suffices), and
+// phase 2 takes each value through E4M3 and sums.  top_k <= 8, hidden a
+// multiple of 8, 16-byte aligned rows, nvec <= C * blockDim.x.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_cta_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// The float at the same shared-memory offset as `p` in CTA `rank` of the cluster.
+__device__ __forceinline__ float ld_cluster_f32(const float* p, uint32_t rank) {
+  uint32_t remote, local = smem_addr(p);
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+template <int C>
+__global__ void __launch_bounds__(256, 2) combine_experts_fp8_cluster_kernel(
+    const CombineExpertsArgs a) {
+  pdl_wait();
+  __shared__ float s_max[8][8];            // [warp][destination]
+  __shared__ float s_part[2][8];           // this CTA's maxima, by token parity
+  __shared__ float s_scale[8], s_inv[8];
+  const int nvec = a.H / 8;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const uint32_t cr = cluster_cta_rank();
+  const int v = (int)cr * blockDim.x + threadIdx.x;   // this thread's column vector
+  const bool has_v = v < nvec;
+  const int64_t clusters = gridDim.x / C;
+  int parity = 0;
+  for (int64_t tok = blockIdx.x / C; tok < a.ntok; tok += clusters) {
+    const int nd = a.plan_nd[tok];                // the same in every CTA of the cluster
+    if (nd == kNoToken) continue;
+    uint16_t* out = a.out + tok * (int64_t)a.H;
+    if (nd == 0) {           // every owner masked off: the sum is empty
+      if (has_v) reinterpret_cast<uint4*>(out)[v] = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const uint64_t w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    if (!plan_row_ok(nd, w0, 0, 0, 0, a.ep, 8, a.err)) continue;
+    int own[8];
+    float wt[8];
+    slot_owners<8>(a, tok, nd, w0, 0, 0, 0, own, wt);
+    uint32_t zr[8][4];
+    float amax[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) amax[q] = 0.0f;
+    if (has_v) {
+      uint4 raw[8];
+      expert_rows_load(raw, a.y + tok * (int64_t)a.k * a.H + (int64_t)v * 8, own, a.H);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q >= nd) break;
+        const int d = (int)((w0 >> (8 * q)) & 0xFFu);
+        float z[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) z[e] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (own[j] != d) continue;
+          const uint32_t wv[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            z[2 * i] = __fmaf_rn(wt[j], bf16_bits_to_f32(wv[i] & 0xFFFFu), z[2 * i]);
+            z[2 * i + 1] = __fmaf_rn(wt[j], bf16_bits_to_f32(wv[i] >> 16), z[2 * i + 1]);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          zr[q][i] = pack_bf16x2(z[2 * i], z[2 * i + 1]);
+          amax[q] = fmaxf(amax[q], fabsf(bf16_bits_to_f32(zr[q][i] & 0xFFFFu)));
+          amax[q] = fmaxf(amax[q], fabsf(bf16_bits_to_f32(zr[q][i] >> 16)));
+        }
+      }
+    }
+    // the CTA's maxima, then the cluster's
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+        amax[q] = fmaxf(amax[q], __shfl_xor_sync(0xFFFFFFFFu, amax[q], o));
+      if (lane == 0) s_max[warp][q] = amax[q];
+    }
+    __syncthreads();
+    if (threadIdx.x < 8) {
+      float m = 0.0f;
+      for (int i = 0; i < nwarps; ++i) m = fmaxf(m, s_max[i][threadIdx.x]);
+      s_part[parity][threadIdx.x] = m;
+    }
+    cluster_sync_all();
+    if (threadIdx.x < 8) {
+      float m = 0.0f;
+      for (uint32_t r = 0; r < (uint32_t)C; ++r)
+        m = fmaxf(m, ld_cluster_f32(&s_part[parity][threadIdx.x], r));
+      row_scale_of(m, s_scale[threadIdx.x], s_inv[threadIdx.x]);
+    }
+    __syncthreads();
+    if (has_v) {
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q >= nd) break;
+        fp8_roundtrip_acc(acc, make_uint4(zr[q][0], zr[q][1], zr[q][2], zr[q][3]), s_inv[q],
+                          s_scale[q]);
+      }
+      uint4 pk;
+      pk.x = pack_bf16x2(acc[0], acc[1]);
+      pk.y = pack_bf16x2(acc[2], acc[3]);
+      pk.z = pack_bf16x2(acc[4], acc[5]);
+      pk.w = pack_bf16x2(acc[6], acc[7]);
+      reinterpret_cast<uint4*>(out)[v] = pk;
+    }
+    parity ^= 1;
+  }
+  cluster_sync_all();        // no CTA leaves while a partner may still read its maxima
+}
+
 // Any top_k (<= 32) and hidden size, no shared-memory rows: for each
 // destination a first pass recomputes z_d over the row to find its maximum;
 // a second pass recomputes z_d, takes it through E4M3 and sums.
@@ -1336,6 +1470,38 @@ cudaError_t launch_combine_experts_staged(const CombineExpertsArgs& a, int grid,
   if (e != cudaSuccess) return e;
   return launch_kernel(combine_experts_staged_kernel<NCW>, dim3(grid), dim3(32 * (NCW + 1)), smem,
                        stream, pdl, a, stages);
+}
+
+template <int C>
+cudaError_t launch_fp8_cluster(const CombineExpertsArgs& a, int clusters, int threads,
+                               cudaStream_t stream, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(clusters * C);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, combine_experts_fp8_cluster_kernel<C>, a);
+}
+
+cudaError_t launch_combine_experts_fp8_cluster(const CombineExpertsArgs& a, int cluster,
+                                               int threads, int clusters, cudaStream_t stream,
+                                               bool pdl) {
+  switch (cluster) {
+    case 1: return launch_fp8_cluster<1>(a, clusters, threads, stream, pdl);
+    case 2: return launch_fp8_cluster<2>(a, clusters, threads, stream, pdl);
+    case 4: return launch_fp8_cluster<4>(a, clusters, threads, stream, pdl);
+    case 8: return launch_fp8_cluster<8>(a, clusters, threads, stream, pdl);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_combine_experts_fp8(const CombineExpertsArgs& a, bool smem_rows, int threads,

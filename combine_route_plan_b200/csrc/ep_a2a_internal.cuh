@@ -175,6 +175,13 @@ cudaError_t launch_combine_experts_staged(const CombineExpertsArgs& a, int grid,
 // else the element kernel (threads <= 256).
 cudaError_t launch_combine_experts_fp8(const CombineExpertsArgs& a, bool smem_rows, int threads,
                                        int grid, size_t smem, cudaStream_t stream, bool pdl);
+// The same with a cluster of `cluster` (1, 2, 4, 8) CTAs of `threads` (<= 256)
+// threads per token, each thread one 16-byte column vector (top_k <= 8, hidden
+// % 8 == 0, hidden / 8 <= cluster * threads, 16-byte aligned rows); `clusters`
+// clusters stride over the tokens.
+cudaError_t launch_combine_experts_fp8_cluster(const CombineExpertsArgs& a, int cluster,
+                                               int threads, int clusters, cudaStream_t stream,
+                                               bool pdl);
 cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n, cudaStream_t stream);
 cudaError_t launch_quantize_e4m3_rows(const uint16_t* in, uint8_t* out, float* scales,
                                       int64_t rows, int hidden, cudaStream_t stream);

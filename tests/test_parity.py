@@ -985,6 +985,25 @@ def test_combine_experts_fp8_edge_shapes(ep, E, k, tpr, H):
     _check_combine_experts_fp8(w, x, y, wts)
 
 
+@pytest.mark.parametrize("case", ["c2_ep8_decode", (4, 16, 5, 33, 40), (2, 8, 8, 16, 8192)])
+def test_combine_experts_fp8_shared_rows_kernel(case):
+    """The one-CTA-per-token kernel that keeps the rows z_d in shared memory (the
+    default is a cluster per token with the rows in registers)."""
+    from combine_route_plan_b200 import ep_a2a
+    if isinstance(case, str):
+        w = W.BY_NAME[case]
+        x = _inputs(w.name)
+        wts = x.payloads[-1].view(torch.float32).view(w.ep_size, w.tokens_per_rank, w.top_k)
+        y = _expert_outputs(w, seed=w.seed + 93)
+    else:
+        ep, E, k, tpr, H = case
+        w, x = _custom(ep, E, k, tpr, H, [16], seed=ep * 19 + k)
+        g = torch.Generator().manual_seed(k + 5)
+        wts = torch.randn((ep, tpr, k), generator=g)
+        y = torch.randn((ep, tpr, k, H), generator=g).to(torch.bfloat16)
+    _check_combine_experts_fp8(w, x, y, wts, options={ep_a2a.OPT_FP8_EXPERTS_CLUSTER: 0})
+
+
 def test_combine_experts_fp8_masks_invalid_ids_and_zero_rows():
     ep, E, k, tpr, H = 8, 64, 6, 40, 64
     mask = [0b10110111, 0, 0, 0]
