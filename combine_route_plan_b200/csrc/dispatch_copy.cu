@@ -302,63 +302,35 @@ __device__ __forceinline__ void copy_row(const uint8_t* __restrict__ src, int64_
 
 constexpr int kVecThreads = 256;
 
-// Destinations of token `tok` (all lanes of the warp call it together): lanes
-// j < k look at expert slot j, the owners are de-duplicated with a warp match,
-// and the distinct live owners are packed as bytes into w0..w3.  The same rule
-// as the routing kernel (owner = e / epr for e in [0, E), live ranks only);
-// returns the number of destinations, or 0 for a token that does not exist.
-__device__ __forceinline__ int token_destinations(const CopyArgs& a, int64_t tok, int lane,
-                                                  uint64_t& w0, uint64_t& w1, uint64_t& w2,
-                                                  uint64_t& w3) {
-  const int r = (int)(tok / a.tpr);
-  const int t = (int)(tok - (int64_t)r * a.tpr);
-  w0 = w1 = w2 = w3 = 0;
-  if (t >= a.n[r]) return 0;              // n[r] is 0 for masked-off ranks
-  int d = -1;
-  if (lane < a.k) {
-    const int32_t e = a.ids[tok * a.k + lane];
-    if (e >= 0 && e < a.E) {
-      const int owner = e / a.epr;
-      if (!a.use_mask || ((a.live[owner >> 6] >> (owner & 63)) & 1ull)) d = owner;
-    }
-  }
-  const unsigned peers = __match_any_sync(kFull, d);
-  const bool leader = d >= 0 && (__ffs(peers) - 1) == lane;
-  unsigned leaders = __ballot_sync(kFull, leader);
-  int nd = 0;
-  while (leaders) {
-    const int l = __ffs(leaders) - 1;
-    leaders &= leaders - 1u;
-    const uint64_t dd = (uint64_t)(__shfl_sync(kFull, d, l) & 0xFF);
-    const int sh = (nd & 7) * 8;
-    if (nd < 8) w0 |= dd << sh;
-    else if (nd < 16) w1 |= dd << sh;
-    else if (nd < 24) w2 |= dd << sh;
-    else w3 |= dd << sh;
-    ++nd;
-  }
-  return nd;
-}
-
 __device__ __forceinline__ bool rank_is_live(const CopyArgs& a, int r) {
   return !a.use_mask || ((a.live[r >> 6] >> (r & 63)) & 1ull);
 }
 
-// The routing outputs of token slot `tok`, the same as the routing kernel
-// writes for it: plan_nd / plan_dst (destinations in ascending rank order),
-// the send counts, and for every live rank d its valid byte and received ids
-// (the token's ids if d is a destination, else invalid_id).  Every warp of
-// the token's group calls it (all 32 lanes); warp gw of nw writes the plan
-// row and counts if gw == 0, and its share of the per-rank ids and valid
-// bytes.  Lane j < k holds expert slot j; owners are de-duplicated with a
-// warp match; a leader's position in the ascending list is the number of
-// leaders with a smaller rank; lane w < 8 holds bits 32w..32w+31 of the
-// destination set, which the lanes writing rank d's row read by shuffle.
-__device__ __forceinline__ void route_token(const CopyArgs& a, int64_t tok, int lane, int gw,
-                                            int nw) {
+// Destinations of token slot `tok` (all lanes of the warp call it together),
+// by the routing kernel's rule: lanes j < k look at expert slot j (owner =
+// e / epr for e in [0, E), live ranks only), the owners are de-duplicated with
+// a warp match, and the distinct owners are packed as bytes into w0..w3 (for
+// the copy; lane order).  Returns their number, 0 for a token that does not
+// exist.
+//
+// With a.route set, the same pass also writes the token's routing outputs,
+// those of the routing kernel: plan_nd / plan_dst (destinations in ascending
+// rank order), the send counts, and for every live rank d its valid byte and
+// received ids (the token's ids if d is a destination, else invalid_id), for
+// tokens that do not exist too.  Every warp of the token's group calls it;
+// warp gw of nw writes the plan row and counts if gw == 0, and its share of the
+// per-rank ids and valid bytes.  A leader's position in the ascending list is
+// the number of leaders with a smaller rank; lane w < 8 holds bits
+// 32w..32w+31 of the destination set, which the lanes writing rank d's row read
+// by shuffle.  The ids are loaded once for both uses.
+__device__ __forceinline__ int token_route(const CopyArgs& a, int64_t tok, int lane, int gw,
+                                           int nw, uint64_t& w0, uint64_t& w1, uint64_t& w2,
+                                           uint64_t& w3) {
   const int r = (int)(tok / a.tpr);
   const int t = (int)(tok - (int64_t)r * a.tpr);
   const bool exists = t < a.n[r];          // n[r] is 0 for masked-off ranks
+  w0 = w1 = w2 = w3 = 0;
+  if (!exists && !a.route) return 0;
   int32_t e = 0;
   int d = -1;
   if (exists && lane < a.k) {
@@ -372,6 +344,21 @@ __device__ __forceinline__ void route_token(const CopyArgs& a, int64_t tok, int 
   const bool leader = d >= 0 && (__ffs(peers) - 1) == lane;
   const unsigned leaders = __ballot_sync(kFull, leader);
   const int nd = __popc(leaders);
+  {
+    unsigned rest = leaders;
+    for (int q = 0; rest; ++q) {
+      const int l = __ffs(rest) - 1;
+      rest &= rest - 1u;
+      const uint64_t dd = (uint64_t)(__shfl_sync(kFull, d, l) & 0xFF);
+      const int sh = (q & 7) * 8;
+      if (q < 8) w0 |= dd << sh;
+      else if (q < 16) w1 |= dd << sh;
+      else if (q < 24) w2 |= dd << sh;
+      else w3 |= dd << sh;
+    }
+  }
+  if (!a.route) return nd;
+
   int pos = 0;
   uint32_t word = 0;                       // lane w: set bits 32w..32w+31
   for (int i = 0; i < a.k; ++i) {
@@ -407,6 +394,7 @@ __device__ __forceinline__ void route_token(const CopyArgs& a, int64_t tok, int 
     if (dd < a.ep && rank_is_live(a, dd))
       a.rank0[(int64_t)dd * a.rank_stride + a.off_valid + tok] = (uint8_t)((wd >> (dd & 31)) & 1u);
   }
+  return exists ? nd : 0;
 }
 
 // EPLB gather: gathered[d][r][:] = live(r) ? stats[r][:] : 0 for live d, as
@@ -475,9 +463,8 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
       for (int p = 0; p < a.np; ++p)
         prefetch_l2(a.src[p] + (tok + tok_step) * a.rb[p], (uint32_t)a.rb[p]);
     }
-    if (a.route) route_token(a, tok, lane, gl >> 5, TPT / 32);
     uint64_t w0, w1, w2, w3;
-    const int nd = token_destinations(a, tok, lane, w0, w1, w2, w3);
+    const int nd = token_route(a, tok, lane, gl >> 5, TPT / 32, w0, w1, w2, w3);
     if (nd == 0) continue;
     for (int p = 0; p < a.np; ++p) {
       const uint8_t* src = a.src[p] + tok * a.rb[p];
