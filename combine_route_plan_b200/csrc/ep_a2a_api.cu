@@ -372,8 +372,14 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   h->copy_vec_bytes = 32;
   h->combine_pipeline = -1;
   h->copy_ctas_per_sm = 1;
-  h->route_in_copy = 1;
-  h->fp8_experts_cluster = 1;
+  // Measured on the decode, Zipf, wide-EP and prefill workloads: the separate
+  // routing kernel, running beside the copy (programmatic dependent launch), beat
+  // routing inside the copy kernel on every one (decode 47.2 against 49.4 us,
+  // wide EP 115.9 against 123.9 us, Zipf 135.6 against 146.8 us per step), and
+  // the sender-side FP8 expert combine with its rows in shared memory beat the
+  // cluster kernel (decode 83 against 175 us).
+  h->route_in_copy = 0;
+  h->fp8_experts_cluster = 0;
   h->copy_stages = 4;
   h->combine_threads = 0;
   h->bulk_min_row = 0;

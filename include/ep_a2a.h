@@ -379,18 +379,19 @@ typedef enum {
   EP_A2A_OPT_COPY_VEC_BYTES = 16, /* vector copy: widest access per thread, 16 or 32
                                      (default) bytes (sm_100 256-bit loads and stores,
                                      for rows and addresses that are 32-byte multiples) */
-  EP_A2A_OPT_ROUTE_IN_COPY = 17,  /* vector copy path (COPY_PATH 1): 1 (default) = the
-                                     copy kernel also writes the routing plan, valid
-                                     bytes, received ids, send counts and EPLB gather,
-                                     so a dispatch is one kernel; 0 = a separate
-                                     routing kernel runs first (the bulk paths always
-                                     use it) */
+  EP_A2A_OPT_ROUTE_IN_COPY = 17,  /* vector copy path (COPY_PATH 1): 1 = the copy kernel
+                                     also writes the routing plan, valid bytes, received
+                                     ids, send counts and EPLB gather, so a dispatch is
+                                     one kernel; 0 (default, measured faster) = a
+                                     separate routing kernel runs first, beside the copy
+                                     (the bulk paths always use it) */
   EP_A2A_OPT_FP8_EXPERTS_CLUSTER = 18 /* ep_a2a_combine_experts_fp8 with top_k <= 8 and
-                                     hidden a multiple of 8 up to 16384: 1 (default) = a
-                                     cluster of CTAs per token, one column vector per
-                                     thread, the rows z_d in registers and the row maxima
-                                     exchanged through distributed shared memory; 0 = one
-                                     CTA per token with the rows z_d in shared memory */
+                                     hidden a multiple of 8 up to 16384: 1 = a cluster of
+                                     CTAs per token, one column vector per thread, the rows
+                                     z_d in registers and the row maxima exchanged through
+                                     distributed shared memory; 0 (default, measured
+                                     faster) = one CTA per token with the rows z_d in
+                                     shared memory */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

@@ -54,14 +54,15 @@ def test_workload_bit_exact(name):
 
 @pytest.mark.parametrize("name", ["c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked",
                                   "c4_ep8_prefill"])
-def test_separate_routing_kernel_bit_exact(name):
-    """The vector copy after a separate routing kernel (the default routes inside
-    the copy kernel): plan, counts, valid bytes, ids, EPLB rows, the combine, and
-    the payload rows of the first and last destination ranks."""
+def test_routing_inside_the_copy_bit_exact(name):
+    """The vector copy kernel that also routes (one launch per dispatch; the
+    default runs a separate routing kernel beside the copy): plan, counts, valid
+    bytes, ids, EPLB rows, the combine, and the payload rows of the first and
+    last destination ranks."""
     from combine_route_plan_b200 import ep_a2a
     w = W.BY_NAME[name]
     x = _inputs(w.name)
-    run = U.Run(w, x, options={ep_a2a.OPT_ROUTE_IN_COPY: 0})
+    run = U.Run(w, x, options={ep_a2a.OPT_ROUTE_IN_COPY: 1})
     plan = U.oracle_plan(w, x)
     U.check_plan(run, plan, w)
     U.check_eplb(run, w, x)
@@ -985,10 +986,12 @@ def test_combine_experts_fp8_edge_shapes(ep, E, k, tpr, H):
     _check_combine_experts_fp8(w, x, y, wts)
 
 
-@pytest.mark.parametrize("case", ["c2_ep8_decode", (4, 16, 5, 33, 40), (2, 8, 8, 16, 8192)])
-def test_combine_experts_fp8_shared_rows_kernel(case):
-    """The one-CTA-per-token kernel that keeps the rows z_d in shared memory (the
-    default is a cluster per token with the rows in registers)."""
+@pytest.mark.parametrize("case", ["c2_ep8_decode", "c5_ep64_wide_masked", (4, 16, 5, 33, 40),
+                                  (2, 8, 8, 16, 8192), (4, 16, 4, 20, 7168 + 256)])
+def test_combine_experts_fp8_cluster_kernel(case):
+    """The kernel with a thread-block cluster per token, the rows z_d in registers
+    and the row maxima exchanged through distributed shared memory (the default
+    keeps the rows in shared memory, one CTA per token)."""
     from combine_route_plan_b200 import ep_a2a
     if isinstance(case, str):
         w = W.BY_NAME[case]
@@ -1001,7 +1004,7 @@ def test_combine_experts_fp8_shared_rows_kernel(case):
         g = torch.Generator().manual_seed(k + 5)
         wts = torch.randn((ep, tpr, k), generator=g)
         y = torch.randn((ep, tpr, k, H), generator=g).to(torch.bfloat16)
-    _check_combine_experts_fp8(w, x, y, wts, options={ep_a2a.OPT_FP8_EXPERTS_CLUSTER: 0})
+    _check_combine_experts_fp8(w, x, y, wts, options={ep_a2a.OPT_FP8_EXPERTS_CLUSTER: 1})
 
 
 def test_combine_experts_fp8_masks_invalid_ids_and_zero_rows():
