@@ -308,6 +308,7 @@ __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
 // At most 8 destinations per token; rows of 16-byte multiples at 16-byte
 // aligned addresses.
 constexpr int kStageChunk = 4096;                 // bytes of one row per item
+constexpr unsigned kFullMask32 = 0xFFFFFFFFu;
 constexpr int kCombineMaxStages = 8;
 
 template <int kMode, int NCW>
@@ -342,47 +343,78 @@ __global__ void __launch_bounds__(32 * (NCW + 1)) combine_staged_kernel(
   __syncthreads();
 
   if (warp == 0) {
-    // producer: items blockIdx.x, blockIdx.x + gridDim.x, ...; after the last
-    // one a sentinel (item -1) tells the consumers to stop
-    if (lane != 0) return;
+    // producer warp: items blockIdx.x, blockIdx.x + gridDim.x, ... in batches
+    // of 32 (lane l reads the plan row of the batch's item l, one load round
+    // per batch); for each item that exists, lane 0 takes a free stage and sets
+    // the bytes to expect, then lanes q < nd each issue the load of row q.
+    // After the last item a sentinel (item -1) tells the consumers to stop.
     int64_t n = 0;
-    for (int64_t it = blockIdx.x;; it += gridDim.x) {
-      int nd = 0;
-      uint64_t w0 = 0;
-      if (it < items) {
+    for (int64_t base = blockIdx.x;; base += 32 * (int64_t)gridDim.x) {
+      const int64_t my_it = base + (int64_t)lane * gridDim.x;
+      int my_nd = kNoToken;
+      uint64_t my_w0 = 0;
+      if (my_it < items) {
+        const int64_t tok = my_it / chunks;
+        my_nd = a.plan_nd[tok];
+        if (my_nd != kNoToken) {
+          my_w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+          if (!plan_row_ok(my_nd, my_w0, 0, 0, 0, a.ep, 8, a.err)) my_nd = kNoToken;
+        }
+      }
+      const bool last_batch = base + 32 * (int64_t)gridDim.x >= items;   // no items after it
+      unsigned todo = __ballot_sync(kFullMask32, my_nd != kNoToken);
+      bool stop = false;
+      while (!stop) {
+        int64_t it;
+        int nd;
+        uint64_t w0;
+        if (todo) {
+          const int l = __ffs(todo) - 1;
+          todo &= todo - 1u;
+          it = base + (int64_t)l * gridDim.x;
+          nd = __shfl_sync(kFullMask32, my_nd, l);
+          w0 = __shfl_sync(kFullMask32, my_w0, l);
+        } else if (last_batch) {
+          it = -1;                                     // the sentinel
+          nd = 0;
+          w0 = 0;
+          stop = true;
+        } else {
+          break;                                       // next batch
+        }
+        const int s = (int)(n % stages);
+        const uint32_t use = (uint32_t)(n / stages);
+        bool ok = true;
+        if (lane == 0) {
+          if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1u, kWaitLimitNs)) {
+            atomicOr(a.err, kErrWaitTimeout);
+            ok = false;
+          } else {
+            st_item[s] = it;
+            st_nd[s] = nd;
+            st_w0[s] = w0;
+          }
+        }
+        if (!__shfl_sync(kFullMask32, ok, 0)) return;
+        ++n;
+        if (it < 0 || nd == 0) {
+          if (lane == 0) mbar_arrive(full0 + 8 * s);
+          continue;
+        }
         const int64_t tok = it / chunks;
-        nd = a.plan_nd[tok];
-        if (nd == kNoToken) continue;
-        w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
-        if (!plan_row_ok(nd, w0, 0, 0, 0, a.ep, 8, a.err)) continue;
+        const int c = (int)(it - tok * chunks);
+        const int64_t off = (int64_t)c * kStageChunk;
+        const int64_t left = row_bytes - off;
+        const uint32_t cb = (uint32_t)(left < kStageChunk ? left : kStageChunk);
+        if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * s, cb * (uint32_t)nd);
+        __syncwarp();
+        if (lane < nd) {
+          const int d = (int)((w0 >> (8 * lane)) & 0xFFu);
+          bulk_load(smem0 + (uint32_t)s * stage_bytes + (uint32_t)lane * kStageChunk,
+                    a.x + tok * row_bytes + off + (int64_t)d * rank_stride, cb, full0 + 8 * s);
+        }
       }
-      const int s = (int)(n % stages);
-      const uint32_t use = (uint32_t)(n / stages);
-      if (use > 0 && !mbar_wait_bounded(empty0 + 8 * s, (use - 1) & 1u, kWaitLimitNs)) {
-        atomicOr(a.err, kErrWaitTimeout);
-        return;
-      }
-      ++n;
-      st_item[s] = it < items ? it : -1;
-      st_nd[s] = nd;
-      st_w0[s] = w0;
-      if (it >= items || nd == 0) {
-        mbar_arrive(full0 + 8 * s);
-        if (it >= items) return;
-        continue;
-      }
-      const int64_t tok = it / chunks;
-      const int c = (int)(it - tok * chunks);
-      const int64_t off = (int64_t)c * kStageChunk;
-      const int64_t left = row_bytes - off;
-      const uint32_t cb = (uint32_t)(left < kStageChunk ? left : kStageChunk);
-      mbar_arrive_expect_tx(full0 + 8 * s, cb * (uint32_t)nd);
-      const uint8_t* src = a.x + tok * row_bytes + off;
-      for (int q = 0; q < nd; ++q) {
-        const int d = (int)((w0 >> (8 * q)) & 0xFFu);
-        bulk_load(smem0 + (uint32_t)s * stage_bytes + (uint32_t)q * kStageChunk,
-                  src + (int64_t)d * rank_stride, cb, full0 + 8 * s);
-      }
+      if (stop) return;
     }
   }
 
