@@ -876,6 +876,14 @@ __device__ __forceinline__ float ld_cluster_f32(const float* p, uint32_t rank) {
   return v;
 }
 
+// The u32 at the same shared-memory offset as `p` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t ld_cluster_u32(const uint32_t* p, uint32_t rank) {
+  uint32_t remote, local = smem_addr(p), v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+  return v;
+}
+
 template <int C>
 __global__ void __launch_bounds__(256, 2) combine_experts_fp8_cluster_kernel(
     const CombineExpertsArgs a) {
@@ -979,6 +987,178 @@ __global__ void __launch_bounds__(256, 2) combine_experts_fp8_cluster_kernel(
     parity ^= 1;
   }
   cluster_sync_all();        // no CTA leaves while a partner may still read its maxima
+}
+
+// The sender-side FP8 expert combine, split over a cluster of C CTAs per
+// token (each CTA a slice of the row's 16-byte column vectors, two per thread)
+// with the rows z_d of its slice in shared memory.  Per token, warp 0 orders
+// the participating slots destination-major (ascending slot within each
+// destination, destinations in ascending rank), so phase 1 is one run of
+// fused multiply-adds over the slots with a uniform branch where a
+// destination's slots end; there z_d is rounded to bf16, stored, and its
+// maximum |z_d| taken on the packed bf16 bits (non-negative bf16 values order
+// like their bit patterns): a packed 16-bit max per pair, a warp max
+// reduction (redux) and a shared atomic max per warp.  The CTAs of the cluster
+// exchange their maxima through distributed shared memory (one cluster
+// barrier per token; the slots alternate between tokens), then phase 2 takes
+// the values through E4M3 and sums in ascending rank order.  top_k <= 8,
+// hidden a multiple of 8, 16-byte aligned rows, hidden / 8 <= C * 2 * blockDim.x.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+template <int C>
+__global__ void __launch_bounds__(256, 3) combine_experts_fp8_split_kernel(
+    const CombineExpertsArgs a, int cols) {
+  pdl_wait();
+  extern __shared__ __align__(16) uint8_t zsplit_mem[];    // [8][cols] bf16
+  __shared__ int s_slot[8];          // slot of position p (destination-major order)
+  __shared__ float s_wt[8];
+  __shared__ uint32_t s_end;         // 4 bits per destination: its slots end before this position
+  __shared__ int s_ns;               // participating slots
+  __shared__ uint32_t s_amax[2][8];  // per destination, by token parity: max |z| as bf16 bits
+  __shared__ float s_scale[8], s_inv[8];
+  uint16_t* zs = reinterpret_cast<uint16_t*>(zsplit_mem);
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const uint32_t cr = C > 1 ? cluster_cta_rank() : 0u;
+  const int nvec = a.H / 8;
+  const int cvec = cols / 8;                       // vectors of this CTA's slice
+  const int vbase = (int)cr * cvec;
+  const int64_t clusters = gridDim.x / C;
+  int parity = 0;
+  for (int64_t tok = blockIdx.x / C; tok < a.ntok; tok += clusters) {
+    const int nd = a.plan_nd[tok];                 // the same in every CTA of the cluster
+    if (nd == kNoToken) continue;
+    uint16_t* out = a.out + tok * (int64_t)a.H;
+    if (nd == 0) {           // every owner masked off: the sum is empty
+      for (int i = threadIdx.x; i < cvec; i += blockDim.x)
+        if (vbase + i < nvec) reinterpret_cast<uint4*>(out)[vbase + i] = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const uint64_t w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    if (!plan_row_ok(nd, w0, 0, 0, 0, a.ep, 8, a.err)) continue;
+    if (warp == 0) {
+      // lane j < k: slot j's destination index q (its owner's position in the
+      // plan row) and weight; its position in the destination-major order
+      int q = -1;
+      float wj = 0.0f;
+      if (lane < a.k) {
+        const int first = (int)(w0 & 0xFFu);
+        const int32_t e = reinterpret_cast<const int32_t*>(
+            a.recv_ids0 + (int64_t)first * a.rank_stride)[tok * a.k + lane];
+        const int o = (e >= 0 && e < a.E) ? e / a.epr : -1;
+        for (int i = 0; i < nd; ++i)
+          if ((int)((w0 >> (8 * i)) & 0xFFu) == o) q = i;
+        wj = a.w[tok * a.k + lane];
+      }
+      const unsigned part = __ballot_sync(0xFFFFFFFFu, q >= 0);
+      int pos = 0, cnt = 0;
+      for (int i = 0; i < 8; ++i) {
+        const int qi = __shfl_sync(0xFFFFFFFFu, q, i);
+        if (q >= 0 && qi >= 0 && (qi < q || (qi == q && i < lane))) ++pos;
+        if (lane < 8 && qi >= 0 && qi <= lane) ++cnt;   // slots of destinations 0..lane
+      }
+      if (q >= 0) {
+        s_slot[pos] = lane;
+        s_wt[pos] = wj;
+      }
+      uint32_t endw = (lane < 8 && lane < nd) ? ((uint32_t)cnt << (4 * lane)) : 0u;
+      endw = __reduce_or_sync(0xFFFFFFFFu, endw);
+      if (lane == 0) {
+        s_end = endw;
+        s_ns = __popc(part);
+      }
+      if (lane < 8) s_amax[parity][lane] = 0u;
+    }
+    __syncthreads();
+    int slot[8];
+    float wt[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      slot[p] = s_slot[p];
+      wt[p] = s_wt[p];
+    }
+    const int ns = s_ns;
+    const uint32_t endw = s_end;
+    const uint16_t* yt = a.y + tok * (int64_t)a.k * a.H;
+    // phase 1: this thread's vectors i = threadIdx.x, threadIdx.x + blockDim.x
+    for (int i = threadIdx.x; i < 2 * (int)blockDim.x; i += blockDim.x) {
+      const int v = vbase + i;
+      const bool has = i < cvec && v < nvec;       // warp-uniform except at the edge
+      uint4 raw[8];
+#pragma unroll
+      for (int p = 0; p < 8; ++p)
+        if (p < ns && has) raw[p] = ld_stream_v4(yt + (int64_t)slot[p] * a.H + (int64_t)v * 8);
+      float z[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z[e] = 0.0f;
+      int q = 0;
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        if (p >= ns) break;
+        if (has) {
+          const uint32_t wv[4] = {raw[p].x, raw[p].y, raw[p].z, raw[p].w};
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) {
+            z[2 * k2] = __fmaf_rn(wt[p], bf16_bits_to_f32(wv[k2] & 0xFFFFu), z[2 * k2]);
+            z[2 * k2 + 1] = __fmaf_rn(wt[p], bf16_bits_to_f32(wv[k2] >> 16), z[2 * k2 + 1]);
+          }
+        }
+        if ((int)((endw >> (4 * q)) & 0xFu) == p + 1) {   // destination q's slots end here
+          uint32_t m = 0u;
+          if (has) {
+            const uint32_t pk0 = pack_bf16x2(z[0], z[1]), pk1 = pack_bf16x2(z[2], z[3]);
+            const uint32_t pk2 = pack_bf16x2(z[4], z[5]), pk3 = pack_bf16x2(z[6], z[7]);
+            *reinterpret_cast<uint4*>(zs + (int64_t)q * cols + (int64_t)i * 8) =
+                make_uint4(pk0, pk1, pk2, pk3);
+            const uint32_t mm = max_u16x2(max_u16x2(pk0 & 0x7FFF7FFFu, pk1 & 0x7FFF7FFFu),
+                                          max_u16x2(pk2 & 0x7FFF7FFFu, pk3 & 0x7FFF7FFFu));
+            m = max(mm & 0xFFFFu, mm >> 16);
+          }
+          m = __reduce_max_sync(0xFFFFFFFFu, m);
+          if (lane == 0) atomicMax(&s_amax[parity][q], m);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) z[e] = 0.0f;
+          ++q;
+        }
+      }
+    }
+    __syncthreads();
+    if (C > 1) cluster_sync_all();
+    if (threadIdx.x < nd) {
+      uint32_t m = 0u;
+      for (uint32_t r = 0; r < (uint32_t)C; ++r)
+        m = max(m, C > 1 ? ld_cluster_u32(&s_amax[parity][threadIdx.x], r)
+                         : s_amax[parity][threadIdx.x]);
+      row_scale_of(__uint_as_float(m << 16), s_scale[threadIdx.x], s_inv[threadIdx.x]);
+    }
+    __syncthreads();
+    // phase 2
+    for (int i = threadIdx.x; i < cvec; i += blockDim.x) {
+      const int v = vbase + i;
+      if (v >= nvec) break;
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q >= nd) break;
+        const uint4 zb = *reinterpret_cast<const uint4*>(zs + (int64_t)q * cols + (int64_t)i * 8);
+        fp8_roundtrip_acc(acc, zb, s_inv[q], s_scale[q]);
+      }
+      uint4 pk;
+      pk.x = pack_bf16x2(acc[0], acc[1]);
+      pk.y = pack_bf16x2(acc[2], acc[3]);
+      pk.z = pack_bf16x2(acc[4], acc[5]);
+      pk.w = pack_bf16x2(acc[6], acc[7]);
+      reinterpret_cast<uint4*>(out)[v] = pk;
+    }
+    parity ^= 1;
+  }
+  if (C > 1) cluster_sync_all();   // no CTA leaves while a partner may still read its maxima
 }
 
 // Any top_k (<= 32) and hidden size, no shared-memory rows: for each
@@ -1532,6 +1712,48 @@ cudaError_t launch_combine_experts_fp8_cluster(const CombineExpertsArgs& a, int 
     case 2: return launch_fp8_cluster<2>(a, clusters, threads, stream, pdl);
     case 4: return launch_fp8_cluster<4>(a, clusters, threads, stream, pdl);
     case 8: return launch_fp8_cluster<8>(a, clusters, threads, stream, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int C>
+cudaError_t launch_fp8_split(const CombineExpertsArgs& a, int clusters, int threads, int cols,
+                             size_t smem, cudaStream_t stream, bool pdl) {
+  cudaError_t e = cudaFuncSetAttribute(combine_experts_fp8_split_kernel<C>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(clusters * C);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (C > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = C;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, combine_experts_fp8_split_kernel<C>, a, cols);
+}
+
+cudaError_t launch_combine_experts_fp8_split(const CombineExpertsArgs& a, int cluster, int threads,
+                                             int cols, int clusters, size_t smem,
+                                             cudaStream_t stream, bool pdl) {
+  switch (cluster) {
+    case 1: return launch_fp8_split<1>(a, clusters, threads, cols, smem, stream, pdl);
+    case 2: return launch_fp8_split<2>(a, clusters, threads, cols, smem, stream, pdl);
+    case 4: return launch_fp8_split<4>(a, clusters, threads, cols, smem, stream, pdl);
+    case 8: return launch_fp8_split<8>(a, clusters, threads, cols, smem, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -147,7 +147,7 @@ struct ep_a2a_handle_s {
   int combine_pipeline;       // 1: the two-deep pipelined kernels
   int copy_ctas_per_sm;
   int route_in_copy;      // vector copy path: 1 = the copy kernel also routes (one launch)
-  int fp8_experts_cluster;  // sender-side FP8 expert combine: 1 = cluster kernel
+  int fp8_experts_kernel;   // sender-side FP8 expert combine: 0 split, 1 cluster, 2 one CTA
   int copy_stages;        // 0 = choose from the row size
   int combine_threads;
   int64_t bulk_min_row;   // rows below this go to the vector copy
@@ -379,7 +379,7 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   // the sender-side FP8 expert combine with its rows in shared memory beat the
   // cluster kernel (decode 83 against 175 us).
   h->route_in_copy = 0;
-  h->fp8_experts_cluster = 0;
+  h->fp8_experts_kernel = 0;
   h->copy_stages = 4;
   h->combine_threads = 0;
   h->bulk_min_row = 0;
@@ -475,10 +475,10 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
         return fail(EP_A2A_ERR_INVALID_ARG, "combine CTAs per SM must be 0..1024");
       h->combine_ctas_per_sm = (int)value;
       return EP_A2A_OK;
-    case EP_A2A_OPT_FP8_EXPERTS_CLUSTER:
-      if (value != 0 && value != 1)
-        return fail(EP_A2A_ERR_INVALID_ARG, "FP8 experts cluster must be 0 or 1");
-      h->fp8_experts_cluster = (int)value;
+    case EP_A2A_OPT_FP8_EXPERTS_KERNEL:
+      if (value < 0 || value > 2)
+        return fail(EP_A2A_ERR_INVALID_ARG, "FP8 experts kernel must be 0, 1 or 2");
+      h->fp8_experts_kernel = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_ROUTE_IN_COPY:
       if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "route in copy must be 0 or 1");
@@ -817,7 +817,31 @@ EP_API ep_a2a_status ep_a2a_combine_experts_fp8(ep_a2a_handle h, const float* to
   const bool vec8 = a.k <= 8 && a.H % 8 == 0 && aligned(expert_output_per_slot, 16) &&
                     aligned(output, 16);
   const int nvec = a.H / 8;
-  if (vec8 && h->fp8_experts_cluster && nvec <= 8 * 256) {
+  const int rows = std::min(h->p.top_k, h->p.ep_size);
+  if (vec8 && h->fp8_experts_kernel == 0) {
+    // a cluster of C CTAs per token, each a slice of at most 512 column vectors
+    // (two per thread) with its rows z_d in shared memory; C the fewest that
+    // keep a slice's rows within 72 KB (three CTAs per SM)
+    int C = 1;
+    while (C < 8 && ((nvec + C - 1) / C > 512 ||
+                     (int64_t)rows * ((nvec + C - 1) / C) * 16 > 72 * 1024))
+      C *= 2;
+    const int cvec = (nvec + C - 1) / C;
+    if (cvec <= 512 && (int64_t)rows * cvec * 16 <= 72 * 1024) {
+      const int threads = std::max(32, ((cvec + 1) / 2 + 31) / 32 * 32);
+      const int cps = h->combine_ctas_per_sm > 0 ? h->combine_ctas_per_sm : 3;
+      const int clusters = (int)std::max<int64_t>(
+          1, std::min<int64_t>(a.ntok, std::max<int64_t>(1, (int64_t)h->num_sms * cps / C)));
+      const size_t smem = (size_t)rows * cvec * 16;
+      const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE_EXPERTS_FP8, (cudaStream_t)stream_v);
+      cudaError_t e = launch_combine_experts_fp8_split(a, C, threads, cvec * 8, clusters, smem,
+                                                       (cudaStream_t)stream_v, h->pdl != 0);
+      prof_end(h, slot, (cudaStream_t)stream_v);
+      if (e != cudaSuccess) return cuda_fail(e, "FP8 expert combine (split) kernel launch");
+      return EP_A2A_OK;
+    }
+  }
+  if (vec8 && h->fp8_experts_kernel == 1 && nvec <= 8 * 256) {
     // a cluster of C CTAs per token, one column vector per thread (the rows
     // z_d stay in registers); two CTAs per SM
     int C = 1;
@@ -836,7 +860,6 @@ EP_API ep_a2a_status ep_a2a_combine_experts_fp8(ep_a2a_handle h, const float* to
   // The shared-memory kernel keeps a token's rows z_d (one per destination, at
   // most min(top_k, ep_size)) as bf16; two CTAs of at most 448 threads share an
   // SM when the rows take at most half of its shared memory.
-  const int rows = std::min(h->p.top_k, h->p.ep_size);
   const size_t smem = (size_t)rows * a.H * 2;
   const bool smem_rows = a.k <= 8 && a.H % 8 == 0 && aligned(expert_output_per_slot, 16) &&
                          aligned(output, 16) && (int64_t)smem <= h->max_smem_optin - 2048;

@@ -182,6 +182,12 @@ cudaError_t launch_combine_experts_fp8(const CombineExpertsArgs& a, bool smem_ro
 cudaError_t launch_combine_experts_fp8_cluster(const CombineExpertsArgs& a, int cluster,
                                                int threads, int clusters, cudaStream_t stream,
                                                bool pdl);
+// The same split over a cluster of `cluster` CTAs per token, each a slice of
+// `cols` elements (two 16-byte vectors per thread, threads <= 256) with its
+// rows z_d in `smem` bytes of shared memory (min(top_k, ep) rows x cols bf16).
+cudaError_t launch_combine_experts_fp8_split(const CombineExpertsArgs& a, int cluster, int threads,
+                                             int cols, int clusters, size_t smem,
+                                             cudaStream_t stream, bool pdl);
 cudaError_t launch_quantize_e4m3(const uint16_t* in, uint8_t* out, int64_t n, cudaStream_t stream);
 cudaError_t launch_quantize_e4m3_rows(const uint16_t* in, uint8_t* out, float* scales,
                                       int64_t rows, int hidden, cudaStream_t stream);

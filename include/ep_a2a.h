@@ -385,13 +385,14 @@ typedef enum {
                                      one kernel; 0 (default, measured faster) = a
                                      separate routing kernel runs first, beside the copy
                                      (the bulk paths always use it) */
-  EP_A2A_OPT_FP8_EXPERTS_CLUSTER = 18 /* ep_a2a_combine_experts_fp8 with top_k <= 8 and
-                                     hidden a multiple of 8 up to 16384: 1 = a cluster of
-                                     CTAs per token, one column vector per thread, the rows
-                                     z_d in registers and the row maxima exchanged through
-                                     distributed shared memory; 0 (default, measured
-                                     faster) = one CTA per token with the rows z_d in
-                                     shared memory */
+  EP_A2A_OPT_FP8_EXPERTS_KERNEL = 18 /* ep_a2a_combine_experts_fp8 with top_k <= 8 and
+                                     hidden a multiple of 8: 0 (default) = a cluster of
+                                     CTAs per token, each a slice of the row with its
+                                     rows z_d in shared memory, the row maxima exchanged
+                                     through distributed shared memory; 1 = a cluster per
+                                     token with one column vector per thread and the rows
+                                     in registers (hidden up to 16384); 2 = one CTA per
+                                     token with the whole rows in shared memory */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

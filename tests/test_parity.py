@@ -986,12 +986,15 @@ def test_combine_experts_fp8_edge_shapes(ep, E, k, tpr, H):
     _check_combine_experts_fp8(w, x, y, wts)
 
 
+@pytest.mark.parametrize("kernel", [1, 2])
 @pytest.mark.parametrize("case", ["c2_ep8_decode", "c5_ep64_wide_masked", (4, 16, 5, 33, 40),
                                   (2, 8, 8, 16, 8192), (4, 16, 4, 20, 7168 + 256)])
-def test_combine_experts_fp8_cluster_kernel(case):
-    """The kernel with a thread-block cluster per token, the rows z_d in registers
-    and the row maxima exchanged through distributed shared memory (the default
-    keeps the rows in shared memory, one CTA per token)."""
+def test_combine_experts_fp8_other_kernels(case, kernel):
+    """The two other kernels of the sender-side FP8 expert combine: a cluster per
+    token with one column vector per thread and the rows z_d in registers (1),
+    and one CTA per token with the whole rows in shared memory (2); the default
+    splits each token over a cluster with the rows of each slice in shared
+    memory."""
     from combine_route_plan_b200 import ep_a2a
     if isinstance(case, str):
         w = W.BY_NAME[case]
@@ -1004,7 +1007,7 @@ def test_combine_experts_fp8_cluster_kernel(case):
         g = torch.Generator().manual_seed(k + 5)
         wts = torch.randn((ep, tpr, k), generator=g)
         y = torch.randn((ep, tpr, k, H), generator=g).to(torch.bfloat16)
-    _check_combine_experts_fp8(w, x, y, wts, options={ep_a2a.OPT_FP8_EXPERTS_CLUSTER: 1})
+    _check_combine_experts_fp8(w, x, y, wts, options={ep_a2a.OPT_FP8_EXPERTS_KERNEL: kernel})
 
 
 def test_combine_experts_fp8_masks_invalid_ids_and_zero_rows():
