@@ -430,10 +430,14 @@ class DeviceCase:
         self.comm.destroy()
 
 
-def measure_case(case, kind, steps, warmup, stream, flush_buf, graph, peak):
+def measure_case(case, kind, steps, warmup, stream, flush_buf, graph, peak, clean_buf=None):
     """Step time (CUDA events; with flush_buf, L2 is flushed before every step
     and each step is timed alone), per-kernel times from an eager pass with
-    events around each launch, and the roofline figures of both."""
+    events around each launch, and the roofline figures of both.  With
+    clean_buf, a second timed loop flushes the same way and then reads
+    clean_buf (larger than L2), so each step also starts with no dirty lines
+    in L2: the write flush leaves L2 full of dirty lines that the step would
+    otherwise write back to DRAM on its own time."""
     import torch
     from combine_route_plan_b200 import ep_a2a
     step = case.step(kind)
@@ -465,6 +469,12 @@ def measure_case(case, kind, steps, warmup, stream, flush_buf, graph, peak):
         ms = run_timed_flushed(timed, lambda: flush_buf.zero_(), steps, warmup, stream, None)
     else:
         ms = run_timed(timed, steps, warmup, CudaTimer(stream), None)
+    ms_clean = None
+    if flush_buf is not None and clean_buf is not None:
+        def clean_flush():
+            flush_buf.zero_()
+            clean_buf.amax()
+        ms_clean = run_timed_flushed(timed, clean_flush, steps, warmup, stream, None)
     torch.cuda.synchronize()
     del g
     if case.comm.get_status() != ep_a2a.OK:
@@ -483,11 +493,16 @@ def measure_case(case, kind, steps, warmup, stream, flush_buf, graph, peak):
             kernels[name] = {"avg_us": avg_s * 1e6, "algorithmic_bytes": kbytes[name],
                              "gbs": kbytes[name] / avg_s / 1e9,
                              "frac": kbytes[name] / avg_s / 1e9 / peak}
-    return {"workload": case.w.name, "combine": kind, "step_us": step_s * 1e6,
-            "tokens_per_s": case.n_tok / step_s, "step_algorithmic_bytes": by.step,
-            "step_gbs": by.step / step_s / 1e9, "step_frac": by.step / step_s / 1e9 / peak,
-            "tokens": case.n_tok, "mean_distinct_ranks": case.sum_d / max(case.n_tok, 1),
-            "kernels": kernels}
+    rec = {"workload": case.w.name, "combine": kind, "step_us": step_s * 1e6,
+           "tokens_per_s": case.n_tok / step_s, "step_algorithmic_bytes": by.step,
+           "step_gbs": by.step / step_s / 1e9, "step_frac": by.step / step_s / 1e9 / peak,
+           "tokens": case.n_tok, "mean_distinct_ranks": case.sum_d / max(case.n_tok, 1),
+           "kernels": kernels}
+    if ms_clean is not None:
+        clean_s = ms_clean / steps / 1e3
+        rec["clean_l2"] = {"step_us": clean_s * 1e6, "tokens_per_s": case.n_tok / clean_s,
+                           "step_frac": by.step / clean_s / 1e9 / peak}
+    return rec
 
 
 def workloads_record(args, device, stream, peak, prefill_case=None):
@@ -498,19 +513,23 @@ def workloads_record(args, device, stream, peak, prefill_case=None):
     import torch
     from combine_route_plan_b200 import workloads as W
     flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    clean_buf = torch.ones(512 << 20, dtype=torch.uint8, device=device)
     out = []
     for name, kinds in RECORD_CASES:
         w = W.BY_NAME[name]
         case = DeviceCase(w, W.make_inputs(w, with_expert_output=False), device, kinds)
         for kind in kinds:
-            r = measure_case(case, kind, args.workload_steps, 5, stream, flush_buf, True, peak)
-            r["timing"] = "CUDA-graph replay, 512 MB L2 flush before each step, steps timed alone"
+            r = measure_case(case, kind, args.workload_steps, 5, stream, flush_buf, True, peak,
+                             clean_buf=clean_buf)
+            r["timing"] = ("CUDA-graph replay, 512 MB L2 flush (written) before each step, steps "
+                           "timed alone; clean_l2: the same flush followed by a 512 MB read, so "
+                           "the step also starts with no dirty lines in L2")
             out.append(r)
         case.destroy()
         del case
         gc.collect()
         torch.cuda.empty_cache()
-    del flush_buf
+    del flush_buf, clean_buf
     if prefill_case is not None:
         for kind in ("fp8", "fp8s", "experts", "experts_fp8"):
             r = measure_case(prefill_case, kind, args.workload_steps, 5, stream, None, False, peak)
