@@ -306,6 +306,44 @@ __device__ __forceinline__ bool rank_is_live(const CopyArgs& a, int r) {
   return !a.use_mask || ((a.live[r >> 6] >> (r & 63)) & 1ull);
 }
 
+// Destinations of token `tok` (all lanes of the warp call it together): lanes
+// j < k look at expert slot j, the owners are de-duplicated with a warp match,
+// and the distinct live owners are packed as bytes into w0..w3.  The same rule
+// as the routing kernel (owner = e / epr for e in [0, E), live ranks only);
+// returns the number of destinations, or 0 for a token that does not exist.
+__device__ __forceinline__ int token_destinations(const CopyArgs& a, int64_t tok, int lane,
+                                                  uint64_t& w0, uint64_t& w1, uint64_t& w2,
+                                                  uint64_t& w3) {
+  const int r = (int)(tok / a.tpr);
+  const int t = (int)(tok - (int64_t)r * a.tpr);
+  w0 = w1 = w2 = w3 = 0;
+  if (t >= a.n[r]) return 0;              // n[r] is 0 for masked-off ranks
+  int d = -1;
+  if (lane < a.k) {
+    const int32_t e = a.ids[tok * a.k + lane];
+    if (e >= 0 && e < a.E) {
+      const int owner = e / a.epr;
+      if (!a.use_mask || ((a.live[owner >> 6] >> (owner & 63)) & 1ull)) d = owner;
+    }
+  }
+  const unsigned peers = __match_any_sync(kFull, d);
+  const bool leader = d >= 0 && (__ffs(peers) - 1) == lane;
+  unsigned leaders = __ballot_sync(kFull, leader);
+  int nd = 0;
+  while (leaders) {
+    const int l = __ffs(leaders) - 1;
+    leaders &= leaders - 1u;
+    const uint64_t dd = (uint64_t)(__shfl_sync(kFull, d, l) & 0xFF);
+    const int sh = (nd & 7) * 8;
+    if (nd < 8) w0 |= dd << sh;
+    else if (nd < 16) w1 |= dd << sh;
+    else if (nd < 24) w2 |= dd << sh;
+    else w3 |= dd << sh;
+    ++nd;
+  }
+  return nd;
+}
+
 // Destinations of token slot `tok` (all lanes of the warp call it together),
 // by the routing kernel's rule: lanes j < k look at expert slot j (owner =
 // e / epr for e in [0, E), live ranks only), the owners are de-duplicated with
@@ -323,14 +361,15 @@ __device__ __forceinline__ bool rank_is_live(const CopyArgs& a, int r) {
 // the number of leaders with a smaller rank; lane w < 8 holds bits
 // 32w..32w+31 of the destination set, which the lanes writing rank d's row read
 // by shuffle.  The ids are loaded once for both uses.
+template <bool kRoute>
 __device__ __forceinline__ int token_route(const CopyArgs& a, int64_t tok, int lane, int gw,
                                            int nw, uint64_t& w0, uint64_t& w1, uint64_t& w2,
                                            uint64_t& w3) {
   const int r = (int)(tok / a.tpr);
   const int t = (int)(tok - (int64_t)r * a.tpr);
+  if (!kRoute) return token_destinations(a, tok, lane, w0, w1, w2, w3);
   const bool exists = t < a.n[r];          // n[r] is 0 for masked-off ranks
   w0 = w1 = w2 = w3 = 0;
-  if (!exists && !a.route) return 0;
   int32_t e = 0;
   int d = -1;
   if (exists && lane < a.k) {
@@ -357,8 +396,6 @@ __device__ __forceinline__ int token_route(const CopyArgs& a, int64_t tok, int l
       else w3 |= dd << sh;
     }
   }
-  if (!a.route) return nd;
-
   int pos = 0;
   uint32_t word = 0;                       // lane w: set bits 32w..32w+31
   for (int i = 0; i < a.k; ++i) {
@@ -442,7 +479,7 @@ __device__ __forceinline__ void finish_counts(const CopyArgs& a) {
 // after it sees the plan complete.  kAll = 16 or 32: every payload of the
 // launch moves in vectors of that many bytes (one code path, fewer registers);
 // kAll = 0: each payload picks its own vector width.
-template <int U, int kAll, bool kStreaming, int TPT>
+template <int U, int kAll, bool kStreaming, int TPT, bool kRoute>
 __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArgs a) {
   constexpr bool kUniform = kAll != 0;
   constexpr int kGroups = kVecThreads / TPT;
@@ -450,7 +487,7 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
   const int group = threadIdx.x / TPT;
   const int lane = threadIdx.x & 31;
   const int64_t tok_step = (int64_t)gridDim.x * kGroups;
-  if (a.route) {
+  if (kRoute) {
     // this launch is the whole dispatch: it reads the caller's ids and rows and
     // rewrites the plan the previous combine read, so it waits for the
     // preceding grid first
@@ -464,7 +501,7 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
         prefetch_l2(a.src[p] + (tok + tok_step) * a.rb[p], (uint32_t)a.rb[p]);
     }
     uint64_t w0, w1, w2, w3;
-    const int nd = token_route(a, tok, lane, gl >> 5, TPT / 32, w0, w1, w2, w3);
+    const int nd = token_route<kRoute>(a, tok, lane, gl >> 5, TPT / 32, w0, w1, w2, w3);
     if (nd == 0) continue;
     for (int p = 0; p < a.np; ++p) {
       const uint8_t* src = a.src[p] + tok * a.rb[p];
@@ -507,7 +544,7 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
       }
     }
   }
-  if (a.route)
+  if (kRoute)
     finish_counts(a);
   else
     pdl_wait();
@@ -697,9 +734,9 @@ cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t strea
   }
 }
 
-template <int U, int TPT>
-cudaError_t launch_vec_ut(const CopyArgs& a, int grid, bool streaming, cudaStream_t stream,
-                          bool pdl) {
+template <int U, int TPT, bool kRoute>
+cudaError_t launch_vec_utr(const CopyArgs& a, int grid, bool streaming, cudaStream_t stream,
+                           bool pdl) {
   bool all16 = true, all32 = true;
   for (int p = 0; p < a.np; ++p) {
     all16 &= a.vec[p] == 16;
@@ -708,17 +745,26 @@ cudaError_t launch_vec_ut(const CopyArgs& a, int grid, bool streaming, cudaStrea
   const dim3 g(grid), b(kVecThreads);
   if (all32) {
     if (streaming)
-      return launch_kernel(dispatch_vec_kernel<U, 32, true, TPT>, g, b, 0, stream, pdl, a);
-    return launch_kernel(dispatch_vec_kernel<U, 32, false, TPT>, g, b, 0, stream, pdl, a);
+      return launch_kernel(dispatch_vec_kernel<U, 32, true, TPT, kRoute>, g, b, 0, stream, pdl,
+                           a);
+    return launch_kernel(dispatch_vec_kernel<U, 32, false, TPT, kRoute>, g, b, 0, stream, pdl, a);
   }
   if (all16) {
     if (streaming)
-      return launch_kernel(dispatch_vec_kernel<U, 16, true, TPT>, g, b, 0, stream, pdl, a);
-    return launch_kernel(dispatch_vec_kernel<U, 16, false, TPT>, g, b, 0, stream, pdl, a);
+      return launch_kernel(dispatch_vec_kernel<U, 16, true, TPT, kRoute>, g, b, 0, stream, pdl,
+                           a);
+    return launch_kernel(dispatch_vec_kernel<U, 16, false, TPT, kRoute>, g, b, 0, stream, pdl, a);
   }
   if (streaming)
-    return launch_kernel(dispatch_vec_kernel<U, 0, true, TPT>, g, b, 0, stream, pdl, a);
-  return launch_kernel(dispatch_vec_kernel<U, 0, false, TPT>, g, b, 0, stream, pdl, a);
+    return launch_kernel(dispatch_vec_kernel<U, 0, true, TPT, kRoute>, g, b, 0, stream, pdl, a);
+  return launch_kernel(dispatch_vec_kernel<U, 0, false, TPT, kRoute>, g, b, 0, stream, pdl, a);
+}
+
+template <int U, int TPT>
+cudaError_t launch_vec_ut(const CopyArgs& a, int grid, bool streaming, cudaStream_t stream,
+                          bool pdl) {
+  if (a.route) return launch_vec_utr<U, TPT, true>(a, grid, streaming, stream, pdl);
+  return launch_vec_utr<U, TPT, false>(a, grid, streaming, stream, pdl);
 }
 
 template <int U>

@@ -240,7 +240,8 @@ CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
   CombineLaunch c;
   c.pipe = fits && (h->combine_pipeline < 0 ? kind != kKindBf16 : h->combine_pipeline == 1);
   c.staged = fits && h->combine_pipeline == 2;
-  c.staged_ctas_per_sm = h->combine_ctas_per_sm > 0 ? std::min(h->combine_ctas_per_sm, 4) : 2;
+  // a staged CTA needs two stages of 32 KB: at most three CTAs per SM
+  c.staged_ctas_per_sm = h->combine_ctas_per_sm > 0 ? std::min(h->combine_ctas_per_sm, 3) : 2;
   const bool mid = !big && ntok >= 8192;
   int threads = 64, cps = 128, prefetch = 0;
   if (kind == kKindFp8) {
