@@ -313,6 +313,14 @@ def kernel_sources_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def device_mb_in_use(device) -> float:
+    """Device memory in use (total minus free, cudaMemGetInfo) in MB: torch's
+    tensors plus the library's own workspace, which torch does not see."""
+    import torch
+    free, total = torch.cuda.mem_get_info(device)
+    return round((total - free) / 1e6, 1)
+
+
 def committed_traffic(kernel: str, workload: str):
     """dram bytes per launch from profiles/dram_traffic.json, if it was taken on
     these exact kernel sources; else None."""
@@ -801,6 +809,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "cpu_baseline_all_cores": cpu_all,
             "kernel_sources": kernel_sources_hash(),
+            "device_mb_in_use": device_mb_in_use(device),
         }
         if fp8_ctx:
             rec["fp8_combine"] = fp8_ctx
