@@ -116,6 +116,7 @@ __device__ __forceinline__ void prefetch_token_rows(const CombineArgs& a, int64_
 template <bool kFp8>
 __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   constexpr int kElems = kFp8 ? 16 : 8;       // elements per 16-byte input vector
   constexpr int kElemBytes = kFp8 ? 1 : 2;
   const int nvec = a.H / kElems;
@@ -249,6 +250,7 @@ template <int kMode>
 __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
                                                            const float* __restrict__ scales) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   constexpr int kElems = kMode == kCombineBf16 ? 8 : 16;
   constexpr int kElemBytes = kMode == kCombineBf16 ? 2 : 1;
   const int nvec = a.H / kElems;
@@ -315,6 +317,7 @@ template <int kMode, int NCW>
 __global__ void __launch_bounds__(32 * (NCW + 1)) combine_staged_kernel(
     const CombineArgs a, const float* __restrict__ scales, int stages, int stage_rows) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   extern __shared__ __align__(128) uint8_t cs_mem[];
   __shared__ __align__(8) uint64_t full_bar[kCombineMaxStages];
   __shared__ __align__(8) uint64_t empty_bar[kCombineMaxStages];
@@ -462,6 +465,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1)) combine_staged_kernel(
 template <bool kFp8>
 __global__ void __launch_bounds__(512) combine_scalar_kernel(const CombineArgs a) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   const int words = a.plan_stride / 8;
   for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
     const int nd = a.plan_nd[tok];
@@ -524,6 +528,7 @@ __device__ __forceinline__ void slot_owners(const CombineExpertsArgs& a, int64_t
 // 16-byte column vectors; the loads of all needed slots are issued first.
 __global__ void __launch_bounds__(512) combine_experts_vec_kernel(const CombineExpertsArgs a) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   constexpr int KMAX = 8;
   const int nvec = a.H / 8;
   const int words = a.plan_stride / 8;
@@ -644,6 +649,7 @@ __device__ __forceinline__ void expert_rows_reduce_store(const uint4 (&raw)[8],
 // current one.  top_k <= 8, so a token has at most 8 destinations.
 __global__ void __launch_bounds__(512) combine_experts_pipe_kernel(const CombineExpertsArgs a) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   const int nvec = a.H / 8;
   const uint32_t tok_bytes = (uint32_t)a.k * a.H * 2;
   if (a.prefetch && threadIdx.x == 0)
@@ -749,6 +755,7 @@ constexpr int kFp8ExpertsMaxWarps = 32;
 // through E4M3 and sums in ascending rank order.
 __global__ void __launch_bounds__(448, 2) combine_experts_fp8_kernel(const CombineExpertsArgs a) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   extern __shared__ __align__(16) uint8_t z_mem[];       // [rows][H] bf16
   __shared__ float s_max[kFp8ExpertsMaxWarps][8];
   __shared__ float s_scale[8], s_inv[8];
@@ -888,6 +895,7 @@ template <int C>
 __global__ void __launch_bounds__(256, 2) combine_experts_fp8_cluster_kernel(
     const CombineExpertsArgs a) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   __shared__ float s_max[8][8];            // [warp][destination]
   __shared__ float s_part[2][8];           // this CTA's maxima, by token parity
   __shared__ float s_scale[8], s_inv[8];
@@ -1013,6 +1021,7 @@ template <int C>
 __global__ void __launch_bounds__(256, 3) combine_experts_fp8_split_kernel(
     const CombineExpertsArgs a, int cols) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   extern __shared__ __align__(16) uint8_t zsplit_mem[];    // [8][cols] bf16
   __shared__ int s_slot[8];          // slot of position p (destination-major order)
   __shared__ float s_wt[8];
@@ -1166,6 +1175,7 @@ __global__ void __launch_bounds__(256, 3) combine_experts_fp8_split_kernel(
 // a second pass recomputes z_d, takes it through E4M3 and sums.
 __global__ void __launch_bounds__(256) combine_experts_fp8_any_kernel(const CombineExpertsArgs a) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   constexpr int KMAX = kMaxTopK;
   __shared__ float s_max[8];
   __shared__ float s_scale[KMAX], s_inv[KMAX];
@@ -1229,6 +1239,7 @@ template <int NCW>
 __global__ void __launch_bounds__(32 * (NCW + 1)) combine_experts_staged_kernel(
     const CombineExpertsArgs a, int stages) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   extern __shared__ __align__(128) uint8_t es_mem[];
   __shared__ __align__(8) uint64_t full_bar[kCombineMaxStages];
   __shared__ __align__(8) uint64_t empty_bar[kCombineMaxStages];
@@ -1351,6 +1362,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1)) combine_experts_staged_kernel(
 // Any top_k (<= 32) and hidden size: one element per thread step.
 __global__ void __launch_bounds__(512) combine_experts_any_kernel(const CombineExpertsArgs a) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   constexpr int KMAX = kMaxTopK;
   const int words = a.plan_stride / 8;
   for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
@@ -1387,6 +1399,7 @@ template <bool kVec>
 __global__ void __launch_bounds__(512) combine_scaled_kernel(const CombineArgs a,
                                                              const float* __restrict__ scales) {
   pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
   const int words = a.plan_stride / 8;
   const int nvec = kVec ? a.H / 16 : 0;
   if (kVec && a.prefetch && threadIdx.x == 0)

@@ -31,6 +31,8 @@
 //     addresses; the SM only issues.
 // The two staged kernels read the plan (plan_nd / plan_dst) the routing kernel
 // wrote just before them.
+#include <type_traits>
+
 #include "ep_a2a_internal.cuh"
 
 namespace ep_a2a {
@@ -272,31 +274,49 @@ __device__ __forceinline__ void store_dst<Vec32>(Vec32* p, const Vec32& v, bool 
                  : "memory");
 }
 
+// One round of a token group's row copy: the vectors i0, i0 + TPT, ...
+// (U of them) of a row of n vectors, loaded into v, then stored to each of
+// the nd destinations.
+template <typename T, int U, int TPT>
+__device__ __forceinline__ void load_round(const T* __restrict__ s, int64_t n, int64_t i0,
+                                           T (&v)[U]) {
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int64_t i = i0 + (int64_t)u * TPT;
+    if (i < n) v[u] = load_src<T>(s + i);
+  }
+}
+
+template <typename T, int U, int TPT>
+__device__ __forceinline__ void store_round(const T (&v)[U], int64_t n, int64_t i0,
+                                            uint8_t* rank0, int64_t rank_stride, int64_t off,
+                                            uint64_t w0, uint64_t w1, uint64_t w2, uint64_t w3,
+                                            int nd, bool streaming) {
+  for (int q = 0; q < nd; ++q) {
+    T* d = reinterpret_cast<T*>(rank0 + (int64_t)dst_rank(w0, w1, w2, w3, q) * rank_stride +
+                                off);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + (int64_t)u * TPT;
+      if (i < n) store_dst<T>(d + i, v[u], streaming);
+    }
+  }
+}
+
 // Copy one payload row of a token to its nd destinations: the TPT threads of a
-// token group each take vectors gl, gl + TPT, ... (U of them in flight).
+// token group each take vectors gl, gl + TPT, ... (U of them in flight),
+// starting at vector `first` (gl, or later when the first round is done).
 template <typename T, int U, int TPT>
 __device__ __forceinline__ void copy_row(const uint8_t* __restrict__ src, int64_t rb,
                                          uint8_t* rank0, int64_t rank_stride, int64_t off,
                                          uint64_t w0, uint64_t w1, uint64_t w2, uint64_t w3,
-                                         int nd, int gl, bool streaming) {
+                                         int nd, int64_t first, bool streaming) {
   const int64_t n = rb / (int64_t)sizeof(T);
   const T* s = reinterpret_cast<const T*>(src);
-  for (int64_t i0 = gl; i0 < n; i0 += TPT * U) {
+  for (int64_t i0 = first; i0 < n; i0 += TPT * U) {
     T v[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t i = i0 + (int64_t)u * TPT;
-      if (i < n) v[u] = load_src<T>(s + i);
-    }
-    for (int q = 0; q < nd; ++q) {
-      T* d = reinterpret_cast<T*>(rank0 + (int64_t)dst_rank(w0, w1, w2, w3, q) * rank_stride +
-                                  off);
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t i = i0 + (int64_t)u * TPT;
-        if (i < n) store_dst<T>(d + i, v[u], streaming);
-      }
-    }
+    load_round<T, U, TPT>(s, n, i0, v);
+    store_round<T, U, TPT>(v, n, i0, rank0, rank_stride, off, w0, w1, w2, w3, nd, streaming);
   }
 }
 
@@ -479,14 +499,18 @@ __device__ __forceinline__ void finish_counts(const CopyArgs& a) {
 // after it sees the plan complete.  kAll = 16 or 32: every payload of the
 // launch moves in vectors of that many bytes (one code path, fewer registers);
 // kAll = 0: each payload picks its own vector width.
-template <int U, int kAll, bool kStreaming, int TPT, bool kRoute>
-__global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArgs a) {
+template <int U, int kAll, bool kStreaming, int TPT, bool kRoute, bool kEarly>
+__device__ __forceinline__ void dispatch_vec_body(const CopyArgs& a) {
   constexpr bool kUniform = kAll != 0;
   constexpr int kGroups = kVecThreads / TPT;
   const int gl = threadIdx.x % TPT;
   const int group = threadIdx.x / TPT;
   const int lane = threadIdx.x & 31;
   const int64_t tok_step = (int64_t)gridDim.x * kGroups;
+  // the first round of a token's first row can be loaded before the token is
+  // routed (the row's address does not depend on its destinations)
+  static_assert(!kEarly || (!kRoute && kUniform && TPT > 32), "early load: vector copy only");
+  using TU = typename std::conditional<kAll == 32, Vec32, uint4>::type;
   if (kRoute) {
     // this launch is the whole dispatch: it reads the caller's ids and rows and
     // rewrites the plan the previous combine read, so it waits for the
@@ -494,11 +518,33 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
     pdl_wait();
     if (a.eplb_stats != nullptr) eplb_gather_rows(a);
   }
+  // the next kernel may launch now; it waits for this grid's completion before
+  // it touches memory
+  if (a.trigger) pdl_launch_dependents();
   for (int64_t tok = (int64_t)blockIdx.x * kGroups + group; tok < a.ntok; tok += tok_step) {
     if (kUniform && a.prefetch && gl == 0 && tok + tok_step < a.ntok) {
       // the group's next token: its rows into L2 while this one is copied
       for (int p = 0; p < a.np; ++p)
         prefetch_l2(a.src[p] + (tok + tok_step) * a.rb[p], (uint32_t)a.rb[p]);
+    }
+    if (kEarly) {
+      const int64_t n0 = a.rb[0] / (int64_t)sizeof(TU);
+      TU v[U];
+      load_round<TU, U, TPT>(reinterpret_cast<const TU*>(a.src[0] + tok * a.rb[0]), n0, gl, v);
+      uint64_t w0, w1, w2, w3;
+      const int nd = token_route<false>(a, tok, lane, gl >> 5, TPT / 32, w0, w1, w2, w3);
+      if (nd == 0) continue;
+      const int64_t off0 = a.dst_off[0] + tok * a.rb[0];
+      const TU* s0 = reinterpret_cast<const TU*>(a.src[0] + tok * a.rb[0]);
+      for (int64_t i0 = gl; i0 < n0; i0 += TPT * U) {
+        if (i0 != gl) load_round<TU, U, TPT>(s0, n0, i0, v);
+        store_round<TU, U, TPT>(v, n0, i0, a.rank0, a.rank_stride, off0, w0, w1, w2, w3, nd,
+                                kStreaming);
+      }
+      for (int p = 1; p < a.np; ++p)
+        copy_row<TU, U, TPT>(a.src[p] + tok * a.rb[p], a.rb[p], a.rank0, a.rank_stride,
+                             a.dst_off[p] + tok * a.rb[p], w0, w1, w2, w3, nd, gl, kStreaming);
+      continue;
     }
     uint64_t w0, w1, w2, w3;
     const int nd = token_route<kRoute>(a, tok, lane, gl >> 5, TPT / 32, w0, w1, w2, w3);
@@ -548,6 +594,20 @@ __global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArg
     finish_counts(a);
   else
     pdl_wait();
+}
+
+template <int U, int kAll, bool kStreaming, int TPT, bool kRoute>
+__global__ void __launch_bounds__(kVecThreads)
+    dispatch_vec_kernel(const __grid_constant__ CopyArgs a) {
+  dispatch_vec_body<U, kAll, kStreaming, TPT, kRoute, false>(a);
+}
+
+// The copy with the early load, two vectors per thread: held to 64 registers,
+// four CTAs per SM, as the copy without it.
+template <int kAll, bool kStreaming, int TPT>
+__global__ void __launch_bounds__(kVecThreads, 4)
+    dispatch_vec_early_kernel(const __grid_constant__ CopyArgs a) {
+  dispatch_vec_body<2, kAll, kStreaming, TPT, false, true>(a);
 }
 
 template <int NCW, int MAXV>
@@ -743,6 +803,16 @@ cudaError_t launch_vec_utr(const CopyArgs& a, int grid, bool streaming, cudaStre
     all32 &= a.vec[p] == 32;
   }
   const dim3 g(grid), b(kVecThreads);
+  if constexpr (!kRoute && TPT > 32 && U == 2) {
+    if (a.early && all32)
+      return launch_kernel(streaming ? dispatch_vec_early_kernel<32, true, TPT>
+                                     : dispatch_vec_early_kernel<32, false, TPT>,
+                           g, b, 0, stream, pdl, a);
+    if (a.early && all16)
+      return launch_kernel(streaming ? dispatch_vec_early_kernel<16, true, TPT>
+                                     : dispatch_vec_early_kernel<16, false, TPT>,
+                           g, b, 0, stream, pdl, a);
+  }
   if (all32) {
     if (streaming)
       return launch_kernel(dispatch_vec_kernel<U, 32, true, TPT, kRoute>, g, b, 0, stream, pdl,

@@ -148,6 +148,8 @@ struct ep_a2a_handle_s {
   int copy_ctas_per_sm;
   int route_in_copy;      // vector copy path: 1 = the copy kernel also routes (one launch)
   int fp8_experts_kernel;   // sender-side FP8 expert combine: 0 split, 1 cluster, 2 one CTA
+  int pdl_trigger;          // copy and combines trigger the next launch at their start
+  int copy_early_load;      // vector copy: first row vectors loaded before routing
   int copy_stages;        // 0 = choose from the row size
   int combine_threads;
   int64_t bulk_min_row;   // rows below this go to the vector copy
@@ -381,6 +383,8 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   // cluster kernel (decode 83 against 175 us).
   h->route_in_copy = 0;
   h->fp8_experts_kernel = 0;
+  h->pdl_trigger = 0;
+  h->copy_early_load = 0;
   h->copy_stages = 4;
   h->combine_threads = 0;
   h->bulk_min_row = 0;
@@ -480,6 +484,14 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       if (value < 0 || value > 2)
         return fail(EP_A2A_ERR_INVALID_ARG, "FP8 experts kernel must be 0, 1 or 2");
       h->fp8_experts_kernel = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_PDL_TRIGGER:
+      if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "PDL trigger must be 0 or 1");
+      h->pdl_trigger = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_COPY_EARLY_LOAD:
+      if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "early load must be 0 or 1");
+      h->copy_early_load = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_ROUTE_IN_COPY:
       if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "route in copy must be 0 or 1");
@@ -607,6 +619,8 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
   std::memcpy(bulk.live, ra.live, sizeof(bulk.live));
   bulk.ep = ep;
   vec = bulk;
+  vec.trigger = pdl && h->pdl_trigger != 0;
+  vec.early = h->copy_early_load;
   if (fused) {
     vec.route = 1;
     vec.invalid_id = ra.invalid_id;
@@ -720,7 +734,7 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   if (dtype != EP_A2A_COMBINE_BF16 && dtype != EP_A2A_COMBINE_FP8_E4M3)
     return fail(EP_A2A_ERR_INVALID_ARG, "unknown combine dtype %d", (int)dtype);
   const bool fp8 = dtype == EP_A2A_COMBINE_FP8_E4M3;
-  CombineArgs a;
+  CombineArgs a{};
   a.plan_nd = h->ws + h->L.off_plan_nd;
   a.plan_dst = h->ws + h->L.off_plan_dst;
   a.x = static_cast<const uint8_t*>(expert_output);
@@ -730,6 +744,7 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   a.plan_stride = h->L.plan_stride;
   a.ep = h->p.ep_size;
   a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
+  a.trigger = h->pdl != 0 && h->pdl_trigger != 0;
   const CombineLaunch c = combine_launch(h, fp8 ? kKindFp8 : kKindBf16, a.ntok);
   a.prefetch = c.prefetch;
   a.out32 = aligned(output, 32) ? 1 : 0;
@@ -757,7 +772,7 @@ EP_API ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle h, const float* topk_w
   if (!h->have_plan) return fail(EP_A2A_ERR_NO_PLAN, "combine needs a preceding dispatch");
   if (!topk_weights || !expert_output_per_slot || !output)
     return fail(EP_A2A_ERR_INVALID_ARG, "topk_weights / expert output / output is NULL");
-  CombineExpertsArgs a;
+  CombineExpertsArgs a{};
   a.plan_nd = h->ws + h->L.off_plan_nd;
   a.plan_dst = h->ws + h->L.off_plan_dst;
   a.recv_ids0 = h->ws + h->L.rank_base + h->L.off_ids;
@@ -773,6 +788,7 @@ EP_API ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle h, const float* topk_w
   a.plan_stride = h->L.plan_stride;
   a.ep = h->p.ep_size;
   a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
+  a.trigger = h->pdl != 0 && h->pdl_trigger != 0;
   const CombineLaunch c = combine_launch(h, kKindExperts, a.ntok);
   a.prefetch = c.prefetch;
   const bool vec = a.k <= 8 && a.H % 8 == 0 && aligned(expert_output_per_slot, 16) &&
@@ -798,7 +814,7 @@ EP_API ep_a2a_status ep_a2a_combine_experts_fp8(ep_a2a_handle h, const float* to
   if (!h->have_plan) return fail(EP_A2A_ERR_NO_PLAN, "combine needs a preceding dispatch");
   if (!topk_weights || !expert_output_per_slot || !output)
     return fail(EP_A2A_ERR_INVALID_ARG, "topk_weights / expert output / output is NULL");
-  CombineExpertsArgs a;
+  CombineExpertsArgs a{};
   a.plan_nd = h->ws + h->L.off_plan_nd;
   a.plan_dst = h->ws + h->L.off_plan_dst;
   a.recv_ids0 = h->ws + h->L.rank_base + h->L.off_ids;
@@ -814,6 +830,7 @@ EP_API ep_a2a_status ep_a2a_combine_experts_fp8(ep_a2a_handle h, const float* to
   a.plan_stride = h->L.plan_stride;
   a.ep = h->p.ep_size;
   a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
+  a.trigger = h->pdl != 0 && h->pdl_trigger != 0;
   a.prefetch = 0;
   const bool vec8 = a.k <= 8 && a.H % 8 == 0 && aligned(expert_output_per_slot, 16) &&
                     aligned(output, 16);
@@ -892,7 +909,7 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
   if (!h->have_plan) return fail(EP_A2A_ERR_NO_PLAN, "combine needs a preceding dispatch");
   if (!expert_output_e4m3 || !row_scales || !output)
     return fail(EP_A2A_ERR_INVALID_ARG, "expert_output / row_scales / output is NULL");
-  CombineArgs a;
+  CombineArgs a{};
   a.plan_nd = h->ws + h->L.off_plan_nd;
   a.plan_dst = h->ws + h->L.off_plan_dst;
   a.x = static_cast<const uint8_t*>(expert_output_e4m3);
@@ -902,6 +919,7 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
   a.plan_stride = h->L.plan_stride;
   a.ep = h->p.ep_size;
   a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
+  a.trigger = h->pdl != 0 && h->pdl_trigger != 0;
   const CombineLaunch c = combine_launch(h, kKindFp8, a.ntok);
   a.prefetch = c.prefetch;
   a.out32 = aligned(output, 32) ? 1 : 0;

@@ -112,6 +112,9 @@ struct CopyArgs {
   int eplb_n;
   int32_t n[kMaxRanks];                  // local_num_tokens (0 for masked-off ranks)
   uint64_t live[kMaskWords];
+  int trigger;                           // 1 = let the next kernel launch at this one's start
+  int early;                             // vector path, 64..256 threads per token: load the
+                                         // first row vectors before routing the token
 };
 
 cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t stream, bool pdl);
@@ -139,6 +142,7 @@ struct CombineArgs {
   uint32_t* err;               // device error word (checked builds)
   int out32;                   // pipelined E4M3 combines: one 32-byte store per
                                // vector (output 32-byte aligned)
+  int trigger;                 // 1 = let the next kernel launch at this one's start
 };
 
 // pipe: the two-deep pipelined kernel (needs at most 8 destinations per token)
@@ -161,6 +165,7 @@ struct CombineExpertsArgs {
                                // grid strides ahead into L2
   int ep;
   uint32_t* err;               // device error word (checked builds)
+  int trigger;                 // 1 = let the next kernel launch at this one's start
 };
 
 cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, bool pipe, int threads,

@@ -392,7 +392,20 @@ typedef enum {
                                      through distributed shared memory; 1 = a cluster per
                                      token with one column vector per thread and the rows
                                      in registers (hidden up to 16384); 2 = one CTA per
-                                     token with the whole rows in shared memory */
+                                     token with the whole rows in shared memory */,
+  EP_A2A_OPT_PDL_TRIGGER = 19,    /* with PDL on: 1 = the copy and combine kernels also
+                                     let the next kernel of the stream launch as soon
+                                     as all their CTAs are running (griddepcontrol.
+                                     launch_dependents at their start), so its CTAs are
+                                     resident and waiting when they finish; 0 = only
+                                     the routing kernel does (the next kernel launches
+                                     when they end).  The next kernel still waits for
+                                     their completion before it touches memory, so
+                                     results do not change */
+  EP_A2A_OPT_COPY_EARLY_LOAD = 20 /* vector copy with 64..256 threads per token: 1 =
+                                     each token's first row vectors are loaded before
+                                     its destinations are worked out (the two loads
+                                     overlap); 0 = after */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

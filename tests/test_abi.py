@@ -32,6 +32,21 @@ def test_header_declares_the_entry_points():
         assert required in names
 
 
+def _header_enum(prefix):
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    return {m.group(1): int(m.group(2))
+            for m in re.finditer(rf"\b{prefix}([A-Z0-9_]+)\s*=\s*(-?\d+)", text)}
+
+
+def test_python_option_and_status_numbers_match_the_header(ep):
+    opts = _header_enum("EP_A2A_OPT_")
+    assert opts and sorted(opts.values()) == list(range(len(opts)))
+    for name, value in opts.items():
+        assert getattr(ep, "OPT_" + name) == value, name
+    for name, value in _header_enum("EP_A2A_ERR_").items():
+        assert getattr(ep, "ERR_" + name) == value, name
+
+
 def test_library_exports_every_declared_symbol(ep):
     lib = ctypes.CDLL(ep.LIB_PATH)
     missing = [n for n in _declared_functions() if not hasattr(lib, n)]
