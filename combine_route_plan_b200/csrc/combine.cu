@@ -300,6 +300,99 @@ __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
   }
 }
 
+// Item `it` of the flat combine: token tok = it / nvec, column vector v; its
+// destination count (-1: no output) and rows' loads, the row scales (scaled
+// mode) and the output address.  The token's plan comes from shared memory.
+template <int kMode>
+__device__ __forceinline__ void flat_item_load(const CombineArgs& a, const float* __restrict__ scales,
+                                               const int* s_nd, const uint64_t* s_w0, int64_t t0,
+                                               uint32_t nvec, int64_t rank_stride, uint32_t it,
+                                               uint4 (&r)[8], float (&sc)[8], int& nd,
+                                               uint16_t*& o) {
+  constexpr int kElems = kMode == kCombineBf16 ? 8 : 16;
+  constexpr int kElemBytes = kMode == kCombineBf16 ? 2 : 1;
+  const uint32_t tok = it / nvec;
+  const uint32_t v = it - tok * nvec;
+  const int rel = (int)((int64_t)tok - t0);
+  const int n = s_nd[rel];
+  const uint64_t w0 = s_w0[rel];
+  nd = n == kNoToken ? -1 : n;
+  o = a.out + (int64_t)tok * a.H + (int64_t)v * kElems;
+  const uint8_t* xt = a.x + ((int64_t)tok * a.H + (int64_t)v * kElems) * kElemBytes;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    sc[i] = 1.0f;
+    if (i < nd) {
+      const int d = (int)((w0 >> (8 * i)) & 0xFFu);
+      r[i] = ld_stream_v4(xt + (int64_t)d * rank_stride);
+      if (kMode == kCombineFp8Scaled) sc[i] = scales[(int64_t)d * a.ntok + tok];
+    }
+  }
+}
+
+// The combines for steps with few tokens per SM (at most 8 destinations per
+// token, 16-byte vectors): a persistent grid, every CTA resident from the
+// start, where CTA c takes the (token, column vector) items [c*I/G,
+// (c+1)*I/G) of all I = tokens x vectors items.  Every CTA has the same
+// number of items, so the SMs finish together instead of waiting on the last
+// tokens the hardware scheduler handed out; the CTA reads the plan rows of its
+// tokens into shared memory once; each thread walks its items (stride
+// blockDim) with the next item's row loads in flight while it sums the current
+// one.  The sums are those of combine_vec_kernel / combine_scaled_kernel.
+template <int kMode>
+__global__ void __launch_bounds__(256) combine_flat_kernel(const CombineArgs a,
+                                                           const float* __restrict__ scales,
+                                                           int max_tok) {
+  pdl_wait();
+  if (a.trigger) pdl_launch_dependents();
+  extern __shared__ __align__(8) uint8_t flat_mem[];
+  uint64_t* s_w0 = reinterpret_cast<uint64_t*>(flat_mem);
+  int* s_nd = reinterpret_cast<int*>(flat_mem + sizeof(uint64_t) * (size_t)max_tok);
+  constexpr int kElems = kMode == kCombineBf16 ? 8 : 16;
+  constexpr int kElemBytes = kMode == kCombineBf16 ? 2 : 1;
+  const uint32_t nvec = (uint32_t)(a.H / kElems);
+  const int64_t items = a.ntok * (int64_t)nvec;                  // < 2^31 (host)
+  const int64_t lo = items * blockIdx.x / gridDim.x;
+  const int64_t hi = items * (blockIdx.x + 1) / gridDim.x;
+  const int64_t t0 = lo / nvec;
+  const int nt = hi > lo ? (int)((hi - 1) / nvec - t0 + 1) : 0;  // <= max_tok (host)
+  for (int i = threadIdx.x; i < nt; i += blockDim.x) {
+    const int64_t tok = t0 + i;
+    int nd = a.plan_nd[tok];
+    const uint64_t w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
+    if (nd != kNoToken && (nd > 8 || !plan_row_ok(nd, w0, 0, 0, 0, a.ep, 8, a.err)))
+      nd = kNoToken;
+    s_nd[i] = nd;
+    s_w0[i] = w0;
+  }
+  __syncthreads();
+  const int64_t rank_stride = a.ntok * (int64_t)a.H * kElemBytes;
+  const bool wide = a.out32 != 0;
+  uint32_t it = (uint32_t)(lo + threadIdx.x);
+  if (it >= hi) return;
+  uint4 ra[8], rb[8];
+  float sca[8], scb[8];
+  int nda, ndb;
+  uint16_t *oa, *ob;
+  flat_item_load<kMode>(a, scales, s_nd, s_w0, t0, nvec, rank_stride, it, ra, sca, nda, oa);
+  for (;;) {
+    const uint32_t nb = it + blockDim.x;
+    const bool more_b = nb < hi;
+    if (more_b)
+      flat_item_load<kMode>(a, scales, s_nd, s_w0, t0, nvec, rank_stride, nb, rb, scb, ndb, ob);
+    if (nda >= 0) reduce_store<kMode>(ra, sca, nda, oa, wide);
+    if (!more_b) break;
+    it = nb;
+    const uint32_t na = it + blockDim.x;
+    const bool more_a = na < hi;
+    if (more_a)
+      flat_item_load<kMode>(a, scales, s_nd, s_w0, t0, nvec, rank_stride, na, ra, sca, nda, oa);
+    if (ndb >= 0) reduce_store<kMode>(rb, scb, ndb, ob, wide);
+    if (!more_a) break;
+    it = na;
+  }
+}
+
 // The combines with their rows staged in shared memory by bulk-async copies
 // (cp.async.bulk, completion counted on an mbarrier): a work item is one
 // chunk of kChunk bytes of a token's row; the producer warp's lane 0 loads the
@@ -1613,6 +1706,48 @@ cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, bool pipe, 
   }
   if (fp8) return launch_kernel(combine_scalar_kernel<true>, g, b, 0, stream, pdl, a);
   return launch_kernel(combine_scalar_kernel<false>, g, b, 0, stream, pdl, a);
+}
+
+namespace {
+template <int kMode>
+cudaError_t launch_flat_mode(const CombineArgs& a, const float* scales, int ctas_per_sm,
+                             int num_sms, cudaStream_t stream, bool pdl) {
+  constexpr int kThreads = 256;
+  constexpr int kElems = kMode == kCombineBf16 ? 8 : 16;
+  const int64_t nvec = a.H / kElems;
+  // every CTA resident at once: the grid is the SMs times the CTAs that fit
+  int fit = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+      &fit, combine_flat_kernel<kMode>, kThreads, 12 * 64);
+  if (e != cudaSuccess) return e;
+  const int cps = std::max(1, ctas_per_sm > 0 ? std::min(ctas_per_sm, fit) : fit);
+  const int64_t items = a.ntok * nvec;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(items, (int64_t)num_sms * cps));
+  const int max_tok = (int)((items / grid + 1) / nvec + 2);
+  const size_t smem = (size_t)max_tok * (sizeof(uint64_t) + sizeof(int));
+  if (smem > 48 * 1024) return cudaErrorInvalidValue;
+  return launch_kernel(combine_flat_kernel<kMode>, dim3(grid), dim3(kThreads), smem, stream, pdl,
+                       a, scales, max_tok);
+}
+}  // namespace
+
+bool combine_flat_ok(const CombineArgs& a, int elems) {
+  const int64_t nvec = a.H / elems;
+  return a.H % elems == 0 && a.ntok * nvec < ((int64_t)1 << 31);
+}
+
+cudaError_t launch_combine_flat(const CombineArgs& a, int mode, const float* scales,
+                                int ctas_per_sm, int num_sms, cudaStream_t stream, bool pdl) {
+  switch (mode) {
+    case kCombineBf16:
+      return launch_flat_mode<kCombineBf16>(a, scales, ctas_per_sm, num_sms, stream, pdl);
+    case kCombineFp8:
+      return launch_flat_mode<kCombineFp8>(a, scales, ctas_per_sm, num_sms, stream, pdl);
+    case kCombineFp8Scaled:
+      return launch_flat_mode<kCombineFp8Scaled>(a, scales, ctas_per_sm, num_sms, stream, pdl);
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_combine_staged(const CombineArgs& a, int mode, const float* scales,

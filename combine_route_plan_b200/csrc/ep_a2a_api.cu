@@ -150,6 +150,7 @@ struct ep_a2a_handle_s {
   int fp8_experts_kernel;   // sender-side FP8 expert combine: 0 split, 1 cluster, 2 one CTA
   int pdl_trigger;          // copy and combines trigger the next launch at their start
   int copy_early_load;      // vector copy: first row vectors loaded before routing
+  int combine_flat;         // -1 auto, 0 off, 1 on: balanced persistent combine
   int copy_stages;        // 0 = choose from the row size
   int combine_threads;
   int64_t bulk_min_row;   // rows below this go to the vector copy
@@ -216,6 +217,7 @@ enum CombineKind { kKindBf16, kKindFp8, kKindExperts };
 
 struct CombineLaunch {
   bool pipe;
+  bool flat;                 // balanced persistent grid (BF16 / FP8 / scaled FP8)
   bool staged;               // rows staged in shared memory by bulk-async copies
   int threads, grid, prefetch;
   int staged_ctas_per_sm;
@@ -242,6 +244,8 @@ CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
   CombineLaunch c;
   c.pipe = fits && (h->combine_pipeline < 0 ? kind != kKindBf16 : h->combine_pipeline == 1);
   c.staged = fits && h->combine_pipeline == 2;
+  c.flat = fits && kind != kKindExperts && !c.staged &&
+           (h->combine_flat < 0 ? false : h->combine_flat == 1);
   // a staged CTA needs two stages of 32 KB: at most three CTAs per SM
   c.staged_ctas_per_sm = h->combine_ctas_per_sm > 0 ? std::min(h->combine_ctas_per_sm, 3) : 2;
   const bool mid = !big && ntok >= 8192;
@@ -385,6 +389,7 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   h->fp8_experts_kernel = 0;
   h->pdl_trigger = 0;
   h->copy_early_load = 0;
+  h->combine_flat = -1;
   h->copy_stages = 4;
   h->combine_threads = 0;
   h->bulk_min_row = 0;
@@ -492,6 +497,10 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
     case EP_A2A_OPT_COPY_EARLY_LOAD:
       if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "early load must be 0 or 1");
       h->copy_early_load = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_COMBINE_FLAT:
+      if (value < -1 || value > 1) return fail(EP_A2A_ERR_INVALID_ARG, "flat combine must be -1, 0 or 1");
+      h->combine_flat = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_ROUTE_IN_COPY:
       if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "route in copy must be 0 or 1");
@@ -756,6 +765,9 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
     e = launch_combine_staged(a, fp8 ? 1 : 0, nullptr, h->num_sms * c.staged_ctas_per_sm,
                               c.staged_ctas_per_sm, h->max_smem_optin, (cudaStream_t)stream_v,
                               h->pdl != 0);
+  else if (vec && c.flat && combine_flat_ok(a, elems))
+    e = launch_combine_flat(a, fp8 ? 1 : 0, nullptr, h->combine_ctas_per_sm, h->num_sms,
+                            (cudaStream_t)stream_v, h->pdl != 0);
   else
     e = launch_combine(a, fp8, vec, c.pipe, c.threads, c.grid, (cudaStream_t)stream_v,
                        h->pdl != 0);
@@ -930,6 +942,9 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
     e = launch_combine_staged(a, 2, row_scales, h->num_sms * c.staged_ctas_per_sm,
                               c.staged_ctas_per_sm, h->max_smem_optin, (cudaStream_t)stream_v,
                               h->pdl != 0);
+  else if (vec && c.flat && combine_flat_ok(a, 16))
+    e = launch_combine_flat(a, 2, row_scales, h->combine_ctas_per_sm, h->num_sms,
+                            (cudaStream_t)stream_v, h->pdl != 0);
   else
     e = launch_combine_scaled(a, row_scales, vec, c.pipe, c.threads, c.grid,
                               (cudaStream_t)stream_v, h->pdl != 0);

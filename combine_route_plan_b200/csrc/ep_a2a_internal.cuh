@@ -202,6 +202,13 @@ cudaError_t launch_quantize_e4m3_rows(const uint16_t* in, uint8_t* out, float* s
 cudaError_t launch_combine_staged(const CombineArgs& a, int mode, const float* scales,
                                   int grid, int ctas_per_sm, int max_smem, cudaStream_t stream,
                                   bool pdl);
+// The BF16 (mode 0), FP8 (1) or scaled FP8 (2) combine on a persistent grid of
+// num_sms x min(ctas_per_sm, what fits) CTAs (0: what fits), each summing an
+// equal share of the (token, column vector) items; at most 8 destinations per
+// token, 16-byte vectors, combine_flat_ok(a, elements per vector).
+bool combine_flat_ok(const CombineArgs& a, int elems);
+cudaError_t launch_combine_flat(const CombineArgs& a, int mode, const float* scales,
+                                int ctas_per_sm, int num_sms, cudaStream_t stream, bool pdl);
 // FP8 combine with one fp32 scale per row (scales [ep, ep*tpr]).
 cudaError_t launch_combine_scaled(const CombineArgs& a, const float* scales, bool vec, bool pipe,
                                   int threads, int grid, cudaStream_t stream, bool pdl);

@@ -402,10 +402,17 @@ typedef enum {
                                      when they end).  The next kernel still waits for
                                      their completion before it touches memory, so
                                      results do not change */
-  EP_A2A_OPT_COPY_EARLY_LOAD = 20 /* vector copy with 64..256 threads per token: 1 =
+  EP_A2A_OPT_COPY_EARLY_LOAD = 20,/* vector copy with 64..256 threads per token: 1 =
                                      each token's first row vectors are loaded before
                                      its destinations are worked out (the two loads
                                      overlap); 0 = after */
+  EP_A2A_OPT_COMBINE_FLAT = 21    /* BF16 / FP8 / scaled FP8 combines of 16-byte vectors
+                                     with at most 8 destinations per token: 1 = a
+                                     persistent grid (every CTA resident) in which each
+                                     CTA sums an equal share of the (token, column
+                                     vector) items, so all SMs finish together; 0 = one
+                                     token per CTA at a time, as the hardware hands
+                                     CTAs out; -1 (default) = automatic */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

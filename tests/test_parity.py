@@ -438,6 +438,31 @@ def test_pipelined_combines_match_the_oracle(case, prefetch, threads):
     """BF16, FP8, scaled-FP8 and expert-output combines with the two-deep
     pipelined kernels."""
     from combine_route_plan_b200 import ep_a2a
+    _check_all_combines(case, {ep_a2a.OPT_COMBINE_PIPELINE: 1, ep_a2a.OPT_COMBINE_PREFETCH: prefetch,
+                               ep_a2a.OPT_COMBINE_THREADS: threads})
+
+
+@pytest.mark.parametrize("case", [
+    ("c2_ep8_decode", None),
+    ("c5_ep64_wide_masked", None),
+    ("c1_ep4_tiny", None),
+    ("c3_ep16_zipf_nvfp4", None),
+    ("mask", [0b10100101, 0, 0, 0]),
+    ("odd", None),
+    ("wide_k", None),
+])
+@pytest.mark.parametrize("ctas", [0, 1])
+def test_flat_combines_match_the_oracle(case, ctas):
+    """BF16, FP8 and scaled-FP8 combines on the balanced persistent grid (each
+    CTA an equal share of the (token, vector) items; shares that start and end
+    inside a token), next to the expert-output combine."""
+    from combine_route_plan_b200 import ep_a2a
+    _check_all_combines(case, {ep_a2a.OPT_COMBINE_FLAT: 1, ep_a2a.OPT_COMBINE_CTAS_PER_SM: ctas,
+                               ep_a2a.OPT_PDL_TRIGGER: 1})
+
+
+def _check_all_combines(case, opts):
+    from combine_route_plan_b200 import ep_a2a
     name, mask = case
     if name in W.BY_NAME:
         w = W.BY_NAME[name]
@@ -448,8 +473,6 @@ def test_pipelined_combines_match_the_oracle(case, prefetch, threads):
         w, x = _custom(4, 16, 4, 30, 40, [32], seed=19)
     else:
         w, x = _custom(16, 64, 16, 20, 64, [32], seed=23)
-    opts = {ep_a2a.OPT_COMBINE_PIPELINE: 1, ep_a2a.OPT_COMBINE_PREFETCH: prefetch,
-            ep_a2a.OPT_COMBINE_THREADS: threads}
     run = U.Run(w, W.Inputs(w, x.token_selected_experts, x.local_num_tokens, x.payloads,
                             x.eplb_local_stats, x.active_rank_mask, None), options=opts)
     plan = U.oracle_plan(w, x)
