@@ -124,8 +124,15 @@ __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
   if (a.prefetch && threadIdx.x == 0)
     for (int p = 0; p < a.prefetch; ++p)
       prefetch_token_rows<kElemBytes>(a, blockIdx.x + (int64_t)p * gridDim.x);
-  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
-    if (a.prefetch && threadIdx.x == 0)
+  // a work item is one of a.split column ranges of a token's row (the whole
+  // row when split is 1)
+  const int split = a.split > 1 ? a.split : 1;
+  for (int64_t item = blockIdx.x; item < a.ntok * split; item += gridDim.x) {
+    const int64_t tok = split == 1 ? item : item / split;
+    const int part = (int)(item - tok * split);
+    const int vbeg = (int)((int64_t)nvec * part / split);
+    const int vend = (int)((int64_t)nvec * (part + 1) / split);
+    if (split == 1 && a.prefetch && threadIdx.x == 0)
       prefetch_token_rows<kElemBytes>(a, tok + (int64_t)a.prefetch * gridDim.x);
     const int nd = a.plan_nd[tok];
     if (nd == kNoToken) continue;
@@ -138,7 +145,7 @@ __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
     const uint8_t* xt = a.x + tok * (int64_t)a.H * kElemBytes;           // rank 0's row
     const int64_t rank_stride = a.ntok * (int64_t)a.H * kElemBytes;      // bytes per rank
     uint16_t* out = a.out + tok * (int64_t)a.H;
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+    for (int v = vbeg + (int)threadIdx.x; v < vend; v += blockDim.x) {
       float acc[kElems];
 #pragma unroll
       for (int e = 0; e < kElems; ++e) acc[e] = 0.0f;
@@ -259,14 +266,20 @@ __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
   if (a.prefetch && threadIdx.x == 0)
     for (int p = 0; p < a.prefetch; ++p)
       prefetch_token_rows<kElemBytes>(a, blockIdx.x + (int64_t)p * gridDim.x);
-  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
-    if (a.prefetch && threadIdx.x == 0)
+  const int split = a.split > 1 ? a.split : 1;
+  for (int64_t item = blockIdx.x; item < a.ntok * split; item += gridDim.x) {
+    const int64_t tok = split == 1 ? item : item / split;
+    const int part = (int)(item - tok * split);
+    const int vbeg = (int)((int64_t)nvec * part / split);
+    const int nv = (int)((int64_t)nvec * (part + 1) / split) - vbeg;   // vectors of the item
+    if (split == 1 && a.prefetch && threadIdx.x == 0)
       prefetch_token_rows<kElemBytes>(a, tok + (int64_t)a.prefetch * gridDim.x);
     const int nd = a.plan_nd[tok];
-    if (nd == kNoToken || (int)threadIdx.x >= nvec) continue;
+    if (nd == kNoToken || (int)threadIdx.x >= nv) continue;
     const uint64_t w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
     if (!plan_row_ok(nd, w0, 0, 0, 0, a.ep, 8, a.err)) continue;
-    const uint8_t* xt = a.x + tok * (int64_t)a.H * kElemBytes + (int64_t)threadIdx.x * 16;
+    const uint8_t* xt =
+        a.x + tok * (int64_t)a.H * kElemBytes + ((int64_t)vbeg + threadIdx.x) * 16;
     const uint8_t* src[8];
     float sc[8];
 #pragma unroll
@@ -276,20 +289,20 @@ __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
       sc[i] = 1.0f;
       if (kMode == kCombineFp8Scaled && i < nd) sc[i] = scales[(int64_t)d * a.ntok + tok];
     }
-    uint16_t* o = a.out + tok * (int64_t)a.H + (int64_t)threadIdx.x * kElems;
+    uint16_t* o = a.out + tok * (int64_t)a.H + ((int64_t)vbeg + threadIdx.x) * kElems;
     const int64_t ostep = (int64_t)blockDim.x * kElems;
     uint4 ra[8], rb[8];
     load_rows(ra, src, nd, 0);
     int64_t off = 0;
     for (int v = threadIdx.x;;) {
-      const bool more_b = v + (int)blockDim.x < nvec;
+      const bool more_b = v + (int)blockDim.x < nv;
       if (more_b) load_rows(rb, src, nd, off + step);
       reduce_store<kMode>(ra, sc, nd, o, a.out32 != 0);
       if (!more_b) break;
       v += blockDim.x;
       off += step;
       o += ostep;
-      const bool more_a = v + (int)blockDim.x < nvec;
+      const bool more_a = v + (int)blockDim.x < nv;
       if (more_a) load_rows(ra, src, nd, off + step);
       reduce_store<kMode>(rb, sc, nd, o, a.out32 != 0);
       if (!more_a) break;

@@ -151,6 +151,9 @@ struct ep_a2a_handle_s {
   int pdl_trigger;          // copy and combines trigger the next launch at their start
   int copy_early_load;      // vector copy: first row vectors loaded before routing
   int combine_flat;         // -1 auto, 0 off, 1 on: balanced persistent combine
+  int copy_flat;            // -1 auto, 0 off, 1 on: balanced persistent vector copy
+  int combine_split;        // vector combines: column ranges per token
+  int copy_split;           // vector copy: column ranges per token
   int copy_stages;        // 0 = choose from the row size
   int combine_threads;
   int64_t bulk_min_row;   // rows below this go to the vector copy
@@ -218,6 +221,7 @@ enum CombineKind { kKindBf16, kKindFp8, kKindExperts };
 struct CombineLaunch {
   bool pipe;
   bool flat;                 // balanced persistent grid (BF16 / FP8 / scaled FP8)
+  int split;                 // column ranges per token (BF16 / FP8 / scaled FP8)
   bool staged;               // rows staged in shared memory by bulk-async copies
   int threads, grid, prefetch;
   int staged_ctas_per_sm;
@@ -261,8 +265,9 @@ CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
   }
   c.threads = h->combine_threads > 0 ? h->combine_threads : threads;
   if (h->combine_ctas_per_sm > 0) cps = h->combine_ctas_per_sm;
-  c.grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntok, (int64_t)h->num_sms * cps));
-  c.prefetch = h->combine_prefetch >= 0 ? h->combine_prefetch : prefetch;
+  c.split = kind == kKindExperts ? 1 : h->combine_split;
+  c.grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntok * c.split, (int64_t)h->num_sms * cps));
+  c.prefetch = c.split > 1 ? 0 : (h->combine_prefetch >= 0 ? h->combine_prefetch : prefetch);
   return c;
 }
 
@@ -390,6 +395,9 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   h->pdl_trigger = 0;
   h->copy_early_load = 0;
   h->combine_flat = -1;
+  h->copy_flat = -1;
+  h->combine_split = 1;
+  h->copy_split = 1;
   h->copy_stages = 4;
   h->combine_threads = 0;
   h->bulk_min_row = 0;
@@ -501,6 +509,18 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
     case EP_A2A_OPT_COMBINE_FLAT:
       if (value < -1 || value > 1) return fail(EP_A2A_ERR_INVALID_ARG, "flat combine must be -1, 0 or 1");
       h->combine_flat = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_COPY_FLAT:
+      if (value < -1 || value > 1) return fail(EP_A2A_ERR_INVALID_ARG, "flat copy must be -1, 0 or 1");
+      h->copy_flat = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_COMBINE_SPLIT:
+      if (value < 1 || value > 8) return fail(EP_A2A_ERR_INVALID_ARG, "combine split must be 1..8");
+      h->combine_split = (int)value;
+      return EP_A2A_OK;
+    case EP_A2A_OPT_COPY_SPLIT:
+      if (value < 1 || value > 8) return fail(EP_A2A_ERR_INVALID_ARG, "copy split must be 1..8");
+      h->copy_split = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_ROUTE_IN_COPY:
       if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "route in copy must be 0 or 1");
@@ -705,12 +725,20 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
     const int tpt = h->vec_threads_per_token > 0 ? h->vec_threads_per_token
                                                  : copy_threads_per_token(ntok, row_vectors);
     const int64_t groups_per_cta = 256 / tpt;
+    vec.split = (fused || tpt == 32) ? 1 : h->copy_split;
+    const int64_t items = ntok * vec.split;
     const int grid = (int)std::max<int64_t>(
-        1, std::min<int64_t>((ntok + groups_per_cta - 1) / groups_per_cta,
+        1, std::min<int64_t>((items + groups_per_cta - 1) / groups_per_cta,
                              (int64_t)h->num_sms * h->vec_ctas_per_sm));
     const int unroll = h->vec_unroll > 0 ? h->vec_unroll : copy_unroll(row_vectors, tpt);
+    const bool flat = !fused && (h->copy_flat < 0 ? false : h->copy_flat == 1) &&
+                      dispatch_flat_ok(vec);
     slot = prof_begin(h, EP_A2A_KERNEL_COPY_VEC, stream);
-    e = launch_dispatch_vec(vec, grid, unroll, tpt, h->store_streaming != 0, stream, pdl);
+    if (flat)
+      e = launch_dispatch_flat(vec, 0, h->num_sms,
+                               h->store_streaming != 0, stream, pdl);
+    else
+      e = launch_dispatch_vec(vec, grid, unroll, tpt, h->store_streaming != 0, stream, pdl);
     prof_end(h, slot, stream);
     if (e != cudaSuccess) return cuda_fail(e, "vector copy kernel launch");
   }
@@ -756,6 +784,7 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   a.trigger = h->pdl != 0 && h->pdl_trigger != 0;
   const CombineLaunch c = combine_launch(h, fp8 ? kKindFp8 : kKindBf16, a.ntok);
   a.prefetch = c.prefetch;
+  a.split = c.split;
   a.out32 = aligned(output, 32) ? 1 : 0;
   const int elems = fp8 ? 16 : 8;
   const bool vec = a.H % elems == 0 && aligned(expert_output, 16) && aligned(output, 16);
@@ -934,6 +963,7 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
   a.trigger = h->pdl != 0 && h->pdl_trigger != 0;
   const CombineLaunch c = combine_launch(h, kKindFp8, a.ntok);
   a.prefetch = c.prefetch;
+  a.split = c.split;
   a.out32 = aligned(output, 32) ? 1 : 0;
   const bool vec = a.H % 16 == 0 && aligned(expert_output_e4m3, 16) && aligned(output, 16);
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);

@@ -113,6 +113,8 @@ struct CopyArgs {
   int32_t n[kMaxRanks];                  // local_num_tokens (0 for masked-off ranks)
   uint64_t live[kMaskWords];
   int trigger;                           // 1 = let the next kernel launch at this one's start
+  int split;                             // vector path without routing: column ranges per
+                                         // token row (work items)
   int early;                             // vector path, 64..256 threads per token: load the
                                          // first row vectors before routing the token
 };
@@ -124,6 +126,13 @@ constexpr int kStagedMaxVec = 8;         // 16-byte vectors per consumer thread 
 cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, int unroll, int threads_per_token,
                                 bool streaming, cudaStream_t stream, bool pdl);
 int bulk_queue_depth(int stages);        // groups allowed in flight for `stages`
+// The vector copy on a persistent grid of num_sms x min(ctas_per_sm, what
+// fits) CTAs (0: what fits), each copying an equal share of the (token,
+// vector) items; every payload row with the same vector width (16 or 32
+// bytes), no routing in the copy (dispatch_flat_ok).
+bool dispatch_flat_ok(const CopyArgs& a);
+cudaError_t launch_dispatch_flat(const CopyArgs& a, int ctas_per_sm, int num_sms, bool streaming,
+                                 cudaStream_t stream, bool pdl);
 
 // ---------------------------------------------------------------------------
 // Combine and the E4M3 helper
@@ -143,6 +152,7 @@ struct CombineArgs {
   int out32;                   // pipelined E4M3 combines: one 32-byte store per
                                // vector (output 32-byte aligned)
   int trigger;                 // 1 = let the next kernel launch at this one's start
+  int split;                   // vector kernels: column ranges per token (work items)
 };
 
 // pipe: the two-deep pipelined kernel (needs at most 8 destinations per token)

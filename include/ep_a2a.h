@@ -412,7 +412,20 @@ typedef enum {
                                      CTA sums an equal share of the (token, column
                                      vector) items, so all SMs finish together; 0 = one
                                      token per CTA at a time, as the hardware hands
-                                     CTAs out; -1 (default) = automatic */
+                                     CTAs out; -1 (default) = automatic */,
+  EP_A2A_OPT_COPY_FLAT = 22       /* vector copy (no routing in the copy) whose payload
+                                     rows all use the same vector width: 1 = a
+                                     persistent grid in which each CTA copies an equal
+                                     share of the (token, vector) items; 0 = token groups
+                                     as the hardware hands CTAs out; -1 (default) =
+                                     automatic */,
+  EP_A2A_OPT_COMBINE_SPLIT = 23,  /* BF16 / FP8 / scaled FP8 vector combines: each
+                                     token's row is summed as this many column ranges,
+                                     each its own work item (1..8; default 1) */
+  EP_A2A_OPT_COPY_SPLIT = 24      /* vector copy with more than 32 threads per token
+                                     and no routing in the copy: each token's rows are
+                                     copied as this many column ranges, each its own
+                                     work item (1..8; default 1) */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

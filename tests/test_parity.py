@@ -461,6 +461,43 @@ def test_flat_combines_match_the_oracle(case, ctas):
                                ep_a2a.OPT_PDL_TRIGGER: 1})
 
 
+@pytest.mark.parametrize("case", [
+    ("c2_ep8_decode", None),
+    ("c5_ep64_wide_masked", None),
+    ("c1_ep4_tiny", None),
+    ("mask", [0b10100101, 0, 0, 0]),
+    ("odd", None),
+])
+@pytest.mark.parametrize("split", [2, 3, 8])
+def test_split_rows_match_the_oracle(case, split):
+    """Combines and the copy with each token's row taken as `split` column
+    ranges (work items), including ranges with no vectors (hidden 40)."""
+    from combine_route_plan_b200 import ep_a2a
+    opts = {ep_a2a.OPT_COMBINE_SPLIT: split, ep_a2a.OPT_COPY_SPLIT: split}
+    for pipe in (0, 1):
+        _check_all_combines(case, dict(opts, **{ep_a2a.OPT_COMBINE_PIPELINE: pipe}))
+    name = case[0]
+    if name in W.BY_NAME:
+        _full_check(W.BY_NAME[name], options=dict(opts, **{ep_a2a.OPT_VEC_THREADS_PER_TOKEN: 256}))
+
+
+@pytest.mark.parametrize("tpt", [64, 128, 256])
+@pytest.mark.parametrize("split", [2, 5])
+def test_split_copy_rows_and_payloads(tpt, split):
+    """The copy's column ranges over payload rows of different widths (some
+    shorter than the range count), ragged token counts and a masked rank."""
+    from combine_route_plan_b200 import ep_a2a
+    ep, E, k, tpr, H = 8, 64, 8, 37, 32
+    rows = [14336, 64, 16, 4]
+    w, x = _custom(ep, E, k, tpr, H, rows, n=[37, 0, 36, 5, 37, 1, 30, 37],
+                   mask=_mask_of(ep, [0, 1, 2, 4, 5, 6, 7]), seed=tpt + split)
+    run = U.Run(w, x, copy_path=1, options={ep_a2a.OPT_COPY_SPLIT: split,
+                                            ep_a2a.OPT_VEC_THREADS_PER_TOKEN: tpt})
+    plan = U.oracle_plan(w, x)
+    U.check_plan(run, plan, w)
+    U.check_payloads(run, plan, w, x)
+
+
 def _check_all_combines(case, opts):
     from combine_route_plan_b200 import ep_a2a
     name, mask = case
