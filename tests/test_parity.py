@@ -498,6 +498,44 @@ def test_split_copy_rows_and_payloads(tpt, split):
     U.check_payloads(run, plan, w, x)
 
 
+@pytest.mark.parametrize("name", ["c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked",
+                                  "c3_ep16_zipf_nvfp4"])
+def test_flat_copy_bit_exact(name):
+    """The vector copy on the balanced persistent grid (equal shares of the
+    (token, vector) items, routed per CTA into shared memory)."""
+    from combine_route_plan_b200 import ep_a2a
+    _full_check(W.BY_NAME[name], options={ep_a2a.OPT_COPY_FLAT: 1})
+
+
+@pytest.mark.parametrize("rows,shift", [([14336, 64, 32], 0), ([4096 + 16, 48, 16], 0),
+                                        ([14336, 32], 16)])
+def test_flat_copy_rows(rows, shift):
+    """Several payload rows per item range, 16- and 32-byte vectors, ragged
+    token counts and a masked rank."""
+    from combine_route_plan_b200 import ep_a2a
+    ep, E, k, tpr, H = 8, 64, 8, 45, 32
+    w, x = _custom(ep, E, k, tpr, H, rows, n=[45, 44, 0, 3, 45, 17, 45, 9],
+                   mask=_mask_of(ep, [0, 1, 2, 3, 5, 6, 7]), seed=sum(rows) % 101 + shift)
+    comm = ep_a2a.EpA2A(ep, E, k, tpr, H, rows, enable_rank_mask=True, workspace_fill=U.CANARY)
+    comm.set_option(ep_a2a.OPT_COPY_FLAT, 1)
+    srcs = []
+    for p in x.payloads:
+        buf = torch.empty(p.numel() + 64, dtype=torch.uint8, device="cuda")
+        v = buf[shift: shift + p.numel()].view(p.shape)
+        v.copy_(p.cuda())
+        srcs.append(v)
+    d = comm.dispatch(x.token_selected_experts.cuda(), x.local_num_tokens, srcs, tpr,
+                      active_rank_mask=x.active_rank_mask)
+    torch.cuda.synchronize()
+    assert comm.get_status() == ep_a2a.OK
+    plan = U.oracle_plan(w, x)
+    for i, p in enumerate(x.payloads):
+        for dst in range(ep):
+            want = U.oracle.dispatch_payload(plan, p.numpy(), only_dst=dst, recv_init=np.full(
+                (1, ep * tpr, p.shape[2]), U.CANARY, np.uint8))
+            U.assert_equal(d.recv_payloads[i][dst], want, f"payload {i} rank {dst}")
+
+
 def _check_all_combines(case, opts):
     from combine_route_plan_b200 import ep_a2a
     name, mask = case
