@@ -85,10 +85,49 @@ __device__ __forceinline__ void add_e4m3x16(float* acc, const uint4& v) {
   }
 }
 
+// Two fp32 values in one 64-bit register, for sm_100's packed fp32 arithmetic
+// (fma.rn.f32x2, mul.rn.f32x2): each lane is rounded as by the scalar
+// instruction, so a packed operation gives the same two results as two scalar
+// ones with one instruction.
+__device__ __forceinline__ uint64_t f32x2_of(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f32x2_parts(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// The two bf16 of w (lo in the low half), widened exactly, as a packed pair.
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+  return f32x2_of(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// a * b + c lane by lane, one rounding per lane.
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// a * b lane by lane, one rounding per lane.
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 // Two fp32 -> packed bf16x2 (lo in the low half), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(uint64_t pair) {
+  float lo, hi;
+  f32x2_parts(pair, lo, hi);
+  return pack_bf16x2(lo, hi);
 }
 
 // Thread 0 asks for the rows of token `tok` (if it exists) to be brought into
@@ -725,22 +764,20 @@ __device__ __forceinline__ void expert_rows_reduce_store(const uint4 (&raw)[8],
   for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
   for (int q = 0; q < nd; ++q) {
     const int d = (int)((w0 >> (8 * q)) & 0xFFu);
-    float z[8];
+    uint64_t z[4];                        // z_d's 8 values as packed pairs
 #pragma unroll
-    for (int e = 0; e < 8; ++e) z[e] = 0.0f;
+    for (int e = 0; e < 4; ++e) z[e] = 0ull;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (own[j] != d) continue;
+      const uint64_t w2 = f32x2_of(wt[j], wt[j]);
       const uint32_t wv[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        z[2 * i] = __fmaf_rn(wt[j], bf16_bits_to_f32(wv[i] & 0xFFFFu), z[2 * i]);
-        z[2 * i + 1] = __fmaf_rn(wt[j], bf16_bits_to_f32(wv[i] >> 16), z[2 * i + 1]);
-      }
+      for (int i = 0; i < 4; ++i) z[i] = fma_f32x2(w2, bf16x2_to_f32x2(wv[i]), z[i]);
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e)           // z_d to bf16 in pairs, then added exactly widened
-      add_bf16x2(acc[2 * e], acc[2 * e + 1], pack_bf16x2(z[2 * e], z[2 * e + 1]));
+      add_bf16x2(acc[2 * e], acc[2 * e + 1], pack_bf16x2(z[e]));
   }
   uint4 pk;
   pk.x = pack_bf16x2(acc[0], acc[1]);
@@ -821,17 +858,20 @@ __global__ void __launch_bounds__(512) combine_experts_pipe_kernel(const Combine
 __device__ __forceinline__ void fp8_roundtrip_acc(float* acc, const uint4& zb, float inv,
                                                   float scale) {
   const uint32_t w[4] = {zb.x, zb.y, zb.z, zb.w};
+  const uint64_t inv2 = f32x2_of(inv, inv);
+  const uint64_t scale2 = f32x2_of(scale, scale);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float2 f = make_float2(__fmul_rn(bf16_bits_to_f32(w[i] & 0xFFFFu), inv),
-                                 __fmul_rn(bf16_bits_to_f32(w[i] >> 16), inv));
+    float2 f;
+    f32x2_parts(mul_f32x2(bf16x2_to_f32x2(w[i]), inv2), f.x, f.y);
     const __nv_fp8x2_storage_t code = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
     const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(code, __NV_E4M3);
     __half_raw lo, hi;
     lo.x = hr.x;
     hi.x = hr.y;
-    acc[2 * i] = __fmaf_rn(__half2float(__half(lo)), scale, acc[2 * i]);
-    acc[2 * i + 1] = __fmaf_rn(__half2float(__half(hi)), scale, acc[2 * i + 1]);
+    const uint64_t dec = f32x2_of(__half2float(__half(lo)), __half2float(__half(hi)));
+    const uint64_t r = fma_f32x2(dec, scale2, f32x2_of(acc[2 * i], acc[2 * i + 1]));
+    f32x2_parts(r, acc[2 * i], acc[2 * i + 1]);
   }
 }
 
@@ -1207,26 +1247,24 @@ __global__ void __launch_bounds__(256, 3) combine_experts_fp8_split_kernel(
 #pragma unroll
       for (int p = 0; p < 8; ++p)
         if (p < ns && has) raw[p] = ld_stream_v4(yt + (int64_t)slot[p] * a.H + (int64_t)v * 8);
-      float z[8];
+      uint64_t z[4];                                  // packed pairs
 #pragma unroll
-      for (int e = 0; e < 8; ++e) z[e] = 0.0f;
+      for (int e = 0; e < 4; ++e) z[e] = 0ull;
       int q = 0;
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
         if (p >= ns) break;
         if (has) {
+          const uint64_t w2 = f32x2_of(wt[p], wt[p]);
           const uint32_t wv[4] = {raw[p].x, raw[p].y, raw[p].z, raw[p].w};
 #pragma unroll
-          for (int k2 = 0; k2 < 4; ++k2) {
-            z[2 * k2] = __fmaf_rn(wt[p], bf16_bits_to_f32(wv[k2] & 0xFFFFu), z[2 * k2]);
-            z[2 * k2 + 1] = __fmaf_rn(wt[p], bf16_bits_to_f32(wv[k2] >> 16), z[2 * k2 + 1]);
-          }
+          for (int k2 = 0; k2 < 4; ++k2) z[k2] = fma_f32x2(w2, bf16x2_to_f32x2(wv[k2]), z[k2]);
         }
         if ((int)((endw >> (4 * q)) & 0xFu) == p + 1) {   // destination q's slots end here
           uint32_t m = 0u;
           if (has) {
-            const uint32_t pk0 = pack_bf16x2(z[0], z[1]), pk1 = pack_bf16x2(z[2], z[3]);
-            const uint32_t pk2 = pack_bf16x2(z[4], z[5]), pk3 = pack_bf16x2(z[6], z[7]);
+            const uint32_t pk0 = pack_bf16x2(z[0]), pk1 = pack_bf16x2(z[1]);
+            const uint32_t pk2 = pack_bf16x2(z[2]), pk3 = pack_bf16x2(z[3]);
             *reinterpret_cast<uint4*>(zs + (int64_t)q * cols + (int64_t)i * 8) =
                 make_uint4(pk0, pk1, pk2, pk3);
             const uint32_t mm = max_u16x2(max_u16x2(pk0 & 0x7FFF7FFFu, pk1 & 0x7FFF7FFFu),
@@ -1236,7 +1274,7 @@ __global__ void __launch_bounds__(256, 3) combine_experts_fp8_split_kernel(
           m = __reduce_max_sync(0xFFFFFFFFu, m);
           if (lane == 0) atomicMax(&s_amax[parity][q], m);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) z[e] = 0.0f;
+          for (int e = 0; e < 4; ++e) z[e] = 0ull;
           ++q;
         }
       }

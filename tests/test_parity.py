@@ -475,10 +475,10 @@ def test_split_rows_match_the_oracle(case, split):
     from combine_route_plan_b200 import ep_a2a
     opts = {ep_a2a.OPT_COMBINE_SPLIT: split, ep_a2a.OPT_COPY_SPLIT: split}
     for pipe in (0, 1):
-        _check_all_combines(case, dict(opts, **{ep_a2a.OPT_COMBINE_PIPELINE: pipe}))
+        _check_all_combines(case, {**opts, ep_a2a.OPT_COMBINE_PIPELINE: pipe})
     name = case[0]
     if name in W.BY_NAME:
-        _full_check(W.BY_NAME[name], options=dict(opts, **{ep_a2a.OPT_VEC_THREADS_PER_TOKEN: 256}))
+        _full_check(W.BY_NAME[name], options={**opts, ep_a2a.OPT_VEC_THREADS_PER_TOKEN: 256})
 
 
 @pytest.mark.parametrize("tpt", [64, 128, 256])
