@@ -85,49 +85,10 @@ __device__ __forceinline__ void add_e4m3x16(float* acc, const uint4& v) {
   }
 }
 
-// Two fp32 values in one 64-bit register, for sm_100's packed fp32 arithmetic
-// (fma.rn.f32x2, mul.rn.f32x2): each lane is rounded as by the scalar
-// instruction, so a packed operation gives the same two results as two scalar
-// ones with one instruction.
-__device__ __forceinline__ uint64_t f32x2_of(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-
-__device__ __forceinline__ void f32x2_parts(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-
-// The two bf16 of w (lo in the low half), widened exactly, as a packed pair.
-__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
-  return f32x2_of(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-}
-
-// a * b + c lane by lane, one rounding per lane.
-__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-
-// a * b lane by lane, one rounding per lane.
-__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
 // Two fp32 -> packed bf16x2 (lo in the low half), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&p);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(uint64_t pair) {
-  float lo, hi;
-  f32x2_parts(pair, lo, hi);
-  return pack_bf16x2(lo, hi);
 }
 
 // Thread 0 asks for the rows of token `tok` (if it exists) to be brought into
@@ -155,7 +116,6 @@ __device__ __forceinline__ void prefetch_token_rows(const CombineArgs& a, int64_
 template <bool kFp8>
 __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   constexpr int kElems = kFp8 ? 16 : 8;       // elements per 16-byte input vector
   constexpr int kElemBytes = kFp8 ? 1 : 2;
   const int nvec = a.H / kElems;
@@ -163,15 +123,8 @@ __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
   if (a.prefetch && threadIdx.x == 0)
     for (int p = 0; p < a.prefetch; ++p)
       prefetch_token_rows<kElemBytes>(a, blockIdx.x + (int64_t)p * gridDim.x);
-  // a work item is one of a.split column ranges of a token's row (the whole
-  // row when split is 1)
-  const int split = a.split > 1 ? a.split : 1;
-  for (int64_t item = blockIdx.x; item < a.ntok * split; item += gridDim.x) {
-    const int64_t tok = split == 1 ? item : item / split;
-    const int part = (int)(item - tok * split);
-    const int vbeg = (int)((int64_t)nvec * part / split);
-    const int vend = (int)((int64_t)nvec * (part + 1) / split);
-    if (split == 1 && a.prefetch && threadIdx.x == 0)
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    if (a.prefetch && threadIdx.x == 0)
       prefetch_token_rows<kElemBytes>(a, tok + (int64_t)a.prefetch * gridDim.x);
     const int nd = a.plan_nd[tok];
     if (nd == kNoToken) continue;
@@ -184,7 +137,7 @@ __global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
     const uint8_t* xt = a.x + tok * (int64_t)a.H * kElemBytes;           // rank 0's row
     const int64_t rank_stride = a.ntok * (int64_t)a.H * kElemBytes;      // bytes per rank
     uint16_t* out = a.out + tok * (int64_t)a.H;
-    for (int v = vbeg + (int)threadIdx.x; v < vend; v += blockDim.x) {
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
       float acc[kElems];
 #pragma unroll
       for (int e = 0; e < kElems; ++e) acc[e] = 0.0f;
@@ -296,7 +249,6 @@ template <int kMode>
 __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
                                                            const float* __restrict__ scales) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   constexpr int kElems = kMode == kCombineBf16 ? 8 : 16;
   constexpr int kElemBytes = kMode == kCombineBf16 ? 2 : 1;
   const int nvec = a.H / kElems;
@@ -305,20 +257,14 @@ __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
   if (a.prefetch && threadIdx.x == 0)
     for (int p = 0; p < a.prefetch; ++p)
       prefetch_token_rows<kElemBytes>(a, blockIdx.x + (int64_t)p * gridDim.x);
-  const int split = a.split > 1 ? a.split : 1;
-  for (int64_t item = blockIdx.x; item < a.ntok * split; item += gridDim.x) {
-    const int64_t tok = split == 1 ? item : item / split;
-    const int part = (int)(item - tok * split);
-    const int vbeg = (int)((int64_t)nvec * part / split);
-    const int nv = (int)((int64_t)nvec * (part + 1) / split) - vbeg;   // vectors of the item
-    if (split == 1 && a.prefetch && threadIdx.x == 0)
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
+    if (a.prefetch && threadIdx.x == 0)
       prefetch_token_rows<kElemBytes>(a, tok + (int64_t)a.prefetch * gridDim.x);
     const int nd = a.plan_nd[tok];
-    if (nd == kNoToken || (int)threadIdx.x >= nv) continue;
+    if (nd == kNoToken || (int)threadIdx.x >= nvec) continue;
     const uint64_t w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
     if (!plan_row_ok(nd, w0, 0, 0, 0, a.ep, 8, a.err)) continue;
-    const uint8_t* xt =
-        a.x + tok * (int64_t)a.H * kElemBytes + ((int64_t)vbeg + threadIdx.x) * 16;
+    const uint8_t* xt = a.x + tok * (int64_t)a.H * kElemBytes + (int64_t)threadIdx.x * 16;
     const uint8_t* src[8];
     float sc[8];
 #pragma unroll
@@ -328,20 +274,20 @@ __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
       sc[i] = 1.0f;
       if (kMode == kCombineFp8Scaled && i < nd) sc[i] = scales[(int64_t)d * a.ntok + tok];
     }
-    uint16_t* o = a.out + tok * (int64_t)a.H + ((int64_t)vbeg + threadIdx.x) * kElems;
+    uint16_t* o = a.out + tok * (int64_t)a.H + (int64_t)threadIdx.x * kElems;
     const int64_t ostep = (int64_t)blockDim.x * kElems;
     uint4 ra[8], rb[8];
     load_rows(ra, src, nd, 0);
     int64_t off = 0;
     for (int v = threadIdx.x;;) {
-      const bool more_b = v + (int)blockDim.x < nv;
+      const bool more_b = v + (int)blockDim.x < nvec;
       if (more_b) load_rows(rb, src, nd, off + step);
       reduce_store<kMode>(ra, sc, nd, o, a.out32 != 0);
       if (!more_b) break;
       v += blockDim.x;
       off += step;
       o += ostep;
-      const bool more_a = v + (int)blockDim.x < nv;
+      const bool more_a = v + (int)blockDim.x < nvec;
       if (more_a) load_rows(ra, src, nd, off + step);
       reduce_store<kMode>(rb, sc, nd, o, a.out32 != 0);
       if (!more_a) break;
@@ -349,99 +295,6 @@ __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
       off += step;
       o += ostep;
     }
-  }
-}
-
-// Item `it` of the flat combine: token tok = it / nvec, column vector v; its
-// destination count (-1: no output) and rows' loads, the row scales (scaled
-// mode) and the output address.  The token's plan comes from shared memory.
-template <int kMode>
-__device__ __forceinline__ void flat_item_load(const CombineArgs& a, const float* __restrict__ scales,
-                                               const int* s_nd, const uint64_t* s_w0, int64_t t0,
-                                               uint32_t nvec, int64_t rank_stride, uint32_t it,
-                                               uint4 (&r)[8], float (&sc)[8], int& nd,
-                                               uint16_t*& o) {
-  constexpr int kElems = kMode == kCombineBf16 ? 8 : 16;
-  constexpr int kElemBytes = kMode == kCombineBf16 ? 2 : 1;
-  const uint32_t tok = it / nvec;
-  const uint32_t v = it - tok * nvec;
-  const int rel = (int)((int64_t)tok - t0);
-  const int n = s_nd[rel];
-  const uint64_t w0 = s_w0[rel];
-  nd = n == kNoToken ? -1 : n;
-  o = a.out + (int64_t)tok * a.H + (int64_t)v * kElems;
-  const uint8_t* xt = a.x + ((int64_t)tok * a.H + (int64_t)v * kElems) * kElemBytes;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    sc[i] = 1.0f;
-    if (i < nd) {
-      const int d = (int)((w0 >> (8 * i)) & 0xFFu);
-      r[i] = ld_stream_v4(xt + (int64_t)d * rank_stride);
-      if (kMode == kCombineFp8Scaled) sc[i] = scales[(int64_t)d * a.ntok + tok];
-    }
-  }
-}
-
-// The combines for steps with few tokens per SM (at most 8 destinations per
-// token, 16-byte vectors): a persistent grid, every CTA resident from the
-// start, where CTA c takes the (token, column vector) items [c*I/G,
-// (c+1)*I/G) of all I = tokens x vectors items.  Every CTA has the same
-// number of items, so the SMs finish together instead of waiting on the last
-// tokens the hardware scheduler handed out; the CTA reads the plan rows of its
-// tokens into shared memory once; each thread walks its items (stride
-// blockDim) with the next item's row loads in flight while it sums the current
-// one.  The sums are those of combine_vec_kernel / combine_scaled_kernel.
-template <int kMode>
-__global__ void __launch_bounds__(256) combine_flat_kernel(const CombineArgs a,
-                                                           const float* __restrict__ scales,
-                                                           int max_tok) {
-  pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
-  extern __shared__ __align__(8) uint8_t flat_mem[];
-  uint64_t* s_w0 = reinterpret_cast<uint64_t*>(flat_mem);
-  int* s_nd = reinterpret_cast<int*>(flat_mem + sizeof(uint64_t) * (size_t)max_tok);
-  constexpr int kElems = kMode == kCombineBf16 ? 8 : 16;
-  constexpr int kElemBytes = kMode == kCombineBf16 ? 2 : 1;
-  const uint32_t nvec = (uint32_t)(a.H / kElems);
-  const int64_t items = a.ntok * (int64_t)nvec;                  // < 2^31 (host)
-  const int64_t lo = items * blockIdx.x / gridDim.x;
-  const int64_t hi = items * (blockIdx.x + 1) / gridDim.x;
-  const int64_t t0 = lo / nvec;
-  const int nt = hi > lo ? (int)((hi - 1) / nvec - t0 + 1) : 0;  // <= max_tok (host)
-  for (int i = threadIdx.x; i < nt; i += blockDim.x) {
-    const int64_t tok = t0 + i;
-    int nd = a.plan_nd[tok];
-    const uint64_t w0 = *reinterpret_cast<const uint64_t*>(a.plan_dst + tok * a.plan_stride);
-    if (nd != kNoToken && (nd > 8 || !plan_row_ok(nd, w0, 0, 0, 0, a.ep, 8, a.err)))
-      nd = kNoToken;
-    s_nd[i] = nd;
-    s_w0[i] = w0;
-  }
-  __syncthreads();
-  const int64_t rank_stride = a.ntok * (int64_t)a.H * kElemBytes;
-  const bool wide = a.out32 != 0;
-  uint32_t it = (uint32_t)(lo + threadIdx.x);
-  if (it >= hi) return;
-  uint4 ra[8], rb[8];
-  float sca[8], scb[8];
-  int nda, ndb;
-  uint16_t *oa, *ob;
-  flat_item_load<kMode>(a, scales, s_nd, s_w0, t0, nvec, rank_stride, it, ra, sca, nda, oa);
-  for (;;) {
-    const uint32_t nb = it + blockDim.x;
-    const bool more_b = nb < hi;
-    if (more_b)
-      flat_item_load<kMode>(a, scales, s_nd, s_w0, t0, nvec, rank_stride, nb, rb, scb, ndb, ob);
-    if (nda >= 0) reduce_store<kMode>(ra, sca, nda, oa, wide);
-    if (!more_b) break;
-    it = nb;
-    const uint32_t na = it + blockDim.x;
-    const bool more_a = na < hi;
-    if (more_a)
-      flat_item_load<kMode>(a, scales, s_nd, s_w0, t0, nvec, rank_stride, na, ra, sca, nda, oa);
-    if (ndb >= 0) reduce_store<kMode>(rb, scb, ndb, ob, wide);
-    if (!more_a) break;
-    it = na;
   }
 }
 
@@ -462,7 +315,6 @@ template <int kMode, int NCW>
 __global__ void __launch_bounds__(32 * (NCW + 1)) combine_staged_kernel(
     const CombineArgs a, const float* __restrict__ scales, int stages, int stage_rows) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   extern __shared__ __align__(128) uint8_t cs_mem[];
   __shared__ __align__(8) uint64_t full_bar[kCombineMaxStages];
   __shared__ __align__(8) uint64_t empty_bar[kCombineMaxStages];
@@ -610,7 +462,6 @@ __global__ void __launch_bounds__(32 * (NCW + 1)) combine_staged_kernel(
 template <bool kFp8>
 __global__ void __launch_bounds__(512) combine_scalar_kernel(const CombineArgs a) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   const int words = a.plan_stride / 8;
   for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
     const int nd = a.plan_nd[tok];
@@ -673,7 +524,6 @@ __device__ __forceinline__ void slot_owners(const CombineExpertsArgs& a, int64_t
 // 16-byte column vectors; the loads of all needed slots are issued first.
 __global__ void __launch_bounds__(512) combine_experts_vec_kernel(const CombineExpertsArgs a) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   constexpr int KMAX = 8;
   const int nvec = a.H / 8;
   const int words = a.plan_stride / 8;
@@ -764,20 +614,22 @@ __device__ __forceinline__ void expert_rows_reduce_store(const uint4 (&raw)[8],
   for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
   for (int q = 0; q < nd; ++q) {
     const int d = (int)((w0 >> (8 * q)) & 0xFFu);
-    uint64_t z[4];                        // z_d's 8 values as packed pairs
+    float z[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) z[e] = 0ull;
+    for (int e = 0; e < 8; ++e) z[e] = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (own[j] != d) continue;
-      const uint64_t w2 = f32x2_of(wt[j], wt[j]);
       const uint32_t wv[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) z[i] = fma_f32x2(w2, bf16x2_to_f32x2(wv[i]), z[i]);
+      for (int i = 0; i < 4; ++i) {
+        z[2 * i] = __fmaf_rn(wt[j], bf16_bits_to_f32(wv[i] & 0xFFFFu), z[2 * i]);
+        z[2 * i + 1] = __fmaf_rn(wt[j], bf16_bits_to_f32(wv[i] >> 16), z[2 * i + 1]);
+      }
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e)           // z_d to bf16 in pairs, then added exactly widened
-      add_bf16x2(acc[2 * e], acc[2 * e + 1], pack_bf16x2(z[e]));
+      add_bf16x2(acc[2 * e], acc[2 * e + 1], pack_bf16x2(z[2 * e], z[2 * e + 1]));
   }
   uint4 pk;
   pk.x = pack_bf16x2(acc[0], acc[1]);
@@ -792,7 +644,6 @@ __device__ __forceinline__ void expert_rows_reduce_store(const uint4 (&raw)[8],
 // current one.  top_k <= 8, so a token has at most 8 destinations.
 __global__ void __launch_bounds__(512) combine_experts_pipe_kernel(const CombineExpertsArgs a) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   const int nvec = a.H / 8;
   const uint32_t tok_bytes = (uint32_t)a.k * a.H * 2;
   if (a.prefetch && threadIdx.x == 0)
@@ -858,20 +709,17 @@ __global__ void __launch_bounds__(512) combine_experts_pipe_kernel(const Combine
 __device__ __forceinline__ void fp8_roundtrip_acc(float* acc, const uint4& zb, float inv,
                                                   float scale) {
   const uint32_t w[4] = {zb.x, zb.y, zb.z, zb.w};
-  const uint64_t inv2 = f32x2_of(inv, inv);
-  const uint64_t scale2 = f32x2_of(scale, scale);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    float2 f;
-    f32x2_parts(mul_f32x2(bf16x2_to_f32x2(w[i]), inv2), f.x, f.y);
+    const float2 f = make_float2(__fmul_rn(bf16_bits_to_f32(w[i] & 0xFFFFu), inv),
+                                 __fmul_rn(bf16_bits_to_f32(w[i] >> 16), inv));
     const __nv_fp8x2_storage_t code = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
     const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(code, __NV_E4M3);
     __half_raw lo, hi;
     lo.x = hr.x;
     hi.x = hr.y;
-    const uint64_t dec = f32x2_of(__half2float(__half(lo)), __half2float(__half(hi)));
-    const uint64_t r = fma_f32x2(dec, scale2, f32x2_of(acc[2 * i], acc[2 * i + 1]));
-    f32x2_parts(r, acc[2 * i], acc[2 * i + 1]);
+    acc[2 * i] = __fmaf_rn(__half2float(__half(lo)), scale, acc[2 * i]);
+    acc[2 * i + 1] = __fmaf_rn(__half2float(__half(hi)), scale, acc[2 * i + 1]);
   }
 }
 
@@ -901,7 +749,6 @@ constexpr int kFp8ExpertsMaxWarps = 32;
 // through E4M3 and sums in ascending rank order.
 __global__ void __launch_bounds__(448, 2) combine_experts_fp8_kernel(const CombineExpertsArgs a) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   extern __shared__ __align__(16) uint8_t z_mem[];       // [rows][H] bf16
   __shared__ float s_max[kFp8ExpertsMaxWarps][8];
   __shared__ float s_scale[8], s_inv[8];
@@ -1041,7 +888,6 @@ template <int C>
 __global__ void __launch_bounds__(256, 2) combine_experts_fp8_cluster_kernel(
     const CombineExpertsArgs a) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   __shared__ float s_max[8][8];            // [warp][destination]
   __shared__ float s_part[2][8];           // this CTA's maxima, by token parity
   __shared__ float s_scale[8], s_inv[8];
@@ -1167,7 +1013,6 @@ template <int C>
 __global__ void __launch_bounds__(256, 3) combine_experts_fp8_split_kernel(
     const CombineExpertsArgs a, int cols) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   extern __shared__ __align__(16) uint8_t zsplit_mem[];    // [8][cols] bf16
   __shared__ int s_slot[8];          // slot of position p (destination-major order)
   __shared__ float s_wt[8];
@@ -1247,24 +1092,26 @@ __global__ void __launch_bounds__(256, 3) combine_experts_fp8_split_kernel(
 #pragma unroll
       for (int p = 0; p < 8; ++p)
         if (p < ns && has) raw[p] = ld_stream_v4(yt + (int64_t)slot[p] * a.H + (int64_t)v * 8);
-      uint64_t z[4];                                  // packed pairs
+      float z[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) z[e] = 0ull;
+      for (int e = 0; e < 8; ++e) z[e] = 0.0f;
       int q = 0;
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
         if (p >= ns) break;
         if (has) {
-          const uint64_t w2 = f32x2_of(wt[p], wt[p]);
           const uint32_t wv[4] = {raw[p].x, raw[p].y, raw[p].z, raw[p].w};
 #pragma unroll
-          for (int k2 = 0; k2 < 4; ++k2) z[k2] = fma_f32x2(w2, bf16x2_to_f32x2(wv[k2]), z[k2]);
+          for (int k2 = 0; k2 < 4; ++k2) {
+            z[2 * k2] = __fmaf_rn(wt[p], bf16_bits_to_f32(wv[k2] & 0xFFFFu), z[2 * k2]);
+            z[2 * k2 + 1] = __fmaf_rn(wt[p], bf16_bits_to_f32(wv[k2] >> 16), z[2 * k2 + 1]);
+          }
         }
         if ((int)((endw >> (4 * q)) & 0xFu) == p + 1) {   // destination q's slots end here
           uint32_t m = 0u;
           if (has) {
-            const uint32_t pk0 = pack_bf16x2(z[0]), pk1 = pack_bf16x2(z[1]);
-            const uint32_t pk2 = pack_bf16x2(z[2]), pk3 = pack_bf16x2(z[3]);
+            const uint32_t pk0 = pack_bf16x2(z[0], z[1]), pk1 = pack_bf16x2(z[2], z[3]);
+            const uint32_t pk2 = pack_bf16x2(z[4], z[5]), pk3 = pack_bf16x2(z[6], z[7]);
             *reinterpret_cast<uint4*>(zs + (int64_t)q * cols + (int64_t)i * 8) =
                 make_uint4(pk0, pk1, pk2, pk3);
             const uint32_t mm = max_u16x2(max_u16x2(pk0 & 0x7FFF7FFFu, pk1 & 0x7FFF7FFFu),
@@ -1274,7 +1121,7 @@ __global__ void __launch_bounds__(256, 3) combine_experts_fp8_split_kernel(
           m = __reduce_max_sync(0xFFFFFFFFu, m);
           if (lane == 0) atomicMax(&s_amax[parity][q], m);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) z[e] = 0ull;
+          for (int e = 0; e < 8; ++e) z[e] = 0.0f;
           ++q;
         }
       }
@@ -1319,7 +1166,6 @@ __global__ void __launch_bounds__(256, 3) combine_experts_fp8_split_kernel(
 // a second pass recomputes z_d, takes it through E4M3 and sums.
 __global__ void __launch_bounds__(256) combine_experts_fp8_any_kernel(const CombineExpertsArgs a) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   constexpr int KMAX = kMaxTopK;
   __shared__ float s_max[8];
   __shared__ float s_scale[KMAX], s_inv[KMAX];
@@ -1383,7 +1229,6 @@ template <int NCW>
 __global__ void __launch_bounds__(32 * (NCW + 1)) combine_experts_staged_kernel(
     const CombineExpertsArgs a, int stages) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   extern __shared__ __align__(128) uint8_t es_mem[];
   __shared__ __align__(8) uint64_t full_bar[kCombineMaxStages];
   __shared__ __align__(8) uint64_t empty_bar[kCombineMaxStages];
@@ -1506,7 +1351,6 @@ __global__ void __launch_bounds__(32 * (NCW + 1)) combine_experts_staged_kernel(
 // Any top_k (<= 32) and hidden size: one element per thread step.
 __global__ void __launch_bounds__(512) combine_experts_any_kernel(const CombineExpertsArgs a) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   constexpr int KMAX = kMaxTopK;
   const int words = a.plan_stride / 8;
   for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
@@ -1543,7 +1387,6 @@ template <bool kVec>
 __global__ void __launch_bounds__(512) combine_scaled_kernel(const CombineArgs a,
                                                              const float* __restrict__ scales) {
   pdl_wait();
-  if (a.trigger) pdl_launch_dependents();
   const int words = a.plan_stride / 8;
   const int nvec = kVec ? a.H / 16 : 0;
   if (kVec && a.prefetch && threadIdx.x == 0)
@@ -1757,48 +1600,6 @@ cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, bool pipe, 
   }
   if (fp8) return launch_kernel(combine_scalar_kernel<true>, g, b, 0, stream, pdl, a);
   return launch_kernel(combine_scalar_kernel<false>, g, b, 0, stream, pdl, a);
-}
-
-namespace {
-template <int kMode>
-cudaError_t launch_flat_mode(const CombineArgs& a, const float* scales, int ctas_per_sm,
-                             int num_sms, cudaStream_t stream, bool pdl) {
-  constexpr int kThreads = 256;
-  constexpr int kElems = kMode == kCombineBf16 ? 8 : 16;
-  const int64_t nvec = a.H / kElems;
-  // every CTA resident at once: the grid is the SMs times the CTAs that fit
-  int fit = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-      &fit, combine_flat_kernel<kMode>, kThreads, 12 * 64);
-  if (e != cudaSuccess) return e;
-  const int cps = std::max(1, ctas_per_sm > 0 ? std::min(ctas_per_sm, fit) : fit);
-  const int64_t items = a.ntok * nvec;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(items, (int64_t)num_sms * cps));
-  const int max_tok = (int)((items / grid + 1) / nvec + 2);
-  const size_t smem = (size_t)max_tok * (sizeof(uint64_t) + sizeof(int));
-  if (smem > 48 * 1024) return cudaErrorInvalidValue;
-  return launch_kernel(combine_flat_kernel<kMode>, dim3(grid), dim3(kThreads), smem, stream, pdl,
-                       a, scales, max_tok);
-}
-}  // namespace
-
-bool combine_flat_ok(const CombineArgs& a, int elems) {
-  const int64_t nvec = a.H / elems;
-  return a.H % elems == 0 && a.ntok * nvec < ((int64_t)1 << 31);
-}
-
-cudaError_t launch_combine_flat(const CombineArgs& a, int mode, const float* scales,
-                                int ctas_per_sm, int num_sms, cudaStream_t stream, bool pdl) {
-  switch (mode) {
-    case kCombineBf16:
-      return launch_flat_mode<kCombineBf16>(a, scales, ctas_per_sm, num_sms, stream, pdl);
-    case kCombineFp8:
-      return launch_flat_mode<kCombineFp8>(a, scales, ctas_per_sm, num_sms, stream, pdl);
-    case kCombineFp8Scaled:
-      return launch_flat_mode<kCombineFp8Scaled>(a, scales, ctas_per_sm, num_sms, stream, pdl);
-    default:
-      return cudaErrorInvalidValue;
-  }
 }
 
 cudaError_t launch_combine_staged(const CombineArgs& a, int mode, const float* scales,

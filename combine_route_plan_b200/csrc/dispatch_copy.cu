@@ -31,8 +31,6 @@
 //     addresses; the SM only issues.
 // The two staged kernels read the plan (plan_nd / plan_dst) the routing kernel
 // wrote just before them.
-#include <type_traits>
-
 #include "ep_a2a_internal.cuh"
 
 namespace ep_a2a {
@@ -274,53 +272,31 @@ __device__ __forceinline__ void store_dst<Vec32>(Vec32* p, const Vec32& v, bool 
                  : "memory");
 }
 
-// One round of a token group's row copy: the vectors i0, i0 + TPT, ...
-// (U of them) of a row of n vectors, loaded into v, then stored to each of
-// the nd destinations.
-template <typename T, int U, int TPT>
-__device__ __forceinline__ void load_round(const T* __restrict__ s, int64_t n, int64_t i0,
-                                           T (&v)[U]) {
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int64_t i = i0 + (int64_t)u * TPT;
-    if (i < n) v[u] = load_src<T>(s + i);
-  }
-}
-
-template <typename T, int U, int TPT>
-__device__ __forceinline__ void store_round(const T (&v)[U], int64_t n, int64_t i0,
-                                            uint8_t* rank0, int64_t rank_stride, int64_t off,
-                                            uint64_t w0, uint64_t w1, uint64_t w2, uint64_t w3,
-                                            int nd, bool streaming) {
-  for (int q = 0; q < nd; ++q) {
-    T* d = reinterpret_cast<T*>(rank0 + (int64_t)dst_rank(w0, w1, w2, w3, q) * rank_stride +
-                                off);
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t i = i0 + (int64_t)u * TPT;
-      if (i < n) store_dst<T>(d + i, v[u], streaming);
-    }
-  }
-}
-
 // Copy one payload row of a token to its nd destinations: the TPT threads of a
-// token group each take vectors gl, gl + TPT, ... (U of them in flight),
-// starting at vector `first` (gl, or later when the first round is done) of
-// column range `part` of `split` equal ranges of the row.
+// token group each take vectors gl, gl + TPT, ... (U of them in flight).
 template <typename T, int U, int TPT>
 __device__ __forceinline__ void copy_row(const uint8_t* __restrict__ src, int64_t rb,
                                          uint8_t* rank0, int64_t rank_stride, int64_t off,
                                          uint64_t w0, uint64_t w1, uint64_t w2, uint64_t w3,
-                                         int nd, int64_t first, bool streaming, int part = 0,
-                                         int split = 1) {
-  const int64_t all = rb / (int64_t)sizeof(T);
-  const int64_t beg = split == 1 ? 0 : all * part / split;
-  const int64_t n = split == 1 ? all : all * (part + 1) / split;
+                                         int nd, int gl, bool streaming) {
+  const int64_t n = rb / (int64_t)sizeof(T);
   const T* s = reinterpret_cast<const T*>(src);
-  for (int64_t i0 = beg + first; i0 < n; i0 += TPT * U) {
+  for (int64_t i0 = gl; i0 < n; i0 += TPT * U) {
     T v[U];
-    load_round<T, U, TPT>(s, n, i0, v);
-    store_round<T, U, TPT>(v, n, i0, rank0, rank_stride, off, w0, w1, w2, w3, nd, streaming);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + (int64_t)u * TPT;
+      if (i < n) v[u] = load_src<T>(s + i);
+    }
+    for (int q = 0; q < nd; ++q) {
+      T* d = reinterpret_cast<T*>(rank0 + (int64_t)dst_rank(w0, w1, w2, w3, q) * rank_stride +
+                                  off);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t i = i0 + (int64_t)u * TPT;
+        if (i < n) store_dst<T>(d + i, v[u], streaming);
+      }
+    }
   }
 }
 
@@ -503,18 +479,14 @@ __device__ __forceinline__ void finish_counts(const CopyArgs& a) {
 // after it sees the plan complete.  kAll = 16 or 32: every payload of the
 // launch moves in vectors of that many bytes (one code path, fewer registers);
 // kAll = 0: each payload picks its own vector width.
-template <int U, int kAll, bool kStreaming, int TPT, bool kRoute, bool kEarly>
-__device__ __forceinline__ void dispatch_vec_body(const CopyArgs& a) {
+template <int U, int kAll, bool kStreaming, int TPT, bool kRoute>
+__global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArgs a) {
   constexpr bool kUniform = kAll != 0;
   constexpr int kGroups = kVecThreads / TPT;
   const int gl = threadIdx.x % TPT;
   const int group = threadIdx.x / TPT;
   const int lane = threadIdx.x & 31;
   const int64_t tok_step = (int64_t)gridDim.x * kGroups;
-  // the first round of a token's first row can be loaded before the token is
-  // routed (the row's address does not depend on its destinations)
-  static_assert(!kEarly || (!kRoute && kUniform && TPT > 32), "early load: vector copy only");
-  using TU = typename std::conditional<kAll == 32, Vec32, uint4>::type;
   if (kRoute) {
     // this launch is the whole dispatch: it reads the caller's ids and rows and
     // rewrites the plan the previous combine read, so it waits for the
@@ -522,40 +494,11 @@ __device__ __forceinline__ void dispatch_vec_body(const CopyArgs& a) {
     pdl_wait();
     if (a.eplb_stats != nullptr) eplb_gather_rows(a);
   }
-  // the next kernel may launch now; it waits for this grid's completion before
-  // it touches memory
-  if (a.trigger) pdl_launch_dependents();
-  // a work item is one of `split` column ranges of a token's rows (the whole
-  // rows when split is 1; groups of more than a warp only, and never when the
-  // copy also routes)
-  const int split = (kRoute || kEarly || TPT == 32 || a.split <= 1) ? 1 : a.split;
-  for (int64_t item = (int64_t)blockIdx.x * kGroups + group; item < a.ntok * split;
-       item += tok_step) {
-    const int64_t tok = split == 1 ? item : item / split;
-    const int part = (int)(item - tok * split);
-    if (split == 1 && kUniform && a.prefetch && gl == 0 && tok + tok_step < a.ntok) {
+  for (int64_t tok = (int64_t)blockIdx.x * kGroups + group; tok < a.ntok; tok += tok_step) {
+    if (kUniform && a.prefetch && gl == 0 && tok + tok_step < a.ntok) {
       // the group's next token: its rows into L2 while this one is copied
       for (int p = 0; p < a.np; ++p)
         prefetch_l2(a.src[p] + (tok + tok_step) * a.rb[p], (uint32_t)a.rb[p]);
-    }
-    if (kEarly) {
-      const int64_t n0 = a.rb[0] / (int64_t)sizeof(TU);
-      TU v[U];
-      load_round<TU, U, TPT>(reinterpret_cast<const TU*>(a.src[0] + tok * a.rb[0]), n0, gl, v);
-      uint64_t w0, w1, w2, w3;
-      const int nd = token_route<false>(a, tok, lane, gl >> 5, TPT / 32, w0, w1, w2, w3);
-      if (nd == 0) continue;
-      const int64_t off0 = a.dst_off[0] + tok * a.rb[0];
-      const TU* s0 = reinterpret_cast<const TU*>(a.src[0] + tok * a.rb[0]);
-      for (int64_t i0 = gl; i0 < n0; i0 += TPT * U) {
-        if (i0 != gl) load_round<TU, U, TPT>(s0, n0, i0, v);
-        store_round<TU, U, TPT>(v, n0, i0, a.rank0, a.rank_stride, off0, w0, w1, w2, w3, nd,
-                                kStreaming);
-      }
-      for (int p = 1; p < a.np; ++p)
-        copy_row<TU, U, TPT>(a.src[p] + tok * a.rb[p], a.rb[p], a.rank0, a.rank_stride,
-                             a.dst_off[p] + tok * a.rb[p], w0, w1, w2, w3, nd, gl, kStreaming);
-      continue;
     }
     uint64_t w0, w1, w2, w3;
     const int nd = token_route<kRoute>(a, tok, lane, gl >> 5, TPT / 32, w0, w1, w2, w3);
@@ -565,38 +508,38 @@ __device__ __forceinline__ void dispatch_vec_body(const CopyArgs& a) {
       const int64_t off = a.dst_off[p] + tok * a.rb[p];
       if (kAll == 32) {
         copy_row<Vec32, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
-                                gl, kStreaming, part, split);
+                                gl, kStreaming);
         continue;
       }
       if (kAll == 16) {
         copy_row<uint4, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
-                                gl, kStreaming, part, split);
+                                gl, kStreaming);
         continue;
       }
       switch (a.vec[p]) {
         case 32:
           copy_row<Vec32, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
-                                  gl, kStreaming, part, split);
+                                  gl, kStreaming);
           break;
         case 16:
           copy_row<uint4, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
-                                  gl, kStreaming, part, split);
+                                  gl, kStreaming);
           break;
         case 8:
           copy_row<uint2, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3, nd,
-                                  gl, false, part, split);
+                                  gl, false);
           break;
         case 4:
           copy_row<uint32_t, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3,
-                                     nd, gl, false, part, split);
+                                     nd, gl, false);
           break;
         case 2:
           copy_row<uint16_t, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3,
-                                     nd, gl, false, part, split);
+                                     nd, gl, false);
           break;
         default:
           copy_row<uint8_t, U, TPT>(src, a.rb[p], a.rank0, a.rank_stride, off, w0, w1, w2, w3,
-                                    nd, gl, false, part, split);
+                                    nd, gl, false);
           break;
       }
     }
@@ -605,116 +548,6 @@ __device__ __forceinline__ void dispatch_vec_body(const CopyArgs& a) {
     finish_counts(a);
   else
     pdl_wait();
-}
-
-template <int U, int kAll, bool kStreaming, int TPT, bool kRoute>
-__global__ void __launch_bounds__(kVecThreads)
-    dispatch_vec_kernel(const __grid_constant__ CopyArgs a) {
-  dispatch_vec_body<U, kAll, kStreaming, TPT, kRoute, false>(a);
-}
-
-// The copy with the early load, two vectors per thread: held to 64 registers,
-// four CTAs per SM, as the copy without it.
-template <int kAll, bool kStreaming, int TPT>
-__global__ void __launch_bounds__(kVecThreads, 4)
-    dispatch_vec_early_kernel(const __grid_constant__ CopyArgs a) {
-  dispatch_vec_body<2, kAll, kStreaming, TPT, false, true>(a);
-}
-
-// The vector copy for steps with few tokens per SM: a persistent grid, every
-// CTA resident from the start, where CTA c copies the (token, vector) items
-// [c*I/G, (c+1)*I/G) of all I = tokens x (vectors of all the token's payload
-// rows) items, so that every CTA has the same number of items and the SMs
-// finish together.  The CTA's warps first route its tokens (token_destinations,
-// one warp per token) into shared memory; each thread then walks its items
-// (stride blockDim) with the next item's load in flight while it stores the
-// current one to every destination.  All payload rows use vectors of T.
-template <typename T, bool kStreaming>
-__device__ __forceinline__ void flat_copy_item(const CopyArgs& a, const uint32_t (&pv)[kMaxPayloads],
-                                               uint32_t tvec, int64_t t0, uint32_t it,
-                                               const int* s_nd, T& v, int& rel, int64_t& off) {
-  const uint32_t tok = it / tvec;
-  uint32_t j = it - tok * tvec;
-  int p = 0;
-  while (p + 1 < a.np && j >= pv[p]) {
-    j -= pv[p];
-    ++p;
-  }
-  rel = (int)((int64_t)tok - t0);
-  off = a.dst_off[p] + (int64_t)tok * a.rb[p] + (int64_t)j * (int64_t)sizeof(T);
-  if (s_nd[rel] > 0)
-    v = load_src<T>(reinterpret_cast<const T*>(a.src[p] + (int64_t)tok * a.rb[p]) + j);
-}
-
-template <typename T, bool kStreaming>
-__global__ void __launch_bounds__(kVecThreads)
-    dispatch_flat_kernel(const __grid_constant__ CopyArgs a, int max_tok) {
-  if (a.trigger) pdl_launch_dependents();
-  extern __shared__ __align__(8) uint8_t cf_mem[];
-  uint64_t* s_w = reinterpret_cast<uint64_t*>(cf_mem);                      // [max_tok][4]
-  int* s_nd = reinterpret_cast<int*>(cf_mem + 4 * sizeof(uint64_t) * (size_t)max_tok);
-  uint32_t pv[kMaxPayloads];
-  uint32_t tvec = 0;
-#pragma unroll
-  for (int p = 0; p < kMaxPayloads; ++p) {
-    pv[p] = p < a.np ? (uint32_t)(a.rb[p] / (int64_t)sizeof(T)) : 0u;
-    tvec += pv[p];
-  }
-  const int64_t items = a.ntok * (int64_t)tvec;                 // < 2^31 (host)
-  const int64_t lo = items * blockIdx.x / gridDim.x;
-  const int64_t hi = items * (blockIdx.x + 1) / gridDim.x;
-  const int64_t t0 = lo / tvec;
-  const int nt = hi > lo ? (int)((hi - 1) / tvec - t0 + 1) : 0;  // <= max_tok (host)
-  const int lane = threadIdx.x & 31;
-  for (int i = threadIdx.x >> 5; i < nt; i += blockDim.x >> 5) {
-    uint64_t w0, w1, w2, w3;
-    const int nd = token_destinations(a, t0 + i, lane, w0, w1, w2, w3);
-    if (lane == 0) {
-      s_nd[i] = nd;
-      s_w[4 * i + 0] = w0;
-      s_w[4 * i + 1] = w1;
-      s_w[4 * i + 2] = w2;
-      s_w[4 * i + 3] = w3;
-    }
-  }
-  __syncthreads();
-  uint32_t it = (uint32_t)(lo + threadIdx.x);
-  if (it < hi) {
-    T va, vb;
-    int ra, rb;
-    int64_t oa, ob;
-    flat_copy_item<T, kStreaming>(a, pv, tvec, t0, it, s_nd, va, ra, oa);
-    for (;;) {
-      const uint32_t nb = it + blockDim.x;
-      const bool more_b = nb < hi;
-      if (more_b) flat_copy_item<T, kStreaming>(a, pv, tvec, t0, nb, s_nd, vb, rb, ob);
-      {
-        const int nd = s_nd[ra];
-        for (int q = 0; q < nd; ++q) {
-          const int d = dst_rank(s_w[4 * ra], s_w[4 * ra + 1], s_w[4 * ra + 2], s_w[4 * ra + 3], q);
-          store_dst<T>(reinterpret_cast<T*>(a.rank0 + (int64_t)d * a.rank_stride + oa), va,
-                       kStreaming);
-        }
-      }
-      if (!more_b) break;
-      it = nb;
-      const uint32_t na = it + blockDim.x;
-      const bool more_a = na < hi;
-      if (more_a) flat_copy_item<T, kStreaming>(a, pv, tvec, t0, na, s_nd, va, ra, oa);
-      {
-        const int nd = s_nd[rb];
-        for (int q = 0; q < nd; ++q) {
-          const int d = dst_rank(s_w[4 * rb], s_w[4 * rb + 1], s_w[4 * rb + 2], s_w[4 * rb + 3], q);
-          store_dst<T>(reinterpret_cast<T*>(a.rank0 + (int64_t)d * a.rank_stride + ob), vb,
-                       kStreaming);
-        }
-      }
-      if (!more_a) break;
-      it = na;
-    }
-  }
-  // completes after the routing kernel it ran beside (see dispatch_vec_kernel)
-  pdl_wait();
 }
 
 template <int NCW, int MAXV>
@@ -910,16 +743,6 @@ cudaError_t launch_vec_utr(const CopyArgs& a, int grid, bool streaming, cudaStre
     all32 &= a.vec[p] == 32;
   }
   const dim3 g(grid), b(kVecThreads);
-  if constexpr (!kRoute && TPT > 32 && U == 2) {
-    if (a.early && all32)
-      return launch_kernel(streaming ? dispatch_vec_early_kernel<32, true, TPT>
-                                     : dispatch_vec_early_kernel<32, false, TPT>,
-                           g, b, 0, stream, pdl, a);
-    if (a.early && all16)
-      return launch_kernel(streaming ? dispatch_vec_early_kernel<16, true, TPT>
-                                     : dispatch_vec_early_kernel<16, false, TPT>,
-                           g, b, 0, stream, pdl, a);
-  }
   if (all32) {
     if (streaming)
       return launch_kernel(dispatch_vec_kernel<U, 32, true, TPT, kRoute>, g, b, 0, stream, pdl,
@@ -954,46 +777,6 @@ cudaError_t launch_vec_u(const CopyArgs& a, int grid, int tpt, bool streaming,
     case 256: return launch_vec_ut<U, 256>(a, grid, streaming, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
-}
-
-namespace {
-template <typename T, bool kStreaming>
-cudaError_t launch_flat_t(const CopyArgs& a, int ctas_per_sm, int num_sms, cudaStream_t stream,
-                          bool pdl) {
-  int fit = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-      &fit, dispatch_flat_kernel<T, kStreaming>, kVecThreads, 36 * 64);
-  if (e != cudaSuccess) return e;
-  const int cps = std::max(1, ctas_per_sm > 0 ? std::min(ctas_per_sm, fit) : fit);
-  int64_t tvec = 0;
-  for (int p = 0; p < a.np; ++p) tvec += a.rb[p] / (int64_t)sizeof(T);
-  const int64_t items = a.ntok * tvec;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(items, (int64_t)num_sms * cps));
-  const int max_tok = (int)((items / grid + 1) / tvec + 2);
-  const size_t smem = (size_t)max_tok * (4 * sizeof(uint64_t) + sizeof(int));
-  if (smem > 48 * 1024) return cudaErrorInvalidValue;
-  return launch_kernel(dispatch_flat_kernel<T, kStreaming>, dim3(grid), dim3(kVecThreads), smem,
-                       stream, pdl, a, max_tok);
-}
-}  // namespace
-
-bool dispatch_flat_ok(const CopyArgs& a) {
-  if (a.np < 1 || a.route) return false;
-  int64_t tvec = 0;
-  for (int p = 0; p < a.np; ++p) {
-    if (a.vec[p] != a.vec[0] || (a.vec[0] != 16 && a.vec[0] != 32)) return false;
-    tvec += a.rb[p] / a.vec[p];
-  }
-  return tvec > 0 && a.ntok * tvec < ((int64_t)1 << 31);
-}
-
-cudaError_t launch_dispatch_flat(const CopyArgs& a, int ctas_per_sm, int num_sms, bool streaming,
-                                 cudaStream_t stream, bool pdl) {
-  if (a.vec[0] == 32)
-    return streaming ? launch_flat_t<Vec32, true>(a, ctas_per_sm, num_sms, stream, pdl)
-                     : launch_flat_t<Vec32, false>(a, ctas_per_sm, num_sms, stream, pdl);
-  return streaming ? launch_flat_t<uint4, true>(a, ctas_per_sm, num_sms, stream, pdl)
-                   : launch_flat_t<uint4, false>(a, ctas_per_sm, num_sms, stream, pdl);
 }
 
 cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, int unroll, int threads_per_token,

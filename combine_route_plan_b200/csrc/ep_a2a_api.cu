@@ -148,12 +148,6 @@ struct ep_a2a_handle_s {
   int copy_ctas_per_sm;
   int route_in_copy;      // vector copy path: 1 = the copy kernel also routes (one launch)
   int fp8_experts_kernel;   // sender-side FP8 expert combine: 0 split, 1 cluster, 2 one CTA
-  int pdl_trigger;          // copy and combines trigger the next launch at their start
-  int copy_early_load;      // vector copy: first row vectors loaded before routing
-  int combine_flat;         // -1 auto, 0 off, 1 on: balanced persistent combine
-  int copy_flat;            // -1 auto, 0 off, 1 on: balanced persistent vector copy
-  int combine_split;        // vector combines: column ranges per token
-  int copy_split;           // vector copy: column ranges per token
   int copy_stages;        // 0 = choose from the row size
   int combine_threads;
   int64_t bulk_min_row;   // rows below this go to the vector copy
@@ -220,8 +214,6 @@ enum CombineKind { kKindBf16, kKindFp8, kKindExperts };
 
 struct CombineLaunch {
   bool pipe;
-  bool flat;                 // balanced persistent grid (BF16 / FP8 / scaled FP8)
-  int split;                 // column ranges per token (BF16 / FP8 / scaled FP8)
   bool staged;               // rows staged in shared memory by bulk-async copies
   int threads, grid, prefetch;
   int staged_ctas_per_sm;
@@ -248,8 +240,6 @@ CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
   CombineLaunch c;
   c.pipe = fits && (h->combine_pipeline < 0 ? kind != kKindBf16 : h->combine_pipeline == 1);
   c.staged = fits && h->combine_pipeline == 2;
-  c.flat = fits && kind != kKindExperts && !c.staged &&
-           (h->combine_flat < 0 ? false : h->combine_flat == 1);
   // a staged CTA needs two stages of 32 KB: at most three CTAs per SM
   c.staged_ctas_per_sm = h->combine_ctas_per_sm > 0 ? std::min(h->combine_ctas_per_sm, 3) : 2;
   const bool mid = !big && ntok >= 8192;
@@ -265,9 +255,8 @@ CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
   }
   c.threads = h->combine_threads > 0 ? h->combine_threads : threads;
   if (h->combine_ctas_per_sm > 0) cps = h->combine_ctas_per_sm;
-  c.split = kind == kKindExperts ? 1 : h->combine_split;
-  c.grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntok * c.split, (int64_t)h->num_sms * cps));
-  c.prefetch = c.split > 1 ? 0 : (h->combine_prefetch >= 0 ? h->combine_prefetch : prefetch);
+  c.grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntok, (int64_t)h->num_sms * cps));
+  c.prefetch = h->combine_prefetch >= 0 ? h->combine_prefetch : prefetch;
   return c;
 }
 
@@ -392,12 +381,6 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   // cluster kernel (decode 83 against 175 us).
   h->route_in_copy = 0;
   h->fp8_experts_kernel = 0;
-  h->pdl_trigger = 0;
-  h->copy_early_load = 0;
-  h->combine_flat = -1;
-  h->copy_flat = -1;
-  h->combine_split = 1;
-  h->copy_split = 1;
   h->copy_stages = 4;
   h->combine_threads = 0;
   h->bulk_min_row = 0;
@@ -497,30 +480,6 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       if (value < 0 || value > 2)
         return fail(EP_A2A_ERR_INVALID_ARG, "FP8 experts kernel must be 0, 1 or 2");
       h->fp8_experts_kernel = (int)value;
-      return EP_A2A_OK;
-    case EP_A2A_OPT_PDL_TRIGGER:
-      if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "PDL trigger must be 0 or 1");
-      h->pdl_trigger = (int)value;
-      return EP_A2A_OK;
-    case EP_A2A_OPT_COPY_EARLY_LOAD:
-      if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "early load must be 0 or 1");
-      h->copy_early_load = (int)value;
-      return EP_A2A_OK;
-    case EP_A2A_OPT_COMBINE_FLAT:
-      if (value < -1 || value > 1) return fail(EP_A2A_ERR_INVALID_ARG, "flat combine must be -1, 0 or 1");
-      h->combine_flat = (int)value;
-      return EP_A2A_OK;
-    case EP_A2A_OPT_COPY_FLAT:
-      if (value < -1 || value > 1) return fail(EP_A2A_ERR_INVALID_ARG, "flat copy must be -1, 0 or 1");
-      h->copy_flat = (int)value;
-      return EP_A2A_OK;
-    case EP_A2A_OPT_COMBINE_SPLIT:
-      if (value < 1 || value > 8) return fail(EP_A2A_ERR_INVALID_ARG, "combine split must be 1..8");
-      h->combine_split = (int)value;
-      return EP_A2A_OK;
-    case EP_A2A_OPT_COPY_SPLIT:
-      if (value < 1 || value > 8) return fail(EP_A2A_ERR_INVALID_ARG, "copy split must be 1..8");
-      h->copy_split = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_ROUTE_IN_COPY:
       if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "route in copy must be 0 or 1");
@@ -648,8 +607,6 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
   std::memcpy(bulk.live, ra.live, sizeof(bulk.live));
   bulk.ep = ep;
   vec = bulk;
-  vec.trigger = pdl && h->pdl_trigger != 0;
-  vec.early = h->copy_early_load;
   if (fused) {
     vec.route = 1;
     vec.invalid_id = ra.invalid_id;
@@ -725,20 +682,12 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
     const int tpt = h->vec_threads_per_token > 0 ? h->vec_threads_per_token
                                                  : copy_threads_per_token(ntok, row_vectors);
     const int64_t groups_per_cta = 256 / tpt;
-    vec.split = (fused || tpt == 32) ? 1 : h->copy_split;
-    const int64_t items = ntok * vec.split;
     const int grid = (int)std::max<int64_t>(
-        1, std::min<int64_t>((items + groups_per_cta - 1) / groups_per_cta,
+        1, std::min<int64_t>((ntok + groups_per_cta - 1) / groups_per_cta,
                              (int64_t)h->num_sms * h->vec_ctas_per_sm));
     const int unroll = h->vec_unroll > 0 ? h->vec_unroll : copy_unroll(row_vectors, tpt);
-    const bool flat = !fused && (h->copy_flat < 0 ? false : h->copy_flat == 1) &&
-                      dispatch_flat_ok(vec);
     slot = prof_begin(h, EP_A2A_KERNEL_COPY_VEC, stream);
-    if (flat)
-      e = launch_dispatch_flat(vec, 0, h->num_sms,
-                               h->store_streaming != 0, stream, pdl);
-    else
-      e = launch_dispatch_vec(vec, grid, unroll, tpt, h->store_streaming != 0, stream, pdl);
+    e = launch_dispatch_vec(vec, grid, unroll, tpt, h->store_streaming != 0, stream, pdl);
     prof_end(h, slot, stream);
     if (e != cudaSuccess) return cuda_fail(e, "vector copy kernel launch");
   }
@@ -771,7 +720,7 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   if (dtype != EP_A2A_COMBINE_BF16 && dtype != EP_A2A_COMBINE_FP8_E4M3)
     return fail(EP_A2A_ERR_INVALID_ARG, "unknown combine dtype %d", (int)dtype);
   const bool fp8 = dtype == EP_A2A_COMBINE_FP8_E4M3;
-  CombineArgs a{};
+  CombineArgs a;
   a.plan_nd = h->ws + h->L.off_plan_nd;
   a.plan_dst = h->ws + h->L.off_plan_dst;
   a.x = static_cast<const uint8_t*>(expert_output);
@@ -781,10 +730,8 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   a.plan_stride = h->L.plan_stride;
   a.ep = h->p.ep_size;
   a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
-  a.trigger = h->pdl != 0 && h->pdl_trigger != 0;
   const CombineLaunch c = combine_launch(h, fp8 ? kKindFp8 : kKindBf16, a.ntok);
   a.prefetch = c.prefetch;
-  a.split = c.split;
   a.out32 = aligned(output, 32) ? 1 : 0;
   const int elems = fp8 ? 16 : 8;
   const bool vec = a.H % elems == 0 && aligned(expert_output, 16) && aligned(output, 16);
@@ -794,9 +741,6 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
     e = launch_combine_staged(a, fp8 ? 1 : 0, nullptr, h->num_sms * c.staged_ctas_per_sm,
                               c.staged_ctas_per_sm, h->max_smem_optin, (cudaStream_t)stream_v,
                               h->pdl != 0);
-  else if (vec && c.flat && combine_flat_ok(a, elems))
-    e = launch_combine_flat(a, fp8 ? 1 : 0, nullptr, h->combine_ctas_per_sm, h->num_sms,
-                            (cudaStream_t)stream_v, h->pdl != 0);
   else
     e = launch_combine(a, fp8, vec, c.pipe, c.threads, c.grid, (cudaStream_t)stream_v,
                        h->pdl != 0);
@@ -813,7 +757,7 @@ EP_API ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle h, const float* topk_w
   if (!h->have_plan) return fail(EP_A2A_ERR_NO_PLAN, "combine needs a preceding dispatch");
   if (!topk_weights || !expert_output_per_slot || !output)
     return fail(EP_A2A_ERR_INVALID_ARG, "topk_weights / expert output / output is NULL");
-  CombineExpertsArgs a{};
+  CombineExpertsArgs a;
   a.plan_nd = h->ws + h->L.off_plan_nd;
   a.plan_dst = h->ws + h->L.off_plan_dst;
   a.recv_ids0 = h->ws + h->L.rank_base + h->L.off_ids;
@@ -829,7 +773,6 @@ EP_API ep_a2a_status ep_a2a_combine_experts(ep_a2a_handle h, const float* topk_w
   a.plan_stride = h->L.plan_stride;
   a.ep = h->p.ep_size;
   a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
-  a.trigger = h->pdl != 0 && h->pdl_trigger != 0;
   const CombineLaunch c = combine_launch(h, kKindExperts, a.ntok);
   a.prefetch = c.prefetch;
   const bool vec = a.k <= 8 && a.H % 8 == 0 && aligned(expert_output_per_slot, 16) &&
@@ -855,7 +798,7 @@ EP_API ep_a2a_status ep_a2a_combine_experts_fp8(ep_a2a_handle h, const float* to
   if (!h->have_plan) return fail(EP_A2A_ERR_NO_PLAN, "combine needs a preceding dispatch");
   if (!topk_weights || !expert_output_per_slot || !output)
     return fail(EP_A2A_ERR_INVALID_ARG, "topk_weights / expert output / output is NULL");
-  CombineExpertsArgs a{};
+  CombineExpertsArgs a;
   a.plan_nd = h->ws + h->L.off_plan_nd;
   a.plan_dst = h->ws + h->L.off_plan_dst;
   a.recv_ids0 = h->ws + h->L.rank_base + h->L.off_ids;
@@ -871,7 +814,6 @@ EP_API ep_a2a_status ep_a2a_combine_experts_fp8(ep_a2a_handle h, const float* to
   a.plan_stride = h->L.plan_stride;
   a.ep = h->p.ep_size;
   a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
-  a.trigger = h->pdl != 0 && h->pdl_trigger != 0;
   a.prefetch = 0;
   const bool vec8 = a.k <= 8 && a.H % 8 == 0 && aligned(expert_output_per_slot, 16) &&
                     aligned(output, 16);
@@ -950,7 +892,7 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
   if (!h->have_plan) return fail(EP_A2A_ERR_NO_PLAN, "combine needs a preceding dispatch");
   if (!expert_output_e4m3 || !row_scales || !output)
     return fail(EP_A2A_ERR_INVALID_ARG, "expert_output / row_scales / output is NULL");
-  CombineArgs a{};
+  CombineArgs a;
   a.plan_nd = h->ws + h->L.off_plan_nd;
   a.plan_dst = h->ws + h->L.off_plan_dst;
   a.x = static_cast<const uint8_t*>(expert_output_e4m3);
@@ -960,10 +902,8 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
   a.plan_stride = h->L.plan_stride;
   a.ep = h->p.ep_size;
   a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
-  a.trigger = h->pdl != 0 && h->pdl_trigger != 0;
   const CombineLaunch c = combine_launch(h, kKindFp8, a.ntok);
   a.prefetch = c.prefetch;
-  a.split = c.split;
   a.out32 = aligned(output, 32) ? 1 : 0;
   const bool vec = a.H % 16 == 0 && aligned(expert_output_e4m3, 16) && aligned(output, 16);
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);
@@ -972,9 +912,6 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
     e = launch_combine_staged(a, 2, row_scales, h->num_sms * c.staged_ctas_per_sm,
                               c.staged_ctas_per_sm, h->max_smem_optin, (cudaStream_t)stream_v,
                               h->pdl != 0);
-  else if (vec && c.flat && combine_flat_ok(a, 16))
-    e = launch_combine_flat(a, 2, row_scales, h->combine_ctas_per_sm, h->num_sms,
-                            (cudaStream_t)stream_v, h->pdl != 0);
   else
     e = launch_combine_scaled(a, row_scales, vec, c.pipe, c.threads, c.grid,
                               (cudaStream_t)stream_v, h->pdl != 0);

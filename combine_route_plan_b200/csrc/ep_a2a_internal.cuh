@@ -112,11 +112,6 @@ struct CopyArgs {
   int eplb_n;
   int32_t n[kMaxRanks];                  // local_num_tokens (0 for masked-off ranks)
   uint64_t live[kMaskWords];
-  int trigger;                           // 1 = let the next kernel launch at this one's start
-  int split;                             // vector path without routing: column ranges per
-                                         // token row (work items)
-  int early;                             // vector path, 64..256 threads per token: load the
-                                         // first row vectors before routing the token
 };
 
 cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t stream, bool pdl);
@@ -126,13 +121,6 @@ constexpr int kStagedMaxVec = 8;         // 16-byte vectors per consumer thread 
 cudaError_t launch_dispatch_vec(const CopyArgs& a, int grid, int unroll, int threads_per_token,
                                 bool streaming, cudaStream_t stream, bool pdl);
 int bulk_queue_depth(int stages);        // groups allowed in flight for `stages`
-// The vector copy on a persistent grid of num_sms x min(ctas_per_sm, what
-// fits) CTAs (0: what fits), each copying an equal share of the (token,
-// vector) items; every payload row with the same vector width (16 or 32
-// bytes), no routing in the copy (dispatch_flat_ok).
-bool dispatch_flat_ok(const CopyArgs& a);
-cudaError_t launch_dispatch_flat(const CopyArgs& a, int ctas_per_sm, int num_sms, bool streaming,
-                                 cudaStream_t stream, bool pdl);
 
 // ---------------------------------------------------------------------------
 // Combine and the E4M3 helper
@@ -151,8 +139,6 @@ struct CombineArgs {
   uint32_t* err;               // device error word (checked builds)
   int out32;                   // pipelined E4M3 combines: one 32-byte store per
                                // vector (output 32-byte aligned)
-  int trigger;                 // 1 = let the next kernel launch at this one's start
-  int split;                   // vector kernels: column ranges per token (work items)
 };
 
 // pipe: the two-deep pipelined kernel (needs at most 8 destinations per token)
@@ -175,7 +161,6 @@ struct CombineExpertsArgs {
                                // grid strides ahead into L2
   int ep;
   uint32_t* err;               // device error word (checked builds)
-  int trigger;                 // 1 = let the next kernel launch at this one's start
 };
 
 cudaError_t launch_combine_experts(const CombineExpertsArgs& a, bool vec, bool pipe, int threads,
@@ -212,13 +197,6 @@ cudaError_t launch_quantize_e4m3_rows(const uint16_t* in, uint8_t* out, float* s
 cudaError_t launch_combine_staged(const CombineArgs& a, int mode, const float* scales,
                                   int grid, int ctas_per_sm, int max_smem, cudaStream_t stream,
                                   bool pdl);
-// The BF16 (mode 0), FP8 (1) or scaled FP8 (2) combine on a persistent grid of
-// num_sms x min(ctas_per_sm, what fits) CTAs (0: what fits), each summing an
-// equal share of the (token, column vector) items; at most 8 destinations per
-// token, 16-byte vectors, combine_flat_ok(a, elements per vector).
-bool combine_flat_ok(const CombineArgs& a, int elems);
-cudaError_t launch_combine_flat(const CombineArgs& a, int mode, const float* scales,
-                                int ctas_per_sm, int num_sms, cudaStream_t stream, bool pdl);
 // FP8 combine with one fp32 scale per row (scales [ep, ep*tpr]).
 cudaError_t launch_combine_scaled(const CombineArgs& a, const float* scales, bool vec, bool pipe,
                                   int threads, int grid, cudaStream_t stream, bool pdl);

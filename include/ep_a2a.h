@@ -392,40 +392,7 @@ typedef enum {
                                      through distributed shared memory; 1 = a cluster per
                                      token with one column vector per thread and the rows
                                      in registers (hidden up to 16384); 2 = one CTA per
-                                     token with the whole rows in shared memory */,
-  EP_A2A_OPT_PDL_TRIGGER = 19,    /* with PDL on: 1 = the copy and combine kernels also
-                                     let the next kernel of the stream launch as soon
-                                     as all their CTAs are running (griddepcontrol.
-                                     launch_dependents at their start), so its CTAs are
-                                     resident and waiting when they finish; 0 = only
-                                     the routing kernel does (the next kernel launches
-                                     when they end).  The next kernel still waits for
-                                     their completion before it touches memory, so
-                                     results do not change */
-  EP_A2A_OPT_COPY_EARLY_LOAD = 20,/* vector copy with 64..256 threads per token: 1 =
-                                     each token's first row vectors are loaded before
-                                     its destinations are worked out (the two loads
-                                     overlap); 0 = after */
-  EP_A2A_OPT_COMBINE_FLAT = 21    /* BF16 / FP8 / scaled FP8 combines of 16-byte vectors
-                                     with at most 8 destinations per token: 1 = a
-                                     persistent grid (every CTA resident) in which each
-                                     CTA sums an equal share of the (token, column
-                                     vector) items, so all SMs finish together; 0 = one
-                                     token per CTA at a time, as the hardware hands
-                                     CTAs out; -1 (default) = automatic */,
-  EP_A2A_OPT_COPY_FLAT = 22       /* vector copy (no routing in the copy) whose payload
-                                     rows all use the same vector width: 1 = a
-                                     persistent grid in which each CTA copies an equal
-                                     share of the (token, vector) items; 0 = token groups
-                                     as the hardware hands CTAs out; -1 (default) =
-                                     automatic */,
-  EP_A2A_OPT_COMBINE_SPLIT = 23,  /* BF16 / FP8 / scaled FP8 vector combines: each
-                                     token's row is summed as this many column ranges,
-                                     each its own work item (1..8; default 1) */
-  EP_A2A_OPT_COPY_SPLIT = 24      /* vector copy with more than 32 threads per token
-                                     and no routing in the copy: each token's rows are
-                                     copied as this many column ranges, each its own
-                                     work item (1..8; default 1) */
+                                     token with the whole rows in shared memory */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

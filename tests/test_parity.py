@@ -80,109 +80,6 @@ def test_routing_inside_the_copy_bit_exact(name):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("name", ["c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked",
-                                  "c3_ep16_zipf_nvfp4", "c3_ep16_zipf_mxfp8"])
-def test_early_load_and_pdl_trigger_bit_exact(name):
-    """The copy that loads each token's first row vectors before routing it, and
-    the copy and combine that let the next kernel launch at their start: the
-    same plan, rows, EPLB rows and combine as the oracle."""
-    from combine_route_plan_b200 import ep_a2a
-    _full_check(W.BY_NAME[name], options={ep_a2a.OPT_COPY_EARLY_LOAD: 1,
-                                          ep_a2a.OPT_PDL_TRIGGER: 1})
-
-
-@pytest.mark.parametrize("tpt", [64, 128, 256])
-@pytest.mark.parametrize("rows,shift", [([14336, 64], 0), ([4096 + 16, 48], 0),
-                                        ([14336, 32], 16), ([64 * 32 + 32], 0)])
-def test_early_load_rows_and_threads(tpt, rows, shift):
-    """Early load with every group size, rows of one and of several rounds,
-    256-bit and 128-bit vectors, ragged token counts and a masked rank."""
-    from combine_route_plan_b200 import ep_a2a
-    ep, E, k, tpr, H = 8, 64, 8, 41, 32
-    n = [41, 40, 0, 17, 41, 3, 41, 29]
-    mask = _mask_of(ep, [0, 1, 2, 3, 4, 6, 7])
-    w, x = _custom(ep, E, k, tpr, H, rows, n=n, mask=mask, seed=tpt + sum(rows) % 97 + shift)
-    comm = ep_a2a.EpA2A(ep, E, k, tpr, H, rows, enable_rank_mask=True, workspace_fill=U.CANARY)
-    comm.set_option(ep_a2a.OPT_COPY_EARLY_LOAD, 1)
-    comm.set_option(ep_a2a.OPT_PDL_TRIGGER, 1)
-    comm.set_option(ep_a2a.OPT_VEC_THREADS_PER_TOKEN, tpt)
-    comm.set_option(ep_a2a.OPT_VEC_UNROLL, 2)       # the early-load kernel's unroll
-    srcs = []
-    for p in x.payloads:
-        buf = torch.empty(p.numel() + 64, dtype=torch.uint8, device="cuda")
-        v = buf[shift: shift + p.numel()].view(p.shape)
-        v.copy_(p.cuda())
-        srcs.append(v)
-    d = comm.dispatch(x.token_selected_experts.cuda(), x.local_num_tokens, srcs, tpr,
-                      active_rank_mask=x.active_rank_mask)
-    torch.cuda.synchronize()
-    assert comm.get_status() == ep_a2a.OK
-    plan = U.oracle_plan(w, x)
-    for i, p in enumerate(x.payloads):
-        for dst in range(ep):
-            want = U.oracle.dispatch_payload(plan, p.numpy(), only_dst=dst, recv_init=np.full(
-                (1, ep * tpr, p.shape[2]), U.CANARY, np.uint8))
-            U.assert_equal(d.recv_payloads[i][dst], want, f"payload {i} rank {dst} tpt {tpt}")
-
-
-def test_pdl_trigger_chain_of_every_combine():
-    """With the early trigger, dispatch and every combine back to back on one
-    stream, then a second dispatch with other routing: each result is the
-    oracle's (a kernel never reads what its predecessor has not finished)."""
-    from combine_route_plan_b200 import ep_a2a
-    w = W.C2
-    x = _inputs(w.name)
-    stats = x.eplb_local_stats.cuda() if x.eplb_local_stats is not None else None
-    comm = ep_a2a.EpA2A(w.ep_size, w.num_experts, w.top_k, w.tokens_per_rank, w.hidden,
-                        w.payload_row_bytes(),
-                        eplb_stats_num_experts=w.num_experts if stats is not None else 0,
-                        workspace_fill=U.CANARY)
-    comm.set_option(ep_a2a.OPT_PDL_TRIGGER, 1)
-    comm.set_option(ep_a2a.OPT_COPY_EARLY_LOAD, 1)
-    H, ep, tpr, k = w.hidden, w.ep_size, w.tokens_per_rank, w.top_k
-    xo = x.expert_output.cuda()
-    xq = ep_a2a.quantize_e4m3(xo)
-    codes, scales = ep_a2a.quantize_e4m3_rows(xo)
-    g = torch.Generator(device="cuda").manual_seed(5)
-    wts = torch.randn((ep, tpr, k), generator=g, device="cuda")
-    y = torch.randn((ep, tpr, k, H), generator=g, device="cuda").to(torch.bfloat16)
-
-    def fresh():
-        return torch.full((ep, tpr, H), U.OUT_CANARY, dtype=torch.int16,
-                          device="cuda").view(torch.bfloat16)
-    outs = [fresh() for _ in range(5)]
-    ids2 = torch.roll(x.token_selected_experts, 1, dims=1)
-    pays = [p.cuda() for p in x.payloads]
-    comm.dispatch(x.token_selected_experts.cuda(), x.local_num_tokens, pays, tpr, stats,
-                  views=False)
-    comm.combine(xo, outs[0])
-    comm.combine(xq, outs[1])
-    comm.combine_scaled(codes, scales, outs[2])
-    comm.combine_experts(wts, y, outs[3])
-    comm.combine_experts_fp8(wts, y, outs[4])
-    d2 = comm.dispatch(ids2.cuda(), x.local_num_tokens, pays, tpr, stats)
-    torch.cuda.synchronize()
-    assert comm.get_status() == ep_a2a.OK
-    plan = U.oracle_plan(w, x)
-    init = U.oracle_out_init(w)
-    ids = x.token_selected_experts.numpy()
-    y_np, w_np = U.to_np(y), wts.cpu().numpy()
-    U.assert_equal(outs[0], U.oracle.combine(plan, U.to_np(xo), H, out_init=init), "bf16")
-    xq_want = U.oracle_e4m3_rows_read(U.to_np(xo), plan, U.oracle_e4m3_table())
-    U.assert_equal(outs[1], U.oracle.combine(plan, xq_want, H, input_is_e4m3=True,
-                                             out_init=init), "fp8")
-    oc, osc = U.oracle_row_quantize_read(U.to_np(xo), plan, H)
-    U.assert_equal(outs[2], U.oracle.combine_scaled(plan, oc, osc, H, out_init=init), "scaled")
-    U.assert_equal(outs[3], U.oracle.combine_experts(plan, w.num_experts, ids, w_np, y_np, H,
-                                                     out_init=init), "experts")
-    U.assert_equal(outs[4], U.oracle.combine_experts_fp8(plan, w.num_experts, ids, w_np, y_np, H,
-                                                         out_init=init), "experts fp8")
-    x2 = W.Inputs(w, ids2, x.local_num_tokens, x.payloads, x.eplb_local_stats, None, None)
-    # the second dispatch: its plan in full, its rows where it says received
-    # (other rows keep the first dispatch's bytes)
-    _check_valid_rows(d2, U.oracle_plan(w, x2), x2, w.ep_size)
-
-
 @pytest.mark.parametrize("name,path", [
     (n, p) for n in ("c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked", "c3_ep16_zipf_nvfp4")
     for p in (0, 2)])
@@ -438,106 +335,6 @@ def test_pipelined_combines_match_the_oracle(case, prefetch, threads):
     """BF16, FP8, scaled-FP8 and expert-output combines with the two-deep
     pipelined kernels."""
     from combine_route_plan_b200 import ep_a2a
-    _check_all_combines(case, {ep_a2a.OPT_COMBINE_PIPELINE: 1, ep_a2a.OPT_COMBINE_PREFETCH: prefetch,
-                               ep_a2a.OPT_COMBINE_THREADS: threads})
-
-
-@pytest.mark.parametrize("case", [
-    ("c2_ep8_decode", None),
-    ("c5_ep64_wide_masked", None),
-    ("c1_ep4_tiny", None),
-    ("c3_ep16_zipf_nvfp4", None),
-    ("mask", [0b10100101, 0, 0, 0]),
-    ("odd", None),
-    ("wide_k", None),
-])
-@pytest.mark.parametrize("ctas", [0, 1])
-def test_flat_combines_match_the_oracle(case, ctas):
-    """BF16, FP8 and scaled-FP8 combines on the balanced persistent grid (each
-    CTA an equal share of the (token, vector) items; shares that start and end
-    inside a token), next to the expert-output combine."""
-    from combine_route_plan_b200 import ep_a2a
-    _check_all_combines(case, {ep_a2a.OPT_COMBINE_FLAT: 1, ep_a2a.OPT_COMBINE_CTAS_PER_SM: ctas,
-                               ep_a2a.OPT_PDL_TRIGGER: 1})
-
-
-@pytest.mark.parametrize("case", [
-    ("c2_ep8_decode", None),
-    ("c5_ep64_wide_masked", None),
-    ("c1_ep4_tiny", None),
-    ("mask", [0b10100101, 0, 0, 0]),
-    ("odd", None),
-])
-@pytest.mark.parametrize("split", [2, 3, 8])
-def test_split_rows_match_the_oracle(case, split):
-    """Combines and the copy with each token's row taken as `split` column
-    ranges (work items), including ranges with no vectors (hidden 40)."""
-    from combine_route_plan_b200 import ep_a2a
-    opts = {ep_a2a.OPT_COMBINE_SPLIT: split, ep_a2a.OPT_COPY_SPLIT: split}
-    for pipe in (0, 1):
-        _check_all_combines(case, {**opts, ep_a2a.OPT_COMBINE_PIPELINE: pipe})
-    name = case[0]
-    if name in W.BY_NAME:
-        _full_check(W.BY_NAME[name], options={**opts, ep_a2a.OPT_VEC_THREADS_PER_TOKEN: 256})
-
-
-@pytest.mark.parametrize("tpt", [64, 128, 256])
-@pytest.mark.parametrize("split", [2, 5])
-def test_split_copy_rows_and_payloads(tpt, split):
-    """The copy's column ranges over payload rows of different widths (some
-    shorter than the range count), ragged token counts and a masked rank."""
-    from combine_route_plan_b200 import ep_a2a
-    ep, E, k, tpr, H = 8, 64, 8, 37, 32
-    rows = [14336, 64, 16, 4]
-    w, x = _custom(ep, E, k, tpr, H, rows, n=[37, 0, 36, 5, 37, 1, 30, 37],
-                   mask=_mask_of(ep, [0, 1, 2, 4, 5, 6, 7]), seed=tpt + split)
-    run = U.Run(w, x, copy_path=1, options={ep_a2a.OPT_COPY_SPLIT: split,
-                                            ep_a2a.OPT_VEC_THREADS_PER_TOKEN: tpt})
-    plan = U.oracle_plan(w, x)
-    U.check_plan(run, plan, w)
-    U.check_payloads(run, plan, w, x)
-
-
-@pytest.mark.parametrize("name", ["c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked",
-                                  "c3_ep16_zipf_nvfp4"])
-def test_flat_copy_bit_exact(name):
-    """The vector copy on the balanced persistent grid (equal shares of the
-    (token, vector) items, routed per CTA into shared memory)."""
-    from combine_route_plan_b200 import ep_a2a
-    _full_check(W.BY_NAME[name], options={ep_a2a.OPT_COPY_FLAT: 1})
-
-
-@pytest.mark.parametrize("rows,shift", [([14336, 64, 32], 0), ([4096 + 16, 48, 16], 0),
-                                        ([14336, 32], 16)])
-def test_flat_copy_rows(rows, shift):
-    """Several payload rows per item range, 16- and 32-byte vectors, ragged
-    token counts and a masked rank."""
-    from combine_route_plan_b200 import ep_a2a
-    ep, E, k, tpr, H = 8, 64, 8, 45, 32
-    w, x = _custom(ep, E, k, tpr, H, rows, n=[45, 44, 0, 3, 45, 17, 45, 9],
-                   mask=_mask_of(ep, [0, 1, 2, 3, 5, 6, 7]), seed=sum(rows) % 101 + shift)
-    comm = ep_a2a.EpA2A(ep, E, k, tpr, H, rows, enable_rank_mask=True, workspace_fill=U.CANARY)
-    comm.set_option(ep_a2a.OPT_COPY_FLAT, 1)
-    srcs = []
-    for p in x.payloads:
-        buf = torch.empty(p.numel() + 64, dtype=torch.uint8, device="cuda")
-        v = buf[shift: shift + p.numel()].view(p.shape)
-        v.copy_(p.cuda())
-        srcs.append(v)
-    d = comm.dispatch(x.token_selected_experts.cuda(), x.local_num_tokens, srcs, tpr,
-                      active_rank_mask=x.active_rank_mask)
-    torch.cuda.synchronize()
-    assert comm.get_status() == ep_a2a.OK
-    plan = U.oracle_plan(w, x)
-    for i, p in enumerate(x.payloads):
-        for dst in range(ep):
-            want = U.oracle.dispatch_payload(plan, p.numpy(), only_dst=dst, recv_init=np.full(
-                (1, ep * tpr, p.shape[2]), U.CANARY, np.uint8))
-            U.assert_equal(d.recv_payloads[i][dst], want, f"payload {i} rank {dst}")
-
-
-def _check_all_combines(case, opts):
-    from combine_route_plan_b200 import ep_a2a
     name, mask = case
     if name in W.BY_NAME:
         w = W.BY_NAME[name]
@@ -548,6 +345,8 @@ def _check_all_combines(case, opts):
         w, x = _custom(4, 16, 4, 30, 40, [32], seed=19)
     else:
         w, x = _custom(16, 64, 16, 20, 64, [32], seed=23)
+    opts = {ep_a2a.OPT_COMBINE_PIPELINE: 1, ep_a2a.OPT_COMBINE_PREFETCH: prefetch,
+            ep_a2a.OPT_COMBINE_THREADS: threads}
     run = U.Run(w, W.Inputs(w, x.token_selected_experts, x.local_num_tokens, x.payloads,
                             x.eplb_local_stats, x.active_rank_mask, None), options=opts)
     plan = U.oracle_plan(w, x)
