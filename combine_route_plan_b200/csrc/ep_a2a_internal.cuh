@@ -67,6 +67,7 @@ struct RouteArgs {
   int32_t invalid_id;
   int32_t n[kMaxRanks];        // local_num_tokens, 0 for masked-off ranks
   uint64_t live[kMaskWords];   // bit r = rank r active
+  int vec_ids;                 // set by launch_route_plan: ids rows as 16-byte stores
 };
 
 cudaError_t launch_route_plan(const RouteArgs& a, bool use_mask, cudaStream_t stream,

@@ -27,6 +27,11 @@
 // leaders of its token with a smaller rank.  Counts are reduced per block in
 // shared memory; the last block of each source rank (ticket counter) writes the
 // final row and resets the scratch to zero, so no memset is needed per call.
+// The receive-side rows (ids and valid byte of each of the block's slots in
+// every live destination) are written from the block's ids and destination
+// sets, kept in shared memory by the first pass: one thread per (slot,
+// destination) pair, consecutive threads on consecutive slots, so a warp
+// stores contiguous rows.
 #include <algorithm>
 
 #include "ep_a2a_internal.cuh"
@@ -79,7 +84,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteAr
   }
   __shared__ int s_cnt[kMaxRanks];
   __shared__ bool s_last;
+  __shared__ int32_t s_ids[kTokPerBlock][kMaxTopK];          // the block's tokens' ids
+  __shared__ unsigned long long s_dst[kTokPerBlock][kMaskWords];  // their destination sets
   for (int i = threadIdx.x; i < a.ep; i += kRouteThreads) s_cnt[i] = 0;
+  for (int i = threadIdx.x; i < kTokPerBlock * kMaskWords; i += kRouteThreads)
+    (&s_dst[0][0])[i] = 0ull;
   __syncthreads();
 
   constexpr int kTokPerWarp = 32 / G;
@@ -135,9 +144,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteAr
       if (leader) {
         row[pos] = (uint8_t)d;
         atomicAdd(&s_cnt[d], 1);
+        atomicOr(&s_dst[t - t_begin][d >> 6], 1ull << (d & 63));
       }
       for (int c = j; c < a.plan_stride; c += G)
         if (c >= nd) row[c] = kPad;
+      if (j < a.k) s_ids[t - t_begin][j] = e;
     }
   }
 
@@ -164,22 +175,29 @@ __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteAr
     if (threadIdx.x == 0) atomicExch(&a.count_ticket[r], 0u);
   }
 
-  // Pass 2: receive-side rows of every slot in every live destination.
-  for (int t0 = t_begin; t0 < t_end; t0 += kRouteWarps * kTokPerWarp) {
-    const int t = t0 + warp * kTokPerWarp + g;
-    int32_t e;
-    int d;
-    bool in_range, exists;
-    owner_of(t, e, d, in_range, exists);
-    const int64_t s = (int64_t)r * a.tpr + t;
-    for (int dd = 0; dd < a.ep; ++dd) {
-      const bool got = (__ballot_sync(kFull, d == dd) & gmask) != 0u;
-      if (!in_range || !rank_live<kMask>(a.live, dd)) continue;
-      uint8_t* base = a.rank0 + dd * a.rank_stride;
-      if (j < a.k)
-        reinterpret_cast<int32_t*>(base + a.off_ids)[s * a.k + j] = got ? e : a.invalid_id;
-      if (j == 0) base[a.off_valid + s] = got ? 1 : 0;
+  // Pass 2: receive-side rows of every slot in every live destination, one
+  // (slot, destination) pair per thread (the first pass's shared arrays are
+  // visible after the barriers above).
+  const int nt = t_end - t_begin;
+  for (int p = threadIdx.x; p < nt * a.ep; p += kRouteThreads) {
+    const int dd = p / nt;
+    const int tl = p - dd * nt;
+    if (!rank_live<kMask>(a.live, dd)) continue;
+    const bool got = (s_dst[tl][dd >> 6] >> (dd & 63)) & 1ull;
+    const int64_t s = (int64_t)r * a.tpr + t_begin + tl;
+    uint8_t* base = a.rank0 + dd * a.rank_stride;
+    int32_t* ids = reinterpret_cast<int32_t*>(base + a.off_ids) + s * a.k;
+    if (a.vec_ids) {
+      for (int q = 0; q < a.k; q += 4) {
+        const int4 v = got ? make_int4(s_ids[tl][q], s_ids[tl][q + 1], s_ids[tl][q + 2],
+                                       s_ids[tl][q + 3])
+                           : make_int4(a.invalid_id, a.invalid_id, a.invalid_id, a.invalid_id);
+        *reinterpret_cast<int4*>(ids + q) = v;
+      }
+    } else {
+      for (int q = 0; q < a.k; ++q) ids[q] = got ? s_ids[tl][q] : a.invalid_id;
     }
+    base[a.off_valid + s] = got ? 1 : 0;
   }
 }
 
@@ -192,7 +210,12 @@ cudaError_t launch_g(const RouteArgs& a, bool use_mask, dim3 grid, cudaStream_t 
 
 }  // namespace
 
-cudaError_t launch_route_plan(const RouteArgs& a, bool use_mask, cudaStream_t stream, bool pdl) {
+cudaError_t launch_route_plan(const RouteArgs& args, bool use_mask, cudaStream_t stream,
+                              bool pdl) {
+  RouteArgs a = args;
+  // received ids as 16-byte stores when every slot's row allows it
+  a.vec_ids = a.k % 4 == 0 && reinterpret_cast<uintptr_t>(a.rank0 + a.off_ids) % 16 == 0 &&
+              a.rank_stride % 16 == 0;
   const int tok_blocks = (a.tpr + kTokPerBlock - 1) / kTokPerBlock;
   int gx = tok_blocks > 0 ? tok_blocks : 1;
   int gy = a.ep;
