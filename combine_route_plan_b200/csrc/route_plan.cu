@@ -84,11 +84,14 @@ __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteAr
   }
   __shared__ int s_cnt[kMaxRanks];
   __shared__ bool s_last;
-  __shared__ int32_t s_ids[kTokPerBlock][kMaxTopK];          // the block's tokens' ids
-  __shared__ unsigned long long s_dst[kTokPerBlock][kMaskWords];  // their destination sets
+  // the block's tokens' ids (rows padded by 4 words, so that the second pass's
+  // 16-byte reads of consecutive tokens fall on different banks) and their
+  // destination sets (bit d of 32-bit words)
+  __shared__ __align__(16) int32_t s_ids[kTokPerBlock][kMaxTopK + 4];
+  __shared__ uint32_t s_dst[kTokPerBlock][kMaxRanks / 32];
   for (int i = threadIdx.x; i < a.ep; i += kRouteThreads) s_cnt[i] = 0;
-  for (int i = threadIdx.x; i < kTokPerBlock * kMaskWords; i += kRouteThreads)
-    (&s_dst[0][0])[i] = 0ull;
+  for (int i = threadIdx.x; i < kTokPerBlock * (kMaxRanks / 32); i += kRouteThreads)
+    (&s_dst[0][0])[i] = 0u;
   __syncthreads();
 
   constexpr int kTokPerWarp = 32 / G;
@@ -144,7 +147,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteAr
       if (leader) {
         row[pos] = (uint8_t)d;
         atomicAdd(&s_cnt[d], 1);
-        atomicOr(&s_dst[t - t_begin][d >> 6], 1ull << (d & 63));
+        atomicOr(&s_dst[t - t_begin][d >> 5], 1u << (d & 31));
       }
       for (int c = j; c < a.plan_stride; c += G)
         if (c >= nd) row[c] = kPad;
@@ -183,14 +186,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteAr
     const int dd = p / nt;
     const int tl = p - dd * nt;
     if (!rank_live<kMask>(a.live, dd)) continue;
-    const bool got = (s_dst[tl][dd >> 6] >> (dd & 63)) & 1ull;
+    const bool got = (s_dst[tl][dd >> 5] >> (dd & 31)) & 1u;
     const int64_t s = (int64_t)r * a.tpr + t_begin + tl;
     uint8_t* base = a.rank0 + dd * a.rank_stride;
     int32_t* ids = reinterpret_cast<int32_t*>(base + a.off_ids) + s * a.k;
     if (a.vec_ids) {
       for (int q = 0; q < a.k; q += 4) {
-        const int4 v = got ? make_int4(s_ids[tl][q], s_ids[tl][q + 1], s_ids[tl][q + 2],
-                                       s_ids[tl][q + 3])
+        const int4 v = got ? *reinterpret_cast<const int4*>(&s_ids[tl][q])
                            : make_int4(a.invalid_id, a.invalid_id, a.invalid_id, a.invalid_id);
         *reinterpret_cast<int4*>(ids + q) = v;
       }
