@@ -394,10 +394,11 @@ typedef enum {
                                      in registers (hidden up to 16384); 2 = one CTA per
                                      token with the whole rows in shared memory */,
   EP_A2A_OPT_COPY_TAIL_EARLY = 19 /* vector copy with more than 32 threads per token and
-                                     two payloads whose second row is at most one
-                                     vector per thread: 1 = that row is loaded before
-                                     the token is routed and stored after the first
-                                     row; 0 (default) = in payload order */
+                                     two or three payloads whose rows after the first
+                                     are at most one vector per thread each: 1 = those
+                                     rows are loaded before the token is routed and
+                                     stored after the first row; 0 (default) = in
+                                     payload order */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

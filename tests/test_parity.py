@@ -90,10 +90,13 @@ def test_copy_tail_row_loaded_early_bit_exact(name):
 
 @pytest.mark.parametrize("tpt", [64, 128, 256])
 @pytest.mark.parametrize("rows,shift", [([3584, 224], 0), ([3584, 32], 0), ([4096 + 16, 48], 0),
-                                        ([7168, 448], 16), ([512, 64, 32], 0)])
+                                        ([7168, 448], 16), ([512, 64, 32], 0),
+                                        ([3584, 448, 32], 0), ([7168, 224, 32], 16),
+                                        ([512, 64, 32, 32], 0), ([512, 4096, 32], 0)])
 def test_copy_tail_rows_and_threads(tpt, rows, shift):
-    """Second rows from one vector to one per thread, 16- and 32-byte vectors,
-    ragged token counts, a masked rank, and three payloads (not taken early)."""
+    """Rows after the first from one vector to one per thread, 16- and 32-byte
+    vectors, two and three payloads, ragged token counts and a masked rank;
+    four payloads and a long later row (not taken early)."""
     from combine_route_plan_b200 import ep_a2a
     ep, E, k, tpr, H = 8, 64, 8, 43, 32
     w, x = _custom(ep, E, k, tpr, H, rows, n=[43, 42, 0, 7, 43, 1, 43, 30],
