@@ -31,8 +31,6 @@
 //     addresses; the SM only issues.
 // The two staged kernels read the plan (plan_nd / plan_dst) the routing kernel
 // wrote just before them.
-#include <type_traits>
-
 #include "ep_a2a_internal.cuh"
 
 namespace ep_a2a {
@@ -481,11 +479,8 @@ __device__ __forceinline__ void finish_counts(const CopyArgs& a) {
 // after it sees the plan complete.  kAll = 16 or 32: every payload of the
 // launch moves in vectors of that many bytes (one code path, fewer registers);
 // kAll = 0: each payload picks its own vector width.
-// (The instances with the early tail loads keep at least four CTAs per SM at
-// 256 threads per token and three below, where four would spill.)
-template <int U, int kAll, bool kStreaming, int TPT, bool kRoute, bool kTail = false>
-__global__ void __launch_bounds__(kVecThreads, kTail ? (TPT == 256 ? 4 : 3) : 0)
-    dispatch_vec_kernel(const CopyArgs a) {
+template <int U, int kAll, bool kStreaming, int TPT, bool kRoute>
+__global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArgs a) {
   constexpr bool kUniform = kAll != 0;
   constexpr int kGroups = kVecThreads / TPT;
   const int gl = threadIdx.x % TPT;
@@ -505,34 +500,9 @@ __global__ void __launch_bounds__(kVecThreads, kTail ? (TPT == 256 ? 4 : 3) : 0)
       for (int p = 0; p < a.np; ++p)
         prefetch_l2(a.src[p] + (tok + tok_step) * a.rb[p], (uint32_t)a.rb[p]);
     }
-    // the rows after the first (scales, weights, extra bytes), when each is at
-    // most one vector per thread, are loaded before the token is routed and
-    // stored after the first row, so their load latency overlaps the others
-    using TT = typename std::conditional<kAll == 16, uint4, Vec32>::type;
-    static_assert(!kTail || (kUniform && !kRoute && TPT > 32), "tail load: vector copy only");
-    TT tail[2];
-#pragma unroll
-    for (int p = 1; p < 3; ++p)
-      if (kTail && p < a.np && gl < a.rb[p] / (int64_t)sizeof(TT))
-        tail[p - 1] = load_src<TT>(reinterpret_cast<const TT*>(a.src[p] + tok * a.rb[p]) + gl);
     uint64_t w0, w1, w2, w3;
     const int nd = token_route<kRoute>(a, tok, lane, gl >> 5, TPT / 32, w0, w1, w2, w3);
     if (nd == 0) continue;
-    if (kTail) {
-      copy_row<TT, U, TPT>(a.src[0] + tok * a.rb[0], a.rb[0], a.rank0, a.rank_stride,
-                           a.dst_off[0] + tok * a.rb[0], w0, w1, w2, w3, nd, gl, kStreaming);
-#pragma unroll
-      for (int p = 1; p < 3; ++p) {
-        if (p >= a.np || gl >= a.rb[p] / (int64_t)sizeof(TT)) continue;
-        const int64_t offp = a.dst_off[p] + tok * a.rb[p];
-        for (int q = 0; q < nd; ++q)
-          store_dst<TT>(reinterpret_cast<TT*>(a.rank0 +
-                                              (int64_t)dst_rank(w0, w1, w2, w3, q) * a.rank_stride +
-                                              offp) + gl,
-                        tail[p - 1], kStreaming);
-      }
-      continue;
-    }
     for (int p = 0; p < a.np; ++p) {
       const uint8_t* src = a.src[p] + tok * a.rb[p];
       const int64_t off = a.dst_off[p] + tok * a.rb[p];
@@ -773,19 +743,6 @@ cudaError_t launch_vec_utr(const CopyArgs& a, int grid, bool streaming, cudaStre
     all32 &= a.vec[p] == 32;
   }
   const dim3 g(grid), b(kVecThreads);
-  if constexpr (!kRoute && TPT > 32) {
-    // the instance that loads a second row of at most one vector per thread early
-    bool tail_fits = a.np == 2 || a.np == 3;
-    for (int p = 1; p < a.np; ++p) tail_fits = tail_fits && a.rb[p] / (int64_t)a.vec[p] <= TPT;
-    if (a.tail && tail_fits && all32)
-      return launch_kernel(streaming ? dispatch_vec_kernel<U, 32, true, TPT, false, true>
-                                     : dispatch_vec_kernel<U, 32, false, TPT, false, true>,
-                           g, b, 0, stream, pdl, a);
-    if (a.tail && tail_fits && all16)
-      return launch_kernel(streaming ? dispatch_vec_kernel<U, 16, true, TPT, false, true>
-                                     : dispatch_vec_kernel<U, 16, false, TPT, false, true>,
-                           g, b, 0, stream, pdl, a);
-  }
   if (all32) {
     if (streaming)
       return launch_kernel(dispatch_vec_kernel<U, 32, true, TPT, kRoute>, g, b, 0, stream, pdl,

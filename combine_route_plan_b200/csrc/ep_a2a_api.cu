@@ -148,7 +148,6 @@ struct ep_a2a_handle_s {
   int copy_ctas_per_sm;
   int route_in_copy;      // vector copy path: 1 = the copy kernel also routes (one launch)
   int fp8_experts_kernel;   // sender-side FP8 expert combine: 0 split, 1 cluster, 2 one CTA
-  int copy_tail;            // vector copy: small second payload row loaded early
   int copy_stages;        // 0 = choose from the row size
   int combine_threads;
   int64_t bulk_min_row;   // rows below this go to the vector copy
@@ -382,7 +381,6 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   // cluster kernel (decode 83 against 175 us).
   h->route_in_copy = 0;
   h->fp8_experts_kernel = 0;
-  h->copy_tail = 0;
   h->copy_stages = 4;
   h->combine_threads = 0;
   h->bulk_min_row = 0;
@@ -482,10 +480,6 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       if (value < 0 || value > 2)
         return fail(EP_A2A_ERR_INVALID_ARG, "FP8 experts kernel must be 0, 1 or 2");
       h->fp8_experts_kernel = (int)value;
-      return EP_A2A_OK;
-    case EP_A2A_OPT_COPY_TAIL_EARLY:
-      if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "tail option must be 0 or 1");
-      h->copy_tail = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_ROUTE_IN_COPY:
       if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "route in copy must be 0 or 1");
@@ -613,7 +607,6 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
   std::memcpy(bulk.live, ra.live, sizeof(bulk.live));
   bulk.ep = ep;
   vec = bulk;
-  vec.tail = h->copy_tail;
   if (fused) {
     vec.route = 1;
     vec.invalid_id = ra.invalid_id;

@@ -113,7 +113,6 @@ struct CopyArgs {
   int eplb_n;
   int32_t n[kMaxRanks];                  // local_num_tokens (0 for masked-off ranks)
   uint64_t live[kMaskWords];
-  int tail;                              // vector path: load a small second row early
 };
 
 cudaError_t launch_dispatch_bulk(const CopyArgs& a, int grid, cudaStream_t stream, bool pdl);

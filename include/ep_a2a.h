@@ -392,13 +392,7 @@ typedef enum {
                                      through distributed shared memory; 1 = a cluster per
                                      token with one column vector per thread and the rows
                                      in registers (hidden up to 16384); 2 = one CTA per
-                                     token with the whole rows in shared memory */,
-  EP_A2A_OPT_COPY_TAIL_EARLY = 19 /* vector copy with more than 32 threads per token and
-                                     two or three payloads whose rows after the first
-                                     are at most one vector per thread each: 1 = those
-                                     rows are loaded before the token is routed and
-                                     stored after the first row; 0 (default) = in
-                                     payload order */
+                                     token with the whole rows in shared memory */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

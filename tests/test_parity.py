@@ -80,48 +80,6 @@ def test_routing_inside_the_copy_bit_exact(name):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("name", ["c3_ep16_zipf_nvfp4", "c3_ep16_zipf_mxfp8", "c3_ep16_zipf_dsfp8"])
-def test_copy_tail_row_loaded_early_bit_exact(name):
-    """The copy that loads a small second payload row (block scales) before
-    routing the token and stores it after the first row."""
-    from combine_route_plan_b200 import ep_a2a
-    _full_check(W.BY_NAME[name], options={ep_a2a.OPT_COPY_TAIL_EARLY: 1})
-
-
-@pytest.mark.parametrize("tpt", [64, 128, 256])
-@pytest.mark.parametrize("rows,shift", [([3584, 224], 0), ([3584, 32], 0), ([4096 + 16, 48], 0),
-                                        ([7168, 448], 16), ([512, 64, 32], 0),
-                                        ([3584, 448, 32], 0), ([7168, 224, 32], 16),
-                                        ([512, 64, 32, 32], 0), ([512, 4096, 32], 0)])
-def test_copy_tail_rows_and_threads(tpt, rows, shift):
-    """Rows after the first from one vector to one per thread, 16- and 32-byte
-    vectors, two and three payloads, ragged token counts and a masked rank;
-    four payloads and a long later row (not taken early)."""
-    from combine_route_plan_b200 import ep_a2a
-    ep, E, k, tpr, H = 8, 64, 8, 43, 32
-    w, x = _custom(ep, E, k, tpr, H, rows, n=[43, 42, 0, 7, 43, 1, 43, 30],
-                   mask=_mask_of(ep, [0, 1, 2, 3, 4, 5, 7]), seed=tpt + sum(rows) % 89 + shift)
-    comm = ep_a2a.EpA2A(ep, E, k, tpr, H, rows, enable_rank_mask=True, workspace_fill=U.CANARY)
-    comm.set_option(ep_a2a.OPT_COPY_TAIL_EARLY, 1)
-    comm.set_option(ep_a2a.OPT_VEC_THREADS_PER_TOKEN, tpt)
-    srcs = []
-    for p in x.payloads:
-        buf = torch.empty(p.numel() + 64, dtype=torch.uint8, device="cuda")
-        v = buf[shift: shift + p.numel()].view(p.shape)
-        v.copy_(p.cuda())
-        srcs.append(v)
-    d = comm.dispatch(x.token_selected_experts.cuda(), x.local_num_tokens, srcs, tpr,
-                      active_rank_mask=x.active_rank_mask)
-    torch.cuda.synchronize()
-    assert comm.get_status() == ep_a2a.OK
-    plan = U.oracle_plan(w, x)
-    for i, p in enumerate(x.payloads):
-        for dst in range(ep):
-            want = U.oracle.dispatch_payload(plan, p.numpy(), only_dst=dst, recv_init=np.full(
-                (1, ep * tpr, p.shape[2]), U.CANARY, np.uint8))
-            U.assert_equal(d.recv_payloads[i][dst], want, f"payload {i} rank {dst} tpt {tpt}")
-
-
 @pytest.mark.parametrize("name,path", [
     (n, p) for n in ("c1_ep4_tiny", "c2_ep8_decode", "c5_ep64_wide_masked", "c3_ep16_zipf_nvfp4")
     for p in (0, 2)])
