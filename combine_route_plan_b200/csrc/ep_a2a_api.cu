@@ -225,13 +225,19 @@ struct CombineLaunch {
 //  * BF16: one vector at a time (pipelining was 1-12 % slower); from 16384
 //    token slots 64 threads, 128 CTAs per SM requested, no prefetch; from 8192
 //    128 threads and a one-token prefetch (Zipf step: 98 against 103 us);
-//    below that 256 threads and 16 CTAs per SM (wide-EP step: 51 against
-//    55 us; decode 26.1 against 26.7 us), no prefetch;
-//  * FP8 and scaled FP8: pipelined (27-54 % faster); 64 threads below 16384
-//    token slots and 128 from there; from 8192 slots on, prefetch one token
-//    ahead (faster by 5-10 %, slower by 5-10 % on the small steps); 16 CTAs per
-//    SM requested from 16384 slots on (scaled: 291 against 310 us), else 128;
-//  * expert outputs: pipelined (24-28 % faster), 64 threads, no prefetch.
+//    below that 16 CTAs per SM and no prefetch, with 256 threads (wide-EP
+//    step: 51 against 55 us), or 192 at up to 8 token slots per SM (decode:
+//    five rounds of column vectors per token at four CTAs per SM beat four
+//    rounds at three, the tokens then fitting in two waves instead of three:
+//    44.9 against 46.5 us per step);
+//  * FP8 and scaled FP8: pipelined (27-54 % faster); 64 threads up to 16
+//    token slots per SM, 128 above (wide-EP step: 94.6 against 96.4 us); from
+//    8192 slots on, prefetch one token ahead (faster by 5-10 %, slower by 5-10 %
+//    on the small steps); 16 CTAs per SM requested from 16384 slots on
+//    (scaled: 291 against 310 us), else 128;
+//  * expert outputs: pipelined (24-28 % faster), no prefetch; 128 threads
+//    below 8192 token slots with more than 16 per SM (wide-EP step: 129.8
+//    against 132.7 us), else 64.
 // The pipelined kernels hold at most 8 destination rows per token, and a token
 // has at most min(top_k, ep_size) destinations.
 CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
@@ -243,13 +249,15 @@ CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
   // a staged CTA needs two stages of 32 KB: at most three CTAs per SM
   c.staged_ctas_per_sm = h->combine_ctas_per_sm > 0 ? std::min(h->combine_ctas_per_sm, 3) : 2;
   const bool mid = !big && ntok >= 8192;
-  int threads = 64, cps = 128, prefetch = 0;
+  const bool small = ntok < 8192;
+  const int64_t per_sm = ntok / std::max(1, h->num_sms);     // token slots per SM
+  int threads = (small && per_sm > 16) ? 128 : 64, cps = 128, prefetch = 0;
   if (kind == kKindFp8) {
-    threads = big ? 128 : 64;
+    threads = big ? 128 : threads;
     cps = big ? 16 : 128;
     prefetch = ntok >= 8192 ? 1 : 0;
   } else if (kind == kKindBf16) {
-    threads = big ? 64 : (mid ? 128 : 256);
+    threads = big ? 64 : (mid ? 128 : (per_sm <= 8 ? 192 : 256));
     cps = (big || mid) ? 128 : 16;
     prefetch = mid ? 1 : 0;
   }
