@@ -113,8 +113,10 @@ __device__ __forceinline__ void prefetch_token_rows(const CombineArgs& a, int64_
   }
 }
 
-template <bool kFp8>
-__global__ void __launch_bounds__(512) combine_vec_kernel(const CombineArgs a) {
+// kMaxThreads / kMinBlocks: launch bounds of the instance (the 128-thread
+// BF16 instance is held to 72 registers, so that seven CTAs fit on an SM).
+template <bool kFp8, int kMaxThreads = 512, int kMinBlocks = 0>
+__global__ void __launch_bounds__(kMaxThreads, kMinBlocks) combine_vec_kernel(const CombineArgs a) {
   pdl_wait();
   constexpr int kElems = kFp8 ? 16 : 8;       // elements per 16-byte input vector
   constexpr int kElemBytes = kFp8 ? 1 : 2;
@@ -1596,6 +1598,8 @@ cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, bool pipe, 
   }
   if (vec) {
     if (fp8) return launch_kernel(combine_vec_kernel<true>, g, b, 0, stream, pdl, a);
+    if (threads == 128)
+      return launch_kernel(combine_vec_kernel<false, 128, 7>, g, b, 0, stream, pdl, a);
     return launch_kernel(combine_vec_kernel<false>, g, b, 0, stream, pdl, a);
   }
   if (fp8) return launch_kernel(combine_scalar_kernel<true>, g, b, 0, stream, pdl, a);
