@@ -1588,7 +1588,7 @@ __global__ void wait_timeout_probe_kernel(uint32_t* err, unsigned long long limi
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, bool pipe, int threads,
-                           int grid, cudaStream_t stream, bool pdl) {
+                           int grid, cudaStream_t stream, bool pdl, bool tight) {
   const dim3 g(grid), b(threads);
   const float* no_scales = nullptr;
   if (vec && pipe) {
@@ -1598,7 +1598,7 @@ cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, bool pipe, 
   }
   if (vec) {
     if (fp8) return launch_kernel(combine_vec_kernel<true>, g, b, 0, stream, pdl, a);
-    if (threads == 128)
+    if (tight && threads == 128)
       return launch_kernel(combine_vec_kernel<false, 128, 7>, g, b, 0, stream, pdl, a);
     return launch_kernel(combine_vec_kernel<false>, g, b, 0, stream, pdl, a);
   }

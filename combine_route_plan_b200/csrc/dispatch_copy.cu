@@ -479,13 +479,8 @@ __device__ __forceinline__ void finish_counts(const CopyArgs& a) {
 // after it sees the plan complete.  kAll = 16 or 32: every payload of the
 // launch moves in vectors of that many bytes (one code path, fewer registers);
 // kAll = 0: each payload picks its own vector width.
-// The instance of the small steps (a 256-thread group per token, two 32-byte
-// vectors per thread) is held to 32 registers, so that eight CTAs, eight
-// tokens, fit on an SM and a 1024-token step is a single wave.
 template <int U, int kAll, bool kStreaming, int TPT, bool kRoute>
-__global__ void __launch_bounds__(kVecThreads,
-                                  (TPT == 256 && U == 2 && kAll == 32 && !kRoute) ? 7 : 0)
-    dispatch_vec_kernel(const CopyArgs a) {
+__global__ void __launch_bounds__(kVecThreads) dispatch_vec_kernel(const CopyArgs a) {
   constexpr bool kUniform = kAll != 0;
   constexpr int kGroups = kVecThreads / TPT;
   const int gl = threadIdx.x % TPT;

@@ -216,6 +216,7 @@ struct CombineLaunch {
   bool pipe;
   bool staged;               // rows staged in shared memory by bulk-async copies
   int threads, grid, prefetch;
+  bool tight;                // BF16, 128 threads: the instance held to 7 CTAs per SM
   int staged_ctas_per_sm;
 };
 
@@ -226,10 +227,11 @@ struct CombineLaunch {
 //    token slots 64 threads, 128 CTAs per SM requested, no prefetch; from 8192
 //    128 threads and a one-token prefetch (Zipf step: 98 against 103 us);
 //    below that 16 CTAs per SM and no prefetch, with 256 threads (wide-EP
-//    step: 51 against 55 us), or 192 at up to 8 token slots per SM (decode:
-//    five rounds of column vectors per token at four CTAs per SM beat four
-//    rounds at three, the tokens then fitting in two waves instead of three:
-//    44.9 against 46.5 us per step);
+//    step: 51 against 55 us), or at up to 8 token slots per SM 128 threads in
+//    the instance held to 72 registers, seven CTAs per SM: every token of the
+//    decode step in one wave, seven rounds of column vectors per token
+//    (combine 23.6 against 24.8 us with 192 threads, two waves of five rounds,
+//    and 25.6 with 256, three waves of four);
 //  * FP8 and scaled FP8: pipelined (27-54 % faster); 64 threads up to 16
 //    token slots per SM, 128 above (wide-EP step: 94.6 against 96.4 us); from
 //    8192 slots on, prefetch one token ahead (faster by 5-10 %, slower by 5-10 %
@@ -252,16 +254,19 @@ CombineLaunch combine_launch(ep_a2a_handle h, CombineKind kind, int64_t ntok) {
   const bool small = ntok < 8192;
   const int64_t per_sm = ntok / std::max(1, h->num_sms);     // token slots per SM
   int threads = (small && per_sm > 16) ? 128 : 64, cps = 128, prefetch = 0;
+  bool tight = false;
   if (kind == kKindFp8) {
     threads = big ? 128 : threads;
     cps = big ? 16 : 128;
     prefetch = ntok >= 8192 ? 1 : 0;
   } else if (kind == kKindBf16) {
-    threads = big ? 64 : (mid ? 128 : (per_sm <= 8 ? 192 : 256));
+    threads = big ? 64 : (mid ? 128 : (per_sm <= 8 ? 128 : 256));
+    tight = !big && !mid && per_sm <= 8;
     cps = (big || mid) ? 128 : 16;
     prefetch = mid ? 1 : 0;
   }
   c.threads = h->combine_threads > 0 ? h->combine_threads : threads;
+  c.tight = tight && c.threads == 128;
   if (h->combine_ctas_per_sm > 0) cps = h->combine_ctas_per_sm;
   c.grid = (int)std::max<int64_t>(1, std::min<int64_t>(ntok, (int64_t)h->num_sms * cps));
   c.prefetch = h->combine_prefetch >= 0 ? h->combine_prefetch : prefetch;
@@ -751,7 +756,7 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
                               h->pdl != 0);
   else
     e = launch_combine(a, fp8, vec, c.pipe, c.threads, c.grid, (cudaStream_t)stream_v,
-                       h->pdl != 0);
+                       h->pdl != 0, c.tight);
   prof_end(h, slot, (cudaStream_t)stream_v);
   if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
   return EP_A2A_OK;

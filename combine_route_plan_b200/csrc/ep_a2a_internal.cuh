@@ -142,9 +142,10 @@ struct CombineArgs {
                                // vector (output 32-byte aligned)
 };
 
-// pipe: the two-deep pipelined kernel (needs at most 8 destinations per token)
+// pipe: the two-deep pipelined kernel (needs at most 8 destinations per token);
+// tight with 128 threads: the BF16 one-vector instance held to seven CTAs per SM
 cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, bool pipe, int threads,
-                           int grid, cudaStream_t stream, bool pdl);
+                           int grid, cudaStream_t stream, bool pdl, bool tight = false);
 
 // Combine of per-(token, slot) expert outputs: the weighted reduction over each
 // destination's local experts fused into the combine.
