@@ -597,101 +597,6 @@ __global__ void __launch_bounds__(512) combine_experts_vec_kernel(const CombineE
 }
 
 // Loads of one 16-byte column vector of each slot row that takes part.
-// A token's participating slots in destination-major order (ascending
-// destination position, ascending slot within a destination, the order of the
-// sums): position p holds slot slot_off[p] / H with weight w_at[p]; bit p of
-// ends is set where a destination's last slot sits; ns positions in all.  Every
-// index is static, so the rows and weights stay in registers.
-struct SlotOrder {
-  int32_t slot_off[8];     // slot * H (elements)
-  float w_at[8];
-  uint32_t ends;
-  int ns;
-};
-
-__device__ __forceinline__ SlotOrder order_slots(const int (&own)[8], const float (&wt)[8],
-                                                 int nd, uint64_t w0, int H) {
-  int q[8];                                 // destination position of each slot, -1 if none
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    q[j] = -1;
-    for (int i = 0; i < nd; ++i)
-      if (own[j] >= 0 && (int)((w0 >> (8 * i)) & 0xFFu) == own[j]) q[j] = i;
-  }
-  SlotOrder o;
-  o.ns = 0;
-  o.ends = 0u;
-#pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    o.slot_off[p] = 0;
-    o.w_at[p] = 0.0f;
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (q[j] < 0) continue;
-    int pos = 0;
-    bool last = true;                       // no later slot of the same destination
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      pos += q[i] >= 0 && (q[i] < q[j] || (q[i] == q[j] && i < j));
-      last = last && !(q[i] == q[j] && i > j);
-    }
-#pragma unroll
-    for (int p = 0; p < 8; ++p)
-      if (p == pos) {
-        o.slot_off[p] = j * H;
-        o.w_at[p] = wt[j];
-      }
-    o.ends |= (last ? 1u : 0u) << pos;
-    ++o.ns;
-  }
-  return o;
-}
-
-__device__ __forceinline__ void ordered_rows_load(uint4 (&r)[8], const uint16_t* yv,
-                                                  const SlotOrder& so) {
-#pragma unroll
-  for (int p = 0; p < 8; ++p)
-    if (p < so.ns) r[p] = ld_stream_v4(yv + so.slot_off[p]);
-}
-
-// The sum of combine_experts: z_d over each destination's slots (fused
-// multiply-adds in ascending slot order), rounded to bf16 in pairs and added
-// widened in ascending destination order; the rows in destination-major order.
-__device__ __forceinline__ void ordered_rows_reduce_store(const uint4 (&raw)[8],
-                                                          const SlotOrder& so, uint16_t* o) {
-  float acc[8], z[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    acc[e] = 0.0f;
-    z[e] = 0.0f;
-  }
-#pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    if (p >= so.ns) break;
-    const uint32_t wv[4] = {raw[p].x, raw[p].y, raw[p].z, raw[p].w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      z[2 * i] = __fmaf_rn(so.w_at[p], bf16_bits_to_f32(wv[i] & 0xFFFFu), z[2 * i]);
-      z[2 * i + 1] = __fmaf_rn(so.w_at[p], bf16_bits_to_f32(wv[i] >> 16), z[2 * i + 1]);
-    }
-    if ((so.ends >> p) & 1u) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        add_bf16x2(acc[2 * e], acc[2 * e + 1], pack_bf16x2(z[2 * e], z[2 * e + 1]));
-        z[2 * e] = 0.0f;
-        z[2 * e + 1] = 0.0f;
-      }
-    }
-  }
-  uint4 pk;
-  pk.x = pack_bf16x2(acc[0], acc[1]);
-  pk.y = pack_bf16x2(acc[2], acc[3]);
-  pk.z = pack_bf16x2(acc[4], acc[5]);
-  pk.w = pack_bf16x2(acc[6], acc[7]);
-  *reinterpret_cast<uint4*>(o) = pk;
-}
-
 __device__ __forceinline__ void expert_rows_load(uint4 (&r)[8], const uint16_t* yv,
                                                  const int (&own)[8], int H) {
 #pragma unroll
@@ -767,21 +672,20 @@ __global__ void __launch_bounds__(512) combine_experts_pipe_kernel(const Combine
     int own[8];
     float wt[8];
     slot_owners<8>(a, tok, nd, w0, 0, 0, 0, own, wt);
-    const SlotOrder so = order_slots(own, wt, nd, w0, a.H);
     const uint16_t* yv = a.y + tok * (int64_t)a.k * a.H + (int64_t)threadIdx.x * 8;
     uint4 ra[8], rb[8];
-    ordered_rows_load(ra, yv, so);
+    expert_rows_load(ra, yv, own, a.H);
     for (int v = threadIdx.x;;) {
       const bool more_b = v + (int)blockDim.x < nvec;
-      if (more_b) ordered_rows_load(rb, yv + step, so);
-      ordered_rows_reduce_store(ra, so, o);
+      if (more_b) expert_rows_load(rb, yv + step, own, a.H);
+      expert_rows_reduce_store(ra, own, wt, nd, w0, o);
       if (!more_b) break;
       v += blockDim.x;
       yv += step;
       o += step;
       const bool more_a = v + (int)blockDim.x < nvec;
-      if (more_a) ordered_rows_load(ra, yv + step, so);
-      ordered_rows_reduce_store(rb, so, o);
+      if (more_a) expert_rows_load(ra, yv + step, own, a.H);
+      expert_rows_reduce_store(rb, own, wt, nd, w0, o);
       if (!more_a) break;
       v += blockDim.x;
       yv += step;
