@@ -377,12 +377,12 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   h->copy_consumer_warps = 4;
   h->copy_interleave = 1;
   h->vec_unroll = 0;
-  h->vec_ctas_per_sm = 32;
+  h->vec_ctas_per_sm = 0;        // automatic (copy launch below)
   h->store_streaming = 1;
   h->pdl = 1;
   h->vec_threads_per_token = 0;
   h->combine_prefetch = -1;       // automatic (combine_launch)
-  h->copy_prefetch = 0;
+  h->copy_prefetch = -1;         // automatic
   h->copy_vec_bytes = 32;
   h->combine_pipeline = -1;
   h->copy_ctas_per_sm = 1;
@@ -442,8 +442,9 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       h->vec_unroll = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_VEC_CTAS_PER_SM:
-      if (value < 1 || value > 64)
-        return fail(EP_A2A_ERR_INVALID_ARG, "vector copy CTAs per SM must be 1..64");
+      if (value < 0 || value > 64)
+        return fail(EP_A2A_ERR_INVALID_ARG,
+                    "vector copy CTAs per SM must be 0 (automatic) or 1..64");
       h->vec_ctas_per_sm = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_STORE_STREAMING:
@@ -472,7 +473,8 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       h->combine_pipeline = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_COPY_PREFETCH:
-      if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "prefetch must be 0 or 1");
+      if (value < -1 || value > 1)
+        return fail(EP_A2A_ERR_INVALID_ARG, "prefetch must be -1 (automatic), 0 or 1");
       h->copy_prefetch = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_PDL:
@@ -695,9 +697,18 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
     const int tpt = h->vec_threads_per_token > 0 ? h->vec_threads_per_token
                                                  : copy_threads_per_token(ntok, row_vectors);
     const int64_t groups_per_cta = 256 / tpt;
+    // CTAs per SM and next-token prefetch: with at most 8 token slots per SM
+    // and a 256-thread group per token, the four CTAs an SM holds loop over
+    // the tokens and ask for each one's next token's rows to be brought into
+    // L2 (decode step: 42.6 against 44.2-44.9 us per step; no gain on the
+    // Zipf or wide-EP steps, where the default is 32 CTAs per SM requested and
+    // no prefetch)
+    const bool few = ntok <= (int64_t)8 * h->num_sms && tpt == 256;
+    const int cps = h->vec_ctas_per_sm > 0 ? h->vec_ctas_per_sm : (few ? 4 : 32);
+    vec.prefetch = h->copy_prefetch >= 0 ? h->copy_prefetch : (few ? 1 : 0);
     const int grid = (int)std::max<int64_t>(
         1, std::min<int64_t>((ntok + groups_per_cta - 1) / groups_per_cta,
-                             (int64_t)h->num_sms * h->vec_ctas_per_sm));
+                             (int64_t)h->num_sms * cps));
     const int unroll = h->vec_unroll > 0 ? h->vec_unroll : copy_unroll(row_vectors, tpt);
     slot = prof_begin(h, EP_A2A_KERNEL_COPY_VEC, stream);
     e = launch_dispatch_vec(vec, grid, unroll, tpt, h->store_streaming != 0, stream, pdl);

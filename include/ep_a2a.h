@@ -347,7 +347,9 @@ typedef enum {
   EP_A2A_OPT_VEC_UNROLL = 8,      /* vector copy: vectors per lane in flight (2, 4, 8; 0 =
                                      default: the fewest that move the largest row in
                                      two rounds) */
-  EP_A2A_OPT_VEC_CTAS_PER_SM = 9, /* vector copy grid = SMs x this (1..64; default 32) */
+  EP_A2A_OPT_VEC_CTAS_PER_SM = 9, /* vector copy grid = SMs x this (1..64); 0 (default) =
+                                     automatic: 4 with at most 8 token slots per SM and
+                                     256 threads per token, else 32 */
   EP_A2A_OPT_STORE_STREAMING = 10,/* vector copy: 1 = evict-first (.cs) stores
                                      (default), 0 = plain stores */
   EP_A2A_OPT_PDL = 11,            /* 1 (default): each kernel of the path may start while
@@ -364,7 +366,9 @@ typedef enum {
                                      one; 0 = never; -1 (default) = automatic: 1 for the
                                      FP8 combines from 8192 token slots and the BF16
                                      combine from 8192 to 16383, else 0 */
-  EP_A2A_OPT_COPY_PREFETCH = 14,  /* vector copy: 1 = the same for the next token's rows */
+  EP_A2A_OPT_COPY_PREFETCH = 14,  /* vector copy: 1 = the same for the next token's rows;
+                                     0 = never; -1 (default) = automatic: 1 where the
+                                     automatic grid is 4 CTAs per SM, else 0 */
   EP_A2A_OPT_COMBINE_PIPELINE = 15,/* BF16 / FP8 / scaled FP8 combines of 16-byte vectors
                                      with at most 8 destinations per token (top_k or
                                      ep_size <= 8): 1 = each thread keeps the loads of its
