@@ -115,7 +115,7 @@ __device__ __forceinline__ void prefetch_token_rows(const CombineArgs& a, int64_
 
 // kMaxThreads / kMinBlocks: launch bounds of the instance (the 128-thread
 // BF16 instance is held to 72 registers, so that seven CTAs fit on an SM).
-template <bool kFp8, int kMaxThreads = 512, int kMinBlocks = 0, bool kCompact = false>
+template <bool kFp8, int kMaxThreads = 512, int kMinBlocks = 0>
 __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) combine_vec_kernel(const CombineArgs a) {
   pdl_wait();
   constexpr int kElems = kFp8 ? 16 : 8;       // elements per 16-byte input vector
@@ -125,14 +125,7 @@ __global__ void __launch_bounds__(kMaxThreads, kMinBlocks) combine_vec_kernel(co
   if (a.prefetch && threadIdx.x == 0)
     for (int p = 0; p < a.prefetch; ++p)
       prefetch_token_rows<kElemBytes>(a, blockIdx.x + (int64_t)p * gridDim.x);
-  __shared__ int32_t s_prefix[kCompact ? kMaxRanks + 1 : 1];
-  if (kCompact) {
-    for (int i = threadIdx.x; i <= a.ep; i += blockDim.x) s_prefix[i] = a.prefix[i];
-    __syncthreads();
-  }
-  const int64_t items = kCompact ? (int64_t)s_prefix[a.ep] : a.ntok;
-  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
-    const int64_t tok = kCompact ? existing_slot(s_prefix, a.ep, a.tpr, item) : item;
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
     if (a.prefetch && threadIdx.x == 0)
       prefetch_token_rows<kElemBytes>(a, tok + (int64_t)a.prefetch * gridDim.x);
     const int nd = a.plan_nd[tok];
@@ -254,7 +247,7 @@ __device__ __forceinline__ void reduce_store(const uint4 (&r)[8], const float (&
 // combine_scaled_kernel<true>, with each thread's loads pipelined two deep --
 // the rows of its next column vector are in flight while it adds the current
 // one, so a thread never waits on memory with its adds still to do.
-template <int kMode, bool kCompact = false>
+template <int kMode>
 __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
                                                            const float* __restrict__ scales) {
   pdl_wait();
@@ -266,14 +259,7 @@ __global__ void __launch_bounds__(512) combine_pipe_kernel(const CombineArgs a,
   if (a.prefetch && threadIdx.x == 0)
     for (int p = 0; p < a.prefetch; ++p)
       prefetch_token_rows<kElemBytes>(a, blockIdx.x + (int64_t)p * gridDim.x);
-  __shared__ int32_t s_prefix[kCompact ? kMaxRanks + 1 : 1];
-  if (kCompact) {
-    for (int i = threadIdx.x; i <= a.ep; i += blockDim.x) s_prefix[i] = a.prefix[i];
-    __syncthreads();
-  }
-  const int64_t items = kCompact ? (int64_t)s_prefix[a.ep] : a.ntok;
-  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
-    const int64_t tok = kCompact ? existing_slot(s_prefix, a.ep, a.tpr, item) : item;
+  for (int64_t tok = blockIdx.x; tok < a.ntok; tok += gridDim.x) {
     if (a.prefetch && threadIdx.x == 0)
       prefetch_token_rows<kElemBytes>(a, tok + (int64_t)a.prefetch * gridDim.x);
     const int nd = a.plan_nd[tok];
@@ -1606,9 +1592,6 @@ cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, bool pipe, 
   const dim3 g(grid), b(threads);
   const float* no_scales = nullptr;
   if (vec && pipe) {
-    if (fp8 && a.compact)
-      return launch_kernel(combine_pipe_kernel<kCombineFp8, true>, g, b, 0, stream, pdl, a,
-                           no_scales);
     if (fp8) return launch_kernel(combine_pipe_kernel<kCombineFp8>, g, b, 0, stream, pdl, a,
                                   no_scales);
     return launch_kernel(combine_pipe_kernel<kCombineBf16>, g, b, 0, stream, pdl, a, no_scales);
@@ -1617,8 +1600,6 @@ cudaError_t launch_combine(const CombineArgs& a, bool fp8, bool vec, bool pipe, 
     if (fp8) return launch_kernel(combine_vec_kernel<true>, g, b, 0, stream, pdl, a);
     if (tight && threads == 128)
       return launch_kernel(combine_vec_kernel<false, 128, 7>, g, b, 0, stream, pdl, a);
-    if (a.compact)
-      return launch_kernel(combine_vec_kernel<false, 512, 0, true>, g, b, 0, stream, pdl, a);
     return launch_kernel(combine_vec_kernel<false>, g, b, 0, stream, pdl, a);
   }
   if (fp8) return launch_kernel(combine_scalar_kernel<true>, g, b, 0, stream, pdl, a);
@@ -1665,10 +1646,7 @@ cudaError_t launch_combine_scaled(const CombineArgs& a, const float* scales, boo
                                   int threads, int grid, cudaStream_t stream, bool pdl) {
   const dim3 g(grid), b(threads);
   if (vec && pipe)
-    return a.compact ? launch_kernel(combine_pipe_kernel<kCombineFp8Scaled, true>, g, b, 0,
-                                     stream, pdl, a, scales)
-                     : launch_kernel(combine_pipe_kernel<kCombineFp8Scaled>, g, b, 0, stream,
-                                     pdl, a, scales);
+    return launch_kernel(combine_pipe_kernel<kCombineFp8Scaled>, g, b, 0, stream, pdl, a, scales);
   if (vec) return launch_kernel(combine_scaled_kernel<true>, g, b, 0, stream, pdl, a, scales);
   return launch_kernel(combine_scaled_kernel<false>, g, b, 0, stream, pdl, a, scales);
 }

@@ -39,7 +39,6 @@ ep_a2a_status cuda_fail(cudaError_t e, const char* what) {
 // Byte offsets of everything in the workspace.
 struct Layout {
   int64_t off_err, off_count_acc, off_ticket, off_counts, off_plan_nd, off_plan_dst;
-  int64_t off_prefix;        // [ep + 1] int32: existing tokens per source rank, prefix sums
   int64_t ctrl_bytes;        // [0, ctrl_bytes) is cleared at init
   int64_t rank_base;         // rank 0's region
   int64_t rank_stride;       // bytes per rank region
@@ -95,7 +94,6 @@ Layout make_layout(const ep_a2a_params& p) {
   L.off_count_acc = c;  c = align_up(c + ep * ep * 4, kAlign);
   L.off_ticket = c;     c = align_up(c + ep * 4, kAlign);
   L.off_counts = c;     c = align_up(c + ep * ep * 4, kAlign);
-  L.off_prefix = c;     c = align_up(c + (ep + 1) * 4, kAlign);
   L.off_plan_nd = c;    c = align_up(c + slots, kAlign);
   L.off_plan_dst = c;   c = align_up(c + slots * L.plan_stride, kAlign);
   L.ctrl_bytes = c;
@@ -132,8 +130,6 @@ struct ep_a2a_handle_s {
   int max_smem_optin;
   bool have_plan;
   int last_tpr;
-  int32_t last_n[kMaxRanks];   // the last dispatch's token counts (0 for masked ranks)
-  bool last_routed;            // the last dispatch ran the routing kernel (prefix written)
   int combine_hidden;     // row length of the combines, 1..p.hidden_size
   // tuning
   int copy_path;          // 0 staged, 1 vector only, 2 bulk loads + bulk stores
@@ -152,7 +148,6 @@ struct ep_a2a_handle_s {
   int copy_ctas_per_sm;
   int route_in_copy;      // vector copy path: 1 = the copy kernel also routes (one launch)
   int fp8_experts_kernel;   // sender-side FP8 expert combine: 0 split, 1 cluster, 2 one CTA
-  int combine_compact;      // vector combines below 8192 slots: existing tokens only
   int copy_stages;        // 0 = choose from the row size
   int combine_threads;
   int64_t bulk_min_row;   // rows below this go to the vector copy
@@ -216,20 +211,6 @@ int64_t largest_row_vectors(const CopyArgs& c) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 enum CombineKind { kKindBf16, kKindFp8, kKindExperts };
-
-// Iterate the vector combines over the existing tokens only (ragged or masked
-// ranks leave empty slots, each of which would cost a CTA a load of its plan
-// entry to find it empty) on steps below 8192 token slots; the larger steps
-// prefetch by slot and keep the slot order.
-int64_t set_compact(ep_a2a_handle h, CombineArgs& a) {
-  int64_t total = 0;
-  for (int r = 0; r < h->p.ep_size; ++r) total += h->last_n[r];
-  a.prefix = reinterpret_cast<const int32_t*>(h->ws + h->L.off_prefix);
-  a.tpr = h->last_tpr;
-  a.compact = a.ntok < 8192 && total < a.ntok && h->combine_compact != 0 && h->last_routed ? 1 : 0;
-  if (a.compact) a.prefetch = 0;
-  return total;
-}
 
 struct CombineLaunch {
   bool pipe;
@@ -413,7 +394,6 @@ EP_API ep_a2a_status ep_a2a_init(const ep_a2a_params* params, void* workspace,
   // cluster kernel (decode 83 against 175 us).
   h->route_in_copy = 0;
   h->fp8_experts_kernel = 0;
-  h->combine_compact = 1;
   h->copy_stages = 4;
   h->combine_threads = 0;
   h->bulk_min_row = 0;
@@ -516,10 +496,6 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
         return fail(EP_A2A_ERR_INVALID_ARG, "FP8 experts kernel must be 0, 1 or 2");
       h->fp8_experts_kernel = (int)value;
       return EP_A2A_OK;
-    case EP_A2A_OPT_COMBINE_COMPACT:
-      if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "compact must be 0 or 1");
-      h->combine_compact = (int)value;
-      return EP_A2A_OK;
     case EP_A2A_OPT_ROUTE_IN_COPY:
       if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "route in copy must be 0 or 1");
       h->route_in_copy = (int)value;
@@ -610,7 +586,6 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
   ra.plan_stride = L.plan_stride;
   ra.eplb_n = p.eplb_stats_num_experts;
   ra.invalid_id = p.invalid_expert_id;
-  ra.prefix_out = reinterpret_cast<int32_t*>(h->ws + L.off_prefix);
   // On the vector copy path the copy kernel routes each token itself and writes
   // everything the routing kernel would (one launch per dispatch); the bulk
   // paths read the plan, so they run after the routing kernel.
@@ -756,8 +731,6 @@ EP_API ep_a2a_status ep_a2a_dispatch(ep_a2a_handle h, const int32_t* token_selec
   result->plan_stride = L.plan_stride;
   h->have_plan = true;
   h->last_tpr = tpr;
-  std::memcpy(h->last_n, ra.n, sizeof(int32_t) * ep);
-  h->last_routed = !fused;
   return EP_A2A_OK;
 }
 
@@ -771,7 +744,7 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   if (dtype != EP_A2A_COMBINE_BF16 && dtype != EP_A2A_COMBINE_FP8_E4M3)
     return fail(EP_A2A_ERR_INVALID_ARG, "unknown combine dtype %d", (int)dtype);
   const bool fp8 = dtype == EP_A2A_COMBINE_FP8_E4M3;
-  CombineArgs a{};
+  CombineArgs a;
   a.plan_nd = h->ws + h->L.off_plan_nd;
   a.plan_dst = h->ws + h->L.off_plan_dst;
   a.x = static_cast<const uint8_t*>(expert_output);
@@ -781,10 +754,8 @@ EP_API ep_a2a_status ep_a2a_combine(ep_a2a_handle h, const void* expert_output,
   a.plan_stride = h->L.plan_stride;
   a.ep = h->p.ep_size;
   a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
-  CombineLaunch c = combine_launch(h, fp8 ? kKindFp8 : kKindBf16, a.ntok);
+  const CombineLaunch c = combine_launch(h, fp8 ? kKindFp8 : kKindBf16, a.ntok);
   a.prefetch = c.prefetch;
-  const int64_t existing = set_compact(h, a);
-  if (a.compact) c.grid = (int)std::max<int64_t>(1, std::min<int64_t>(existing, c.grid));
   a.out32 = aligned(output, 32) ? 1 : 0;
   const int elems = fp8 ? 16 : 8;
   const bool vec = a.H % elems == 0 && aligned(expert_output, 16) && aligned(output, 16);
@@ -945,7 +916,7 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
   if (!h->have_plan) return fail(EP_A2A_ERR_NO_PLAN, "combine needs a preceding dispatch");
   if (!expert_output_e4m3 || !row_scales || !output)
     return fail(EP_A2A_ERR_INVALID_ARG, "expert_output / row_scales / output is NULL");
-  CombineArgs a{};
+  CombineArgs a;
   a.plan_nd = h->ws + h->L.off_plan_nd;
   a.plan_dst = h->ws + h->L.off_plan_dst;
   a.x = static_cast<const uint8_t*>(expert_output_e4m3);
@@ -955,10 +926,8 @@ EP_API ep_a2a_status ep_a2a_combine_scaled(ep_a2a_handle h, const void* expert_o
   a.plan_stride = h->L.plan_stride;
   a.ep = h->p.ep_size;
   a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
-  CombineLaunch c = combine_launch(h, kKindFp8, a.ntok);
+  const CombineLaunch c = combine_launch(h, kKindFp8, a.ntok);
   a.prefetch = c.prefetch;
-  const int64_t existing = set_compact(h, a);
-  if (a.compact) c.grid = (int)std::max<int64_t>(1, std::min<int64_t>(existing, c.grid));
   a.out32 = aligned(output, 32) ? 1 : 0;
   const bool vec = a.H % 16 == 0 && aligned(expert_output_e4m3, 16) && aligned(output, 16);
   const int slot = prof_begin(h, EP_A2A_KERNEL_COMBINE, (cudaStream_t)stream_v);

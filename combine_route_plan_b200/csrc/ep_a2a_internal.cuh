@@ -68,7 +68,6 @@ struct RouteArgs {
   int32_t n[kMaxRanks];        // local_num_tokens, 0 for masked-off ranks
   uint64_t live[kMaskWords];   // bit r = rank r active
   int vec_ids;                 // set by launch_route_plan: ids rows as 16-byte stores
-  int32_t* prefix_out;         // [ep + 1] prefix sums of n, or nullptr
 };
 
 cudaError_t launch_route_plan(const RouteArgs& a, bool use_mask, cudaStream_t stream,
@@ -141,25 +140,7 @@ struct CombineArgs {
   uint32_t* err;               // device error word (checked builds)
   int out32;                   // pipelined E4M3 combines: one 32-byte store per
                                // vector (output 32-byte aligned)
-  // compact (the instances that walk the existing tokens only): rank r's
-  // existing tokens are the slots r * tpr + [0, prefix[r + 1] - prefix[r]),
-  // prefix [ep + 1] in device memory, written by the routing kernel
-  const int32_t* prefix;
-  int tpr;
-  int compact;
 };
-
-// Token slot of the item-th existing token: the rank found by binary search
-// over the prefix counts (a copy in shared memory).
-__device__ __forceinline__ int64_t existing_slot(const int32_t* s_prefix, int ep, int tpr,
-                                                 int64_t item) {
-  int lo = 0, hi = ep;                   // prefix[lo] <= item < prefix[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (s_prefix[mid] <= item) lo = mid; else hi = mid;
-  }
-  return (int64_t)lo * tpr + (item - s_prefix[lo]);
-}
 
 // pipe: the two-deep pipelined kernel (needs at most 8 destinations per token);
 // tight with 128 threads: the BF16 one-vector instance held to seven CTAs per SM

@@ -663,7 +663,7 @@ EP_API ep_a2a_status ep_mp_combine_finish(ep_mp_handle h, void* output, ep_a2a_c
   // The ordered sum over the landing rows [ep(d), tpr, H] with this rank's
   // plan: the single-process combine kernels with one source rank.
   const bool fp8 = dtype == EP_A2A_COMBINE_FP8_E4M3;
-  CombineArgs c{};
+  CombineArgs c;
   c.plan_nd = own + h->L.off_plan_nd;
   c.plan_dst = own + h->L.off_plan_dst;
   c.x = own + h->L.off_landing;

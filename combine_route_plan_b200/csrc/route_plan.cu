@@ -77,16 +77,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_plan_kernel(const RouteAr
   // what this kernel writes, so it may run alongside; the combine after it
   // still waits for this grid (through the copy's final wait).
   pdl_launch_dependents();
-  if (a.prefix_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-    // prefix sums of the existing tokens per source rank, for the combines
-    // that walk the existing tokens only
-    int32_t sum = 0;
-    a.prefix_out[0] = 0;
-    for (int q = 0; q < a.ep; ++q) {
-      sum += a.n[q];
-      a.prefix_out[q + 1] = sum;
-    }
-  }
   const int r = blockIdx.y;
   if (r == a.ep) {  // the extra row of blocks gathers EPLB statistics
     eplb_gather<kMask>(a);

@@ -37,7 +37,7 @@ OPT_COPY_PATH, OPT_COPY_CTAS_PER_SM, OPT_COPY_STAGES, OPT_COMBINE_THREADS, \
     OPT_COPY_INTERLEAVE, OPT_VEC_UNROLL, OPT_VEC_CTAS_PER_SM, OPT_STORE_STREAMING, \
     OPT_PDL, OPT_VEC_THREADS_PER_TOKEN, OPT_COMBINE_PREFETCH, OPT_COPY_PREFETCH, \
     OPT_COMBINE_PIPELINE, OPT_COPY_VEC_BYTES, OPT_ROUTE_IN_COPY, \
-    OPT_FP8_EXPERTS_KERNEL, OPT_COMBINE_COMPACT = range(20)
+    OPT_FP8_EXPERTS_KERNEL = range(19)
 
 
 class EpA2AError(RuntimeError):

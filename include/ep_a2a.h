@@ -396,13 +396,7 @@ typedef enum {
                                      through distributed shared memory; 1 = a cluster per
                                      token with one column vector per thread and the rows
                                      in registers (hidden up to 16384); 2 = one CTA per
-                                     token with the whole rows in shared memory */,
-  EP_A2A_OPT_COMBINE_COMPACT = 19 /* BF16 / FP8 / scaled FP8 combines below 8192 token
-                                     slots with empty slots (ragged or masked ranks):
-                                     1 (default) = the CTAs walk the existing tokens
-                                     only (rank r's first n[r] slots, from the last
-                                     dispatch's counts); 0 = every slot, the empty
-                                     ones found from the plan */
+                                     token with the whole rows in shared memory */
 } ep_a2a_option;
 ep_a2a_status ep_a2a_set_option(ep_a2a_handle handle, ep_a2a_option option, int64_t value);
 

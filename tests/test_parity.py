@@ -380,49 +380,6 @@ def test_pipelined_combines_match_the_oracle(case, prefetch, threads):
                                                   U.to_np(y), H, out_init=init), "experts")
 
 
-@pytest.mark.parametrize("compact", [0, 1])
-@pytest.mark.parametrize("name", ["c5_ep64_wide_masked", "mask", "odd", "ragged"])
-def test_combines_over_existing_tokens(name, compact):
-    """BF16, FP8 and scaled-FP8 combines that walk only the existing tokens
-    (ragged counts and masked ranks leave empty slots; the prefix counts come
-    from the routing kernel) against walking every slot: the oracle's output,
-    empty slots untouched."""
-    from combine_route_plan_b200 import ep_a2a
-    if name in W.BY_NAME:
-        w = W.BY_NAME[name]
-        x = _inputs(w.name)
-    elif name == "mask":
-        w, x = _custom(8, 64, 6, 40, 64, [32], n=[40, 1, 0, 39, 17, 40, 2, 33],
-                       mask=[0b10100101, 0, 0, 0], seed=8)
-    elif name == "odd":
-        w, x = _custom(4, 16, 4, 30, 40, [32], n=[30, 0, 7, 29], seed=19)
-    else:
-        w, x = _custom(16, 64, 8, 33, 256, [32], n=[33, 0, 0, 1, 32, 5, 0, 33, 9, 0, 0, 0, 2, 31,
-                                                    0, 17], seed=29)
-    run = U.Run(w, W.Inputs(w, x.token_selected_experts, x.local_num_tokens, x.payloads,
-                            x.eplb_local_stats, x.active_rank_mask, None),
-                options={ep_a2a.OPT_COMBINE_COMPACT: compact})
-    plan = U.oracle_plan(w, x)
-    xo, H = x.expert_output, w.hidden
-
-    def fresh():
-        return torch.full((w.ep_size, w.tokens_per_rank, H), U.OUT_CANARY, dtype=torch.int16,
-                          device="cuda").view(torch.bfloat16)
-    out, out8, outs = fresh(), fresh(), fresh()
-    run.comm.combine(xo.cuda(), out)
-    run.comm.combine(ep_a2a.quantize_e4m3(xo.cuda()), out8)
-    codes, scales = ep_a2a.quantize_e4m3_rows(xo.cuda())
-    run.comm.combine_scaled(codes, scales, outs)
-    torch.cuda.synchronize()
-    assert run.comm.get_status() == ep_a2a.OK
-    init = U.oracle_out_init(w)
-    xq = U.oracle_e4m3_rows_read(U.to_np(xo), plan, U.oracle_e4m3_table())
-    oc, osc = U.oracle_row_quantize_read(U.to_np(xo), plan, H)
-    U.assert_equal(out, U.oracle.combine(plan, U.to_np(xo), H, out_init=init), "bf16")
-    U.assert_equal(out8, U.oracle.combine(plan, xq, H, input_is_e4m3=True, out_init=init), "fp8")
-    U.assert_equal(outs, U.oracle.combine_scaled(plan, oc, osc, H, out_init=init), "scaled")
-
-
 @pytest.mark.parametrize("case,ctas", [
     (("c2_ep8_decode", None), 0),
     (("c2_ep8_decode", None), 3),
