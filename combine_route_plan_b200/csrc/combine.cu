@@ -1030,8 +1030,17 @@ __global__ void __launch_bounds__(256, 3) combine_experts_fp8_split_kernel(
   const int cvec = cols / 8;                       // vectors of this CTA's slice
   const int vbase = (int)cr * cvec;
   const int64_t clusters = gridDim.x / C;
+  const int pf_bytes = (min(cvec, nvec - vbase) > 0 ? min(cvec, nvec - vbase) : 0) * 16;
   int parity = 0;
   for (int64_t tok = blockIdx.x / C; tok < a.ntok; tok += clusters) {
+    if (a.prefetch && (int)threadIdx.x < a.k && pf_bytes > 0) {
+      // this CTA's slice of each slot row of the token a.prefetch steps ahead
+      // into L2 while this one is summed
+      const int64_t nt = tok + (int64_t)a.prefetch * clusters;
+      if (nt < a.ntok)
+        prefetch_l2(a.y + (nt * a.k + threadIdx.x) * (int64_t)a.H + (int64_t)vbase * 8,
+                    (uint32_t)pf_bytes);
+    }
     const int nd = a.plan_nd[tok];                 // the same in every CTA of the cluster
     if (nd == kNoToken) continue;
     uint16_t* out = a.out + tok * (int64_t)a.H;

@@ -838,7 +838,11 @@ EP_API ep_a2a_status ep_a2a_combine_experts_fp8(ep_a2a_handle h, const float* to
   a.plan_stride = h->L.plan_stride;
   a.ep = h->p.ep_size;
   a.err = reinterpret_cast<uint32_t*>(h->ws + h->L.off_err);
-  a.prefetch = 0;
+  // the split kernel (below) prefetches a CTA's slice of the slot rows of the
+  // token this many steps ahead: automatic 1 from 8192 token slots (prefill:
+  // 1389 against 1426 us; Zipf 328 against 336 us), 0 below (slower by 4-5 %
+  // on the decode and wide-EP steps)
+  a.prefetch = h->combine_prefetch >= 0 ? h->combine_prefetch : (a.ntok >= 8192 ? 1 : 0);
   const bool vec8 = a.k <= 8 && a.H % 8 == 0 && aligned(expert_output_per_slot, 16) &&
                     aligned(output, 16);
   const int nvec = a.H / 8;

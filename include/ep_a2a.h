@@ -364,8 +364,9 @@ typedef enum {
                                      its token p grid strides ahead to be brought into L2
                                      (cp.async.bulk.prefetch.L2) while it sums the current
                                      one; 0 = never; -1 (default) = automatic: 1 for the
-                                     FP8 combines from 8192 token slots and the BF16
-                                     combine from 8192 to 16383, else 0 */
+                                     FP8 combines from 8192 token slots, the BF16
+                                     combine from 8192 to 16383 and the sender-side FP8
+                                     expert combine (its split kernel) from 8192, else 0 */
   EP_A2A_OPT_COPY_PREFETCH = 14,  /* vector copy: 1 = the same for the next token's rows;
                                      0 = never; -1 (default) = automatic: 1 where the
                                      automatic grid is 4 CTAs per SM, else 0 */
