@@ -806,6 +806,34 @@ def test_ones_combine_counts_destinations():
 # Host validation that needs a live handle, and the bounded-wait status path
 # --------------------------------------------------------------------------- #
 
+@pytest.mark.parametrize("option,good,bad", [
+    ("VEC_CTAS_PER_SM", [0, 1, 4, 64], [-1, 65]),
+    ("COPY_PREFETCH", [-1, 0, 1], [-2, 2]),
+    ("COMBINE_PREFETCH", [-1, 0, 1, 4], [-2, 5]),
+    ("COMBINE_THREADS", [0, 64, 96, 128, 192, 512], [32, 100, 544]),
+    ("COMBINE_CTAS_PER_SM", [0, 1, 1024], [-1, 1025]),
+    ("VEC_THREADS_PER_TOKEN", [0, 32, 64, 128, 256], [16, 48, 512]),
+    ("FP8_EXPERTS_KERNEL", [0, 1, 2], [-1, 3]),
+])
+def test_option_ranges(option, good, bad):
+    """Every value an option documents is accepted and the ones outside are
+    rejected with EP_A2A_ERR_INVALID_ARG, leaving the handle usable."""
+    from combine_route_plan_b200 import ep_a2a
+    comm = ep_a2a.EpA2A(4, 16, 2, 8, 32, [32])
+    opt = getattr(ep_a2a, "OPT_" + option)
+    for v in good:
+        comm.set_option(opt, v)
+    for v in bad:
+        with pytest.raises(ep_a2a.EpA2AError) as e:
+            comm.set_option(opt, v)
+        assert e.value.status == ep_a2a.ERR_INVALID_ARG
+    ids = torch.zeros((4, 8, 2), dtype=torch.int32, device="cuda")
+    pay = torch.zeros((4, 8, 32), dtype=torch.uint8, device="cuda")
+    comm.dispatch(ids, [8] * 4, [pay], 8)
+    torch.cuda.synchronize()
+    assert comm.get_status() == ep_a2a.OK
+
+
 def test_dispatch_and_combine_validation():
     from combine_route_plan_b200 import ep_a2a
     ep, E, k, tpr, H = 4, 16, 2, 8, 32
