@@ -1,8 +1,9 @@
 // Combine of rank-major MoE dispatch (flashinfer.moe_ep.NVLinkTwoSidedAlltoAll,
 // combine()): each existing token (src, t) gets the sum of the rows its
 // destination ranks return, each row being that rank's experts' outputs for the
-// token with the routing weights applied and summed.  The sum is an fp32 accumulator that starts at +0.0f and adds the
-// rows in ascending destination-rank order with round-to-nearest adds, then is
+// token with the routing weights applied and summed.  The sum is an fp32
+// accumulator that starts at +0.0f and adds the rows in ascending
+// destination-rank order with round-to-nearest adds, then is
 // rounded once to bf16 (nearest-even).  With the low-precision combine
 // (flashinfer.moe_ep.NVLinkOneSidedConfig, use_low_precision_combine) the rows
 // are E4M3, widened exactly to fp32 before the same sum.

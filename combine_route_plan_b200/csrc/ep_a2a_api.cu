@@ -409,7 +409,8 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
   if (st != EP_A2A_OK) return st;
   switch (option) {
     case EP_A2A_OPT_COPY_PATH:
-      if (value < 0 || value > 2) return fail(EP_A2A_ERR_INVALID_ARG, "copy path must be 0, 1 or 2");
+      if (value < 0 || value > 2)
+        return fail(EP_A2A_ERR_INVALID_ARG, "copy path must be 0, 1 or 2");
       h->copy_path = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_COPY_CTAS_PER_SM:
@@ -433,7 +434,8 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       h->copy_consumer_warps = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_COPY_INTERLEAVE:
-      if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "interleave must be 0 or 1");
+      if (value != 0 && value != 1)
+        return fail(EP_A2A_ERR_INVALID_ARG, "interleave must be 0 or 1");
       h->copy_interleave = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_VEC_UNROLL:
@@ -497,7 +499,8 @@ EP_API ep_a2a_status ep_a2a_set_option(ep_a2a_handle h, ep_a2a_option option, in
       h->fp8_experts_kernel = (int)value;
       return EP_A2A_OK;
     case EP_A2A_OPT_ROUTE_IN_COPY:
-      if (value != 0 && value != 1) return fail(EP_A2A_ERR_INVALID_ARG, "route in copy must be 0 or 1");
+      if (value != 0 && value != 1)
+        return fail(EP_A2A_ERR_INVALID_ARG, "route in copy must be 0 or 1");
       h->route_in_copy = (int)value;
       return EP_A2A_OK;
   }
@@ -1034,7 +1037,8 @@ EP_API ep_a2a_status ep_a2a_profile_stop(ep_a2a_handle h, ep_a2a_kernel_times* t
   for (size_t i = 0; i < h->prof_kernel.size(); ++i) {
     cudaError_t e = cudaEventSynchronize(h->prof_events[2 * i + 1]);
     float ms = 0.f;
-    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, h->prof_events[2 * i], h->prof_events[2 * i + 1]);
+    if (e == cudaSuccess)
+      e = cudaEventElapsedTime(&ms, h->prof_events[2 * i], h->prof_events[2 * i + 1]);
     if (e != cudaSuccess) {
       prof_free(h);
       return cuda_fail(e, "reading profiling events");

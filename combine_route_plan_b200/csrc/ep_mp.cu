@@ -445,7 +445,8 @@ EP_API ep_a2a_status ep_mp_init(const ep_a2a_params* params, int32_t rank, void*
   if (st != EP_A2A_OK) return st;
   if (!out_handle) return mp_fail(EP_A2A_ERR_INVALID_ARG, "out_handle is NULL");
   *out_handle = nullptr;
-  if (rank < 0 || rank >= params->ep_size) return mp_fail(EP_A2A_ERR_INVALID_ARG, "rank out of range");
+  if (rank < 0 || rank >= params->ep_size)
+    return mp_fail(EP_A2A_ERR_INVALID_ARG, "rank out of range");
   if (!window || !peers) return mp_fail(EP_A2A_ERR_INVALID_ARG, "window / peers is NULL");
   if (reinterpret_cast<uintptr_t>(window) % kMpAlign != 0)
     return mp_fail(EP_A2A_ERR_INVALID_ARG, "window must be 256-byte aligned");
